@@ -1,0 +1,8 @@
+"""FP4 (E2M1) microscaling with FP8 (E4M3 / UE5M3) block scales on B200 (sm_100a).
+
+The CUDA library (libmxfp4_b200.so, C ABI in include/mx.h) does the work: quantize + pack,
+dequantize, the three-term block-error reduction and the per-tensor FP16 scale.  This package is a
+thin binding over it; importing it fails when the library is missing.
+"""
+from .api import (E4M3, UE5M3, ErrorStats, MXError, dequantize, error_stats,  # noqa: F401
+                  fmt_code, g_bits, global_scale, kernel_launches, quantize, stats_workspace)

@@ -1,0 +1,59 @@
+"""ctypes binding of libmxfp4_b200.so (the C ABI in include/mx.h).
+
+Argument marshalling only: every step of the method runs in the library's CUDA kernels.  PyTorch is
+used for device memory and streams.  Importing this module fails loudly when the library has not
+been built; there is no fallback.
+"""
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxfp4_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m fp4_microscaling_tensor_b200.build` "
+        "(nvcc, sm_100a) or __graft_entry__.build()")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+MX_OK, MX_ERR_INVALID_ARG, MX_ERR_UNSUPPORTED, MX_ERR_MISALIGNED, MX_ERR_WORKSPACE, MX_ERR_CUDA = \
+    range(6)
+MX_F32, MX_BF16 = 0, 1
+MX_SCALE_E4M3, MX_SCALE_UE5M3 = 0, 1
+
+# every symbol declared in include/mx.h
+EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_error_stats",
+           "mx_global_scale_workspace_size", "mx_global_scale", "mx_status_string",
+           "mx_kernel_launches")
+
+_i, _i64, _u16, _vp, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_uint16, ctypes.c_void_p, ctypes.c_size_t
+
+lib.mx_quantize.restype = _i
+lib.mx_quantize.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp]
+lib.mx_dequantize.restype = _i
+lib.mx_dequantize.argtypes = [_vp, _vp, _i64, _i64, _i, _i, _u16, _vp, _i, _vp]
+lib.mx_error_stats_workspace_size.restype = _sz
+lib.mx_error_stats_workspace_size.argtypes = [_i64, _i64, _i]
+lib.mx_error_stats.restype = _i
+lib.mx_error_stats.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.mx_global_scale_workspace_size.restype = _sz
+lib.mx_global_scale_workspace_size.argtypes = [_i64, _i64]
+lib.mx_global_scale.restype = _i
+lib.mx_global_scale.argtypes = [_vp, _i, _i64, _i64, _i, _vp, _vp, _sz, _vp]
+lib.mx_status_string.restype = ctypes.c_char_p
+lib.mx_status_string.argtypes = [_i]
+lib.mx_kernel_launches.restype = ctypes.c_longlong
+lib.mx_kernel_launches.argtypes = []
+
+
+class MXError(RuntimeError):
+    """A non-OK mx_status returned by the library."""
+
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {lib.mx_status_string(status).decode()}")
+
+
+def check(status, where):
+    if status != MX_OK:
+        raise MXError(status, where)

@@ -1,0 +1,151 @@
+"""Python API over the C ABI: quantize, dequantize, error_stats, global_scale.
+
+Tensors are CUDA tensors, contiguous, row-major, with blocks along the last dimension.  Outputs are
+allocated with torch on the tensor's device unless given.  Calls are asynchronous on the current
+torch stream (or `stream=`); nothing here synchronizes except ErrorStats.to_dict().
+"""
+import struct
+
+import numpy as np
+import torch
+
+from ._lib import (MX_BF16, MX_F32, MX_SCALE_E4M3, MX_SCALE_UE5M3, MXError, check,  # noqa: F401
+                   lib)
+
+E4M3, UE5M3 = MX_SCALE_E4M3, MX_SCALE_UE5M3
+_FMT = {"e4m3": E4M3, "ue5m3": UE5M3, E4M3: E4M3, UE5M3: UE5M3}
+_DT = {torch.float32: MX_F32, torch.bfloat16: MX_BF16}
+STATS_BYTES = 64
+STATS_FIELDS = ("sse_elem", "sse_max", "sse_zero", "numel", "n_blocks", "n_zero_blocks",
+                "n_scale_sat", "n_elem_sat")
+
+
+def fmt_code(fmt):
+    try:
+        return _FMT[fmt.lower() if isinstance(fmt, str) else fmt]
+    except KeyError:
+        raise ValueError(f"unknown scale format {fmt!r}") from None
+
+
+def g_bits(g):
+    """binary16 bit pattern of the per-tensor scale: a float (rounded to fp16) or an int pattern."""
+    if g is None:
+        return 0x3C00
+    if isinstance(g, (int, np.integer)) and not isinstance(g, bool):
+        return int(g) & 0xFFFF
+    return int(np.array([g], np.float16).view(np.uint16)[0])
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes_stream(stream)
+
+
+def ctypes_stream(stream):
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _shape2d(t, what):
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if t.dim() == 0:
+        raise ValueError(f"{what} must have at least one dimension")
+    cols = t.shape[-1]
+    rows = t.numel() // cols if cols else 0
+    return rows, cols
+
+
+def quantize(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, stream=None):
+    """Quantize + pack.  Returns (packed uint8 [..., cols/2], scales uint8 [..., cols/block])."""
+    rows, cols = _shape2d(x, "x")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    lead = tuple(x.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+                             device=x.device)
+    check(lib.mx_quantize(x.data_ptr(), _DT[x.dtype], rows, cols, int(block), fmt_code(fmt),
+                          g_bits(g), packed.data_ptr(), scales.data_ptr(),
+                          _stream(stream, x.device)), "mx_quantize")
+    return packed, scales
+
+
+def dequantize(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=torch.bfloat16, out=None,
+               stream=None):
+    """Dequantize packed codes and block scales into a [..., cols] tensor of out_dtype."""
+    if out_dtype not in _DT:
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    prow, pcols = _shape2d(packed, "packed")
+    _shape2d(scales, "scales")
+    cols = 2 * pcols
+    if out is None:
+        out = torch.empty(tuple(packed.shape[:-1]) + (cols,), dtype=out_dtype, device=packed.device)
+    check(lib.mx_dequantize(packed.data_ptr(), scales.data_ptr(), prow, cols, int(block),
+                            fmt_code(fmt), g_bits(g), out.data_ptr(), _DT[out.dtype],
+                            _stream(stream, packed.device)), "mx_dequantize")
+    return out
+
+
+class ErrorStats:
+    """Device-resident mx_error_stats_t (64 bytes); to_dict() copies it to the host."""
+
+    def __init__(self, tensor):
+        self.tensor = tensor
+
+    def to_dict(self):
+        raw = self.tensor.cpu().numpy().tobytes()
+        vals = struct.unpack("<3d5q", raw)
+        d = dict(zip(STATS_FIELDS, vals))
+        n = d["numel"] or 1
+        d.update(mse_elem=d["sse_elem"] / n, mse_max=d["sse_max"] / n, mse_zero=d["sse_zero"] / n)
+        d["mse_total"] = d["mse_elem"] + d["mse_max"] + d["mse_zero"]
+        return d
+
+
+def stats_workspace(device, rows=0, cols=0, block=32):
+    n = lib.mx_error_stats_workspace_size(rows, cols, block)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def error_stats(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, out=None,
+                workspace=None, stream=None):
+    """Three-term error sums of quantizing x (codes recomputed when packed is None)."""
+    rows, cols = _shape2d(x, "x")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(STATS_BYTES, dtype=torch.uint8, device=x.device)
+    if workspace is None:
+        workspace = stats_workspace(x.device, rows, cols, block)
+    check(lib.mx_error_stats(x.data_ptr(), _DT[x.dtype], rows, cols, int(block), fmt_code(fmt),
+                             g_bits(g), None if packed is None else packed.data_ptr(),
+                             None if scales is None else scales.data_ptr(), out.data_ptr(),
+                             workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)),
+          "mx_error_stats")
+    return ErrorStats(out)
+
+
+def global_scale(x, fmt="e4m3", out=None, workspace=None, stream=None):
+    """Per-tensor FP16 scale of x, as a device uint16 tensor of one element (bit pattern)."""
+    rows, cols = _shape2d(x, "x")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(8, dtype=torch.uint8, device=x.device)  # 16-byte aligned allocation
+    if workspace is None:
+        workspace = torch.empty(lib.mx_global_scale_workspace_size(rows, cols), dtype=torch.uint8,
+                                device=x.device)
+    check(lib.mx_global_scale(x.data_ptr(), _DT[x.dtype], rows, cols, fmt_code(fmt),
+                              out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              _stream(stream, x.device)), "mx_global_scale")
+    return out[:2].view(torch.uint16)
+
+
+def kernel_launches():
+    """Number of kernels the library has enqueued in this process (diagnostic)."""
+    return int(lib.mx_kernel_launches())

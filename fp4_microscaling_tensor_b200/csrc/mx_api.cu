@@ -1,0 +1,151 @@
+// mx_api.cu -- the C ABI declared in include/mx.h: argument checks on the host, then the kernel
+// launches of mx_quantize.cu, mx_dequantize.cu, mx_error_stats.cu and mx_global_scale.cu on the
+// caller's stream.  Nothing is allocated and nothing is synchronized here.
+#include <atomic>
+
+#include "../../include/mx.h"
+#include "mx_device.cuh"
+#include "mx_launch.h"
+
+static_assert(sizeof(mx_error_stats_t) == 64, "mx_error_stats_t layout");
+
+namespace {
+
+std::atomic<long long> g_launches{0};  // diagnostic: kernels enqueued by this library
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_block(int block) {
+  return block == 4 || block == 8 || block == 16 || block == 32 || block == 64 || block == 128 ||
+         block == 256;
+}
+
+// g must be a finite, positive binary16 (subnormals allowed).
+bool valid_g(uint16_t g) {
+  const unsigned e = (g >> 10) & 31u;
+  return (g & 0x8000u) == 0 && e != 31u && (g & 0x7FFFu) != 0;
+}
+
+bool valid_dtype(int t) { return t == MX_F32 || t == MX_BF16; }
+bool valid_fmt(int f) { return f == MX_SCALE_E4M3 || f == MX_SCALE_UE5M3; }
+
+// rows, cols >= 0, product representable; returns false on overflow.
+bool shape_ok(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return false;
+  if (rows != 0 && cols > (int64_t(1) << 62) / rows) return false;
+  return true;
+}
+
+mx_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
+
+size_t stats_ws_bytes() { return (size_t)mxk::kMaxReduceCtas * 64; }
+size_t amax_ws_bytes() { return (size_t)mxk::kMaxReduceCtas * 4; }
+
+}  // namespace
+
+extern "C" {
+
+mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                      mx_scale_fmt fmt, uint16_t global_scale_fp16, uint8_t* packed,
+                      uint8_t* scales, cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  if (cols % block != 0) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel == 0) return MX_OK;
+  if (!x || !packed || !scales) return MX_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales)) return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
+                                          global_scale_fp16, packed, scales, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t cols,
+                        int block, mx_scale_fmt fmt, uint16_t global_scale_fp16, void* y,
+                        mx_dtype yt, cudaStream_t stream) {
+  if (!valid_dtype(yt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  if (cols % block != 0) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel == 0) return MX_OK;
+  if (!packed || !scales || !y) return MX_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(y)) return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_dequantize(packed, scales, numel, block, (int)fmt,
+                                            global_scale_fp16, y, yt == MX_BF16, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int block) {
+  (void)rows;
+  (void)cols;
+  (void)block;
+  return stats_ws_bytes();
+}
+
+mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                         mx_scale_fmt fmt, uint16_t global_scale_fp16, const uint8_t* packed,
+                         const uint8_t* scales, mx_error_stats_t* out_dev, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  if (cols % block != 0) return MX_ERR_INVALID_ARG;
+  if ((packed == nullptr) != (scales == nullptr)) return MX_ERR_INVALID_ARG;
+  if (!out_dev) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel != 0 && !x) return MX_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < stats_ws_bytes()) return MX_ERR_WORKSPACE;
+  if ((numel != 0 && !aligned16(x)) || !aligned16(out_dev) || !aligned16(workspace) ||
+      (packed && (!aligned16(packed) || !aligned16(scales))))
+    return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e =
+      mxk::run_error_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
+                           global_scale_fp16, packed, scales, out_dev, workspace, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols) {
+  (void)rows;
+  (void)cols;
+  return amax_ws_bytes();
+}
+
+mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols, mx_scale_fmt fmt,
+                          uint16_t* out_fp16_dev, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt) || !shape_ok(rows, cols)) return MX_ERR_INVALID_ARG;
+  if (!out_fp16_dev) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel != 0 && !x) return MX_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < amax_ws_bytes()) return MX_ERR_WORKSPACE;
+  if ((numel != 0 && !aligned16(x)) || !aligned16(workspace)) return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_global_scale(x, xt == MX_BF16, numel, (int)fmt, out_fp16_dev,
+                                              workspace, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+const char* mx_status_string(mx_status status) {
+  switch (status) {
+    case MX_OK: return "MX_OK";
+    case MX_ERR_INVALID_ARG: return "MX_ERR_INVALID_ARG: invalid argument";
+    case MX_ERR_UNSUPPORTED: return "MX_ERR_UNSUPPORTED: block size not in {4,8,16,32,64,128,256}";
+    case MX_ERR_MISALIGNED: return "MX_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case MX_ERR_WORKSPACE: return "MX_ERR_WORKSPACE: workspace missing or too small";
+    case MX_ERR_CUDA: return "MX_ERR_CUDA: CUDA runtime error while enqueueing";
+    default: return "unknown mx_status";
+  }
+}
+
+long long mx_kernel_launches(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+// mx_dequantize.cu -- dequantize kernel (sm_100a).
+//
+// Method: the microscaling article (hotelren.com/news/2192771) §1 and §3.1 item 3: the stored value
+// is FP4 x FP8_scale x FP16_scale.  The product of an E2M1 value (<= 2 significant bits), an FP8
+// scale (<= 4) and the FP16 g (<= 11) has at most 17 significant bits and stays inside the fp32
+// normal range, so y = e2m1 * (S g) is exact in fp32; bf16 output is its round-to-nearest-even.
+//
+// Layout mirrors the quantize kernel: a thread owns EPT consecutive codes (16 for bf16 output with
+// N >= 16, else 8), reads EPT/2 packed bytes and the scale byte(s) of its block(s), decodes the
+// codes, multiplies by the per-code constant S g from a
+// shared-memory table and writes 16-byte vectors.  Codes are decoded with exact bit arithmetic
+// (e2m1_scaled_bits_at), not with a conversion instruction.
+#include "mx_device.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+
+template <int N, bool BF16OUT>
+struct DShape {
+  static constexpr int EPT = (BF16OUT && N >= 16) ? 16 : 8;
+  static constexpr int L = (N >= EPT) ? N / EPT : 1;
+  static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
+  static constexpr int U = 2;
+};
+
+template <int N, int FMT, bool BF16OUT>
+__global__ void __launch_bounds__(kThreads) k_dequantize(const uint8_t* __restrict__ packed,
+                                                          const uint8_t* __restrict__ scales,
+                                                          int64_t nitems, uint16_t g_bits,
+                                                          void* __restrict__ y) {
+  using S = DShape<N, BF16OUT>;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U;
+  __shared__ float s_D[256];
+  const float g = fp16_bits_to_float(g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+  __syncthreads();
+
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t base = tid; base < nitems; base += T * U) {
+    uint32_t cw[U][EPT / 8];
+    uint32_t sc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + (int64_t)u * T;
+      cw[u][0] = 0;
+      if (EPT == 16) cw[u][EPT / 8 - 1] = 0;
+      sc[u] = 0;
+      if (i < nitems) {
+        if constexpr (EPT == 16) {
+          const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
+          cw[u][0] = p.x;
+          cw[u][EPT / 8 - 1] = p.y;
+        } else {
+          cw[u][0] = __ldcs(reinterpret_cast<const unsigned int*>(packed) + i);
+        }
+        if constexpr (BPI == 1)
+          sc[u] = __ldg(scales + i / L);
+        else if constexpr (BPI == 2)
+          sc[u] = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + (int64_t)u * T;
+      if (i >= nitems) continue;
+      float out[EPT];
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        const float D = s_D[(sc[u] >> (8 * b)) & 0xFF];
+        constexpr int BE = EPT / BPI;
+#pragma unroll
+        for (int k = 0; k < BE; ++k) {
+          const int e = b * BE + k;  // element index in the item: nibble e % 8 of word e / 8
+          const float f = __uint_as_float(e2m1_scaled_bits_at(cw[u][e / 8], 4 * (e % 8)));
+          out[e] = __fmul_rn(__fmul_rn(f, 0x1p126f), D);
+        }
+      }
+      if constexpr (BF16OUT) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + i * EPT);
+#pragma unroll
+        for (int h = 0; h < EPT / 8; ++h)
+          __stcs(dst + h, make_uint4(pack_bf16x2(out[8 * h], out[8 * h + 1]),
+                                     pack_bf16x2(out[8 * h + 2], out[8 * h + 3]),
+                                     pack_bf16x2(out[8 * h + 4], out[8 * h + 5]),
+                                     pack_bf16x2(out[8 * h + 6], out[8 * h + 7])));
+      } else {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + i * EPT);
+#pragma unroll
+        for (int h = 0; h < EPT / 4; ++h)
+          __stcs(dst + h, make_float4(out[4 * h], out[4 * h + 1], out[4 * h + 2], out[4 * h + 3]));
+      }
+    }
+  }
+}
+
+// The last 4 codes when N = 4 and numel % 8 == 4.
+template <int FMT, bool BF16OUT>
+__global__ void k_dequantize_tail4(const uint8_t* __restrict__ packed,
+                                   const uint8_t* __restrict__ scales, int64_t first,
+                                   uint16_t g_bits, void* __restrict__ y) {
+  if (threadIdx.x >= 4) return;
+  const int64_t e = first + threadIdx.x;
+  const float D = __fmul_rn(scale_value(scales[first / 4], FMT), fp16_bits_to_float(g_bits));
+  const uint32_t nib = (uint32_t)(packed[e / 2] >> (4 * (e & 1))) & 0xFu;
+  const float v = __fmul_rn(e2m1_to_float(nib), D);
+  if (BF16OUT)
+    reinterpret_cast<__nv_bfloat16*>(y)[e] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(y)[e] = v;
+}
+
+template <int N, int FMT, bool BF16OUT>
+static cudaError_t launch_dq(const uint8_t* packed, const uint8_t* scales, int64_t numel,
+                             uint16_t g_bits, void* y, cudaStream_t stream, int* launches) {
+  using S = DShape<N, BF16OUT>;
+  const int64_t nitems = numel / S::EPT;
+  if (nitems > 0) {
+    const int grid = persistent_grid((const void*)k_dequantize<N, FMT, BF16OUT>, nitems, S::U);
+    k_dequantize<N, FMT, BF16OUT><<<grid, kThreads, 0, stream>>>(packed, scales, nitems, g_bits, y);
+    ++*launches;
+  }
+  if (numel % S::EPT != 0) {
+    k_dequantize_tail4<FMT, BF16OUT><<<1, 32, 0, stream>>>(packed, scales, nitems * S::EPT,
+                                                            g_bits, y);
+    ++*launches;
+  }
+  return cudaGetLastError();
+}
+
+template <int FMT, bool BF16OUT>
+static cudaError_t dq_block(int block, const uint8_t* p, const uint8_t* s, int64_t numel,
+                            uint16_t g, void* y, cudaStream_t st, int* n) {
+  switch (block) {
+    case 4: return launch_dq<4, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 8: return launch_dq<8, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 16: return launch_dq<16, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 32: return launch_dq<32, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 64: return launch_dq<64, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 128: return launch_dq<128, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    default: return launch_dq<256, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+  }
+}
+
+cudaError_t run_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t numel, int block,
+                           int fmt, uint16_t g_bits, void* y, bool bf16, cudaStream_t stream,
+                           int* launches) {
+  if (fmt == kUE5M3)
+    return bf16 ? dq_block<kUE5M3, true>(block, packed, scales, numel, g_bits, y, stream, launches)
+                : dq_block<kUE5M3, false>(block, packed, scales, numel, g_bits, y, stream, launches);
+  return bf16 ? dq_block<kE4M3, true>(block, packed, scales, numel, g_bits, y, stream, launches)
+              : dq_block<kE4M3, false>(block, packed, scales, numel, g_bits, y, stream, launches);
+}
+
+}  // namespace mxk

@@ -1,0 +1,569 @@
+// mx_error_stats.cu -- fused three-term block-error reduction (sm_100a).
+//
+// Method: the microscaling article (hotelren.com/news/2192771) §2.2 items 1-3.  Per block with a
+// non-zero scale: the max element (first index of max|x|) contributes (x - y)^2 to SSE_max (the
+// scale-rounding error of item 2), every other element to SSE_elem (item 1).  A block whose scale
+// is zero contributes sum x^2 to SSE_zero (item 3).  y is the exact E2M1 * S * g.
+//
+// Pass 1 (k_error_stats_*): persistent grid; each thread walks items like the quantize kernel,
+// either recomputing the codes in registers (RECOMPUTE: reads x only) or reading stored codes.
+//   Arithmetic: a block is scaled by a power of two s that brings its maximum a into [1, 2); the
+//   scaled errors d' = x s - y s are fp32 differences and their squares are summed in fp32 (at
+//   most 16 terms per lane), then scaled back exactly in double.  Squares below 2^-120 in scaled
+//   units would lose digits to fp32 underflow, so each lane tracks its smallest non-zero |x|; in
+//   the rare lane where one falls below 2^-30 a (a block spanning a huge dynamic range), or where a
+//   stored scale is far from the block maximum, the lane recomputes its slice in double.
+//   Elements whose |x| equals the block maximum are kept out of the per-element sums; with
+//   recomputed codes they all carry the same error, so the block's first lane adds that error
+//   (computed in double) once to SSE_max and (count - 1) times to SSE_elem.  With stored codes the
+//   lane holding the first max element adds it to SSE_max and the others to SSE_elem.  Every added
+//   term is non-negative, so exact zeros stay exact.
+// Pass 2 (k_error_stats_final): one CTA adds the per-CTA partials in a fixed order, so results are
+// deterministic for a given device.  No CTA waits on another.
+#include "mx_device.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+
+struct StatsPartial {  // 64 bytes
+  double sse_elem, sse_max, sse_zero, pad;
+  unsigned long long n_zero_blocks, n_scale_sat, n_elem_sat, pad2;
+};
+
+struct StatsOut {  // layout of mx_error_stats_t
+  double sse_elem, sse_max, sse_zero;
+  long long numel, n_blocks, n_zero_blocks, n_scale_sat, n_elem_sat;
+};
+
+template <int N, typename T>
+struct SShape {
+  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? 16 : 8;
+  static constexpr int L = (N >= EPT) ? N / EPT : 1;
+  static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
+  static constexpr int U = 2;
+};
+
+struct Acc {
+  double elem = 0.0, mx = 0.0, zero = 0.0;
+  unsigned n_zero = 0, n_ssat = 0, n_esat = 0;
+};
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_sum(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// CTA-wide reduction of the accumulators into part[blockIdx.x] (fixed order).
+__device__ void write_partial(const Acc& acc, StatsPartial* part) {
+  __shared__ double sd[3][kThreads / 32];
+  __shared__ unsigned long long su[3][kThreads / 32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const double a0 = warp_sum(acc.elem), a1 = warp_sum(acc.mx), a2 = warp_sum(acc.zero);
+  const unsigned long long c0 = warp_sum((unsigned long long)acc.n_zero);
+  const unsigned long long c1 = warp_sum((unsigned long long)acc.n_ssat);
+  const unsigned long long c2 = warp_sum((unsigned long long)acc.n_esat);
+  if (lane == 0) {
+    sd[0][w] = a0; sd[1][w] = a1; sd[2][w] = a2;
+    su[0][w] = c0; su[1][w] = c1; su[2][w] = c2;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    StatsPartial p{};
+    for (int k = 0; k < kThreads / 32; ++k) {
+      p.sse_elem += sd[0][k]; p.sse_max += sd[1][k]; p.sse_zero += sd[2][k];
+      p.n_zero_blocks += su[0][k]; p.n_scale_sat += su[1][k]; p.n_elem_sat += su[2][k];
+    }
+    part[blockIdx.x] = p;
+  }
+}
+
+// Power of two s with a * s in [1, 2) (s from 2^-127 to 2^126) and back = 1 / s^2, exact in double.
+struct BlockScale {
+  float s;
+  double back;
+};
+__device__ __forceinline__ BlockScale block_scale(float a) {
+  int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);  // biased exponent of a >= 0
+  E = max(E, 1);
+  BlockScale b;
+  b.s = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);  // 2^(127 - E)
+  b.back = __longlong_as_double((long long)(769 + 2 * E) << 52);             // 2^(2E - 254)
+  return b;
+}
+
+// Error sums (unscaled, double) of the NE elements of one block held by this lane.
+struct LaneErr {
+  double lt = 0.0;     // elements with |x| < a
+  double mxs = 0.0;    // elements with |x| == a (stored codes only)
+  double first = 0.0;  // the lowest-index element with |x| == a (stored codes only)
+  unsigned cnt = 0;    // elements with |x| == a
+  unsigned nsat = 0;   // elements with |x| > 6 D
+};
+
+// xv: the lane's NE values; code(k): a word whose low nibble is element k's code.  Elements are
+// visited in descending index order so `first` ends on the lowest-index max element.
+template <int NE, bool GIVEN, typename CodeFn>
+__device__ __forceinline__ LaneErr lane_errors(const float* xv, CodeFn code, float a, float D) {
+  LaneErr r;
+  const BlockScale bs = block_scale(a);
+  const float Ds = __fmul_rn(D, bs.s);
+  const float sat6 = __fmul_rn(6.0f, D);
+  // decoded code bits are value * 2^-126: one multiply by D s 2^126 gives y s exactly.  The fast
+  // path needs D s in [2^-30, 2] (or 0): always true for recomputed codes (1/24 < D s <= 1/3)
+  const bool fast_ok = Ds <= 2.0f && (Ds == 0.0f || Ds >= 0x1p-30f);
+  const float Dq = __fmul_rn(fast_ok ? Ds : 0.0f, 0x1p126f);
+  float lt = 0.0f, mxs = 0.0f, first = 0.0f;
+  // smallest non-zero |x| as (bits * 2 - 2) (zero wraps to the top).  With every non-zero |x| at
+  // least a 2^-30, every non-zero scaled error is at least 2^-54 (one unit in the last place of
+  // x s or y s), so its square is a normal fp32 number and nothing is lost to underflow.
+  uint32_t xmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int k = NE - 1; k >= 0; --k) {
+    const float ys = __fmul_rn(__uint_as_float(e2m1_scaled_bits_at(code(k), 0)), Dq);
+    const float d = __fsub_rn(__fmul_rn(xv[k], bs.s), ys);
+    const bool ism = fabsf(xv[k]) == a;
+    const float dl = ism ? 0.0f : d;
+    lt = __fmaf_rn(dl, dl, lt);
+    r.cnt += ism ? 1u : 0u;
+    r.nsat += (fabsf(xv[k]) > sat6) ? 1u : 0u;
+    xmin = min(xmin, __float_as_uint(xv[k]) * 2u - 2u);
+    if constexpr (GIVEN) {
+      const float e2 = __fmul_rn(d, d);
+      if (ism) {
+        mxs = __fadd_rn(mxs, e2);
+        first = e2;
+      }
+    }
+  }
+  if (fast_ok && xmin >= __float_as_uint(__fmul_rn(a, 0x1p-30f)) * 2u - 2u) {
+    r.lt = (double)lt * bs.back;
+    r.mxs = (double)mxs * bs.back;
+    r.first = (double)first * bs.back;
+    return r;
+  }
+  // exact slice in double (rare: a block spanning more than 2^30, or a stored scale far from a)
+  double ltd = 0.0, mxd = 0.0, fd = 0.0;
+#pragma unroll
+  for (int k = NE - 1; k >= 0; --k) {
+    const float y = __fmul_rn(e2m1_to_float(code(k)), D);  // exact
+    const double d = (double)xv[k] - (double)y;            // exact
+    const double e2 = d * d;
+    if (fabsf(xv[k]) == a) {
+      mxd += e2;
+      fd = e2;
+    } else {
+      ltd += e2;
+    }
+  }
+  r.lt = ltd;
+  r.mxs = GIVEN ? mxd : 0.0;
+  r.first = GIVEN ? fd : 0.0;
+  return r;
+}
+
+// Accounting of one block slice (the block's lanes are the L-lane group around `lane`).
+//  recomputed codes: every max-valued element has the error of y_m; the block's first lane adds it.
+//  stored codes: the lane holding the first max element adds its `first` to SSE_max.
+template <int L, bool GIVEN>
+__device__ __forceinline__ void account(Acc& acc, int lane, bool ok, float a, float D, float y_m,
+                                        LaneErr r, float sat_thr) {
+  if (!ok) r = LaneErr{};
+  unsigned cnt = r.cnt;
+  if constexpr (!GIVEN) {
+#pragma unroll
+    for (int off = 1; off < L; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if (D > 0.0f) {
+      acc.elem += r.lt;
+      acc.n_esat += r.nsat;
+    } else {
+      acc.zero += r.lt;
+    }
+    if (ok && (lane & (L - 1)) == 0) {
+      const double dm = (double)a - (double)y_m;  // exact: difference of two floats
+      const double em = dm * dm;
+      if (D > 0.0f) {
+        acc.mx += em;
+        acc.elem += (double)(cnt - 1u) * em;
+      } else {
+        acc.zero += (double)cnt * em;  // y_m = 0 here: em = a^2
+        acc.n_zero += 1;
+      }
+      acc.n_ssat += (a > sat_thr) ? 1u : 0u;
+    }
+  } else {
+    const unsigned gmask =
+        (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(L - 1)));
+    const unsigned has = __ballot_sync(0xffffffffu, cnt > 0) & gmask;
+    const bool is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
+    if (D > 0.0f) {
+      acc.elem += r.lt + (is_first_lane ? r.mxs - r.first : r.mxs);
+      if (is_first_lane) acc.mx += r.first;
+      acc.n_esat += r.nsat;
+    } else {
+      acc.zero += r.lt + r.mxs;
+    }
+    if (ok && (lane & (L - 1)) == 0) {
+      acc.n_zero += (D > 0.0f) ? 0u : 1u;
+      acc.n_ssat += (a > sat_thr) ? 1u : 0u;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// bf16 input
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT, bool RECOMPUTE>
+__global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
+    const uint16_t* __restrict__ x, int64_t nitems, uint16_t g_bits,
+    const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+    StatsPartial* __restrict__ part) {
+  using S = SShape<N, uint16_t>;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
+  constexpr int BW = NW / BPI;  // words per block inside an item
+  constexpr int BE = 2 * BW;    // elements per block inside an item
+  constexpr bool GIVEN = !RECOMPUTE;
+  __shared__ float s_rcp[256], s_D[256];
+  const float g = fp16_bits_to_float(g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+    const float D = __fmul_rn(scale_value(c, FMT), g);
+    s_D[c] = D;
+    s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;
+  }
+  const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
+  const float sat_thr = __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>());  // exact
+  __syncthreads();
+
+  Acc acc;
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t warp0 = tid - (threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+
+  for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
+    uint32_t w[U][NW];
+    uint32_t cw[U][EPT / 8];
+    uint32_t scw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      const bool ok = i < nitems;
+#pragma unroll
+      for (int h = 0; h < NW / 4; ++h) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ok) v = ld_stream16(x + i * EPT + h * 8);
+        w[u][4 * h + 0] = v.x; w[u][4 * h + 1] = v.y; w[u][4 * h + 2] = v.z; w[u][4 * h + 3] = v.w;
+      }
+      scw[u] = 0;
+#pragma unroll
+      for (int j = 0; j < EPT / 8; ++j) cw[u][j] = 0;
+      if constexpr (GIVEN) {
+        if (ok) {
+          if constexpr (EPT == 16) {
+            const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
+            cw[u][0] = p.x; cw[u][1] = p.y;
+          } else {
+            cw[u][0] = __ldcs(reinterpret_cast<const unsigned int*>(packed) + i);
+          }
+          if constexpr (BPI == 1) scw[u] = __ldg(scales + i / L);
+          else scw[u] = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      const bool ok = i < nitems;
+      float xv[EPT];
+#pragma unroll
+      for (int k = 0; k < NW; ++k) {
+        xv[2 * k] = bf16lo(w[u][k]);
+        xv[2 * k + 1] = bf16hi(w[u][k]);
+      }
+      // phase A: block maxima, scale codes and (recomputing) the element quotients
+      float a_b[BPI], D_b[BPI], ym_b[BPI];
+      float qv[EPT];
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        const uint32_t* wb = &w[u][b * BW];
+        uint32_t t = wb[0];
+#pragma unroll
+        for (int k = 1; k < BW; ++k) t = bf16x2_absmax(t, wb[k]);
+        t &= 0x7FFF7FFFu;
+        uint32_t m = max(t & 0xFFFFu, t >> 16);
+#pragma unroll
+        for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float a = __uint_as_float(m << 16);
+        uint32_t s;
+        if constexpr (RECOMPUTE) {
+          s = encode_scale<FMT>(snap21(__fmul_rn(a, r6)));
+          const float r = s_rcp[s];
+          const uint32_t ca =
+              cvt_e2m1x8(snap21(__fmul_rn(a, r)), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+          ym_b[b] = __fmul_rn(e2m1_to_float(ca), s_D[s]);
+#pragma unroll
+          for (int k = 0; k < BE; ++k) qv[b * BE + k] = snap21(__fmul_rn(xv[b * BE + k], r));
+        } else {
+          s = (scw[u] >> (8 * b)) & 0xFF;
+          ym_b[b] = 0.0f;
+        }
+        a_b[b] = a;
+        D_b[b] = s_D[s];
+      }
+      // phase B: codes of the whole item
+      if constexpr (RECOMPUTE) {
+#pragma unroll
+        for (int j = 0; j < EPT / 8; ++j)
+          cw[u][j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3],
+                                qv[8 * j + 4], qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
+      }
+      // phase C: per-element errors and per-block accounting
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        const uint32_t* cwu = cw[u];
+        auto code = [&](int k) {
+          const int e = b * BE + k;
+          return cwu[e / 8] >> (4 * (e % 8));
+        };
+        const LaneErr r = lane_errors<BE, GIVEN>(&xv[b * BE], code, a_b[b], D_b[b]);
+        account<L, GIVEN>(acc, lane, ok, a_b[b], D_b[b], ym_b[b], r, sat_thr);
+      }
+    }
+  }
+  write_partial(acc, part);
+}
+
+// ------------------------------------------------------------------------------------------------
+// fp32 input (codes recomputed with IEEE division, or read)
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT, bool RECOMPUTE>
+__global__ void __launch_bounds__(kThreads) k_error_stats_f32(
+    const float* __restrict__ x, int64_t nitems, uint16_t g_bits,
+    const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+    StatsPartial* __restrict__ part) {
+  using S = SShape<N, float>;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI;
+  constexpr int BE = EPT / BPI;
+  constexpr bool GIVEN = !RECOMPUTE;
+  __shared__ float s_D[256];
+  const float g = fp16_bits_to_float(g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+  const float g6 = __fmul_rn(6.0f, g);
+  const float sat_thr = __fmul_rn(g6, scale_max<FMT>());
+  __syncthreads();
+
+  Acc acc;
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t warp0 = tid - (threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+
+  for (int64_t base = 0; warp0 + base < nitems; base += T) {
+    const int64_t i = tid + base;
+    const bool ok = i < nitems;
+    float v[EPT];
+#pragma unroll
+    for (int h = 0; h < EPT / 4; ++h) {
+      uint4 t = make_uint4(0, 0, 0, 0);
+      if (ok) t = ld_stream16(x + i * EPT + h * 4);
+      v[4 * h] = __uint_as_float(t.x); v[4 * h + 1] = __uint_as_float(t.y);
+      v[4 * h + 2] = __uint_as_float(t.z); v[4 * h + 3] = __uint_as_float(t.w);
+    }
+    uint32_t cw = 0, scw = 0;
+    if (GIVEN && ok) {
+      cw = reinterpret_cast<const unsigned int*>(packed)[i];
+      scw = (BPI == 1) ? scales[i / L] : reinterpret_cast<const unsigned short*>(scales)[i];
+    }
+#pragma unroll
+    for (int b = 0; b < BPI; ++b) {
+      float a = 0.0f;
+#pragma unroll
+      for (int k = 0; k < BE; ++k) a = fmaxf(a, fabsf(v[b * BE + k]));
+#pragma unroll
+      for (int off = 1; off < L; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      uint32_t s, bc = 0;
+      float y_m = 0.0f;
+      if constexpr (RECOMPUTE) {
+        s = encode_scale<FMT>(__fdiv_rn(a, g6));
+        const float D0 = s_D[s];
+        float q[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          q[k] = (k < BE && D0 > 0.0f) ? __fdiv_rn(v[b * BE + (k < BE ? k : 0)], D0)
+                                       : __fmul_rn(k < BE ? v[b * BE + k] : 0.0f, 0.0f);
+        bc = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+        const float qa = D0 > 0.0f ? __fdiv_rn(a, D0) : 0.0f;
+        y_m = __fmul_rn(e2m1_to_float(cvt_e2m1x8(qa, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f)), D0);
+      } else {
+        s = (scw >> (8 * b)) & 0xFF;
+        bc = cw >> (4 * b * BE);
+      }
+      const float D = s_D[s];
+      auto code = [&](int k) { return bc >> (4 * k); };
+      const LaneErr r = lane_errors<BE, GIVEN>(&v[b * BE], code, a, D);
+      account<L, GIVEN>(acc, lane, ok, a, D, y_m, r, sat_thr);
+    }
+  }
+  write_partial(acc, part);
+}
+
+// ------------------------------------------------------------------------------------------------
+// N = 4 tail (4 elements) and the final reduction
+// ------------------------------------------------------------------------------------------------
+
+template <int FMT, typename T>
+__global__ void k_error_stats_tail4(const T* __restrict__ x, int64_t first, uint16_t g_bits,
+                                    const uint8_t* __restrict__ packed,
+                                    const uint8_t* __restrict__ scales, StatsPartial* part) {
+  if (threadIdx.x != 0) return;
+  const float g = fp16_bits_to_float(g_bits);
+  float v[4], a = 0.0f;
+  int imax = 0;
+  for (int k = 0; k < 4; ++k) {
+    if constexpr (sizeof(T) == 2)
+      v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[first + k] << 16);
+    else
+      v[k] = reinterpret_cast<const float*>(x)[first + k];
+    if (fabsf(v[k]) > a) { a = fabsf(v[k]); imax = k; }
+  }
+  uint32_t s, codes[4];
+  if (packed == nullptr) {
+    s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
+    const float D0 = __fmul_rn(scale_value((int)s, FMT), g);
+    for (int k = 0; k < 4; ++k) {
+      const float q = D0 > 0.0f ? __fdiv_rn(v[k], D0) : __fmul_rn(v[k], 0.0f);
+      codes[k] = cvt_e2m1x8(q, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xF;
+    }
+  } else {
+    s = scales[first / 4];
+    for (int k = 0; k < 4; ++k) codes[k] = (packed[(first + k) / 2] >> (4 * ((first + k) & 1))) & 0xF;
+  }
+  const float D = __fmul_rn(scale_value((int)s, FMT), g);
+  StatsPartial p{};
+  for (int k = 0; k < 4; ++k) {
+    const double y = (double)__fmul_rn(e2m1_to_float(codes[k]), D);
+    const double d = (double)v[k] - y;
+    if (!(D > 0.0f)) p.sse_zero += (double)v[k] * (double)v[k];
+    else if (k == imax) p.sse_max += d * d;
+    else p.sse_elem += d * d;
+    if (D > 0.0f && fabsf(v[k]) > __fmul_rn(6.0f, D)) p.n_elem_sat += 1;
+  }
+  p.n_zero_blocks = (D > 0.0f) ? 0 : 1;
+  p.n_scale_sat = (a > __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>())) ? 1 : 0;
+  part[0] = p;
+}
+
+__global__ void __launch_bounds__(kThreads) k_error_stats_final(const StatsPartial* __restrict__ part,
+                                                                int nparts, int64_t numel,
+                                                                int64_t nblocks,
+                                                                StatsOut* __restrict__ out) {
+  double e = 0.0, m = 0.0, z = 0.0;
+  unsigned long long c0 = 0, c1 = 0, c2 = 0;
+  for (int k = threadIdx.x; k < nparts; k += blockDim.x) {  // fixed assignment and order
+    e += part[k].sse_elem; m += part[k].sse_max; z += part[k].sse_zero;
+    c0 += part[k].n_zero_blocks; c1 += part[k].n_scale_sat; c2 += part[k].n_elem_sat;
+  }
+  __shared__ double sd[3][kThreads / 32];
+  __shared__ unsigned long long su[3][kThreads / 32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  e = warp_sum(e); m = warp_sum(m); z = warp_sum(z);
+  c0 = warp_sum(c0); c1 = warp_sum(c1); c2 = warp_sum(c2);
+  if (lane == 0) {
+    sd[0][w] = e; sd[1][w] = m; sd[2][w] = z;
+    su[0][w] = c0; su[1][w] = c1; su[2][w] = c2;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    StatsOut o{};
+    for (int k = 0; k < kThreads / 32; ++k) {
+      o.sse_elem += sd[0][k]; o.sse_max += sd[1][k]; o.sse_zero += sd[2][k];
+      o.n_zero_blocks += (long long)su[0][k]; o.n_scale_sat += (long long)su[1][k];
+      o.n_elem_sat += (long long)su[2][k];
+    }
+    o.numel = numel;
+    o.n_blocks = nblocks;
+    *out = o;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// launcher
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT, typename T, bool RC>
+static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g_bits,
+                             const uint8_t* packed, const uint8_t* scales, void* out,
+                             StatsPartial* part, cudaStream_t stream, int* launches) {
+  using S = SShape<N, T>;
+  const int64_t nitems = numel / S::EPT;
+  int nparts = 0;
+  if (nitems > 0) {
+    const void* kern = (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, RC>
+                                        : (const void*)k_error_stats_f32<N, FMT, RC>;
+    const int grid = persistent_grid(kern, nitems, sizeof(T) == 2 ? S::U : 1, kMaxReduceCtas - 1);
+    if (sizeof(T) == 2)
+      k_error_stats_bf16<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
+          (const uint16_t*)x, nitems, g_bits, packed, scales, part);
+    else
+      k_error_stats_f32<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
+          (const float*)x, nitems, g_bits, packed, scales, part);
+    ++*launches;
+    nparts = grid;
+  }
+  if (numel % S::EPT != 0) {
+    k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits,
+                                                      RC ? nullptr : packed, scales, part + nparts);
+    ++*launches;
+    ++nparts;
+  }
+  k_error_stats_final<<<1, kThreads, 0, stream>>>(part, nparts, numel, numel / block,
+                                                  (StatsOut*)out);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+template <int FMT, typename T, bool RC>
+static cudaError_t st_block(int block, const void* x, int64_t numel, uint16_t g,
+                            const uint8_t* p, const uint8_t* s, void* out, StatsPartial* part,
+                            cudaStream_t st, int* n) {
+  switch (block) {
+    case 4: return launch_st<4, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 8: return launch_st<8, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 16: return launch_st<16, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 32: return launch_st<32, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 64: return launch_st<64, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 128: return launch_st<128, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    default: return launch_st<256, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+  }
+}
+
+template <int FMT, typename T>
+static cudaError_t st_rc(bool rc, int block, const void* x, int64_t numel, uint16_t g,
+                         const uint8_t* p, const uint8_t* s, void* out, StatsPartial* part,
+                         cudaStream_t st, int* n) {
+  return rc ? st_block<FMT, T, true>(block, x, numel, g, p, s, out, part, st, n)
+            : st_block<FMT, T, false>(block, x, numel, g, p, s, out, part, st, n);
+}
+
+cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                            uint16_t g_bits, const uint8_t* packed, const uint8_t* scales,
+                            void* out, void* workspace, cudaStream_t stream, int* launches) {
+  StatsPartial* part = reinterpret_cast<StatsPartial*>(workspace);
+  const bool rc = packed == nullptr;
+  if (bf16)
+    return fmt == kUE5M3
+               ? st_rc<kUE5M3, uint16_t>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches)
+               : st_rc<kE4M3, uint16_t>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches);
+  return fmt == kUE5M3
+             ? st_rc<kUE5M3, float>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches)
+             : st_rc<kE4M3, float>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches);
+}
+
+}  // namespace mxk

@@ -1,0 +1,41 @@
+// mx_launch.h -- host-side launch helpers and the internal kernel entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mxk {
+
+// Upper bound on the CTAs of any reduction kernel; sizes the workspaces.
+constexpr int kMaxReduceCtas = 4096;
+
+// Persistent grid for a grid-stride kernel with kThreads threads: enough CTAs to fill every SM
+// at the kernel's occupancy, never more than the work needs (items / (threads * items_per_iter)).
+inline int persistent_grid(const void* kern, int64_t nitems, int items_per_iter,
+                           int cap = 1 << 30) {
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t full = (int64_t)sms * per_sm;
+  const int64_t need = (nitems + 256LL * items_per_iter - 1) / (256LL * items_per_iter);
+  int64_t g = need < full ? need : full;
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+
+cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                         uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
+                         int* launches);
+cudaError_t run_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t numel, int block,
+                           int fmt, uint16_t g_bits, void* y, bool bf16, cudaStream_t stream,
+                           int* launches);
+// out: device mx_error_stats_t (layout-compatible struct defined in mx.h)
+cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                            uint16_t g_bits, const uint8_t* packed, const uint8_t* scales,
+                            void* out, void* workspace, cudaStream_t stream, int* launches);
+cudaError_t run_global_scale(const void* x, bool bf16, int64_t numel, int fmt, uint16_t* out,
+                             void* workspace, cudaStream_t stream, int* launches);
+
+}  // namespace mxk

@@ -1,0 +1,280 @@
+// mx_quantize.cu -- quantize + pack kernel (sm_100a).
+//
+// Method: the microscaling article (hotelren.com/news/2192771) §3.1 item 2, quantize_block:
+//   abs_max = max|block|; scale = Q_fp8(abs_max / 6); q = Q_fp4(block / scale)
+// with the FP16 per-tensor factor g of §3.1 item 3 (abs_max / (6 g), block / (scale g)), and two
+// FP4 codes per byte (4-bit float article, gtnt.cn/news/16247, §4.3).
+//
+// Layout: the tensor is contiguous row-major and cols % N == 0, so blocks never straddle rows and
+// the whole tensor is one flat run of blocks.  A thread owns EPT consecutive elements (an "item"):
+// EPT = 16 bf16 (32 bytes, two 16-byte loads) when N >= 16 so a block spans N/16 lanes of a warp
+// and its absmax is finished with warp shuffles; EPT = 8 for N in {4, 8} (one or two blocks per
+// item, no shuffles).  fp32 input uses EPT = 8.  Every CTA first builds a 256-entry table of
+// per-scale-code constants in shared memory (1/(S g) for bf16, S g for fp32), so the per-block work
+// is: absmax, one multiply + snap + FP8 encode, one shared-memory lookup.  The grid is persistent
+// (a multiple of the SM count) and walks the items with a grid stride, two items per thread in
+// flight.  No kernel here waits on another CTA.
+#include "mx_device.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+
+template <int N, typename T>
+struct QShape {
+  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? 16 : 8;  // elements per item
+  static constexpr int L = (N >= EPT) ? N / EPT : 1;                // lanes per block
+  static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;              // blocks per item
+  static constexpr int U = 2;                                       // items in flight per thread
+};
+
+// ------------------------------------------------------------------------------------------------
+// bf16 input
+// ------------------------------------------------------------------------------------------------
+
+// Absmax (as non-negative bf16 bits) of words w[k0 .. k0+nw).
+template <int NW>
+__device__ __forceinline__ uint32_t absmax_bits(const uint32_t* w) {
+  uint32_t t = w[0];
+#pragma unroll
+  for (int k = 1; k < NW; ++k) t = bf16x2_absmax(t, w[k]);
+  if (NW == 1) t = bf16x2_absmax(t, t);
+  t &= 0x7FFF7FFFu;
+  return max(t & 0xFFFFu, t >> 16);
+}
+
+template <int N, int FMT>
+__global__ void __launch_bounds__(kThreads) k_quantize_bf16(const uint16_t* __restrict__ x,
+                                                             int64_t nitems, uint16_t g_bits,
+                                                             uint8_t* __restrict__ packed,
+                                                             uint8_t* __restrict__ scales) {
+  using S = QShape<N, uint16_t>;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
+  __shared__ float s_rcp[256];
+  const float g = fp16_bits_to_float(g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+    const float D = __fmul_rn(scale_value(c, FMT), g);  // exact (<= 15 significant bits)
+    s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;          // zero scale -> every code is +-0
+  }
+  const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
+  __syncthreads();
+
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t warp0 = tid - (threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+
+  for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
+    uint32_t w[U][NW];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      ok[u] = i < nitems;
+#pragma unroll
+      for (int h = 0; h < NW / 4; ++h) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ok[u]) v = ld_stream16(x + i * EPT + h * 8);
+        w[u][4 * h + 0] = v.x;
+        w[u][4 * h + 1] = v.y;
+        w[u][4 * h + 2] = v.z;
+        w[u][4 * h + 3] = v.w;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      float qv[EPT];
+      uint32_t sc = 0;
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        constexpr int BW = NW / BPI;  // words per block inside this item
+        uint32_t m = absmax_bits<BW>(&w[u][b * BW]);
+#pragma unroll
+        for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float a = __uint_as_float(m << 16);
+        const uint32_t s = encode_scale<FMT>(snap21(__fmul_rn(a, r6)));
+        const float r = s_rcp[s];
+        sc |= s << (8 * b);
+#pragma unroll
+        for (int k = 0; k < BW; ++k) {
+          const uint32_t wk = w[u][b * BW + k];
+          qv[2 * (b * BW + k)] = snap21(__fmul_rn(bf16lo(wk), r));
+          qv[2 * (b * BW + k) + 1] = snap21(__fmul_rn(bf16hi(wk), r));
+        }
+      }
+      uint32_t codes[EPT / 8];
+#pragma unroll
+      for (int j = 0; j < EPT / 8; ++j)
+        codes[j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3], qv[8 * j + 4],
+                              qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
+      if (!ok[u]) continue;
+      if constexpr (NW == 8) {
+        *reinterpret_cast<uint2*>(packed + i * 8) = make_uint2(codes[0], codes[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(packed + i * 4) = codes[0];
+      }
+      if constexpr (BPI == 1) {
+        if ((lane & (L - 1)) == 0) scales[i / L] = (uint8_t)sc;
+      } else {
+        *reinterpret_cast<uint16_t*>(scales + i * 2) = (uint16_t)sc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// fp32 input: IEEE division (see mx_device.cuh for why the multiply shortcut is not used here)
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT>
+__global__ void __launch_bounds__(kThreads) k_quantize_f32(const float* __restrict__ x,
+                                                            int64_t nitems, uint16_t g_bits,
+                                                            uint8_t* __restrict__ packed,
+                                                            uint8_t* __restrict__ scales) {
+  using S = QShape<N, float>;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U;
+  __shared__ float s_D[256];
+  const float g = fp16_bits_to_float(g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+  const float g6 = __fmul_rn(6.0f, g);
+  __syncthreads();
+
+  const int64_t T = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t warp0 = tid - (threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+
+  for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
+    float v[U][EPT];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      ok[u] = i < nitems;
+#pragma unroll
+      for (int h = 0; h < EPT / 4; ++h) {
+        uint4 t = make_uint4(0, 0, 0, 0);
+        if (ok[u]) t = ld_stream16(x + i * EPT + h * 4);
+        v[u][4 * h + 0] = __uint_as_float(t.x);
+        v[u][4 * h + 1] = __uint_as_float(t.y);
+        v[u][4 * h + 2] = __uint_as_float(t.z);
+        v[u][4 * h + 3] = __uint_as_float(t.w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = tid + base + (int64_t)u * T;
+      float q[EPT];
+      uint32_t sc = 0;
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        constexpr int BE = EPT / BPI;  // elements per block inside this item
+        float a = 0.0f;
+#pragma unroll
+        for (int k = 0; k < BE; ++k) a = fmaxf(a, fabsf(v[u][b * BE + k]));
+#pragma unroll
+        for (int off = 1; off < L; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        const uint32_t s = encode_scale<FMT>(__fdiv_rn(a, g6));
+        const float D = s_D[s];
+        sc |= s << (8 * b);
+#pragma unroll
+        for (int k = 0; k < BE; ++k) {
+          const float xv = v[u][b * BE + k];
+          q[b * BE + k] = D > 0.0f ? __fdiv_rn(xv, D) : __fmul_rn(xv, 0.0f);
+        }
+      }
+      if (!ok[u]) continue;
+      *reinterpret_cast<uint32_t*>(packed + i * 4) =
+          cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      if constexpr (BPI == 1) {
+        if ((lane & (L - 1)) == 0) scales[i / L] = (uint8_t)sc;
+      } else {
+        *reinterpret_cast<uint16_t*>(scales + i * 2) = (uint16_t)sc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// tail: when N = 4 and the element count is not a multiple of 8, the last 4 elements (one block)
+// do not fill an item.  One warp finishes that block with plain per-element code.
+// ------------------------------------------------------------------------------------------------
+
+template <int FMT, typename T>
+__global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_t g_bits,
+                                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scales) {
+  if (threadIdx.x != 0) return;
+  const float g = fp16_bits_to_float(g_bits);
+  float v[4], a = 0.0f;
+  for (int k = 0; k < 4; ++k) {
+    if constexpr (sizeof(T) == 2)
+      v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[first + k] << 16);
+    else
+      v[k] = reinterpret_cast<const float*>(x)[first + k];
+    a = fmaxf(a, fabsf(v[k]));
+  }
+  const uint32_t s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
+  const float D = __fmul_rn(scale_value((int)s, FMT), g);
+  float q[4];
+  for (int k = 0; k < 4; ++k) q[k] = D > 0.0f ? __fdiv_rn(v[k], D) : __fmul_rn(v[k], 0.0f);
+  const uint32_t c = cvt_e2m1x8(q[0], q[1], q[2], q[3], 0.f, 0.f, 0.f, 0.f);
+  packed[first / 2] = (uint8_t)(c & 0xFF);
+  packed[first / 2 + 1] = (uint8_t)((c >> 8) & 0xFF);
+  scales[first / 4] = (uint8_t)s;
+}
+
+// ------------------------------------------------------------------------------------------------
+// launcher
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT, typename T>
+static cudaError_t launch_q(const void* x, int64_t numel, uint16_t g_bits, uint8_t* packed,
+                            uint8_t* scales, cudaStream_t stream, int* launches) {
+  using S = QShape<N, T>;
+  const int64_t nitems = numel / S::EPT;
+  if (nitems > 0) {
+    auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT> : (void*)k_quantize_f32<N, FMT>;
+    const int grid = persistent_grid(kern, nitems, S::U);
+    if (sizeof(T) == 2)
+      k_quantize_bf16<N, FMT><<<grid, kThreads, 0, stream>>>(
+          (const uint16_t*)x, nitems, g_bits, packed, scales);
+    else
+      k_quantize_f32<N, FMT><<<grid, kThreads, 0, stream>>>((const float*)x, nitems, g_bits,
+                                                            packed, scales);
+    ++*launches;
+  }
+  if (numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
+    k_quantize_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits, packed,
+                                                   scales);
+    ++*launches;
+  }
+  return cudaGetLastError();
+}
+
+template <int FMT, typename T>
+static cudaError_t dispatch_block(int block, const void* x, int64_t numel, uint16_t g,
+                                  uint8_t* p, uint8_t* s, cudaStream_t st, int* n) {
+  switch (block) {
+    case 4: return launch_q<4, FMT, T>(x, numel, g, p, s, st, n);
+    case 8: return launch_q<8, FMT, T>(x, numel, g, p, s, st, n);
+    case 16: return launch_q<16, FMT, T>(x, numel, g, p, s, st, n);
+    case 32: return launch_q<32, FMT, T>(x, numel, g, p, s, st, n);
+    case 64: return launch_q<64, FMT, T>(x, numel, g, p, s, st, n);
+    case 128: return launch_q<128, FMT, T>(x, numel, g, p, s, st, n);
+    default: return launch_q<256, FMT, T>(x, numel, g, p, s, st, n);
+  }
+}
+
+cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                         uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
+                         int* launches) {
+  if (bf16)
+    return fmt == kUE5M3
+               ? dispatch_block<kUE5M3, uint16_t>(block, x, numel, g_bits, packed, scales, stream, launches)
+               : dispatch_block<kE4M3, uint16_t>(block, x, numel, g_bits, packed, scales, stream, launches);
+  return fmt == kUE5M3
+             ? dispatch_block<kUE5M3, float>(block, x, numel, g_bits, packed, scales, stream, launches)
+             : dispatch_block<kE4M3, float>(block, x, numel, g_bits, packed, scales, stream, launches);
+}
+
+}  // namespace mxk

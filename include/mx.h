@@ -1,0 +1,136 @@
+/*
+ * mx.h -- C ABI of the B200 (sm_100a) FP4 microscaling library (libmxfp4_b200.so).
+ *
+ * The method (microscaling article, hotelren.com/news/2192771, page titled "企业官网建设流程全解析";
+ * cited below as [MX]):
+ *   - a tensor is cut into blocks of N consecutive values, N in 4..256 ([MX] §1); here a block is
+ *     N consecutive columns of one row, so cols must be a multiple of N;
+ *   - each block gets one FP8 scale s = Q_fp8(absmax / (6 g)) in E4M3 or UE5M3 ([MX] §3.1 items 1-2);
+ *   - each value becomes the FP4 E2M1 code q = Q_fp4(x / (s g)) ([MX] §1, §3.1 item 2);
+ *   - g is an optional per-tensor FP16 factor, value = FP4 x FP8_scale x FP16_scale ([MX] §3.1 item 3);
+ *   - the quantization error splits into three sums ([MX] §2.2 items 1-3).
+ * Q_* rounds to the nearest representable value, ties to the even code, and saturates at the largest
+ * finite value.  E2M1 has no inf/NaN.  E4M3 is the OCP "FN" variant (bias 7, max 448; 0x7F never
+ * produced).  UE5M3 is unsigned, bias 15, with subnormals, every code finite, max 122880.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are caller-owned DEVICE memory, contiguous and row-major.  The library never
+ *     allocates, never synchronizes and keeps no state between calls.
+ *   - Everything is enqueued on `stream` (0 = the legacy default stream); results are valid after
+ *     the caller synchronizes that stream.
+ *   - Arguments are checked on the host before anything is enqueued; a non-OK status means nothing
+ *     was launched.  MX_ERR_CUDA reports a launch error (cudaGetLastError); faults that happen while
+ *     a kernel runs surface at the caller's next synchronization, as usual in CUDA.
+ *   - Every pointer argument must be 16-byte aligned (MX_ERR_MISALIGNED otherwise).
+ *   - rows == 0 or cols == 0 is an empty tensor: quantize / dequantize enqueue nothing,
+ *     mx_error_stats writes an all-zero result and mx_global_scale writes 1.0.
+ *   - x must be finite: NaN or Inf in x gives unspecified codes (no kernel faults or hangs).
+ *   - global_scale_fp16 is the IEEE binary16 bit pattern of g; it must be finite and > 0
+ *     (0x3C00 = 1.0 = no global scale); anything else is MX_ERR_INVALID_ARG.
+ */
+#ifndef MX_H
+#define MX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MX_API __attribute__((visibility("default")))
+#else
+#define MX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MX_OK = 0,
+  MX_ERR_INVALID_ARG = 1, /* null pointer, negative size, cols % block != 0, bad enum, bad g */
+  MX_ERR_UNSUPPORTED = 2, /* block not one of 4, 8, 16, 32, 64, 128, 256 */
+  MX_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+  MX_ERR_WORKSPACE = 4,   /* workspace pointer NULL or smaller than the *_workspace_size() value */
+  MX_ERR_CUDA = 5         /* the CUDA runtime reported an error while enqueueing */
+} mx_status;
+
+typedef enum { MX_F32 = 0, MX_BF16 = 1 } mx_dtype;
+typedef enum { MX_SCALE_E4M3 = 0, MX_SCALE_UE5M3 = 1 } mx_scale_fmt;
+
+/* Result of mx_error_stats ([MX] §2.2).  The SSE fields are sums over the tensor; the pages' mean
+ * squared errors are sse_* / numel, and the three sum to the total MSE. */
+typedef struct {
+  double sse_elem;       /* item 1: (x - y)^2 over every non-max element of blocks with s > 0 */
+  double sse_max;        /* item 2: (x - y)^2 of the max element (first index of max|x|) of blocks
+                            with s > 0, i.e. the error left by rounding the scale */
+  double sse_zero;       /* item 3: x^2 over every element of blocks whose scale is zero */
+  int64_t numel;         /* rows * cols */
+  int64_t n_blocks;      /* rows * cols / block */
+  int64_t n_zero_blocks; /* blocks whose scale code decodes to 0 */
+  int64_t n_scale_sat;   /* blocks with absmax / (6 g) above the largest scale value */
+  int64_t n_elem_sat;    /* elements of blocks with s > 0 and |x| > 6 s g (clipped at +-6) */
+} mx_error_stats_t;
+
+/* Quantize + pack ([MX] §3.1 item 2, with g from §3.1 item 3; packing from the 4-bit float
+ * article, gtnt.cn/news/16247, §4.3, two FP4 values per byte).
+ *   x       rows x cols values of type xt (MX_BF16 or MX_F32), device.
+ *   block   N, one of 4, 8, 16, 32, 64, 128, 256; cols % block == 0.
+ *   fmt     scale format of the block scales.
+ *   packed  OUT rows*cols/2 bytes, device: element 2k of the flattened tensor in the low nibble of
+ *           byte k, element 2k+1 in the high nibble.  Nibble = sign<<3 | E2M1 magnitude code; the
+ *           sign bit is x's sign bit (also for -0.0 and in zero-scale blocks).
+ *   scales  OUT rows*cols/block bytes, device: the FP8 code of each block, row-major.
+ * A block whose scale rounds to zero (absmax <= 3 g smin) stores magnitude 0 in every element. */
+MX_API mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                      mx_scale_fmt fmt, uint16_t global_scale_fp16, uint8_t* packed,
+                      uint8_t* scales, cudaStream_t stream);
+
+/* Dequantize ([MX] §1 and §3.1 item 3: value = FP4 x FP8_scale x FP16_scale).
+ *   packed, scales  as written by mx_quantize (any byte values are accepted; E4M3 codes with the
+ *                   sign bit decode to negative scales, 0x7F / 0xFF to NaN).
+ *   y       OUT rows x cols values of type yt, device.  MX_F32 holds the exact product
+ *           E2M1 * S * g; MX_BF16 holds its round-to-nearest-even. */
+MX_API mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t cols,
+                        int block, mx_scale_fmt fmt, uint16_t global_scale_fp16, void* y,
+                        mx_dtype yt, cudaStream_t stream);
+
+/* Bytes of device workspace mx_error_stats needs (a bound that holds for any device). */
+MX_API size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int block);
+
+/* Three-term error reduction ([MX] §2.2 items 1-3).
+ *   packed, scales  NULL, NULL: the codes are recomputed from x in registers (same rule as
+ *                   mx_quantize, nothing is written); otherwise the given codes are used and only
+ *                   scale codes the quantizer can produce are meaningful (E4M3 0x00..0x7E).
+ *   out_dev  OUT one mx_error_stats_t in device memory (written by the last kernel).
+ *   workspace, ws_bytes  device scratch of at least mx_error_stats_workspace_size() bytes; its
+ *                   contents need no initialisation and are overwritten.
+ * The reconstruction used for the errors is the exact E2M1 * S * g.  Sums are accumulated in
+ * double in a fixed order for a given device, so repeated calls give identical results. */
+MX_API mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                         mx_scale_fmt fmt, uint16_t global_scale_fp16, const uint8_t* packed,
+                         const uint8_t* scales, mx_error_stats_t* out_dev, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of device workspace mx_global_scale needs. */
+MX_API size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols);
+
+/* Per-tensor FP16 scale for [MX] §3.1 item 3.  The pages do not say how g is chosen; this library
+ * takes the smallest binary16 value g with g * 6 * Smax >= max|x| (so no block scale saturates),
+ * 1.0 when x is all zero, and 65504 when even that is too small.
+ *   out_fp16_dev  OUT one uint16_t (binary16 bit pattern) in device memory. */
+MX_API mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols, mx_scale_fmt fmt,
+                          uint16_t* out_fp16_dev, void* workspace, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+MX_API const char* mx_status_string(mx_status status);
+
+/* Diagnostic: number of kernels this library has enqueued in this process so far (all calls,
+ * all threads).  The only state the library keeps; it never affects results. */
+MX_API long long mx_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MX_H */

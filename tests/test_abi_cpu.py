@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports every symbol include/mx.h declares, and rejects bad arguments
+on the host before enqueueing anything (no compute call is made: every call here is invalid)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_microscaling_tensor_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+L = _lib.lib
+OK, INV, UNS, MIS, WS = (_lib.MX_OK, _lib.MX_ERR_INVALID_ARG, _lib.MX_ERR_UNSUPPORTED,
+                         _lib.MX_ERR_MISALIGNED, _lib.MX_ERR_WORKSPACE)
+A = 0x10000  # a fake 16-byte-aligned device address; never dereferenced (every call fails first)
+BF16, F32, E4, UE = _lib.MX_BF16, _lib.MX_F32, _lib.MX_SCALE_E4M3, _lib.MX_SCALE_UE5M3
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "mx.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"MX_API\s+[\w\s\*]+?\b(mx_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(_lib.EXPORTS) == names
+
+
+def test_status_strings():
+    for s in range(6):
+        assert L.mx_status_string(s)
+    assert b"unknown" in L.mx_status_string(99)
+
+
+def test_workspace_sizes():
+    assert L.mx_error_stats_workspace_size(4096, 4096, 32) >= 64
+    assert L.mx_global_scale_workspace_size(4096, 4096) >= 4
+
+
+def q(x=A, xt=BF16, rows=4, cols=64, block=32, fmt=E4, g=0x3C00, p=A, s=A):
+    return L.mx_quantize(x, xt, rows, cols, block, fmt, g, p, s, None)
+
+
+def test_quantize_rejects_bad_arguments():
+    assert q(x=None) == INV
+    assert q(p=None) == INV
+    assert q(s=None) == INV
+    assert q(rows=-1) == INV
+    assert q(cols=48) == INV                      # 48 % 32 != 0
+    assert q(block=12) == UNS
+    assert q(block=512) == UNS
+    assert q(block=2) == UNS
+    assert q(xt=7) == INV
+    assert q(fmt=3) == INV
+    for g in (0x0000, 0x8000, 0xBC00, 0x7C00, 0x7E00, 0xFC00):  # 0, -0, <0, inf, nan, -inf
+        assert q(g=g) == INV
+    assert q(x=A + 8) == MIS
+    assert q(p=A + 4) == MIS
+    assert q(s=A + 1) == MIS
+    assert q(rows=1 << 40, cols=1 << 40) == INV   # element count overflows
+
+
+def test_dequantize_rejects_bad_arguments():
+    def dq(p=A, s=A, rows=4, cols=64, block=32, fmt=E4, g=0x3C00, y=A, yt=BF16):
+        return L.mx_dequantize(p, s, rows, cols, block, fmt, g, y, yt, None)
+    assert dq(p=None) == INV
+    assert dq(y=None) == INV
+    assert dq(cols=40) == INV
+    assert dq(block=24) == UNS
+    assert dq(yt=2) == INV
+    assert dq(g=0) == INV
+    assert dq(y=A + 2) == MIS
+    assert dq(s=A + 3) == MIS
+
+
+def test_error_stats_rejects_bad_arguments():
+    ws = L.mx_error_stats_workspace_size(4, 64, 32)
+
+    def st(x=A, p=None, s=None, out=A, w=A, n=ws, block=32, cols=64, g=0x3C00):
+        return L.mx_error_stats(x, BF16, 4, cols, block, E4, g, p, s, out, w, n, None)
+    assert st(out=None) == INV
+    assert st(x=None) == INV
+    assert st(p=A, s=None) == INV                 # packed and scales go together
+    assert st(p=None, s=A) == INV
+    assert st(w=None) == WS
+    assert st(n=ws - 1) == WS
+    assert st(cols=50) == INV
+    assert st(block=3) == UNS
+    assert st(g=0xFFFF) == INV
+    assert st(out=A + 8) == MIS
+    assert st(w=A + 4) == MIS
+    assert st(p=A + 1, s=A) == MIS
+
+
+def test_global_scale_rejects_bad_arguments():
+    ws = L.mx_global_scale_workspace_size(4, 64)
+
+    def gs(x=A, out=A, w=A, n=ws, fmt=UE):
+        return L.mx_global_scale(x, BF16, 4, 64, fmt, out, w, n, None)
+    assert gs(out=None) == INV
+    assert gs(x=None) == INV
+    assert gs(fmt=9) == INV
+    assert gs(w=None) == WS
+    assert gs(n=ws - 1) == WS
+    assert gs(x=A + 2) == MIS
+
+
+def test_python_binding_marshalling_errors():
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    with pytest.raises(ValueError):
+        mx.quantize(torch.zeros(4, 64, dtype=torch.bfloat16))  # CPU tensor: not accepted
+    with pytest.raises(ValueError):
+        mx.fmt_code("e5m2")
+    assert mx.g_bits(None) == 0x3C00 and mx.g_bits(1.0) == 0x3C00 and mx.g_bits(0x1234) == 0x1234
