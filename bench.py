@@ -37,8 +37,8 @@ L2_BYTES = 126 * 2 ** 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -76,55 +76,103 @@ def measured_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and throttle reasons sampled every 5 ms (NVML) while the timed region runs.
 
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.proc = None
-        self.tmp = None
+    Sampling starts before and stops after the region.  Falls back to `nvidia-smi -lms 200`."""
+
+    def __init__(self, device):
+        import threading
+        self.device = device
+        self.samples = []
+        self.stop = threading.Event()
+        self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.smi = None
+
+    def _open_nvml(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+        self.nvml = pynvml
+
+    def _loop(self):
+        nv, h = self.nvml, self.handle
+        reasons = {"hw_slowdown": nv.nvmlClocksThrottleReasonHwSlowdown,
+                   "hw_thermal_slowdown": nv.nvmlClocksThrottleReasonHwThermalSlowdown,
+                   "sw_thermal_slowdown": nv.nvmlClocksThrottleReasonSwThermalSlowdown,
+                   "sw_power_cap": nv.nvmlClocksThrottleReasonSwPowerCap}
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                util = nv.nvmlDeviceGetUtilizationRates(h).gpu
+                self.samples.append((sm, [k for k, b in reasons.items() if mask & b], pw, util))
+            except Exception:
+                pass
+            self.stop.wait(0.005)
 
     def __enter__(self):
-        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.tmp, stderr=subprocess.DEVNULL)
-        except FileNotFoundError:
-            self.proc = None
-        time.sleep(0.3)
+            self._open_nvml()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.nvml = None
+            try:
+                self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+                self.smi = subprocess.Popen(
+                    ["nvidia-smi", "--query-gpu=clocks.sm,clocks_event_reasons.active",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=self.tmp, stderr=subprocess.DEVNULL)
+            except FileNotFoundError:
+                self.smi = None
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        time.sleep(0.02)
+        self.stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if self.smi is not None:
+            self.smi.terminate()
+            self.smi.wait(timeout=5)
 
     def summary(self):
-        rows = []
-        try:
+        max_mhz = None
+        if self.nvml is not None:
+            try:
+                max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+            except Exception:
+                pass
+        if self.samples:
+            sm = [s[0] for s in self.samples]
+            busy = [s[0] for s in self.samples if s[3] > 0] or sm
+            reasons = sorted({r for s in self.samples for r in s[1]})
+            return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max_mhz, "reasons": reasons,
+                    "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples),
+                    "source": "nvml 5 ms"}
+        if self.smi is not None:
+            rows = []
             with open(self.tmp.name) as f:
                 for line in f:
                     p = [c.strip() for c in line.split(",")]
-                    if len(p) >= 9 and p[1].isdigit():
-                        rows.append(p)
-        finally:
+                    if p and p[0].isdigit():
+                        rows.append(int(p[0]))
             os.unlink(self.tmp.name)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        sm = [int(r[1]) for r in rows]
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]),
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
-                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+            if rows:
+                return {"sm_mhz": statistics.median(rows), "sm_max_mhz": max_mhz, "reasons": [],
+                        "samples": len(rows), "source": "nvidia-smi 200 ms"}
+        return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": ["no clock samples"]}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -288,7 +336,7 @@ def run_ours(args):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index if world == 1 else local) as clk:
+    with ClockSampler(dev) as clk:
         t_wall = time.perf_counter()
         with torch.cuda.stream(stream):
             for s in range(args.steps):
