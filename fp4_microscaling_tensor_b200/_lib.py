@@ -23,8 +23,8 @@ MX_SCALE_E4M3, MX_SCALE_UE5M3 = 0, 1
 
 # every symbol declared in include/mx.h
 EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_error_stats",
-           "mx_global_scale_workspace_size", "mx_global_scale", "mx_status_string",
-           "mx_kernel_launches")
+           "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
+           "mx_status_string", "mx_kernel_launches")
 
 _i, _i64, _u16, _vp, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_uint16, ctypes.c_void_p, ctypes.c_size_t
 
@@ -40,6 +40,8 @@ lib.mx_global_scale_workspace_size.restype = _sz
 lib.mx_global_scale_workspace_size.argtypes = [_i64, _i64]
 lib.mx_global_scale.restype = _i
 lib.mx_global_scale.argtypes = [_vp, _i, _i64, _i64, _i, _vp, _vp, _sz, _vp]
+lib.mx_error_stats_noalloc.restype = _i
+lib.mx_error_stats_noalloc.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp]
 lib.mx_status_string.restype = ctypes.c_char_p
 lib.mx_status_string.argtypes = [_i]
 lib.mx_kernel_launches.restype = ctypes.c_longlong

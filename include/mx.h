@@ -123,6 +123,24 @@ MX_API mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64
                           uint16_t* out_fp16_dev, void* workspace, size_t ws_bytes,
                           cudaStream_t stream);
 
+/* mx_error_stats without a caller workspace (no counterpart in the pages: a library convenience).
+ * For callers that cannot allocate device memory for a workspace -- a host framework that owns all
+ * device allocations and passes the library only tensors, a real-time loop that must not enter an
+ * allocator, a C caller without a device allocator.  The scratch is a fixed 256 KiB array in this
+ * library's device memory (every GPU that loads the library holds it until the process exits); the
+ * call allocates nothing (no cudaMalloc, cudaFree or allocating library routine).  Arguments,
+ * results and errors are those of mx_error_stats; any rows x cols fits, because the scratch need
+ * does not grow with the tensor (a call that needed more than the array would get MX_ERR_WORKSPACE).
+ *   - The first call on a device resolves the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and keeps it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents behind.  Nothing in it
+ *     needs to start at zero (each call overwrites what it reads), but calls whose kernels overlap
+ *     on the GPU (different streams, no ordering between them) race on it: order them. */
+MX_API mx_status mx_error_stats_noalloc(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
+                                        int block, mx_scale_fmt fmt, uint16_t global_scale_fp16,
+                                        const uint8_t* packed, const uint8_t* scales,
+                                        mx_error_stats_t* out_dev, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 MX_API const char* mx_status_string(mx_status status);
 
