@@ -43,6 +43,13 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    # single-kernel timing / profiling case (not the benchmark line)
+    ap.add_argument("--case", choices=["quantize", "dequantize", "stats", "stats-recompute",
+                                       "global-scale"])
+    ap.add_argument("--shape", type=int, nargs=2, default=[16384, 8192])
+    ap.add_argument("--block", type=int, default=32)
+    ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
+    ap.add_argument("--reps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -435,8 +442,55 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+def run_case(args):
+    """Time one kernel on one bf16 tensor (N(0, 0.02^2), seed 0): CUDA events around each launch,
+    L2 flushed before each launch by writing a 256 MB buffer; prints one JSON line."""
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    from fp4_microscaling_tensor_b200 import inputs
+    dev = torch.device("cuda", 0)
+    rows, cols = args.shape
+    n, fmt = args.block, mx.fmt_code(args.fmt)
+    x = inputs.normal((rows, cols), 0.02, 0, device=dev)
+    numel = rows * cols
+    packed, scales = mx.quantize(x, n, fmt)
+    y = torch.empty(rows, cols, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(64, dtype=torch.uint8, device=dev)
+    ws = mx.stats_workspace(dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    calls = {
+        "quantize": (lambda: mx.quantize(x, n, fmt, packed=packed, scales=scales),
+                     numel * (2.5 + 1.0 / n)),
+        "dequantize": (lambda: mx.dequantize(packed, scales, n, fmt, out=y), numel * (2.5 + 1.0 / n)),
+        "stats": (lambda: mx.error_stats(x, n, fmt, packed=packed, scales=scales, out=out,
+                                         workspace=ws), numel * (2.5 + 1.0 / n)),
+        "stats-recompute": (lambda: mx.error_stats(x, n, fmt, out=out, workspace=ws), numel * 2.0),
+        "global-scale": (lambda: mx.global_scale(x, fmt), numel * 2.0),
+    }
+    fn, nbytes = calls[args.case]
+    fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    peak, kind = measured_peak()
+    print(json.dumps({"case": args.case, "shape": [rows, cols], "block": n, "fmt": args.fmt,
+                      "median_us": t * 1e6, "gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
+                      "peak": peak, "peak_kind": kind, "reps": args.reps}), flush=True)
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

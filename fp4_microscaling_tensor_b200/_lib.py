@@ -7,7 +7,9 @@ been built; there is no fallback.
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxfp4_b200.so")
+# MXFP4_B200_LIB may name another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("MXFP4_B200_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libmxfp4_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

@@ -15,12 +15,20 @@
 
 namespace mxk {
 
+// Item shape (compile-time; the defaults are the tuned values).
+#ifndef MX_DQ_EPT_BF16
+#define MX_DQ_EPT_BF16 8
+#endif
+#ifndef MX_DQ_U
+#define MX_DQ_U 2
+#endif
+
 template <int N, bool BF16OUT>
 struct DShape {
-  static constexpr int EPT = (BF16OUT && N >= 16) ? 16 : 8;
+  static constexpr int EPT = (BF16OUT && N >= 16) ? MX_DQ_EPT_BF16 : 8;
   static constexpr int L = (N >= EPT) ? N / EPT : 1;
   static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
-  static constexpr int U = 2;
+  static constexpr int U = MX_DQ_U;
 };
 
 template <int N, int FMT, bool BF16OUT>

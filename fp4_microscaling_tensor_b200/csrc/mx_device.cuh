@@ -134,6 +134,13 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
   return d;
 }
 
+// min(|a|, |b|) per bf16 half (sign meaningless, as above).
+__device__ __forceinline__ uint32_t bf16x2_absmin(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Streaming 16-byte load of read-only data (not kept in L1).
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;

@@ -7,21 +7,32 @@
 //
 // Pass 1 (k_error_stats_*): persistent grid; each thread walks items like the quantize kernel,
 // either recomputing the codes in registers (RECOMPUTE: reads x only) or reading stored codes.
-//   Arithmetic: a block is scaled by a power of two s that brings its maximum a into [1, 2); the
-//   scaled errors d' = x s - y s are fp32 differences and their squares are summed in fp32 (at
-//   most 16 terms per lane), then scaled back exactly in double.  Squares below 2^-120 in scaled
-//   units would lose digits to fp32 underflow, so each lane tracks its smallest non-zero |x|; in
-//   the rare lane where one falls below 2^-30 a (a block spanning a huge dynamic range), or where a
-//   stored scale is far from the block maximum, the lane recomputes its slice in double.
-//   Elements whose |x| equals the block maximum are kept out of the per-element sums; with
-//   recomputed codes they all carry the same error, so the block's first lane adds that error
-//   (computed in double) once to SSE_max and (count - 1) times to SSE_elem.  With stored codes the
-//   lane holding the first max element adds it to SSE_max and the others to SSE_elem.  Every added
-//   term is non-negative, so exact zeros stay exact.
+// Per block slice held by a lane:
+//   * Scaling.  s = 2^k brings the block maximum a into [1, 2).  d' = x s - code * (S g s) is one
+//     FMA (the code's bits are its value times 2^-126; S g s 2^126 is a per-block constant) and
+//     exact; squares are summed in fp32 (at most 16 terms) and scaled back exactly in double
+//     (integer operations place the fp32 sum, times 1/s^2, into a double).
+//   * Two compares per element: |x| == a (the max-valued elements: their squares go to a second
+//     fp32 sum and a counter) and |x| > 6 S g (clipped elements, counted).  A lane holding one
+//     max-valued element (the usual case) knows its error exactly; the block's first max element
+//     (lowest lane, lowest index) goes to SSE_max, everything else to SSE_elem.  Ties of the
+//     maximum inside one lane take a slower path in double.  All added terms are non-negative,
+//     so exact zeros stay exact.
+//   * Underflow.  Scaled squares below 2^-120 would lose digits.  A lane whose slice holds a value
+//     below 2^-30 a (checked with a min|x| tree, then per element only if the tree fires, because
+//     exact zeros are harmless) or whose stored scale is far from a redoes its slice in double.
 // Pass 2 (k_error_stats_final): one CTA adds the per-CTA partials in a fixed order, so results are
 // deterministic for a given device.  No CTA waits on another.
 #include "mx_device.cuh"
 #include "mx_launch.h"
+
+// Item shape (compile-time; the defaults are the tuned values).
+#ifndef MX_ST_EPT_BF16
+#define MX_ST_EPT_BF16 16
+#endif
+#ifndef MX_ST_U
+#define MX_ST_U 1
+#endif
 
 namespace mxk {
 
@@ -37,10 +48,10 @@ struct StatsOut {  // layout of mx_error_stats_t
 
 template <int N, typename T>
 struct SShape {
-  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? 16 : 8;
+  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? MX_ST_EPT_BF16 : 8;
   static constexpr int L = (N >= EPT) ? N / EPT : 1;
   static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
-  static constexpr int U = 2;
+  static constexpr int U = (sizeof(T) == 2) ? MX_ST_U : 1;
 };
 
 struct Acc {
@@ -83,135 +94,106 @@ __device__ void write_partial(const Acc& acc, StatsPartial* part) {
   }
 }
 
-// Power of two s with a * s in [1, 2) (s from 2^-127 to 2^126) and back = 1 / s^2, exact in double.
-struct BlockScale {
-  float s;
-  double back;
-};
-__device__ __forceinline__ BlockScale block_scale(float a) {
-  int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);  // biased exponent of a >= 0
+// v * 2^(2E - 254) in double for a non-negative fp32 v that is zero or normal, built with integer
+// operations: the fp32 exponent and mantissa move into the double's fields and the block's scale
+// factor is added to the exponent (no conversion or double multiply instructions).
+__device__ __forceinline__ double scaled_to_double(float v, int E) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t hi = (b >> 3) + ((uint32_t)(642 + 2 * E) << 20);
+  const uint32_t lo = b << 29;
+  return b ? __hiloint2double((int)hi, (int)lo) : 0.0;
+}
+
+// One block slice of NE elements held by this lane.
+//   xval(k)  value of element k;  code(k): a word whose low nibble is element k's code (k is a
+//            compile-time constant after unrolling)
+//   lane_max max |x| over this lane's slice (before the cross-lane reduction); min_abs: min |x|
+// Adds its contributions to acc.  `ok` is false for the padding lanes of the last warp.
+template <int NE, int L, typename XF, typename CF>
+__device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a, float D,
+                                            float sat_thr, float lane_max, float min_abs, XF xval,
+                                            CF code) {
+  int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);
   E = max(E, 1);
-  BlockScale b;
-  b.s = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);  // 2^(127 - E)
-  b.back = __longlong_as_double((long long)(769 + 2 * E) << 52);             // 2^(2E - 254)
-  return b;
-}
+  // s = 2^(127 - E) brings a into [1, 2); squares are scaled by s^2 = 2^(254 - 2E)
+  const float sc = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);
+  const float as = __fmul_rn(a, sc);
+  const float Ds = __fmul_rn(D, sc);
+  const float sat6s = __fmul_rn(6.0f, Ds);  // scaled clip level 6 S g s
+  const bool zero_blk = !(D > 0.0f);
+  const float nDq = -__fmul_rn(Ds, 0x1p126f);
+  // fast path valid: stored scale within [2^-30, 2] of the block maximum (recomputed: ~1/24..1/3)
+  const bool scale_ok = zero_blk || (Ds <= 2.0f && Ds >= 0x1p-30f);
+  const float tiny = __fmul_rn(a, 0x1p-30f);
 
-// Error sums (unscaled, double) of the NE elements of one block held by this lane.
-struct LaneErr {
-  double lt = 0.0;     // elements with |x| < a
-  double mxs = 0.0;    // elements with |x| == a (stored codes only)
-  double first = 0.0;  // the lowest-index element with |x| == a (stored codes only)
-  unsigned cnt = 0;    // elements with |x| == a
-  unsigned nsat = 0;   // elements with |x| > 6 D
-};
-
-// xv: the lane's NE values; code(k): a word whose low nibble is element k's code.  Elements are
-// visited in descending index order so `first` ends on the lowest-index max element.
-template <int NE, bool GIVEN, typename CodeFn>
-__device__ __forceinline__ LaneErr lane_errors(const float* xv, CodeFn code, float a, float D) {
-  LaneErr r;
-  const BlockScale bs = block_scale(a);
-  const float Ds = __fmul_rn(D, bs.s);
-  const float sat6 = __fmul_rn(6.0f, D);
-  // decoded code bits are value * 2^-126: one multiply by D s 2^126 gives y s exactly.  The fast
-  // path needs D s in [2^-30, 2] (or 0): always true for recomputed codes (1/24 < D s <= 1/3)
-  const bool fast_ok = Ds <= 2.0f && (Ds == 0.0f || Ds >= 0x1p-30f);
-  const float Dq = __fmul_rn(fast_ok ? Ds : 0.0f, 0x1p126f);
-  float lt = 0.0f, mxs = 0.0f, first = 0.0f;
-  // smallest non-zero |x| as (bits * 2 - 2) (zero wraps to the top).  With every non-zero |x| at
-  // least a 2^-30, every non-zero scaled error is at least 2^-54 (one unit in the last place of
-  // x s or y s), so its square is a normal fp32 number and nothing is lost to underflow.
-  uint32_t xmin = 0xFFFFFFFFu;
+  float lt = 0.0f, ms = 0.0f;  // scaled squares of the other / the max-valued elements
+  unsigned cnt = 0, nsat = 0;  // max-valued elements, clipped elements
 #pragma unroll
-  for (int k = NE - 1; k >= 0; --k) {
-    const float ys = __fmul_rn(__uint_as_float(e2m1_scaled_bits_at(code(k), 0)), Dq);
-    const float d = __fsub_rn(__fmul_rn(xv[k], bs.s), ys);
-    const bool ism = fabsf(xv[k]) == a;
-    const float dl = ism ? 0.0f : d;
-    lt = __fmaf_rn(dl, dl, lt);
-    r.cnt += ism ? 1u : 0u;
-    r.nsat += (fabsf(xv[k]) > sat6) ? 1u : 0u;
-    xmin = min(xmin, __float_as_uint(xv[k]) * 2u - 2u);
-    if constexpr (GIVEN) {
-      const float e2 = __fmul_rn(d, d);
-      if (ism) {
-        mxs = __fadd_rn(mxs, e2);
-        first = e2;
-      }
-    }
-  }
-  if (fast_ok && xmin >= __float_as_uint(__fmul_rn(a, 0x1p-30f)) * 2u - 2u) {
-    r.lt = (double)lt * bs.back;
-    r.mxs = (double)mxs * bs.back;
-    r.first = (double)first * bs.back;
-    return r;
-  }
-  // exact slice in double (rare: a block spanning more than 2^30, or a stored scale far from a)
-  double ltd = 0.0, mxd = 0.0, fd = 0.0;
-#pragma unroll
-  for (int k = NE - 1; k >= 0; --k) {
-    const float y = __fmul_rn(e2m1_to_float(code(k)), D);  // exact
-    const double d = (double)xv[k] - (double)y;            // exact
-    const double e2 = d * d;
-    if (fabsf(xv[k]) == a) {
-      mxd += e2;
-      fd = e2;
+  for (int k = 0; k < NE; ++k) {
+    const float xs = __fmul_rn(xval(k), sc);
+    const float d = __fmaf_rn(__uint_as_float(e2m1_scaled_bits_at(code(k), 0)), nDq, xs);
+    const float ax = fabsf(xs);
+    if (ax >= as) {
+      ms = __fmaf_rn(d, d, ms);
+      ++cnt;
     } else {
-      ltd += e2;
+      lt = __fmaf_rn(d, d, lt);
+    }
+    if (ax > sat6s) ++nsat;
+  }
+  if (!ok) cnt = nsat = 0;
+  const bool has_max = cnt != 0;
+
+  // underflow guard: the tree minimum includes zeros, so confirm per element before giving up
+  bool exact = !scale_ok;
+  if (min_abs < tiny) {
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+      const float ax = fabsf(xval(k));
+      exact |= (ax != 0.0f) && (ax < tiny);
     }
   }
-  r.lt = ltd;
-  r.mxs = GIVEN ? mxd : 0.0;
-  r.first = GIVEN ? fd : 0.0;
-  return r;
-}
-
-// Accounting of one block slice (the block's lanes are the L-lane group around `lane`).
-//  recomputed codes: every max-valued element has the error of y_m; the block's first lane adds it.
-//  stored codes: the lane holding the first max element adds its `first` to SSE_max.
-template <int L, bool GIVEN>
-__device__ __forceinline__ void account(Acc& acc, int lane, bool ok, float a, float D, float y_m,
-                                        LaneErr r, float sat_thr) {
-  if (!ok) r = LaneErr{};
-  unsigned cnt = r.cnt;
-  if constexpr (!GIVEN) {
-#pragma unroll
-    for (int off = 1; off < L; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (D > 0.0f) {
-      acc.elem += r.lt;
-      acc.n_esat += r.nsat;
-    } else {
-      acc.zero += r.lt;
-    }
-    if (ok && (lane & (L - 1)) == 0) {
-      const double dm = (double)a - (double)y_m;  // exact: difference of two floats
-      const double em = dm * dm;
-      if (D > 0.0f) {
-        acc.mx += em;
-        acc.elem += (double)(cnt - 1u) * em;
-      } else {
-        acc.zero += (double)cnt * em;  // y_m = 0 here: em = a^2
-        acc.n_zero += 1;
-      }
-      acc.n_ssat += (a > sat_thr) ? 1u : 0u;
-    }
+  double lt_d, first, others = 0.0;
+  if (!exact && cnt <= 1) {
+    // common case: at most one max-valued element in this lane
+    lt_d = scaled_to_double(lt, E);
+    first = scaled_to_double(ms, E);
   } else {
-    const unsigned gmask =
-        (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(L - 1)));
-    const unsigned has = __ballot_sync(0xffffffffu, cnt > 0) & gmask;
-    const bool is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
-    if (D > 0.0f) {
-      acc.elem += r.lt + (is_first_lane ? r.mxs - r.first : r.mxs);
-      if (is_first_lane) acc.mx += r.first;
-      acc.n_esat += r.nsat;
-    } else {
-      acc.zero += r.lt + r.mxs;
+    // ties of the maximum or the exact path: every element in double, lowest max apart
+    lt_d = first = 0.0;
+    bool seen = false;
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+      const float y = __fmul_rn(e2m1_to_float(code(k)), D);  // exact
+      const double dd = (double)xval(k) - (double)y;          // exact
+      const double e2 = dd * dd;
+      if (fabsf(xval(k)) != a) {
+        lt_d += e2;
+      } else if (!seen) {
+        first = e2;
+        seen = true;
+      } else {
+        others += e2;
+      }
     }
-    if (ok && (lane & (L - 1)) == 0) {
-      acc.n_zero += (D > 0.0f) ? 0u : 1u;
-      acc.n_ssat += (a > sat_thr) ? 1u : 0u;
-    }
+  }
+  bool is_first_lane = has_max;
+  if constexpr (L > 1) {
+    const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
+    const unsigned has = __ballot_sync(0xffffffffu, has_max) & gmask;
+    is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
+  }
+  if (!ok) lt_d = first = others = 0.0;
+  if (zero_blk) {
+    acc.zero += lt_d + first + others;
+  } else {
+    acc.elem += lt_d + others + (is_first_lane ? 0.0 : first);
+    if (is_first_lane) acc.mx += first;
+    acc.n_esat += nsat;
+  }
+  if (ok && (lane & (L - 1)) == 0) {
+    acc.n_zero += zero_blk ? 1u : 0u;
+    acc.n_ssat += (a > sat_thr) ? 1u : 0u;
   }
 }
 
@@ -225,10 +207,9 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
     const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
     StatsPartial* __restrict__ part) {
   using S = SShape<N, uint16_t>;
-  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2, NCW = EPT / 8;
   constexpr int BW = NW / BPI;  // words per block inside an item
   constexpr int BE = 2 * BW;    // elements per block inside an item
-  constexpr bool GIVEN = !RECOMPUTE;
   __shared__ float s_rcp[256], s_D[256];
   const float g = fp16_bits_to_float(g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
@@ -248,7 +229,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
 
   for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
     uint32_t w[U][NW];
-    uint32_t cw[U][EPT / 8];
+    uint32_t cw[U][NCW];
     uint32_t scw[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -262,10 +243,10 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
       }
       scw[u] = 0;
 #pragma unroll
-      for (int j = 0; j < EPT / 8; ++j) cw[u][j] = 0;
-      if constexpr (GIVEN) {
+      for (int j = 0; j < NCW; ++j) cw[u][j] = 0;
+      if constexpr (!RECOMPUTE) {
         if (ok) {
-          if constexpr (EPT == 16) {
+          if constexpr (NCW == 2) {
             const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
             cw[u][0] = p.x; cw[u][1] = p.y;
           } else {
@@ -280,23 +261,24 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
     for (int u = 0; u < U; ++u) {
       const int64_t i = tid + base + (int64_t)u * T;
       const bool ok = i < nitems;
-      float xv[EPT];
-#pragma unroll
-      for (int k = 0; k < NW; ++k) {
-        xv[2 * k] = bf16lo(w[u][k]);
-        xv[2 * k + 1] = bf16hi(w[u][k]);
-      }
-      // phase A: block maxima, scale codes and (recomputing) the element quotients
-      float a_b[BPI], D_b[BPI], ym_b[BPI];
+      const uint32_t* wu = w[u];
+      float a_b[BPI], D_b[BPI], lm_b[BPI];
+      uint32_t mn_b[BPI];
       float qv[EPT];
 #pragma unroll
       for (int b = 0; b < BPI; ++b) {
-        const uint32_t* wb = &w[u][b * BW];
-        uint32_t t = wb[0];
+        const uint32_t* wb = &wu[b * BW];
+        uint32_t t = wb[0], tm = wb[0];
 #pragma unroll
-        for (int k = 1; k < BW; ++k) t = bf16x2_absmax(t, wb[k]);
+        for (int k = 1; k < BW; ++k) {
+          t = bf16x2_absmax(t, wb[k]);
+          tm = bf16x2_absmin(tm, wb[k]);
+        }
         t &= 0x7FFF7FFFu;
+        tm &= 0x7FFF7FFFu;
         uint32_t m = max(t & 0xFFFFu, t >> 16);
+        mn_b[b] = min(tm & 0xFFFFu, tm >> 16);
+        lm_b[b] = __uint_as_float(m << 16);
 #pragma unroll
         for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
         const float a = __uint_as_float(m << 16);
@@ -304,35 +286,34 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
         if constexpr (RECOMPUTE) {
           s = encode_scale<FMT>(snap21(__fmul_rn(a, r6)));
           const float r = s_rcp[s];
-          const uint32_t ca =
-              cvt_e2m1x8(snap21(__fmul_rn(a, r)), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
-          ym_b[b] = __fmul_rn(e2m1_to_float(ca), s_D[s]);
 #pragma unroll
-          for (int k = 0; k < BE; ++k) qv[b * BE + k] = snap21(__fmul_rn(xv[b * BE + k], r));
+          for (int k = 0; k < BW; ++k) {
+            qv[2 * (b * BW + k)] = snap21(__fmul_rn(bf16lo(wb[k]), r));
+            qv[2 * (b * BW + k) + 1] = snap21(__fmul_rn(bf16hi(wb[k]), r));
+          }
         } else {
           s = (scw[u] >> (8 * b)) & 0xFF;
-          ym_b[b] = 0.0f;
         }
         a_b[b] = a;
         D_b[b] = s_D[s];
       }
-      // phase B: codes of the whole item
       if constexpr (RECOMPUTE) {
 #pragma unroll
-        for (int j = 0; j < EPT / 8; ++j)
+        for (int j = 0; j < NCW; ++j)
           cw[u][j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3],
                                 qv[8 * j + 4], qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
       }
-      // phase C: per-element errors and per-block accounting
+      const uint32_t* cwu = cw[u];
 #pragma unroll
       for (int b = 0; b < BPI; ++b) {
-        const uint32_t* cwu = cw[u];
-        auto code = [&](int k) {
-          const int e = b * BE + k;
-          return cwu[e / 8] >> (4 * (e % 8));
+        const int e0 = b * BE;
+        auto xval = [&](int k) {
+          const uint32_t wd = wu[(e0 + k) >> 1];
+          return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
         };
-        const LaneErr r = lane_errors<BE, GIVEN>(&xv[b * BE], code, a_b[b], D_b[b]);
-        account<L, GIVEN>(acc, lane, ok, a_b[b], D_b[b], ym_b[b], r, sat_thr);
+        auto code = [&](int k) { return cwu[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
+        block_slice<BE, L>(acc, lane, ok, a_b[b], D_b[b], sat_thr, lm_b[b],
+                           __uint_as_float(mn_b[b] << 16), xval, code);
       }
     }
   }
@@ -351,7 +332,6 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
   using S = SShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI;
   constexpr int BE = EPT / BPI;
-  constexpr bool GIVEN = !RECOMPUTE;
   __shared__ float s_D[256];
   const float g = fp16_bits_to_float(g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
@@ -377,38 +357,41 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
       v[4 * h + 2] = __uint_as_float(t.z); v[4 * h + 3] = __uint_as_float(t.w);
     }
     uint32_t cw = 0, scw = 0;
-    if (GIVEN && ok) {
+    if (!RECOMPUTE && ok) {
       cw = reinterpret_cast<const unsigned int*>(packed)[i];
       scw = (BPI == 1) ? scales[i / L] : reinterpret_cast<const unsigned short*>(scales)[i];
     }
 #pragma unroll
     for (int b = 0; b < BPI; ++b) {
+      const float* vb = &v[b * BE];
       float a = 0.0f;
+      uint32_t mn = 0x7FFFFFFFu;
 #pragma unroll
-      for (int k = 0; k < BE; ++k) a = fmaxf(a, fabsf(v[b * BE + k]));
+      for (int k = 0; k < BE; ++k) {
+        a = fmaxf(a, fabsf(vb[k]));
+        mn = min(mn, __float_as_uint(vb[k]) & 0x7FFFFFFFu);
+      }
+      const float lane_max = a;
 #pragma unroll
       for (int off = 1; off < L; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       uint32_t s, bc = 0;
-      float y_m = 0.0f;
       if constexpr (RECOMPUTE) {
         s = encode_scale<FMT>(__fdiv_rn(a, g6));
         const float D0 = s_D[s];
         float q[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          q[k] = (k < BE && D0 > 0.0f) ? __fdiv_rn(v[b * BE + (k < BE ? k : 0)], D0)
-                                       : __fmul_rn(k < BE ? v[b * BE + k] : 0.0f, 0.0f);
+          q[k] = (k < BE && D0 > 0.0f) ? __fdiv_rn(vb[k < BE ? k : 0], D0)
+                                       : __fmul_rn(k < BE ? vb[k < BE ? k : 0] : 0.0f, 0.0f);
         bc = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-        const float qa = D0 > 0.0f ? __fdiv_rn(a, D0) : 0.0f;
-        y_m = __fmul_rn(e2m1_to_float(cvt_e2m1x8(qa, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f)), D0);
       } else {
         s = (scw >> (8 * b)) & 0xFF;
         bc = cw >> (4 * b * BE);
       }
       const float D = s_D[s];
+      auto xval = [&](int k) { return vb[k]; };
       auto code = [&](int k) { return bc >> (4 * k); };
-      const LaneErr r = lane_errors<BE, GIVEN>(&v[b * BE], code, a, D);
-      account<L, GIVEN>(acc, lane, ok, a, D, y_m, r, sat_thr);
+      block_slice<BE, L>(acc, lane, ok, a, D, sat_thr, lane_max, __uint_as_float(mn), xval, code);
     }
   }
   write_partial(acc, part);
@@ -507,7 +490,7 @@ static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g
   if (nitems > 0) {
     const void* kern = (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, RC>
                                         : (const void*)k_error_stats_f32<N, FMT, RC>;
-    const int grid = persistent_grid(kern, nitems, sizeof(T) == 2 ? S::U : 1, kMaxReduceCtas - 1);
+    const int grid = persistent_grid(kern, nitems, S::U, kMaxReduceCtas - 1);
     if (sizeof(T) == 2)
       k_error_stats_bf16<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
           (const uint16_t*)x, nitems, g_bits, packed, scales, part);

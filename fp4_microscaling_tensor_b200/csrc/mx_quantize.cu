@@ -19,12 +19,21 @@
 
 namespace mxk {
 
+// Item shape (compile-time; the defaults are the tuned values): elements per item for bf16 input
+// when N >= 16 (8 or 16), and items in flight per thread.
+#ifndef MX_Q_EPT_BF16
+#define MX_Q_EPT_BF16 16
+#endif
+#ifndef MX_Q_U
+#define MX_Q_U 2
+#endif
+
 template <int N, typename T>
 struct QShape {
-  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? 16 : 8;  // elements per item
-  static constexpr int L = (N >= EPT) ? N / EPT : 1;                // lanes per block
-  static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;              // blocks per item
-  static constexpr int U = 2;                                       // items in flight per thread
+  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? MX_Q_EPT_BF16 : 8;  // elements per item
+  static constexpr int L = (N >= EPT) ? N / EPT : 1;                          // lanes per block
+  static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;                        // blocks per item
+  static constexpr int U = (sizeof(T) == 2) ? MX_Q_U : 2;                    // items in flight
 };
 
 // ------------------------------------------------------------------------------------------------
