@@ -246,7 +246,10 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
       for (int j = 0; j < NCW; ++j) cw[u][j] = 0;
       if constexpr (!RECOMPUTE) {
         if (ok) {
-          if constexpr (NCW == 2) {
+          if constexpr (NCW == 4) {
+            const uint4 p = __ldcs(reinterpret_cast<const uint4*>(packed) + i);
+            cw[u][0] = p.x; cw[u][1] = p.y; cw[u][2] = p.z; cw[u][3] = p.w;
+          } else if constexpr (NCW == 2) {
             const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
             cw[u][0] = p.x; cw[u][1] = p.y;
           } else {
