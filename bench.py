@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     # single-kernel timing / profiling case (not the benchmark line)
     ap.add_argument("--case", choices=["quantize", "dequantize", "stats", "stats-recompute",
-                                       "global-scale"])
+                                       "quantize-stats", "global-scale"])
     ap.add_argument("--shape", type=int, nargs=2, default=[16384, 8192])
     ap.add_argument("--block", type=int, default=32)
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
@@ -465,6 +465,9 @@ def run_case(args):
         "stats": (lambda: mx.error_stats(x, n, fmt, packed=packed, scales=scales, out=out,
                                          workspace=ws), numel * (2.5 + 1.0 / n)),
         "stats-recompute": (lambda: mx.error_stats(x, n, fmt, out=out, workspace=ws), numel * 2.0),
+        "quantize-stats": (lambda: mx.quantize_with_stats(x, n, fmt, packed=packed, scales=scales,
+                                                          out=out, workspace=ws),
+                           numel * (2.5 + 1.0 / n)),
         "global-scale": (lambda: mx.global_scale(x, fmt), numel * 2.0),
     }
     fn, nbytes = calls[args.case]

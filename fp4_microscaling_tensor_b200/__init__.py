@@ -5,4 +5,5 @@ dequantize, the three-term block-error reduction and the per-tensor FP16 scale. 
 thin binding over it; importing it fails when the library is missing.
 """
 from .api import (E4M3, UE5M3, ErrorStats, MXError, dequantize, error_stats,  # noqa: F401
-                  fmt_code, g_bits, global_scale, kernel_launches, quantize, stats_workspace)
+                  fmt_code, g_bits, global_scale, kernel_launches, quantize, quantize_with_stats,
+                  stats_workspace)

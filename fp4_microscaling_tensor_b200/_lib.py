@@ -25,6 +25,7 @@ MX_SCALE_E4M3, MX_SCALE_UE5M3 = 0, 1
 
 # every symbol declared in include/mx.h
 EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_error_stats",
+           "mx_quantize_stats",
            "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
            "mx_status_string", "mx_kernel_launches")
 
@@ -38,6 +39,8 @@ lib.mx_error_stats_workspace_size.restype = _sz
 lib.mx_error_stats_workspace_size.argtypes = [_i64, _i64, _i]
 lib.mx_error_stats.restype = _i
 lib.mx_error_stats.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.mx_quantize_stats.restype = _i
+lib.mx_quantize_stats.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.mx_global_scale_workspace_size.restype = _sz
 lib.mx_global_scale_workspace_size.argtypes = [_i64, _i64]
 lib.mx_global_scale.restype = _i

@@ -130,6 +130,32 @@ def error_stats(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, out=N
     return ErrorStats(out)
 
 
+def quantize_with_stats(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, out=None,
+                        workspace=None, stream=None):
+    """Quantize + pack with the three-term error reduction in the same pass over x.
+
+    Returns (packed, scales, ErrorStats); the same values as quantize() followed by
+    error_stats(x, packed=..., scales=...)."""
+    rows, cols = _shape2d(x, "x")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    lead = tuple(x.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+                             device=x.device)
+    if out is None:
+        out = torch.empty(STATS_BYTES, dtype=torch.uint8, device=x.device)
+    if workspace is None:
+        workspace = stats_workspace(x.device, rows, cols, block)
+    check(lib.mx_quantize_stats(x.data_ptr(), _DT[x.dtype], rows, cols, int(block), fmt_code(fmt),
+                                g_bits(g), packed.data_ptr(), scales.data_ptr(), out.data_ptr(),
+                                workspace.data_ptr(), workspace.numel(),
+                                _stream(stream, x.device)), "mx_quantize_stats")
+    return packed, scales, ErrorStats(out)
+
+
 def global_scale(x, fmt="e4m3", out=None, workspace=None, stream=None):
     """Per-tensor FP16 scale of x, as a device uint16 tensor of one element (bit pattern)."""
     rows, cols = _shape2d(x, "x")

@@ -112,6 +112,29 @@ mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
   return from_cuda(e);
 }
 
+mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                            mx_scale_fmt fmt, uint16_t global_scale_fp16, uint8_t* packed,
+                            uint8_t* scales, mx_error_stats_t* out_dev, void* workspace,
+                            size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  if (cols % block != 0) return MX_ERR_INVALID_ARG;
+  if (!out_dev) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel != 0 && (!x || !packed || !scales)) return MX_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < stats_ws_bytes()) return MX_ERR_WORKSPACE;
+  if ((numel != 0 && (!aligned16(x) || !aligned16(packed) || !aligned16(scales))) ||
+      !aligned16(out_dev) || !aligned16(workspace))
+    return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_quantize_stats(numel ? x : nullptr, xt == MX_BF16, numel, block,
+                                                (int)fmt, global_scale_fp16, packed, scales,
+                                                out_dev, workspace, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
 size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols) {
   (void)rows;
   (void)cols;

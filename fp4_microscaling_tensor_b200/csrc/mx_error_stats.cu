@@ -104,60 +104,99 @@ __device__ __forceinline__ double scaled_to_double(float v, int E) {
   return b ? __hiloint2double((int)hi, (int)lo) : 0.0;
 }
 
-// One block slice of NE elements held by this lane.
-//   xval(k)  value of element k;  code(k): a word whose low nibble is element k's code (k is a
-//            compile-time constant after unrolling)
-//   lane_max max |x| over this lane's slice (before the cross-lane reduction); min_abs: min |x|
-// Adds its contributions to acc.  `ok` is false for the padding lanes of the last warp.
-template <int NE, int L, typename XF, typename CF>
-__device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a, float D,
-                                            float sat_thr, float lane_max, float min_abs, XF xval,
-                                            CF code) {
-  int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);
-  E = max(E, 1);
-  // s = 2^(127 - E) brings a into [1, 2); squares are scaled by s^2 = 2^(254 - 2E)
-  const float sc = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);
-  const float as = __fmul_rn(a, sc);
-  const float Ds = __fmul_rn(D, sc);
-  const float sat6s = __fmul_rn(6.0f, Ds);  // scaled clip level 6 S g s
-  const bool zero_blk = !(D > 0.0f);
-  const float nDq = -__fmul_rn(Ds, 0x1p126f);
-  // fast path valid: stored scale within [2^-30, 2] of the block maximum (recomputed: ~1/24..1/3)
-  const bool scale_ok = zero_blk || (Ds <= 2.0f && Ds >= 0x1p-30f);
-  const float tiny = __fmul_rn(a, 0x1p-30f);
+// Per-block constants of one block slice (see the file comment for the scaling).
+struct SliceSetup {
+  int E;           // biased exponent of the block maximum a (at least 1)
+  float sc;        // 2^(127 - E): a * sc in [1, 2)
+  float sat6s;     // 6 S g sc, the scaled clip level
+  float nDq;       // -S g sc 2^126: one FMA with a code's bits gives -y sc
+  float tiny;      // a 2^-30: below it a scaled square could lose digits
+  bool zero_blk;   // S == 0
+  bool scale_ok;   // S g sc in [2^-30, 2] (always true for recomputed codes)
+};
 
-  float lt = 0.0f, ms = 0.0f;  // scaled squares of the other / the max-valued elements
-  unsigned cnt = 0, nsat = 0;  // max-valued elements, clipped elements
-#pragma unroll
-  for (int k = 0; k < NE; ++k) {
-    const float xs = __fmul_rn(xval(k), sc);
-    const float d = __fmaf_rn(__uint_as_float(e2m1_scaled_bits_at(code(k), 0)), nDq, xs);
-    const float ax = fabsf(xs);
-    if (ax >= as) {
-      ms = __fmaf_rn(d, d, ms);
-      ++cnt;
-    } else {
-      lt = __fmaf_rn(d, d, lt);
-    }
-    if (ax > sat6s) ++nsat;
-  }
+__device__ __forceinline__ SliceSetup slice_setup(float a, float D) {
+  SliceSetup st;
+  st.E = max((int)((__float_as_uint(a) >> 23) & 0xFFu), 1);
+  st.sc = __uint_as_float(st.E <= 253 ? (uint32_t)(254 - st.E) << 23 : 0x00400000u);
+  const float Ds = __fmul_rn(D, st.sc);
+  st.sat6s = __fmul_rn(6.0f, Ds);
+  st.nDq = -__fmul_rn(Ds, 0x1p126f);
+  st.tiny = __fmul_rn(a, 0x1p-30f);
+  st.zero_blk = !(D > 0.0f);
+  st.scale_ok = st.zero_blk || (Ds <= 2.0f && Ds >= 0x1p-30f);
+  return st;
+}
+
+// Core of a bf16 block slice, one word (two elements) at a time, in PTX so that every step is one
+// instruction: scaled values (f32x2 multiply), scaled errors (f32x2 FMA with the code bits),
+// |x| >= a and |x| > 6 S g as bf16x2 compares (x is bf16, so |x| > 6 S g holds exactly when |x| is
+// above 6 S g rounded down to bf16), predicated sums and counters.
+//   w: the word; cb: the code byte in bits 0..7; A2 = {a, a}, S2 = {RD(6 S g), same} as bf16x2.
+__device__ __forceinline__ void pair_step(uint32_t w, uint32_t cb, float sc, float nDq,
+                                          uint32_t A2, uint32_t S2, float& lt, float& ms,
+                                          uint32_t& cnt, uint32_t& nsat) {
+  asm("{\n\t"
+      ".reg .b32 lo, hi, blo, bhi, aw, t;\n\t"
+      ".reg .b64 x2, s2, b2, q2, d2;\n\t"
+      ".reg .f32 dlo, dhi;\n\t"
+      ".reg .pred pl, ph, ql, qh;\n\t"
+      "shl.b32 lo, %4, 16;\n\t"
+      "and.b32 hi, %4, 0xffff0000;\n\t"
+      "mov.b64 x2, {lo, hi};\n\t"
+      "mov.b64 s2, {%6, %6};\n\t"
+      "mul.rn.f32x2 x2, x2, s2;\n\t"
+      "shl.b32 t, %5, 28;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 blo, t, 0x81c00000;\n\t"
+      "shl.b32 t, %5, 24;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 bhi, t, 0x81c00000;\n\t"
+      "mov.b64 b2, {blo, bhi};\n\t"
+      "mov.b64 q2, {%7, %7};\n\t"
+      "fma.rn.f32x2 d2, b2, q2, x2;\n\t"
+      "mov.b64 {dlo, dhi}, d2;\n\t"
+      "and.b32 aw, %4, 0x7fff7fff;\n\t"
+      "setp.ge.bf16x2 pl|ph, aw, %8;\n\t"
+      "setp.gt.bf16x2 ql|qh, aw, %9;\n\t"
+      "@pl fma.rn.f32 %1, dlo, dlo, %1;\n\t"
+      "@!pl fma.rn.f32 %0, dlo, dlo, %0;\n\t"
+      "@ph fma.rn.f32 %1, dhi, dhi, %1;\n\t"
+      "@!ph fma.rn.f32 %0, dhi, dhi, %0;\n\t"
+      "@pl add.u32 %2, %2, 1;\n\t"
+      "@ph add.u32 %2, %2, 1;\n\t"
+      "@ql add.u32 %3, %3, 1;\n\t"
+      "@qh add.u32 %3, %3, 1;\n\t"
+      "}"
+      : "+f"(lt), "+f"(ms), "+r"(cnt), "+r"(nsat)
+      : "r"(w), "r"(cb), "f"(sc), "f"(nDq), "r"(A2), "r"(S2));
+}
+
+// Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
+// cnt the number of max-valued elements, nsat the clipped elements.  xval(k) / code(k) (k a
+// compile-time constant) serve the exact path: ties of the maximum in this lane, or a slice that
+// could lose digits to fp32 underflow.
+template <int NE, int L, typename XF, typename CF>
+__device__ __forceinline__ void slice_finish(Acc& acc, int lane, bool ok, float a, float D,
+                                             float sat_thr, float min_abs, const SliceSetup& st,
+                                             float lt, float ms, unsigned cnt, unsigned nsat,
+                                             XF xval, CF code) {
   if (!ok) cnt = nsat = 0;
   const bool has_max = cnt != 0;
-
   // underflow guard: the tree minimum includes zeros, so confirm per element before giving up
-  bool exact = !scale_ok;
-  if (min_abs < tiny) {
+  bool exact = !st.scale_ok;
+  if (min_abs < st.tiny) {
 #pragma unroll
     for (int k = 0; k < NE; ++k) {
       const float ax = fabsf(xval(k));
-      exact |= (ax != 0.0f) && (ax < tiny);
+      exact |= (ax != 0.0f) && (ax < st.tiny);
     }
   }
   double lt_d, first, others = 0.0;
   if (!exact && cnt <= 1) {
     // common case: at most one max-valued element in this lane
-    lt_d = scaled_to_double(lt, E);
-    first = scaled_to_double(ms, E);
+    lt_d = scaled_to_double(lt, st.E);
+    first = scaled_to_double(ms, st.E);
   } else {
     // ties of the maximum or the exact path: every element in double, lowest max apart
     lt_d = first = 0.0;
@@ -184,7 +223,7 @@ __device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a
     is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
   }
   if (!ok) lt_d = first = others = 0.0;
-  if (zero_blk) {
+  if (st.zero_blk) {
     acc.zero += lt_d + first + others;
   } else {
     acc.elem += lt_d + others + (is_first_lane ? 0.0 : first);
@@ -192,20 +231,69 @@ __device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a
     acc.n_esat += nsat;
   }
   if (ok && (lane & (L - 1)) == 0) {
-    acc.n_zero += zero_blk ? 1u : 0u;
+    acc.n_zero += st.zero_blk ? 1u : 0u;
     acc.n_ssat += (a > sat_thr) ? 1u : 0u;
   }
+}
+
+// Generic block slice of NE elements (fp32 input): xval(k) value, code(k) a word whose low nibble
+// is element k's code (k a compile-time constant after unrolling).
+template <int NE, int L, typename XF, typename CF>
+__device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a, float D,
+                                            float sat_thr, float min_abs, XF xval, CF code) {
+  const SliceSetup st = slice_setup(a, D);
+  const float as = __fmul_rn(a, st.sc);
+  float lt = 0.0f, ms = 0.0f;
+  unsigned cnt = 0, nsat = 0;
+#pragma unroll
+  for (int k = 0; k < NE; ++k) {
+    const float xs = __fmul_rn(xval(k), st.sc);
+    const float d = __fmaf_rn(__uint_as_float(e2m1_scaled_bits_at(code(k), 0)), st.nDq, xs);
+    const float ax = fabsf(xs);
+    if (ax >= as) {
+      ms = __fmaf_rn(d, d, ms);
+      ++cnt;
+    } else {
+      lt = __fmaf_rn(d, d, lt);
+    }
+    if (ax > st.sat6s) ++nsat;
+  }
+  slice_finish<NE, L>(acc, lane, ok, a, D, sat_thr, min_abs, st, lt, ms, cnt, nsat, xval, code);
+}
+
+// bf16 block slice: NW words wb[0..NW) of the lane's item, codes from byte `b0` of the item's
+// code words onwards (byte j holds the codes of word j).
+template <int NW, int L, typename XF, typename CF>
+__device__ __forceinline__ void block_slice_bf16(Acc& acc, int lane, bool ok, float a, float D,
+                                                 float sat_thr, float min_abs, const uint32_t* wb,
+                                                 const uint32_t* cwu, int b0, XF xval, CF code) {
+  const SliceSetup st = slice_setup(a, D);
+  const uint32_t ab = __float_as_uint(a) >> 16;              // a is a bf16 value
+  const uint32_t sb = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // 6 S g rounded down to bf16
+  const uint32_t A2 = ab | (ab << 16), S2 = sb | (sb << 16);
+  float lt = 0.0f, ms = 0.0f;
+  uint32_t cnt = 0, nsat = 0;
+#pragma unroll
+  for (int k = 0; k < NW; ++k) {
+    const int bi = b0 + k;
+    pair_step(wb[k], cwu[bi >> 2] >> (8 * (bi & 3)), st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat);
+  }
+  slice_finish<2 * NW, L>(acc, lane, ok, a, D, sat_thr, min_abs, st, lt, ms, cnt, nsat, xval, code);
 }
 
 // ------------------------------------------------------------------------------------------------
 // bf16 input
 // ------------------------------------------------------------------------------------------------
 
-template <int N, int FMT, bool RECOMPUTE>
+// RECOMPUTE: codes computed in registers (same rule as the quantize kernel); with STORE they are
+// also written to packed_out / scales_out, which makes this the fused quantize+pack+reduction pass.
+template <int N, int FMT, bool RECOMPUTE, bool STORE = false>
 __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
     const uint16_t* __restrict__ x, int64_t nitems, uint16_t g_bits,
     const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part) {
+    StatsPartial* __restrict__ part, uint8_t* __restrict__ packed_out = nullptr,
+    uint8_t* __restrict__ scales_out = nullptr) {
+  static_assert(!STORE || RECOMPUTE, "storing needs recomputed codes");
   using S = SShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2, NCW = EPT / 8;
   constexpr int BW = NW / BPI;  // words per block inside an item
@@ -265,8 +353,9 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
       const int64_t i = tid + base + (int64_t)u * T;
       const bool ok = i < nitems;
       const uint32_t* wu = w[u];
-      float a_b[BPI], D_b[BPI], lm_b[BPI];
+      float a_b[BPI], D_b[BPI];
       uint32_t mn_b[BPI];
+      uint32_t sc_all = 0;  // scale codes of the item's blocks, byte b = block b
       float qv[EPT];
 #pragma unroll
       for (int b = 0; b < BPI; ++b) {
@@ -281,7 +370,6 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
         tm &= 0x7FFF7FFFu;
         uint32_t m = max(t & 0xFFFFu, t >> 16);
         mn_b[b] = min(tm & 0xFFFFu, tm >> 16);
-        lm_b[b] = __uint_as_float(m << 16);
 #pragma unroll
         for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
         const float a = __uint_as_float(m << 16);
@@ -299,12 +387,31 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
         }
         a_b[b] = a;
         D_b[b] = s_D[s];
+        sc_all |= s << (8 * b);
       }
       if constexpr (RECOMPUTE) {
 #pragma unroll
         for (int j = 0; j < NCW; ++j)
           cw[u][j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3],
                                 qv[8 * j + 4], qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
+      }
+      if constexpr (STORE) {
+        if (ok) {
+          if constexpr (NCW == 4)
+            *reinterpret_cast<uint4*>(packed_out + i * 16) =
+                make_uint4(cw[u][0], cw[u][1], cw[u][2], cw[u][3]);
+          else if constexpr (NCW == 2)
+            *reinterpret_cast<uint2*>(packed_out + i * 8) = make_uint2(cw[u][0], cw[u][1]);
+          else
+            *reinterpret_cast<uint32_t*>(packed_out + i * 4) = cw[u][0];
+          if constexpr (BPI == 1) {
+            if ((lane & (L - 1)) == 0) scales_out[i / L] = (uint8_t)sc_all;
+          } else if constexpr (BPI == 2) {
+            *reinterpret_cast<uint16_t*>(scales_out + i * 2) = (uint16_t)sc_all;
+          } else {
+            *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
+          }
+        }
       }
       const uint32_t* cwu = cw[u];
 #pragma unroll
@@ -315,8 +422,9 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
           return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
         };
         auto code = [&](int k) { return cwu[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
-        block_slice<BE, L>(acc, lane, ok, a_b[b], D_b[b], sat_thr, lm_b[b],
-                           __uint_as_float(mn_b[b] << 16), xval, code);
+        block_slice_bf16<BW, L>(acc, lane, ok, a_b[b], D_b[b], sat_thr,
+                                __uint_as_float(mn_b[b] << 16), &wu[b * BW], cwu, b * BW, xval,
+                                code);
       }
     }
   }
@@ -374,7 +482,6 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
         a = fmaxf(a, fabsf(vb[k]));
         mn = min(mn, __float_as_uint(vb[k]) & 0x7FFFFFFFu);
       }
-      const float lane_max = a;
 #pragma unroll
       for (int off = 1; off < L; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       uint32_t s, bc = 0;
@@ -394,7 +501,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
       const float D = s_D[s];
       auto xval = [&](int k) { return vb[k]; };
       auto code = [&](int k) { return bc >> (4 * k); };
-      block_slice<BE, L>(acc, lane, ok, a, D, sat_thr, lane_max, __uint_as_float(mn), xval, code);
+      block_slice<BE, L>(acc, lane, ok, a, D, sat_thr, __uint_as_float(mn), xval, code);
     }
   }
   write_partial(acc, part);
@@ -536,6 +643,72 @@ static cudaError_t st_rc(bool rc, int block, const void* x, int64_t numel, uint1
                          cudaStream_t st, int* n) {
   return rc ? st_block<FMT, T, true>(block, x, numel, g, p, s, out, part, st, n)
             : st_block<FMT, T, false>(block, x, numel, g, p, s, out, part, st, n);
+}
+
+// ------------------------------------------------------------------------------------------------
+// fused quantize + pack + error reduction (bf16 input): one pass over x
+// ------------------------------------------------------------------------------------------------
+
+template <int N, int FMT>
+static cudaError_t launch_qs(const uint16_t* x, int64_t numel, int block, uint16_t g_bits,
+                             uint8_t* packed, uint8_t* scales, void* out, StatsPartial* part,
+                             cudaStream_t stream, int* launches) {
+  using S = SShape<N, uint16_t>;
+  const int64_t nitems = numel / S::EPT;
+  int nparts = 0;
+  if (nitems > 0) {
+    const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, true, true>, nitems,
+                                     S::U, kMaxReduceCtas - 1);
+    k_error_stats_bf16<N, FMT, true, true><<<grid, kThreads, 0, stream>>>(
+        x, nitems, g_bits, nullptr, nullptr, part, packed, scales);
+    ++*launches;
+    nparts = grid;
+  }
+  if (numel % S::EPT != 0) {  // N = 4 and 4 elements left: quantize them, then reduce from the codes
+    const cudaError_t e = run_quantize_tail4(x, true, nitems * S::EPT, FMT, g_bits, packed, scales,
+                                             stream, launches);
+    if (e != cudaSuccess) return e;
+    k_error_stats_tail4<FMT, uint16_t><<<1, 32, 0, stream>>>(x, nitems * S::EPT, g_bits, packed,
+                                                             scales, part + nparts);
+    ++*launches;
+    ++nparts;
+  }
+  k_error_stats_final<<<1, kThreads, 0, stream>>>(part, nparts, numel, numel / block,
+                                                  (StatsOut*)out);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t qs_block(int block, const uint16_t* x, int64_t numel, uint16_t g, uint8_t* p,
+                            uint8_t* s, void* out, StatsPartial* part, cudaStream_t st, int* n) {
+  switch (block) {
+    case 4: return launch_qs<4, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    case 8: return launch_qs<8, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    case 16: return launch_qs<16, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    case 32: return launch_qs<32, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    case 64: return launch_qs<64, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    case 128: return launch_qs<128, FMT>(x, numel, block, g, p, s, out, part, st, n);
+    default: return launch_qs<256, FMT>(x, numel, block, g, p, s, out, part, st, n);
+  }
+}
+
+cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                               uint16_t g_bits, uint8_t* packed, uint8_t* scales, void* out,
+                               void* workspace, cudaStream_t stream, int* launches) {
+  StatsPartial* part = reinterpret_cast<StatsPartial*>(workspace);
+  if (!bf16) {  // fp32 input: quantize, then reduce from the stored codes
+    cudaError_t e = run_quantize(x, false, numel, block, fmt, g_bits, packed, scales, stream,
+                                 launches);
+    if (e != cudaSuccess) return e;
+    return run_error_stats(x, false, numel, block, fmt, g_bits, packed, scales, out, workspace,
+                           stream, launches);
+  }
+  const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+  return fmt == kUE5M3 ? qs_block<kUE5M3>(block, xb, numel, g_bits, packed, scales, out, part,
+                                          stream, launches)
+                       : qs_block<kE4M3>(block, xb, numel, g_bits, packed, scales, out, part,
+                                         stream, launches);
 }
 
 cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,

@@ -35,6 +35,15 @@ cudaError_t run_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t
 cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                             uint16_t g_bits, const uint8_t* packed, const uint8_t* scales,
                             void* out, void* workspace, cudaStream_t stream, int* launches);
+// Quantize + pack with the three-term error reduction fused into the same pass (bf16 input; fp32
+// input runs quantize then the reduction from the stored codes).
+cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                               uint16_t g_bits, uint8_t* packed, uint8_t* scales, void* out,
+                               void* workspace, cudaStream_t stream, int* launches);
+// The last 4 elements of an N = 4 tensor whose size is not a multiple of 8 (from element `first`).
+cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt, uint16_t g_bits,
+                               uint8_t* packed, uint8_t* scales, cudaStream_t stream,
+                               int* launches);
 cudaError_t run_global_scale(const void* x, bool bf16, int64_t numel, int fmt, uint16_t* out,
                              void* workspace, cudaStream_t stream, int* launches);
 

@@ -274,6 +274,28 @@ static cudaError_t dispatch_block(int block, const void* x, int64_t numel, uint1
   }
 }
 
+cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt, uint16_t g_bits,
+                               uint8_t* packed, uint8_t* scales, cudaStream_t stream,
+                               int* launches) {
+  if (bf16) {
+    if (fmt == kUE5M3)
+      k_quantize_tail4<kUE5M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, g_bits,
+                                                               packed, scales);
+    else
+      k_quantize_tail4<kE4M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, g_bits,
+                                                              packed, scales);
+  } else {
+    if (fmt == kUE5M3)
+      k_quantize_tail4<kUE5M3, float><<<1, 32, 0, stream>>>((const float*)x, first, g_bits, packed,
+                                                            scales);
+    else
+      k_quantize_tail4<kE4M3, float><<<1, 32, 0, stream>>>((const float*)x, first, g_bits, packed,
+                                                           scales);
+  }
+  ++*launches;
+  return cudaGetLastError();
+}
+
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
                          uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
                          int* launches) {

@@ -112,6 +112,15 @@ MX_API mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_
                          const uint8_t* scales, mx_error_stats_t* out_dev, void* workspace,
                          size_t ws_bytes, cudaStream_t stream);
 
+/* Quantize + pack with the three-term error reduction fused into the same pass over x ([MX] §3.1
+ * item 2 and §2.2 items 1-3).  packed and scales are what mx_quantize writes; out_dev is what
+ * mx_error_stats reports for them.  x is read once instead of twice.  Arguments are those of
+ * mx_quantize plus out_dev, workspace and ws_bytes of mx_error_stats (same size rule). */
+MX_API mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
+                                   int block, mx_scale_fmt fmt, uint16_t global_scale_fp16,
+                                   uint8_t* packed, uint8_t* scales, mx_error_stats_t* out_dev,
+                                   void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Bytes of device workspace mx_global_scale needs. */
 MX_API size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols);
 

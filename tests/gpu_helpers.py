@@ -78,13 +78,24 @@ def stats_both(x, block, fmt, g=0x3C00, packed=None, scales=None, po=None, so=No
     return got, ref
 
 
+def fused_both(x, block, fmt, g, po, so):
+    """mx_quantize_stats: codes and scales bit-exact, error sums as the oracle's."""
+    rows, cols = x.shape
+    p, s, st = mx.quantize_with_stats(x, block, fmt, g)
+    assert_same(u8(s), so, f"fused scales N={block} fmt={fmt} g={g:#x}")
+    assert_same(u8(p), po, f"fused packed N={block} fmt={fmt} g={g:#x}")
+    ref = oracle.error_stats(inputs.to_oracle(x), rows, cols, block, fmt, g)
+    assert_stats(st.to_dict(), ref, f"fused stats N={block} fmt={fmt} g={g:#x}")
+
+
 def full_check(x, block, fmt, g=0x3C00):
-    """Quantize, dequantize, stats (recomputed and from stored codes) against the oracle."""
+    """Quantize, dequantize, stats (recomputed, from stored codes, fused) against the oracle."""
     rows, cols = x.shape
     p, s, po, so = quantize_both(x, block, fmt, g)
     dequantize_both(po, so, rows, cols, block, fmt, g)
     stats_both(x, block, fmt, g)
     stats_both(x, block, fmt, g, packed=p, scales=s, po=po, so=so)
+    fused_both(x, block, fmt, g, po, so)
 
 
 def special_values_bf16(fmt, g_bits, n, seed):

@@ -96,6 +96,25 @@ def test_error_stats_rejects_bad_arguments():
     assert st(p=A + 1, s=A) == MIS
 
 
+def test_quantize_stats_rejects_bad_arguments():
+    ws = L.mx_error_stats_workspace_size(4, 64, 32)
+
+    def qs(x=A, p=A, s=A, out=A, w=A, n=ws, block=32, cols=64, g=0x3C00, xt=BF16):
+        return L.mx_quantize_stats(x, xt, 4, cols, block, E4, g, p, s, out, w, n, None)
+    assert qs(x=None) == INV
+    assert qs(p=None) == INV
+    assert qs(s=None) == INV
+    assert qs(out=None) == INV
+    assert qs(w=None) == WS
+    assert qs(n=ws - 1) == WS
+    assert qs(cols=48) == INV
+    assert qs(block=64 * 8) == UNS
+    assert qs(g=0x7C00) == INV
+    assert qs(xt=5) == INV
+    assert qs(p=A + 2) == MIS
+    assert qs(out=A + 4) == MIS
+
+
 def test_global_scale_rejects_bad_arguments():
     ws = L.mx_global_scale_workspace_size(4, 64)
 
