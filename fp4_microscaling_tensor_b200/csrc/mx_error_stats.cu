@@ -28,10 +28,13 @@
 
 // Item shape (compile-time; the defaults are the tuned values).
 #ifndef MX_ST_EPT_BF16
-#define MX_ST_EPT_BF16 16
+#define MX_ST_EPT_BF16 32
 #endif
 #ifndef MX_ST_U
 #define MX_ST_U 1
+#endif
+#ifndef MX_ST_MINB  // minimum resident CTAs per SM for the bf16 pass (register cap)
+#define MX_ST_MINB 2
 #endif
 
 namespace mxk {
@@ -48,7 +51,8 @@ struct StatsOut {  // layout of mx_error_stats_t
 
 template <int N, typename T>
 struct SShape {
-  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? MX_ST_EPT_BF16 : 8;
+  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? (N < MX_ST_EPT_BF16 ? N : MX_ST_EPT_BF16)
+                                                         : 8;
   static constexpr int L = (N >= EPT) ? N / EPT : 1;
   static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
   static constexpr int U = (sizeof(T) == 2) ? MX_ST_U : 1;
@@ -56,7 +60,8 @@ struct SShape {
 
 struct Acc {
   double elem = 0.0, mx = 0.0, zero = 0.0;
-  unsigned n_zero = 0, n_ssat = 0, n_esat = 0;
+  unsigned n_zero = 0, n_ssat = 0;
+  float n_esat = 0.0f;  // clipped elements (exact: a thread sees far fewer than 2^24)
 };
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -104,6 +109,22 @@ __device__ __forceinline__ double scaled_to_double(float v, int E) {
   return b ? __hiloint2double((int)hi, (int)lo) : 0.0;
 }
 
+// Quotients x / (S g) of two bf16 elements (lo / hi: their fp32 bits), rounded to multiples of
+// 2^-18 on the FMA pipe, for the E2M1 conversion.  r = RN(1 / (S g)), so x r is within 2^-21 of the
+// true quotient t when |t| <= 8.  Adding and subtracting 48 (whose binade [32, 64) has spacing
+// 2^-18) rounds x r to that grid exactly (Sterbenz for the subtraction).  A midpoint of the E2M1
+// grid (a multiple of 1/4) is then hit exactly when t is one; otherwise t is at least 2^-17 away
+// from every midpoint (x has 8 significant bits, S g at most 15), and the rounded value stays on
+// t's side.  Larger |t| only has to stay above 6, which it does.  The sign is copied from x, so that
+// quotients rounding to zero keep the sign of x (the code's sign bit always follows x).
+__device__ __forceinline__ float2 snap_quotient2(uint32_t lo, uint32_t hi, float r) {
+  const float2 q = __fadd2_rn(__ffma2_rn(make_float2(__uint_as_float(lo), __uint_as_float(hi)),
+                                         make_float2(r, r), make_float2(48.0f, 48.0f)),
+                              make_float2(-48.0f, -48.0f));
+  return make_float2(__uint_as_float((__float_as_uint(q.x) & 0x7FFFFFFFu) | (lo & 0x80000000u)),
+                     __uint_as_float((__float_as_uint(q.y) & 0x7FFFFFFFu) | (hi & 0x80000000u)));
+}
+
 // Per-block constants of one block slice (see the file comment for the scaling).
 struct SliceSetup {
   int E;           // biased exponent of the block maximum a (at least 1)
@@ -131,45 +152,61 @@ __device__ __forceinline__ SliceSetup slice_setup(float a, float D) {
 // Core of a bf16 block slice, one word (two elements) at a time, in PTX so that every step is one
 // instruction: scaled values (f32x2 multiply), scaled errors (f32x2 FMA with the code bits),
 // |x| >= a and |x| > 6 S g as bf16x2 compares (x is bf16, so |x| > 6 S g holds exactly when |x| is
-// above 6 S g rounded down to bf16), predicated sums and counters.
-//   w: the word; cb: the code byte in bits 0..7; A2 = {a, a}, S2 = {RD(6 S g), same} as bf16x2.
-__device__ __forceinline__ void pair_step(uint32_t w, uint32_t cb, float sc, float nDq,
-                                          uint32_t A2, uint32_t S2, float& lt, float& ms,
-                                          uint32_t& cnt, uint32_t& nsat) {
-  asm("{\n\t"
-      ".reg .b32 lo, hi, blo, bhi, aw, t;\n\t"
-      ".reg .b64 x2, s2, b2, q2, d2;\n\t"
-      ".reg .f32 dlo, dhi;\n\t"
-      ".reg .pred pl, ph, ql, qh;\n\t"
-      "shl.b32 lo, %4, 16;\n\t"
-      "and.b32 hi, %4, 0xffff0000;\n\t"
-      "mov.b64 x2, {lo, hi};\n\t"
-      "mov.b64 s2, {%6, %6};\n\t"
-      "mul.rn.f32x2 x2, x2, s2;\n\t"
-      "shl.b32 t, %5, 28;\n\t"
-      "shr.s32 t, t, 6;\n\t"
-      "and.b32 blo, t, 0x81c00000;\n\t"
-      "shl.b32 t, %5, 24;\n\t"
-      "shr.s32 t, t, 6;\n\t"
-      "and.b32 bhi, t, 0x81c00000;\n\t"
-      "mov.b64 b2, {blo, bhi};\n\t"
-      "mov.b64 q2, {%7, %7};\n\t"
-      "fma.rn.f32x2 d2, b2, q2, x2;\n\t"
-      "mov.b64 {dlo, dhi}, d2;\n\t"
-      "and.b32 aw, %4, 0x7fff7fff;\n\t"
-      "setp.ge.bf16x2 pl|ph, aw, %8;\n\t"
-      "setp.gt.bf16x2 ql|qh, aw, %9;\n\t"
-      "@pl fma.rn.f32 %1, dlo, dlo, %1;\n\t"
-      "@!pl fma.rn.f32 %0, dlo, dlo, %0;\n\t"
-      "@ph fma.rn.f32 %1, dhi, dhi, %1;\n\t"
-      "@!ph fma.rn.f32 %0, dhi, dhi, %0;\n\t"
-      "@pl add.u32 %2, %2, 1;\n\t"
-      "@ph add.u32 %2, %2, 1;\n\t"
-      "@ql add.u32 %3, %3, 1;\n\t"
-      "@qh add.u32 %3, %3, 1;\n\t"
-      "}"
-      : "+f"(lt), "+f"(ms), "+r"(cnt), "+r"(nsat)
-      : "r"(w), "r"(cb), "f"(sc), "f"(nDq), "r"(A2), "r"(S2));
+// above 6 S g rounded down to bf16), predicated sums and counters (fp32 adds: the counters stay
+// exact and the integer pipe stays free for the decode).  MS: also sum the squares of the
+// max-valued elements (stored codes); with recomputed codes their error is known per block.
+//   w: the word, lo / hi: its elements as fp32 bits; cw: the code word holding the word's code
+//   byte at byte J; A2 = {a, a}, S2 = {RD(6 S g), same} as bf16x2.  The left shifts are written as
+//   multiplies by 2^k.
+template <int J, bool MS>
+__device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
+                                          float sc, float nDq, uint32_t A2, uint32_t S2, float& lt,
+                                          float& ms, float& cnt, float& nsat) {
+#define MX_PAIR_HEAD                                   \
+  "{\n\t"                                             \
+  ".reg .b32 blo, bhi, aw, t;\n\t"                    \
+  ".reg .b64 x2, s2, b2, q2, d2;\n\t"                 \
+  ".reg .f32 dlo, dhi;\n\t"                           \
+  ".reg .pred pl, ph, ql, qh;\n\t"                    \
+  "mov.b64 x2, {%12, %13};\n\t"                       \
+  "mov.b64 s2, {%6, %6};\n\t"                         \
+  "mul.rn.f32x2 x2, x2, s2;\n\t"                      \
+  "mul.lo.u32 t, %5, %10;\n\t"                        \
+  "shr.s32 t, t, 6;\n\t"                              \
+  "and.b32 blo, t, 0x81c00000;\n\t"                   \
+  "mul.lo.u32 t, %5, %11;\n\t"                        \
+  "shr.s32 t, t, 6;\n\t"                              \
+  "and.b32 bhi, t, 0x81c00000;\n\t"                   \
+  "mov.b64 b2, {blo, bhi};\n\t"                       \
+  "mov.b64 q2, {%7, %7};\n\t"                         \
+  "fma.rn.f32x2 d2, b2, q2, x2;\n\t"                  \
+  "mov.b64 {dlo, dhi}, d2;\n\t"                       \
+  "and.b32 aw, %4, 0x7fff7fff;\n\t"                   \
+  "setp.ge.bf16x2 pl|ph, aw, %8;\n\t"                 \
+  "setp.gt.bf16x2 ql|qh, aw, %9;\n\t"                 \
+  "@!pl fma.rn.f32 %0, dlo, dlo, %0;\n\t"             \
+  "@!ph fma.rn.f32 %0, dhi, dhi, %0;\n\t"
+#define MX_PAIR_TAIL                                   \
+  "@pl add.f32 %2, %2, 0f3F800000;\n\t"               \
+  "@ph add.f32 %2, %2, 0f3F800000;\n\t"               \
+  "@ql add.f32 %3, %3, 0f3F800000;\n\t"               \
+  "@qh add.f32 %3, %3, 0f3F800000;\n\t"               \
+  "}"
+  if constexpr (MS) {
+    asm(MX_PAIR_HEAD
+        "@pl fma.rn.f32 %1, dlo, dlo, %1;\n\t"
+        "@ph fma.rn.f32 %1, dhi, dhi, %1;\n\t" MX_PAIR_TAIL
+        : "+f"(lt), "+f"(ms), "+f"(cnt), "+f"(nsat)
+        : "r"(w), "r"(cw), "f"(sc), "f"(nDq), "r"(A2), "r"(S2), "n"(1u << (28 - 8 * J)),
+          "n"(1u << (24 - 8 * J)), "r"(lo), "r"(hi));
+  } else {
+    asm(MX_PAIR_HEAD MX_PAIR_TAIL
+        : "+f"(lt), "+f"(ms), "+f"(cnt), "+f"(nsat)
+        : "r"(w), "r"(cw), "f"(sc), "f"(nDq), "r"(A2), "r"(S2), "n"(1u << (28 - 8 * J)),
+          "n"(1u << (24 - 8 * J)), "r"(lo), "r"(hi));
+  }
+#undef MX_PAIR_HEAD
+#undef MX_PAIR_TAIL
 }
 
 // Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
@@ -178,22 +215,14 @@ __device__ __forceinline__ void pair_step(uint32_t w, uint32_t cb, float sc, flo
 // could lose digits to fp32 underflow.
 template <int NE, int L, typename XF, typename CF>
 __device__ __forceinline__ void slice_finish(Acc& acc, int lane, bool ok, float a, float D,
-                                             float sat_thr, float min_abs, const SliceSetup& st,
-                                             float lt, float ms, unsigned cnt, unsigned nsat,
+                                             float sat_thr, bool exact, const SliceSetup& st,
+                                             float lt, float ms, float cnt, float nsat,
                                              XF xval, CF code) {
-  if (!ok) cnt = nsat = 0;
-  const bool has_max = cnt != 0;
-  // underflow guard: the tree minimum includes zeros, so confirm per element before giving up
-  bool exact = !st.scale_ok;
-  if (min_abs < st.tiny) {
-#pragma unroll
-    for (int k = 0; k < NE; ++k) {
-      const float ax = fabsf(xval(k));
-      exact |= (ax != 0.0f) && (ax < st.tiny);
-    }
-  }
+  if (!ok) cnt = nsat = 0.0f;
+  const bool has_max = cnt != 0.0f;
+  exact |= !st.scale_ok;
   double lt_d, first, others = 0.0;
-  if (!exact && cnt <= 1) {
+  if (!exact && cnt <= 1.0f) {
     // common case: at most one max-valued element in this lane
     lt_d = scaled_to_double(lt, st.E);
     first = scaled_to_double(ms, st.E);
@@ -236,15 +265,95 @@ __device__ __forceinline__ void slice_finish(Acc& acc, int lane, bool ok, float 
   }
 }
 
+// 2^(2E - 254) as a double: the factor that undoes the slice scaling of a sum of squares.
+__device__ __forceinline__ double unscale_sq(int E) {
+  return __hiloint2double((2 * E + 769) << 20, 0);
+}
+
+// Exact errors of a slice in double: every element, or (ONLY_MAX) only the max-valued ones.
+// first: the lowest-index max-valued element; others: the other max-valued ones; rest: the rest.
+template <int NE, bool ONLY_MAX, typename XF, typename CF>
+__device__ __forceinline__ void exact_slice(float a, float D, XF xval, CF code, double& rest,
+                                            double& first, double& others) {
+  bool seen = false;
+#pragma unroll
+  for (int k = 0; k < NE; ++k) {
+    const bool is_max = fabsf(xval(k)) == a;
+    if (ONLY_MAX && !is_max) continue;
+    const float y = __fmul_rn(e2m1_to_float(code(k)), D);  // exact
+    const double dd = (double)xval(k) - (double)y;          // exact
+    const double e2 = dd * dd;
+    if (!is_max) {
+      rest += e2;
+    } else if (!seen) {
+      first = e2;
+      seen = true;
+    } else {
+      others += e2;
+    }
+  }
+}
+
+// Tail of a bf16 block slice: lt is the sum of the scaled squares of the elements below the
+// maximum, cnt the number of max-valued elements, nsat the clipped elements.  Stored codes (!RC):
+// ms sums the scaled squares of the max-valued elements; a lane with ties of the maximum redoes
+// those elements in double, a slice whose stored scale is far from a redoes everything.
+// Recomputed codes (RC): every max-valued element has the same error, dmax (scaled), computed
+// once per block.  Either way a slice whose lt is below 2^-80 may have lost squares below 2^-126
+// and is redone in double (any loss in a larger sum is below 2^-40 of it).  Items past the end
+// hold zeros and an all-zero scale, so they add zeros (their block counters are skipped via ok).
+template <int NE, int L, bool RC, typename XF, typename CF>
+__device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, float a, float D,
+                                                  float sat_thr, const SliceSetup& st, float lt,
+                                                  float ms, float dmax, float cnt, float nsat,
+                                                  XF xval, CF code) {
+  const bool has_max = cnt != 0.0f;
+  bool is_first_lane = has_max;
+  if constexpr (L > 1) {
+    const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
+    const unsigned has = __ballot_sync(0xffffffffu, has_max) & gmask;
+    is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
+  }
+  double rest = 0.0, first = 0.0, others = 0.0;
+  bool all_exact = lt < 0x1p-80f;
+  if constexpr (!RC) all_exact |= !st.scale_ok;
+  if (all_exact) {
+    exact_slice<NE, false>(a, D, xval, code, rest, first, others);
+  } else {
+    const double sd = unscale_sq(st.E);
+    rest = (double)lt * sd;
+    if constexpr (RC) {
+      if (has_max) {
+        first = (double)dmax * (double)dmax * sd;  // exact
+        others = (double)(cnt - 1.0f) * first;
+      }
+    } else {
+      if (cnt <= 1.0f) first = (double)ms * sd;
+      else exact_slice<NE, true>(a, D, xval, code, rest, first, others);
+    }
+  }
+  if (st.zero_blk) {
+    acc.zero += rest + first + others;
+  } else {
+    acc.elem += rest + others + (is_first_lane ? 0.0 : first);
+    if (is_first_lane) acc.mx += first;
+    acc.n_esat += nsat;
+  }
+  if (ok && (lane & (L - 1)) == 0) {
+    acc.n_zero += st.zero_blk ? 1u : 0u;
+    acc.n_ssat += (a > sat_thr) ? 1u : 0u;
+  }
+}
+
 // Generic block slice of NE elements (fp32 input): xval(k) value, code(k) a word whose low nibble
-// is element k's code (k a compile-time constant after unrolling).
+// is element k's code (k a compile-time constant after unrolling).  min_abs: the slice's min|x|
+// (zeros included); a nonzero value below 2^-30 a could lose digits to fp32 underflow.
 template <int NE, int L, typename XF, typename CF>
 __device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a, float D,
                                             float sat_thr, float min_abs, XF xval, CF code) {
   const SliceSetup st = slice_setup(a, D);
   const float as = __fmul_rn(a, st.sc);
-  float lt = 0.0f, ms = 0.0f;
-  unsigned cnt = 0, nsat = 0;
+  float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f;
 #pragma unroll
   for (int k = 0; k < NE; ++k) {
     const float xs = __fmul_rn(xval(k), st.sc);
@@ -252,52 +361,53 @@ __device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a
     const float ax = fabsf(xs);
     if (ax >= as) {
       ms = __fmaf_rn(d, d, ms);
-      ++cnt;
+      cnt += 1.0f;
     } else {
       lt = __fmaf_rn(d, d, lt);
     }
-    if (ax > st.sat6s) ++nsat;
+    if (ax > st.sat6s) nsat += 1.0f;
   }
-  slice_finish<NE, L>(acc, lane, ok, a, D, sat_thr, min_abs, st, lt, ms, cnt, nsat, xval, code);
-}
-
-// bf16 block slice: NW words wb[0..NW) of the lane's item, codes from byte `b0` of the item's
-// code words onwards (byte j holds the codes of word j).
-template <int NW, int L, typename XF, typename CF>
-__device__ __forceinline__ void block_slice_bf16(Acc& acc, int lane, bool ok, float a, float D,
-                                                 float sat_thr, float min_abs, const uint32_t* wb,
-                                                 const uint32_t* cwu, int b0, XF xval, CF code) {
-  const SliceSetup st = slice_setup(a, D);
-  const uint32_t ab = __float_as_uint(a) >> 16;              // a is a bf16 value
-  const uint32_t sb = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // 6 S g rounded down to bf16
-  const uint32_t A2 = ab | (ab << 16), S2 = sb | (sb << 16);
-  float lt = 0.0f, ms = 0.0f;
-  uint32_t cnt = 0, nsat = 0;
+  bool exact = false;
+  if (min_abs < st.tiny) {
 #pragma unroll
-  for (int k = 0; k < NW; ++k) {
-    const int bi = b0 + k;
-    pair_step(wb[k], cwu[bi >> 2] >> (8 * (bi & 3)), st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat);
+    for (int k = 0; k < NE; ++k) {
+      const float ax = fabsf(xval(k));
+      exact |= (ax != 0.0f) && (ax < st.tiny);
+    }
   }
-  slice_finish<2 * NW, L>(acc, lane, ok, a, D, sat_thr, min_abs, st, lt, ms, cnt, nsat, xval, code);
+  slice_finish<NE, L>(acc, lane, ok, a, D, sat_thr, exact, st, lt, ms, cnt, nsat, xval, code);
 }
 
 // ------------------------------------------------------------------------------------------------
 // bf16 input
 // ------------------------------------------------------------------------------------------------
 
-// RECOMPUTE: codes computed in registers (same rule as the quantize kernel); with STORE they are
-// also written to packed_out / scales_out, which makes this the fused quantize+pack+reduction pass.
-template <int N, int FMT, bool RECOMPUTE, bool STORE = false>
-__global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
+// What the bf16 pass does with the codes: read them (kGiven), recompute them in registers with the
+// quantize kernel's rule (kRecompute), or recompute and also write them to packed_out / scales_out
+// (kStore: the fused quantize + pack + reduction pass).
+enum { kGiven = 0, kRecompute = 1, kStore = 2 };
+
+// One thread's item: EPT consecutive elements (NW words), their code words and scale bytes.
+template <int NW, int NCW>
+struct StatsItem {
+  uint32_t w[NW];
+  uint32_t cw[NCW];
+  uint32_t scw;
+};
+
+template <int N, int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
     const uint16_t* __restrict__ x, int64_t nitems, uint16_t g_bits,
     const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part, uint8_t* __restrict__ packed_out = nullptr,
-    uint8_t* __restrict__ scales_out = nullptr) {
-  static_assert(!STORE || RECOMPUTE, "storing needs recomputed codes");
+    StatsPartial* __restrict__ part, uint8_t* __restrict__ packed_out,
+    uint8_t* __restrict__ scales_out) {
+  constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
   using S = SShape<N, uint16_t>;
-  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2, NCW = EPT / 8;
+  constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, NW = EPT / 2, NCW = EPT / 8;
   constexpr int BW = NW / BPI;  // words per block inside an item
   constexpr int BE = 2 * BW;    // elements per block inside an item
+  using Item = StatsItem<NW, NCW>;
+  static_assert(NCW == 1 || NCW == 2 || NCW == 4, "items of 8, 16 or 32 elements");
   __shared__ float s_rcp[256], s_D[256];
   const float g = fp16_bits_to_float(g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
@@ -312,121 +422,150 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_bf16(
   Acc acc;
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t warp0 = tid - (threadIdx.x & 31);
   const int lane = threadIdx.x & 31;
+  const int64_t warp0 = tid - lane;
 
-  for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
-    uint32_t w[U][NW];
-    uint32_t cw[U][NCW];
-    uint32_t scw[U];
+  // Loads of one item (zeros past the end).  Issued one item ahead of the arithmetic.
+  auto load = [&](Item& it, int64_t i) {
+    const bool ok = i < nitems;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t i = tid + base + (int64_t)u * T;
-      const bool ok = i < nitems;
+    for (int h = 0; h < NW / 4; ++h) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (ok) v = ld_stream16(x + i * EPT + h * 8);
+      it.w[4 * h + 0] = v.x; it.w[4 * h + 1] = v.y; it.w[4 * h + 2] = v.z; it.w[4 * h + 3] = v.w;
+    }
+    it.scw = 0;
 #pragma unroll
-      for (int h = 0; h < NW / 4; ++h) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (ok) v = ld_stream16(x + i * EPT + h * 8);
-        w[u][4 * h + 0] = v.x; w[u][4 * h + 1] = v.y; w[u][4 * h + 2] = v.z; w[u][4 * h + 3] = v.w;
+    for (int j = 0; j < NCW; ++j) it.cw[j] = 0;
+    if constexpr (!RECOMPUTE) {
+      if (ok) {
+        if constexpr (NCW == 4) {
+          const uint4 p = __ldcs(reinterpret_cast<const uint4*>(packed) + i);
+          it.cw[0] = p.x; it.cw[1] = p.y; it.cw[2] = p.z; it.cw[3] = p.w;
+        } else if constexpr (NCW == 2) {
+          const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
+          it.cw[0] = p.x; it.cw[1] = p.y;
+        } else {
+          it.cw[0] = __ldcs(reinterpret_cast<const unsigned int*>(packed) + i);
+        }
+        if constexpr (BPI == 1) it.scw = __ldg(scales + i / L);
+        else it.scw = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
       }
-      scw[u] = 0;
+    }
+  };
+
+  auto process = [&](Item& it, int64_t i) {
+    const bool ok = i < nitems;
+    float a_b[BPI], D_b[BPI], r_b[BPI];
+    uint32_t m_b[BPI];
+    uint32_t sc_all = 0;  // scale codes of the item's blocks, byte b = block b
 #pragma unroll
-      for (int j = 0; j < NCW; ++j) cw[u][j] = 0;
-      if constexpr (!RECOMPUTE) {
-        if (ok) {
-          if constexpr (NCW == 4) {
-            const uint4 p = __ldcs(reinterpret_cast<const uint4*>(packed) + i);
-            cw[u][0] = p.x; cw[u][1] = p.y; cw[u][2] = p.z; cw[u][3] = p.w;
-          } else if constexpr (NCW == 2) {
-            const uint2 p = __ldcs(reinterpret_cast<const uint2*>(packed) + i);
-            cw[u][0] = p.x; cw[u][1] = p.y;
-          } else {
-            cw[u][0] = __ldcs(reinterpret_cast<const unsigned int*>(packed) + i);
-          }
-          if constexpr (BPI == 1) scw[u] = __ldg(scales + i / L);
-          else scw[u] = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
+    for (int b = 0; b < BPI; ++b) {
+      const uint32_t* wb = &it.w[b * BW];
+      uint32_t t = wb[0];
+#pragma unroll
+      for (int k = 1; k < BW; ++k) t = bf16x2_absmax(t, wb[k]);
+      t &= 0x7FFF7FFFu;
+      uint32_t m = max(t & 0xFFFFu, t >> 16);
+#pragma unroll
+      for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float a = __uint_as_float(m << 16);
+      uint32_t s;
+      if constexpr (RECOMPUTE) {
+        s = encode_scale<FMT>(snap21(__fmul_rn(a, r6)));
+        r_b[b] = s_rcp[s];
+      } else {
+        s = (it.scw >> (8 * b)) & 0xFF;
+      }
+      a_b[b] = a;
+      m_b[b] = m;
+      D_b[b] = s_D[s];
+      sc_all |= s << (8 * b);
+    }
+    if constexpr (RECOMPUTE) {
+      // codes: eight quotients per code word, converted right away
+#pragma unroll
+      for (int j = 0; j < NCW; ++j) {
+        float q[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int wi = 4 * j + k;
+          const uint32_t w = it.w[wi];
+          const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
+          q[2 * k] = qq.x;
+          q[2 * k + 1] = qq.y;
+        }
+        it.cw[j] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      }
+    }
+    if constexpr (STORE) {
+      if (ok) {
+        if constexpr (NCW == 4)
+          *reinterpret_cast<uint4*>(packed_out + i * 16) =
+              make_uint4(it.cw[0], it.cw[1], it.cw[2], it.cw[3]);
+        else if constexpr (NCW == 2)
+          *reinterpret_cast<uint2*>(packed_out + i * 8) = make_uint2(it.cw[0], it.cw[1]);
+        else
+          *reinterpret_cast<uint32_t*>(packed_out + i * 4) = it.cw[0];
+        if constexpr (BPI == 1) {
+          if ((lane & (L - 1)) == 0) scales_out[i / L] = (uint8_t)sc_all;
+        } else if constexpr (BPI == 2) {
+          *reinterpret_cast<uint16_t*>(scales_out + i * 2) = (uint16_t)sc_all;
+        } else {
+          *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t i = tid + base + (int64_t)u * T;
-      const bool ok = i < nitems;
-      const uint32_t* wu = w[u];
-      float a_b[BPI], D_b[BPI];
-      uint32_t mn_b[BPI];
-      uint32_t sc_all = 0;  // scale codes of the item's blocks, byte b = block b
-      float qv[EPT];
+    for (int b = 0; b < BPI; ++b) {
+      const float a = a_b[b], D = D_b[b];
+      const SliceSetup st = slice_setup(a, D);
+      const uint32_t sb = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // 6 S g rounded down
+      const uint32_t A2 = m_b[b] * 0x10001u, S2 = sb * 0x10001u;
+      float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f, dmax = 0.0f;
 #pragma unroll
-      for (int b = 0; b < BPI; ++b) {
-        const uint32_t* wb = &wu[b * BW];
-        uint32_t t = wb[0], tm = wb[0];
-#pragma unroll
-        for (int k = 1; k < BW; ++k) {
-          t = bf16x2_absmax(t, wb[k]);
-          tm = bf16x2_absmin(tm, wb[k]);
+      for (int k = 0; k < BW; ++k) {
+        const int wi = b * BW + k;
+        const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
+        constexpr bool MS = !RECOMPUTE;
+        switch (wi & 3) {
+          case 0: pair_step<0, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
+          case 1: pair_step<1, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
+          case 2: pair_step<2, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
+          default: pair_step<3, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
         }
-        t &= 0x7FFF7FFFu;
-        tm &= 0x7FFF7FFFu;
-        uint32_t m = max(t & 0xFFFFu, t >> 16);
-        mn_b[b] = min(tm & 0xFFFFu, tm >> 16);
-#pragma unroll
-        for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const float a = __uint_as_float(m << 16);
-        uint32_t s;
-        if constexpr (RECOMPUTE) {
-          s = encode_scale<FMT>(snap21(__fmul_rn(a, r6)));
-          const float r = s_rcp[s];
-#pragma unroll
-          for (int k = 0; k < BW; ++k) {
-            qv[2 * (b * BW + k)] = snap21(__fmul_rn(bf16lo(wb[k]), r));
-            qv[2 * (b * BW + k) + 1] = snap21(__fmul_rn(bf16hi(wb[k]), r));
-          }
-        } else {
-          s = (scw[u] >> (8 * b)) & 0xFF;
-        }
-        a_b[b] = a;
-        D_b[b] = s_D[s];
-        sc_all |= s << (8 * b);
       }
       if constexpr (RECOMPUTE) {
-#pragma unroll
-        for (int j = 0; j < NCW; ++j)
-          cw[u][j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3],
-                                qv[8 * j + 4], qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
+        // the max-valued elements' code magnitude is that of a; their scaled error, as above
+        const float qa = snap_quotient2(__float_as_uint(a), 0u, r_b[b]).x;
+        const uint32_t ca = cvt_e2m1x8(qa, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+        dmax = __fmaf_rn(__uint_as_float(e2m1_scaled_bits_at(ca, 0)), st.nDq,
+                         __fmul_rn(a, st.sc));
       }
-      if constexpr (STORE) {
-        if (ok) {
-          if constexpr (NCW == 4)
-            *reinterpret_cast<uint4*>(packed_out + i * 16) =
-                make_uint4(cw[u][0], cw[u][1], cw[u][2], cw[u][3]);
-          else if constexpr (NCW == 2)
-            *reinterpret_cast<uint2*>(packed_out + i * 8) = make_uint2(cw[u][0], cw[u][1]);
-          else
-            *reinterpret_cast<uint32_t*>(packed_out + i * 4) = cw[u][0];
-          if constexpr (BPI == 1) {
-            if ((lane & (L - 1)) == 0) scales_out[i / L] = (uint8_t)sc_all;
-          } else if constexpr (BPI == 2) {
-            *reinterpret_cast<uint16_t*>(scales_out + i * 2) = (uint16_t)sc_all;
-          } else {
-            *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
-          }
-        }
-      }
-      const uint32_t* cwu = cw[u];
-#pragma unroll
-      for (int b = 0; b < BPI; ++b) {
-        const int e0 = b * BE;
-        auto xval = [&](int k) {
-          const uint32_t wd = wu[(e0 + k) >> 1];
-          return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
-        };
-        auto code = [&](int k) { return cwu[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
-        block_slice_bf16<BW, L>(acc, lane, ok, a_b[b], D_b[b], sat_thr,
-                                __uint_as_float(mn_b[b] << 16), &wu[b * BW], cwu, b * BW, xval,
-                                code);
-      }
+      const int e0 = b * BE;
+      auto xval = [&](int k) {
+        const uint32_t wd = it.w[(e0 + k) >> 1];
+        return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
+      };
+      auto code = [&](int k) { return it.cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
+      slice_finish_bf16<BE, L, RECOMPUTE>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax, cnt,
+                                          nsat, xval, code);
     }
+  };
+
+  // Two items in flight per thread: the loads of the next item are issued before the arithmetic
+  // of the current one.  The trip test is warp-uniform (lanes of a block share shuffles).
+  Item A, B;
+  int64_t i = tid;
+  load(A, i);
+  while (warp0 + (i - tid) < nitems) {
+    load(B, i + T);
+    process(A, i);
+    i += T;
+    if (!(warp0 + (i - tid) < nitems)) break;
+    load(A, i + T);
+    process(B, i);
+    i += T;
   }
   write_partial(acc, part);
 }
@@ -598,12 +737,13 @@ static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g
   const int64_t nitems = numel / S::EPT;
   int nparts = 0;
   if (nitems > 0) {
-    const void* kern = (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, RC>
-                                        : (const void*)k_error_stats_f32<N, FMT, RC>;
+    const void* kern = (sizeof(T) == 2)
+                           ? (const void*)k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>
+                           : (const void*)k_error_stats_f32<N, FMT, RC>;
     const int grid = persistent_grid(kern, nitems, S::U, kMaxReduceCtas - 1);
     if (sizeof(T) == 2)
-      k_error_stats_bf16<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
-          (const uint16_t*)x, nitems, g_bits, packed, scales, part);
+      k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven><<<grid, kThreads, 0, stream>>>(
+          (const uint16_t*)x, nitems, g_bits, packed, scales, part, nullptr, nullptr);
     else
       k_error_stats_f32<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
           (const float*)x, nitems, g_bits, packed, scales, part);
@@ -657,9 +797,9 @@ static cudaError_t launch_qs(const uint16_t* x, int64_t numel, int block, uint16
   const int64_t nitems = numel / S::EPT;
   int nparts = 0;
   if (nitems > 0) {
-    const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, true, true>, nitems,
+    const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, kStore>, nitems,
                                      S::U, kMaxReduceCtas - 1);
-    k_error_stats_bf16<N, FMT, true, true><<<grid, kThreads, 0, stream>>>(
+    k_error_stats_bf16<N, FMT, kStore><<<grid, kThreads, 0, stream>>>(
         x, nitems, g_bits, nullptr, nullptr, part, packed, scales);
     ++*launches;
     nparts = grid;
