@@ -21,8 +21,11 @@
 //   * Underflow.  Scaled squares below 2^-120 would lose digits.  A lane whose slice holds a value
 //     below 2^-30 a (checked with a min|x| tree, then per element only if the tree fires, because
 //     exact zeros are harmless) or whose stored scale is far from a redoes its slice in double.
-// Pass 2 (k_error_stats_final): one CTA adds the per-CTA partials in a fixed order, so results are
-// deterministic for a given device.  No CTA waits on another.
+// Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
+// in a fixed order, so results are deterministic for a given device and grid; with an N = 4 tail a
+// separate one-CTA pass does it.  No CTA waits on another.
+#include <functional>
+
 #include "mx_device.cuh"
 #include "mx_launch.h"
 
@@ -96,6 +99,33 @@ __device__ void write_partial(const Acc& acc, StatsPartial* part) {
       p.n_zero_blocks += su[0][k]; p.n_scale_sat += su[1][k]; p.n_elem_sat += su[2][k];
     }
     part[blockIdx.x] = p;
+  }
+}
+
+struct FinalArgs {
+  unsigned int* counter;  // zeroed before the launch; nullptr: a separate pass adds the partials
+  StatsOut* out;
+  int64_t numel, nblocks;
+};
+
+__device__ void final_reduce(const StatsPartial* part, int nparts, int64_t numel, int64_t nblocks,
+                             StatsOut* out);
+
+// Writes this CTA's partial; the CTA that finishes last (counted with one atomic per CTA after a
+// fence) then adds all partials in a fixed order and resets the counter.  No CTA waits for another.
+__device__ void finish_cta(const Acc& acc, StatsPartial* part, const FinalArgs& fa) {
+  write_partial(acc, part);
+  if (fa.counter == nullptr) return;
+  __shared__ unsigned int s_last;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(fa.counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    final_reduce(part, gridDim.x, fa.numel, fa.nblocks, fa.out);
+    if (threadIdx.x == 0) *fa.counter = 0;
   }
 }
 
@@ -399,7 +429,7 @@ template <int N, int FMT, int MODE>
 __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
     const uint16_t* __restrict__ x, int64_t nitems, uint16_t g_bits,
     const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part, uint8_t* __restrict__ packed_out,
+    StatsPartial* __restrict__ part, FinalArgs fa, uint8_t* __restrict__ packed_out,
     uint8_t* __restrict__ scales_out) {
   constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
   using S = SShape<N, uint16_t>;
@@ -567,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
     process(B, i);
     i += T;
   }
-  write_partial(acc, part);
+  finish_cta(acc, part, fa);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -578,7 +608,7 @@ template <int N, int FMT, bool RECOMPUTE>
 __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
     const float* __restrict__ x, int64_t nitems, uint16_t g_bits,
     const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part) {
+    StatsPartial* __restrict__ part, FinalArgs fa) {
   using S = SShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI;
   constexpr int BE = EPT / BPI;
@@ -643,7 +673,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
       block_slice<BE, L>(acc, lane, ok, a, D, sat_thr, __uint_as_float(mn), xval, code);
     }
   }
-  write_partial(acc, part);
+  finish_cta(acc, part, fa);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -692,15 +722,17 @@ __global__ void k_error_stats_tail4(const T* __restrict__ x, int64_t first, uint
   part[0] = p;
 }
 
-__global__ void __launch_bounds__(kThreads) k_error_stats_final(const StatsPartial* __restrict__ part,
-                                                                int nparts, int64_t numel,
-                                                                int64_t nblocks,
-                                                                StatsOut* __restrict__ out) {
+// Adds nparts partials in a fixed order (thread t takes t, t + 256, ...; then warps, then the 8
+// warp sums in order) and writes the result record.  Run by all threads of one CTA.
+__device__ void final_reduce(const StatsPartial* part, int nparts, int64_t numel, int64_t nblocks,
+                             StatsOut* out) {
   double e = 0.0, m = 0.0, z = 0.0;
   unsigned long long c0 = 0, c1 = 0, c2 = 0;
-  for (int k = threadIdx.x; k < nparts; k += blockDim.x) {  // fixed assignment and order
-    e += part[k].sse_elem; m += part[k].sse_max; z += part[k].sse_zero;
-    c0 += part[k].n_zero_blocks; c1 += part[k].n_scale_sat; c2 += part[k].n_elem_sat;
+  for (int k = threadIdx.x; k < nparts; k += blockDim.x) {
+    const double* pd = reinterpret_cast<const double*>(part + k);
+    const unsigned long long* pu = reinterpret_cast<const unsigned long long*>(part + k);
+    e += __ldcg(pd + 0); m += __ldcg(pd + 1); z += __ldcg(pd + 2);
+    c0 += __ldcg(pu + 4); c1 += __ldcg(pu + 5); c2 += __ldcg(pu + 6);
   }
   __shared__ double sd[3][kThreads / 32];
   __shared__ unsigned long long su[3][kThreads / 32];
@@ -725,46 +757,86 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_final(const StatsParti
   }
 }
 
+__global__ void __launch_bounds__(kThreads) k_error_stats_final(const StatsPartial* __restrict__ part,
+                                                                int nparts, int64_t numel,
+                                                                int64_t nblocks,
+                                                                StatsOut* __restrict__ out) {
+  final_reduce(part, nparts, numel, nblocks, out);
+}
+
 // ------------------------------------------------------------------------------------------------
 // launcher
 // ------------------------------------------------------------------------------------------------
 
-template <int N, int FMT, typename T, bool RC>
-static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g_bits,
-                             const uint8_t* packed, const uint8_t* scales, void* out,
-                             StatsPartial* part, cudaStream_t stream, int* launches) {
-  using S = SShape<N, T>;
-  const int64_t nitems = numel / S::EPT;
+// Workspace layout: a 64-byte header (the last-CTA counter) and then one 64-byte partial per CTA.
+struct Workspace {
+  unsigned int* counter;
+  StatsPartial* part;
+  explicit Workspace(void* ws)
+      : counter(reinterpret_cast<unsigned int*>(ws)),
+        part(reinterpret_cast<StatsPartial*>(reinterpret_cast<char*>(ws) + 64)) {}
+};
+constexpr int kMaxStatsGrid = kMaxReduceCtas - 2;  // header + one slot for the N = 4 tail
+
+// Main pass, then (N = 4 tail) the tail partial and a one-CTA final pass, or (empty) the final
+// pass alone.  Without a tail the main pass adds the partials itself.
+template <typename Launch>
+static cudaError_t stats_passes(int64_t nitems, bool tail, int64_t numel, int block, void* out,
+                                Workspace ws, cudaStream_t stream, int* launches, Launch main,
+                                const std::function<void(StatsPartial*)>& tail_pass) {
   int nparts = 0;
   if (nitems > 0) {
-    const void* kern = (sizeof(T) == 2)
-                           ? (const void*)k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>
-                           : (const void*)k_error_stats_f32<N, FMT, RC>;
-    const int grid = persistent_grid(kern, nitems, S::U, kMaxReduceCtas - 1);
-    if (sizeof(T) == 2)
-      k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven><<<grid, kThreads, 0, stream>>>(
-          (const uint16_t*)x, nitems, g_bits, packed, scales, part, nullptr, nullptr);
-    else
-      k_error_stats_f32<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
-          (const float*)x, nitems, g_bits, packed, scales, part);
+    FinalArgs fa{nullptr, (StatsOut*)out, numel, numel / block};
+    if (!tail) {
+      const cudaError_t e = cudaMemsetAsync(ws.counter, 0, sizeof(unsigned int), stream);
+      if (e != cudaSuccess) return e;
+      fa.counter = ws.counter;
+    }
+    nparts = main(fa);
     ++*launches;
-    nparts = grid;
+    if (!tail) return cudaGetLastError();
   }
-  if (numel % S::EPT != 0) {
-    k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits,
-                                                      RC ? nullptr : packed, scales, part + nparts);
-    ++*launches;
+  if (tail) {
+    tail_pass(ws.part + nparts);
     ++nparts;
   }
-  k_error_stats_final<<<1, kThreads, 0, stream>>>(part, nparts, numel, numel / block,
+  k_error_stats_final<<<1, kThreads, 0, stream>>>(ws.part, nparts, numel, numel / block,
                                                   (StatsOut*)out);
   ++*launches;
   return cudaGetLastError();
 }
 
+template <int N, int FMT, typename T, bool RC>
+static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g_bits,
+                             const uint8_t* packed, const uint8_t* scales, void* out, Workspace ws,
+                             cudaStream_t stream, int* launches) {
+  using S = SShape<N, T>;
+  const int64_t nitems = numel / S::EPT;
+  auto main = [&](FinalArgs fa) {
+    const void* kern = (sizeof(T) == 2)
+                           ? (const void*)k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>
+                           : (const void*)k_error_stats_f32<N, FMT, RC>;
+    const int grid = persistent_grid(kern, nitems, S::U, kMaxStatsGrid);
+    if (sizeof(T) == 2)
+      k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven><<<grid, kThreads, 0, stream>>>(
+          (const uint16_t*)x, nitems, g_bits, packed, scales, ws.part, fa, nullptr, nullptr);
+    else
+      k_error_stats_f32<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
+          (const float*)x, nitems, g_bits, packed, scales, ws.part, fa);
+    return grid;
+  };
+  auto tail = [&](StatsPartial* slot) {
+    k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits,
+                                                      RC ? nullptr : packed, scales, slot);
+    ++*launches;
+  };
+  return stats_passes(nitems, numel % S::EPT != 0, numel, block, out, ws, stream, launches, main,
+                      tail);
+}
+
 template <int FMT, typename T, bool RC>
 static cudaError_t st_block(int block, const void* x, int64_t numel, uint16_t g,
-                            const uint8_t* p, const uint8_t* s, void* out, StatsPartial* part,
+                            const uint8_t* p, const uint8_t* s, void* out, Workspace part,
                             cudaStream_t st, int* n) {
   switch (block) {
     case 4: return launch_st<4, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
@@ -779,7 +851,7 @@ static cudaError_t st_block(int block, const void* x, int64_t numel, uint16_t g,
 
 template <int FMT, typename T>
 static cudaError_t st_rc(bool rc, int block, const void* x, int64_t numel, uint16_t g,
-                         const uint8_t* p, const uint8_t* s, void* out, StatsPartial* part,
+                         const uint8_t* p, const uint8_t* s, void* out, Workspace part,
                          cudaStream_t st, int* n) {
   return rc ? st_block<FMT, T, true>(block, x, numel, g, p, s, out, part, st, n)
             : st_block<FMT, T, false>(block, x, numel, g, p, s, out, part, st, n);
@@ -791,37 +863,31 @@ static cudaError_t st_rc(bool rc, int block, const void* x, int64_t numel, uint1
 
 template <int N, int FMT>
 static cudaError_t launch_qs(const uint16_t* x, int64_t numel, int block, uint16_t g_bits,
-                             uint8_t* packed, uint8_t* scales, void* out, StatsPartial* part,
+                             uint8_t* packed, uint8_t* scales, void* out, Workspace ws,
                              cudaStream_t stream, int* launches) {
   using S = SShape<N, uint16_t>;
   const int64_t nitems = numel / S::EPT;
-  int nparts = 0;
-  if (nitems > 0) {
+  auto main = [&](FinalArgs fa) {
     const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, kStore>, nitems,
-                                     S::U, kMaxReduceCtas - 1);
+                                     S::U, kMaxStatsGrid);
     k_error_stats_bf16<N, FMT, kStore><<<grid, kThreads, 0, stream>>>(
-        x, nitems, g_bits, nullptr, nullptr, part, packed, scales);
-    ++*launches;
-    nparts = grid;
-  }
-  if (numel % S::EPT != 0) {  // N = 4 and 4 elements left: quantize them, then reduce from the codes
-    const cudaError_t e = run_quantize_tail4(x, true, nitems * S::EPT, FMT, g_bits, packed, scales,
-                                             stream, launches);
-    if (e != cudaSuccess) return e;
+        x, nitems, g_bits, nullptr, nullptr, ws.part, fa, packed, scales);
+    return grid;
+  };
+  // N = 4 with 4 elements left: quantize them, then reduce them from the stored codes
+  auto tail = [&](StatsPartial* slot) {
+    run_quantize_tail4(x, true, nitems * S::EPT, FMT, g_bits, packed, scales, stream, launches);
     k_error_stats_tail4<FMT, uint16_t><<<1, 32, 0, stream>>>(x, nitems * S::EPT, g_bits, packed,
-                                                             scales, part + nparts);
+                                                             scales, slot);
     ++*launches;
-    ++nparts;
-  }
-  k_error_stats_final<<<1, kThreads, 0, stream>>>(part, nparts, numel, numel / block,
-                                                  (StatsOut*)out);
-  ++*launches;
-  return cudaGetLastError();
+  };
+  return stats_passes(nitems, numel % S::EPT != 0, numel, block, out, ws, stream, launches, main,
+                      tail);
 }
 
 template <int FMT>
 static cudaError_t qs_block(int block, const uint16_t* x, int64_t numel, uint16_t g, uint8_t* p,
-                            uint8_t* s, void* out, StatsPartial* part, cudaStream_t st, int* n) {
+                            uint8_t* s, void* out, Workspace part, cudaStream_t st, int* n) {
   switch (block) {
     case 4: return launch_qs<4, FMT>(x, numel, block, g, p, s, out, part, st, n);
     case 8: return launch_qs<8, FMT>(x, numel, block, g, p, s, out, part, st, n);
@@ -836,7 +902,7 @@ static cudaError_t qs_block(int block, const uint16_t* x, int64_t numel, uint16_
 cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                                uint16_t g_bits, uint8_t* packed, uint8_t* scales, void* out,
                                void* workspace, cudaStream_t stream, int* launches) {
-  StatsPartial* part = reinterpret_cast<StatsPartial*>(workspace);
+  const Workspace part(workspace);
   if (!bf16) {  // fp32 input: quantize, then reduce from the stored codes
     cudaError_t e = run_quantize(x, false, numel, block, fmt, g_bits, packed, scales, stream,
                                  launches);
@@ -854,7 +920,7 @@ cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int bloc
 cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                             uint16_t g_bits, const uint8_t* packed, const uint8_t* scales,
                             void* out, void* workspace, cudaStream_t stream, int* launches) {
-  StatsPartial* part = reinterpret_cast<StatsPartial*>(workspace);
+  const Workspace part(workspace);
   const bool rc = packed == nullptr;
   if (bf16)
     return fmt == kUE5M3

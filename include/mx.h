@@ -104,7 +104,9 @@ MX_API size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int bloc
  *                   scale codes the quantizer can produce are meaningful (E4M3 0x00..0x7E).
  *   out_dev  OUT one mx_error_stats_t in device memory (written by the last kernel).
  *   workspace, ws_bytes  device scratch of at least mx_error_stats_workspace_size() bytes; its
- *                   contents need no initialisation and are overwritten.
+ *                   contents need no initialisation and are overwritten (a counter, reset by the
+ *                   call, and one partial sum per CTA).  Two calls that share a workspace must
+ *                   not run concurrently (order them on one stream).
  * The reconstruction used for the errors is the exact E2M1 * S * g.  Sums are accumulated in
  * double in a fixed order for a given device, so repeated calls give identical results. */
 MX_API mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
