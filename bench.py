@@ -2,14 +2,15 @@
 
 Default workload (N = 1): the block-size x scale-format sweep on five bf16 4096x4096 tensors
 N(0, sigma^2), sigma in {0.005, 0.01, 0.02, 0.05, 0.1}; block sizes {4..256} x {E4M3, UE5M3} = 70
-points.  One step = quantize+pack of every point, then dequantize (bf16 out) of every point, then
-the three-term error reduction of every point (codes read back), sigma innermost so that no
-buffer is re-read while it could still sit in L2 (inputs 168 MB > 126 MB L2, outputs ~3 GB).
+points.  One step = the fused pass (quantize + pack + three-term error reduction, x read once) of
+every point, then dequantize (bf16 out) of every point; sigma innermost, so that no buffer is
+re-read while it could still sit in L2 (inputs 168 MB > 126 MB L2, outputs ~1.8 GB per step).
 The device-resident number replays one CUDA graph per phase; `e2e` calls the public Python API
 eagerly with the inputs copied from pinned host memory and the 70 error records copied back.
+The plain quantize + pack kernel (no error reduction) is timed beside the step the same way.
 
-Byte accounting (algorithmic, bf16): quantize 2 + 1/2 + 1/N bytes per element, dequantize the same,
-error reduction from stored codes 2 + 1/2 + 1/N.  `roofline` covers the quantize kernel.
+Byte accounting (algorithmic, bf16): fused pass and quantize 2 + 1/2 + 1/N bytes per element,
+dequantize 1/2 + 1/N + 2.  `roofline` covers the fused pass, the dominant kernel of the step.
 
 --gpus N > 1 runs under torchrun, one process per GPU: every rank runs the same sweep on its own
 seeded tensors (weak scaling; the path has no exchange step), timing is the max over ranks.
@@ -69,7 +70,7 @@ def q_bytes(numel, n):
 
 def step_bytes(pts, numel):
     q = sum(q_bytes(numel, n) for _, n, _ in pts)
-    return q, q, q  # quantize, dequantize, error reduction from stored codes
+    return q, q  # fused quantize + pack + error reduction, dequantize
 
 
 def measured_peak():
@@ -187,7 +188,7 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 
 def oracle_sample_step(xs_host, rows, pts, threads):
-    """Quantize, dequantize and error-reduce the first `rows` rows of every point on the CPU."""
+    """Quantize, error-reduce and dequantize the first `rows` rows of every point on the CPU."""
     import oracle
     cols = SHAPE[1]
     for k, n, fmt in pts:
@@ -201,11 +202,11 @@ def oracle_sample(seconds, threads):
     """Pick a row count whose oracle step takes about `seconds`; return (xs_host, rows, pts)."""
     from fp4_microscaling_tensor_b200 import inputs
     pts = points()
-    xs = [inputs.to_oracle(inputs.workload2(k, shape=(256, SHAPE[1]))) for k in range(5)]
+    xs = [inputs.to_oracle(inputs.workload2(k, shape=SHAPE)) for k in range(5)]
     t0 = time.perf_counter()
-    oracle_sample_step(xs, 4, pts, threads)
-    per_row = (time.perf_counter() - t0) / 4
-    rows = int(max(1, min(256, seconds / max(per_row, 1e-9))))
+    oracle_sample_step(xs, 8, pts, threads)
+    per_row = (time.perf_counter() - t0) / 8
+    rows = int(max(1, min(SHAPE[0], seconds / max(per_row, 1e-9))))
     return xs, rows, pts
 
 
@@ -215,8 +216,8 @@ def cpu_rate(xs, rows, pts, threads, reps=1):
         oracle_sample_step(xs, rows, pts, threads)
     dt = (time.perf_counter() - t0) / reps
     numel = rows * SHAPE[1]
-    qb, db, sb = step_bytes(pts, numel)
-    return (qb + db + sb) / dt / 1e9, dt
+    qb, db = step_bytes(pts, numel)
+    return (qb + db) / dt / 1e9, dt
 
 
 def run_reference(args):
@@ -234,9 +235,9 @@ def run_reference(args):
         times.append(time.perf_counter() - t0)
     dt = sum(times) / len(times)
     numel = rows * SHAPE[1]
-    qb, db, sb = step_bytes(pts, numel)
-    v = (qb + db + sb) / dt / 1e9
-    sample = f"first {rows} of 4096 rows of each of the 70 points (quantize, dequantize, error reduction)"
+    qb, db = step_bytes(pts, numel)
+    v = (qb + db) / dt / 1e9
+    sample = f"first {rows} of 4096 rows of each of the 70 points (quantize, error reduction, dequantize)"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
@@ -274,19 +275,35 @@ class Sweep:
         for i, (k, n, fmt) in enumerate(self.pts):
             self.mx.quantize(self.xs[k], n, fmt, packed=self.packed[i], scales=self.scales[i])
 
+    def phase_qs(self):
+        for i, (k, n, fmt) in enumerate(self.pts):
+            self.mx.quantize_with_stats(self.xs[k], n, fmt, packed=self.packed[i],
+                                        scales=self.scales[i], out=self.stats[i],
+                                        workspace=self.ws)
+
     def phase_dq(self):
         for i, (k, n, fmt) in enumerate(self.pts):
             self.mx.dequantize(self.packed[i], self.scales[i], n, fmt, out=self.ys[i])
 
-    def phase_stats(self):
-        for i, (k, n, fmt) in enumerate(self.pts):
-            self.mx.error_stats(self.xs[k], n, fmt, packed=self.packed[i], scales=self.scales[i],
-                                out=self.stats[i], workspace=self.ws)
-
     def step(self):
-        self.phase_q()
+        self.phase_qs()
         self.phase_dq()
-        self.phase_stats()
+
+
+def time_graphs(graphs, steps, stream):
+    """Replay the graphs `steps` times; per-graph device seconds summed over the steps."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+          for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for s in range(steps):
+            ev[s][0].record(stream)
+            for j, g in enumerate(graphs):
+                g.replay()
+                ev[s][j + 1].record(stream)
+    stream.synchronize()
+    return [sum(ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(steps)) / 1e3
+            for j in range(len(graphs))]
 
 
 def run_ours(args):
@@ -315,57 +332,54 @@ def run_ours(args):
         x = inputs.normal(SHAPE, inputs.SWEEP_SIGMAS[k], 100 + k + 1000 * rank, device=dev)
         xs.append(x)
     sw = Sweep(xs, dev)
-    qb, db, sb = step_bytes(sw.pts, numel)
+    qb, db = step_bytes(sw.pts, numel)
 
     # eager warm-up (also loads every kernel), then one graph per phase
     with torch.cuda.stream(stream):
         sw.step()
+        sw.phase_q()
     stream.synchronize()
     graphs = []
     n0 = mx.kernel_launches()
-    for fn in (sw.phase_q, sw.phase_dq, sw.phase_stats):
+    for fn in (sw.phase_qs, sw.phase_dq):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             fn()
         graphs.append(g)
     launches_per_step = mx.kernel_launches() - n0
+    g_q = torch.cuda.CUDAGraph()  # plain quantize + pack, timed beside the step
+    with torch.cuda.graph(g_q, stream=stream):
+        sw.phase_q()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            for g in graphs:
-                g.replay()
-    stream.synchronize()
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    time_graphs(graphs, args.warmup, stream)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
         t_wall = time.perf_counter()
-        with torch.cuda.stream(stream):
-            for s in range(args.steps):
-                ev[s][0].record(stream)
-                for j, g in enumerate(graphs):
-                    g.replay()
-                    ev[s][j + 1].record(stream)
-        stream.synchronize()
+        ph = time_graphs(graphs, args.steps, stream)
         t_wall = time.perf_counter() - t_wall
     barrier()
     torch.cuda.synchronize()
-    ph = [0.0, 0.0, 0.0]
-    for s in range(args.steps):
-        for j in range(3):
-            ph[j] += ev[s][j].elapsed_time(ev[s][j + 1]) / 1e3
     total = sum(ph)
     if world > 1:
         t = torch.tensor([total] + ph, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total, ph = float(t[0]), [float(v) for v in t[1:]]
     step_s = total / args.steps
-    value = world * (qb + db + sb) / step_s / 1e9
+    value = world * (qb + db) / step_s / 1e9
+
+    # plain quantize + pack of the same 70 points (not part of the step)
+    q_steps = max(3, min(args.steps, 50))
+    time_graphs([g_q], 3, stream)
+    t_q = time_graphs([g_q], q_steps, stream)[0] / q_steps
+    if world > 1:
+        t = torch.tensor([t_q], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_q = float(t[0])
 
     # ---- end to end through the public API: pinned H2D of the inputs, eager calls, D2H of stats
     host = [x.cpu().pin_memory() for x in xs]
@@ -394,33 +408,39 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in xs)
     d2h = stats_host.numel()
 
-    # ---- parity spot check of this run's stats against a second replay (deterministic)
+    # ---- a second replay of the fused phase gives the same error records (deterministic sums)
     stats_a = sw.stats.clone()
     with torch.cuda.stream(stream):
-        graphs[2].replay()
+        graphs[0].replay()
     stream.synchronize()
     deterministic = bool(torch.equal(stats_a, sw.stats))
 
     peak, peak_kind = measured_peak()
-    q_gbs = qb / (ph[0] / args.steps) / 1e9
+    per_step = [v / args.steps for v in ph]
+    qs_gbs = qb / per_step[0] / 1e9
+    elems = len(sw.pts) * numel
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "points": len(sw.pts), "elements_per_point": numel,
-                   "phases": "quantize all -> dequantize all -> error reduction all",
+                   "phases": "quantize+pack+error reduction (fused) all -> dequantize all",
                    "launch": "one CUDA graph per phase",
                    "l2": "inputs 168 MB > 126 MB L2; sigma innermost, each buffer reused only "
                          "after >= 4 other points (>150 MB) have streamed",
                    "parallelism": f"dp{world} (independent sweeps)"},
-        "phases_gbs": {"quantize": q_gbs, "dequantize": db / (ph[1] / args.steps) / 1e9,
-                       "error_stats": sb / (ph[2] / args.steps) / 1e9},
-        "gelem_s": {"quantize": len(sw.pts) * numel / (ph[0] / args.steps) / 1e9,
-                    "dequantize": len(sw.pts) * numel / (ph[1] / args.steps) / 1e9},
-        "roofline": {"bound": "hbm", "kernel": "k_quantize_bf16 (all 70 points)",
-                     "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
-                     "peak_kind": peak_kind, "traffic": None},
-        "e2e": {"value": world * (qb + db + sb) / e2e_s / 1e9, "unit": "GB/s",
+        "phases_gbs": {"quantize_pack_stats": qs_gbs, "dequantize": db / per_step[1] / 1e9},
+        "kernels_gbs": {"quantize_pack": qb / t_q / 1e9, "dequantize": db / per_step[1] / 1e9,
+                        "quantize_pack_stats": qs_gbs},
+        "gelem_s": {"quantize_pack_stats": elems / per_step[0] / 1e9,
+                    "quantize_pack": elems / t_q / 1e9,
+                    "dequantize": elems / per_step[1] / 1e9},
+        "roofline": {"bound": "hbm",
+                     "kernel": "k_error_stats_bf16<kStore> (fused quantize+pack+error reduction), "
+                               "all 70 points; per launch avg incl. its 4-byte counter reset",
+                     "achieved": qs_gbs, "peak": peak, "unit": "GB/s", "frac": qs_gbs / peak,
+                     "peak_kind": peak_kind + " (burst copy)", "traffic": None},
+        "e2e": {"value": world * (qb + db) / e2e_s / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "deterministic_stats": deterministic,
@@ -435,7 +455,7 @@ def run_ours(args):
             "value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"first {rows_s} of 4096 rows of each of the 70 points, one step "
                       f"({dt:.1f} s)"}
-    del graphs
+    del graphs, g_q
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -192,35 +192,40 @@ template <int J, bool MS>
 __device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
                                           float sc, float nDq, uint32_t A2, uint32_t S2, float& lt,
                                           float& ms, float& cnt, float& nsat) {
-#define MX_PAIR_HEAD                                   \
-  "{\n\t"                                             \
-  ".reg .b32 blo, bhi, aw, t;\n\t"                    \
-  ".reg .b64 x2, s2, b2, q2, d2;\n\t"                 \
-  ".reg .f32 dlo, dhi;\n\t"                           \
-  ".reg .pred pl, ph, ql, qh;\n\t"                    \
-  "mov.b64 x2, {%12, %13};\n\t"                       \
-  "mov.b64 s2, {%6, %6};\n\t"                         \
-  "mul.rn.f32x2 x2, x2, s2;\n\t"                      \
-  "mul.lo.u32 t, %5, %10;\n\t"                        \
-  "shr.s32 t, t, 6;\n\t"                              \
-  "and.b32 blo, t, 0x81c00000;\n\t"                   \
-  "mul.lo.u32 t, %5, %11;\n\t"                        \
-  "shr.s32 t, t, 6;\n\t"                              \
-  "and.b32 bhi, t, 0x81c00000;\n\t"                   \
-  "mov.b64 b2, {blo, bhi};\n\t"                       \
-  "mov.b64 q2, {%7, %7};\n\t"                         \
-  "fma.rn.f32x2 d2, b2, q2, x2;\n\t"                  \
-  "mov.b64 {dlo, dhi}, d2;\n\t"                       \
-  "and.b32 aw, %4, 0x7fff7fff;\n\t"                   \
-  "setp.ge.bf16x2 pl|ph, aw, %8;\n\t"                 \
-  "setp.gt.bf16x2 ql|qh, aw, %9;\n\t"                 \
-  "@!pl fma.rn.f32 %0, dlo, dlo, %0;\n\t"             \
+  static_assert(J >= 0 && J < 4, "byte index");
+  // The decode of code byte J is bit arithmetic: each code's bits become its value times 2^-126
+  // (sign to bit 31, exponent and mantissa to bits 24..22), and %7 is -S g s 2^126.  (The
+  // E2M1x2 -> f16x2 conversion instruction was tried instead and gave wrong values for some
+  // inputs when its byte came straight from the encoding conversion in registers.)
+#define MX_PAIR_HEAD                            \
+  "{\n\t"                                      \
+  ".reg .b32 blo, bhi, aw, t;\n\t"             \
+  ".reg .b64 x2, s2, b2, q2, d2;\n\t"          \
+  ".reg .f32 dlo, dhi;\n\t"                    \
+  ".reg .pred pl, ph, ql, qh;\n\t"             \
+  "mov.b64 x2, {%12, %13};\n\t"                \
+  "mov.b64 s2, {%6, %6};\n\t"                  \
+  "mul.rn.f32x2 x2, x2, s2;\n\t"               \
+  "mul.lo.u32 t, %5, %10;\n\t"                 \
+  "shr.s32 t, t, 6;\n\t"                       \
+  "and.b32 blo, t, 0x81c00000;\n\t"            \
+  "mul.lo.u32 t, %5, %11;\n\t"                 \
+  "shr.s32 t, t, 6;\n\t"                       \
+  "and.b32 bhi, t, 0x81c00000;\n\t"            \
+  "mov.b64 b2, {blo, bhi};\n\t"                \
+  "mov.b64 q2, {%7, %7};\n\t"                  \
+  "fma.rn.f32x2 d2, b2, q2, x2;\n\t"           \
+  "mov.b64 {dlo, dhi}, d2;\n\t"                \
+  "and.b32 aw, %4, 0x7fff7fff;\n\t"            \
+  "setp.ge.bf16x2 pl|ph, aw, %8;\n\t"          \
+  "setp.gt.bf16x2 ql|qh, aw, %9;\n\t"          \
+  "@!pl fma.rn.f32 %0, dlo, dlo, %0;\n\t"      \
   "@!ph fma.rn.f32 %0, dhi, dhi, %0;\n\t"
-#define MX_PAIR_TAIL                                   \
-  "@pl add.f32 %2, %2, 0f3F800000;\n\t"               \
-  "@ph add.f32 %2, %2, 0f3F800000;\n\t"               \
-  "@ql add.f32 %3, %3, 0f3F800000;\n\t"               \
-  "@qh add.f32 %3, %3, 0f3F800000;\n\t"               \
+#define MX_PAIR_TAIL                            \
+  "@pl add.f32 %2, %2, 0f3F800000;\n\t"        \
+  "@ph add.f32 %2, %2, 0f3F800000;\n\t"        \
+  "@ql add.f32 %3, %3, 0f3F800000;\n\t"        \
+  "@qh add.f32 %3, %3, 0f3F800000;\n\t"        \
   "}"
   if constexpr (MS) {
     asm(MX_PAIR_HEAD
@@ -553,16 +558,17 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
       const uint32_t sb = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // 6 S g rounded down
       const uint32_t A2 = m_b[b] * 0x10001u, S2 = sb * 0x10001u;
       float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f, dmax = 0.0f;
+      const float nD = st.nDq;
 #pragma unroll
       for (int k = 0; k < BW; ++k) {
         const int wi = b * BW + k;
         const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
         constexpr bool MS = !RECOMPUTE;
         switch (wi & 3) {
-          case 0: pair_step<0, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
-          case 1: pair_step<1, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
-          case 2: pair_step<2, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
-          default: pair_step<3, MS>(w, lo, hi, cw, st.sc, st.nDq, A2, S2, lt, ms, cnt, nsat); break;
+          case 0: pair_step<0, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
+          case 1: pair_step<1, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
+          case 2: pair_step<2, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
+          default: pair_step<3, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
         }
       }
       if constexpr (RECOMPUTE) {
