@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(kThreads) k_dequantize(const uint8_t* __restri
   const float g = fp16_bits_to_float(g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
 
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -125,7 +127,9 @@ static cudaError_t launch_dq(const uint8_t* packed, const uint8_t* scales, int64
   const int64_t nitems = numel / S::EPT;
   if (nitems > 0) {
     const int grid = persistent_grid((const void*)k_dequantize<N, FMT, BF16OUT>, nitems, S::U);
-    k_dequantize<N, FMT, BF16OUT><<<grid, kThreads, 0, stream>>>(packed, scales, nitems, g_bits, y);
+    const cudaError_t e = launch_pdl(k_dequantize<N, FMT, BF16OUT>, grid, kThreads, stream, packed,
+                                     scales, nitems, g_bits, y);
+    if (e != cudaSuccess) return e;
     ++*launches;
   }
   if (numel % S::EPT != 0) {

@@ -142,6 +142,13 @@ __device__ __forceinline__ uint32_t bf16x2_absmin(uint32_t a, uint32_t b) {
 }
 
 // Streaming 16-byte load of read-only data (not kept in L1).
+// Programmatic dependent launch: wait until the previous grid in the stream has completed and its
+// memory is visible (a no-op without such a dependency); then allow the next grid to be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;
   asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"

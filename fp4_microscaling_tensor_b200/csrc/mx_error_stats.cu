@@ -453,6 +453,8 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
   const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
   const float sat_thr = __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>());  // exact
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
 
   Acc acc;
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
@@ -624,6 +626,8 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
   const float g6 = __fmul_rn(6.0f, g);
   const float sat_thr = __fmul_rn(g6, scale_max<FMT>());
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
 
   Acc acc;
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
@@ -784,6 +788,15 @@ struct Workspace {
 };
 constexpr int kMaxStatsGrid = kMaxReduceCtas - 2;  // header + one slot for the N = 4 tail
 
+// Zeroes the last-CTA counter once the previous kernel in the stream is done with it (launched
+// with programmatic serialization, so its launch overlaps that kernel's tail and the main pass's
+// launch overlaps it).
+__global__ void k_stats_reset(unsigned int* counter) {
+  griddep_wait();
+  if (threadIdx.x == 0) *counter = 0;
+  griddep_launch_next();
+}
+
 // Main pass, then (N = 4 tail) the tail partial and a one-CTA final pass, or (empty) the final
 // pass alone.  Without a tail the main pass adds the partials itself.
 template <typename Launch>
@@ -794,8 +807,9 @@ static cudaError_t stats_passes(int64_t nitems, bool tail, int64_t numel, int bl
   if (nitems > 0) {
     FinalArgs fa{nullptr, (StatsOut*)out, numel, numel / block};
     if (!tail) {
-      const cudaError_t e = cudaMemsetAsync(ws.counter, 0, sizeof(unsigned int), stream);
+      const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, ws.counter);
       if (e != cudaSuccess) return e;
+      ++*launches;
       fa.counter = ws.counter;
     }
     nparts = main(fa);
@@ -824,11 +838,12 @@ static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g
                            : (const void*)k_error_stats_f32<N, FMT, RC>;
     const int grid = persistent_grid(kern, nitems, S::U, kMaxStatsGrid);
     if (sizeof(T) == 2)
-      k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven><<<grid, kThreads, 0, stream>>>(
-          (const uint16_t*)x, nitems, g_bits, packed, scales, ws.part, fa, nullptr, nullptr);
+      launch_pdl(k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>, grid, kThreads, stream,
+                 (const uint16_t*)x, nitems, g_bits, packed, scales, ws.part, fa,
+                 (uint8_t*)nullptr, (uint8_t*)nullptr);
     else
-      k_error_stats_f32<N, FMT, RC><<<grid, kThreads, 0, stream>>>(
-          (const float*)x, nitems, g_bits, packed, scales, ws.part, fa);
+      launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream, (const float*)x, nitems,
+                 g_bits, packed, scales, ws.part, fa);
     return grid;
   };
   auto tail = [&](StatsPartial* slot) {
@@ -876,8 +891,8 @@ static cudaError_t launch_qs(const uint16_t* x, int64_t numel, int block, uint16
   auto main = [&](FinalArgs fa) {
     const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, kStore>, nitems,
                                      S::U, kMaxStatsGrid);
-    k_error_stats_bf16<N, FMT, kStore><<<grid, kThreads, 0, stream>>>(
-        x, nitems, g_bits, nullptr, nullptr, ws.part, fa, packed, scales);
+    launch_pdl(k_error_stats_bf16<N, FMT, kStore>, grid, kThreads, stream, x, nitems, g_bits,
+               (const uint8_t*)nullptr, (const uint8_t*)nullptr, ws.part, fa, packed, scales);
     return grid;
   };
   // N = 4 with 4 elements left: quantize them, then reduce them from the stored codes

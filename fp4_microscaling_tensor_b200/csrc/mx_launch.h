@@ -25,6 +25,27 @@ inline int persistent_grid(const void* kern, int64_t nitems, int items_per_iter,
   return (int)(g < 1 ? 1 : g);
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel in the stream is still finishing.  Every kernel launched this way executes
+// griddep_wait() (mx_device.cuh) before its first global-memory access, which returns once the
+// previous grid has completed and its writes are visible; so ordering is as for a plain launch and
+// only the launch latency and the shared-memory setup overlap the previous kernel's tail.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
                          uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
                          int* launches);

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const uint16_t* __re
   }
   const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
 
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const float* __restri
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   const float g6 = __fmul_rn(6.0f, g);
   __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
 
   const int64_t T = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -244,12 +248,13 @@ static cudaError_t launch_q(const void* x, int64_t numel, uint16_t g_bits, uint8
   if (nitems > 0) {
     auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT> : (void*)k_quantize_f32<N, FMT>;
     const int grid = persistent_grid(kern, nitems, S::U);
-    if (sizeof(T) == 2)
-      k_quantize_bf16<N, FMT><<<grid, kThreads, 0, stream>>>(
-          (const uint16_t*)x, nitems, g_bits, packed, scales);
-    else
-      k_quantize_f32<N, FMT><<<grid, kThreads, 0, stream>>>((const float*)x, nitems, g_bits,
-                                                            packed, scales);
+    const cudaError_t e =
+        (sizeof(T) == 2)
+            ? launch_pdl(k_quantize_bf16<N, FMT>, grid, kThreads, stream, (const uint16_t*)x,
+                         nitems, g_bits, packed, scales)
+            : launch_pdl(k_quantize_f32<N, FMT>, grid, kThreads, stream, (const float*)x, nitems,
+                         g_bits, packed, scales);
+    if (e != cudaSuccess) return e;
     ++*launches;
   }
   if (numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
