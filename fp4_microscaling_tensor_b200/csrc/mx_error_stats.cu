@@ -330,14 +330,14 @@ __device__ __forceinline__ void exact_slice(float a, float D, XF xval, CF code, 
 }
 
 // Tail of a bf16 block slice: lt is the sum of the scaled squares of the elements below the
-// maximum, cnt the number of max-valued elements, nsat the clipped elements.  Stored codes (!RC):
-// ms sums the scaled squares of the max-valued elements; a lane with ties of the maximum redoes
-// those elements in double, a slice whose stored scale is far from a redoes everything.
-// Recomputed codes (RC): every max-valued element has the same error, dmax (scaled), computed
-// once per block.  Either way a slice whose lt is below 2^-80 may have lost squares below 2^-126
+// maximum, cnt the number of max-valued elements, nsat the clipped elements.  Without CLOSED, ms
+// sums the scaled squares of the max-valued elements and a lane with ties of the maximum redoes
+// those elements in double; with stored codes (!RC) a slice whose stored scale is far from a
+// redoes everything.  CLOSED (recomputed codes): every max-valued element has the same error,
+// dmax (scaled), computed once per block.  Either way a slice whose lt is below 2^-80 may have lost squares below 2^-126
 // and is redone in double (any loss in a larger sum is below 2^-40 of it).  Items past the end
 // hold zeros and an all-zero scale, so they add zeros (their block counters are skipped via ok).
-template <int NE, int L, bool RC, typename XF, typename CF>
+template <int NE, int L, bool RC, bool CLOSED, typename XF, typename CF>
 __device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, float a, float D,
                                                   float sat_thr, const SliceSetup& st, float lt,
                                                   float ms, float dmax, float cnt, float nsat,
@@ -357,7 +357,7 @@ __device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, f
   } else {
     const double sd = unscale_sq(st.E);
     rest = (double)lt * sd;
-    if constexpr (RC) {
+    if constexpr (CLOSED) {
       if (has_max) {
         first = (double)dmax * (double)dmax * sd;  // exact
         others = (double)(cnt - 1.0f) * first;
@@ -437,6 +437,9 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
     StatsPartial* __restrict__ part, FinalArgs fa, uint8_t* __restrict__ packed_out,
     uint8_t* __restrict__ scales_out) {
   constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
+  // Recomputed codes: the max-valued elements' error in closed form per block (blocks of 16 and
+  // more), or summed like the others (small blocks, where the per-block work would cost more).
+  constexpr bool CLOSED = RECOMPUTE && N >= 16;
   using S = SShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, NW = EPT / 2, NCW = EPT / 8;
   constexpr int BW = NW / BPI;  // words per block inside an item
@@ -565,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
       for (int k = 0; k < BW; ++k) {
         const int wi = b * BW + k;
         const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
-        constexpr bool MS = !RECOMPUTE;
+        constexpr bool MS = !CLOSED;
         switch (wi & 3) {
           case 0: pair_step<0, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
           case 1: pair_step<1, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
@@ -573,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
           default: pair_step<3, MS>(w, lo, hi, cw, st.sc, nD, A2, S2, lt, ms, cnt, nsat); break;
         }
       }
-      if constexpr (RECOMPUTE) {
+      if constexpr (CLOSED) {
         // the max-valued elements' code magnitude is that of a; their scaled error, as above
         const float qa = snap_quotient2(__float_as_uint(a), 0u, r_b[b]).x;
         const uint32_t ca = cvt_e2m1x8(qa, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
@@ -586,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
         return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
       };
       auto code = [&](int k) { return it.cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
-      slice_finish_bf16<BE, L, RECOMPUTE>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax, cnt,
+      slice_finish_bf16<BE, L, RECOMPUTE, CLOSED>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax, cnt,
                                           nsat, xval, code);
     }
   };
