@@ -1,26 +1,26 @@
-// mx_error_stats.cu -- fused three-term block-error reduction (sm_100a).
+// mx_error_stats.cu -- three-term block-error reduction, alone or fused with quantize + pack.
 //
 // Method: the microscaling article (hotelren.com/news/2192771) §2.2 items 1-3.  Per block with a
 // non-zero scale: the max element (first index of max|x|) contributes (x - y)^2 to SSE_max (the
 // scale-rounding error of item 2), every other element to SSE_elem (item 1).  A block whose scale
 // is zero contributes sum x^2 to SSE_zero (item 3).  y is the exact E2M1 * S * g.
 //
-// Pass 1 (k_error_stats_*): persistent grid; each thread walks items like the quantize kernel,
-// either recomputing the codes in registers (RECOMPUTE: reads x only) or reading stored codes.
-// Per block slice held by a lane:
+// Main pass (k_error_stats_*): persistent grid; each thread walks items of 8, 16 or 32 elements
+// with the next item's loads issued before the current item's arithmetic.  The codes are read
+// (kGiven), recomputed in registers with the quantize rule (kRecompute), or recomputed and stored
+// (kStore: the fused quantize + pack + reduction pass, x read once).  Per block slice held by a
+// lane:
 //   * Scaling.  s = 2^k brings the block maximum a into [1, 2).  d' = x s - code * (S g s) is one
 //     FMA (the code's bits are its value times 2^-126; S g s 2^126 is a per-block constant) and
-//     exact; squares are summed in fp32 (at most 16 terms) and scaled back exactly in double
-//     (integer operations place the fp32 sum, times 1/s^2, into a double).
-//   * Two compares per element: |x| == a (the max-valued elements: their squares go to a second
-//     fp32 sum and a counter) and |x| > 6 S g (clipped elements, counted).  A lane holding one
-//     max-valued element (the usual case) knows its error exactly; the block's first max element
-//     (lowest lane, lowest index) goes to SSE_max, everything else to SSE_elem.  Ties of the
-//     maximum inside one lane take a slower path in double.  All added terms are non-negative,
-//     so exact zeros stay exact.
-//   * Underflow.  Scaled squares below 2^-120 would lose digits.  A lane whose slice holds a value
-//     below 2^-30 a (checked with a min|x| tree, then per element only if the tree fires, because
-//     exact zeros are harmless) or whose stored scale is far from a redoes its slice in double.
+//     exact; squares are summed in fp32 (at most 32 terms) and scaled back exactly in double.
+//   * Two bf16x2 compares per word: |x| >= a (the max-valued elements) and |x| > 6 S g (clipped
+//     elements, counted).  The max-valued elements stay out of the per-element sum: with
+//     recomputed codes (N >= 16) they all share one error, computed once per block; otherwise
+//     their squares are summed apart, and a lane holding a tie of the maximum redoes them in
+//     double.  The block's first max element (lowest lane, lowest index) goes to SSE_max,
+//     everything else to SSE_elem.  All added terms are non-negative, so exact zeros stay exact.
+//   * Underflow.  A slice whose scaled non-max sum is below 2^-80 (squares below 2^-126 could be
+//     lost), or whose stored scale is far from a, redoes its slice in double.
 // Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
 // in a fixed order, so results are deterministic for a given device and grid; with an N = 4 tail a
 // separate one-CTA pass does it.  No CTA waits on another.
