@@ -39,7 +39,7 @@ L2_BYTES = 126 * 2 ** 20
 FUSED_TRAFFIC_BYTES = 33607424 + 7168
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -55,7 +55,7 @@ def parse():
     ap.add_argument("--block", type=int, default=32)
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
     ap.add_argument("--reps", type=int, default=20)
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def points():
@@ -311,6 +311,22 @@ def time_graphs(graphs, steps, stream):
             for j in range(len(graphs))]
 
 
+def rank_seed(k, rank):
+    """Seed of sigma index k on a rank: every rank draws its own tensors (weak scaling)."""
+    return 100 + k + 1000 * rank
+
+
+def max_over_ranks(vals, device):
+    """Element-wise max over the ranks of the process group (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -334,7 +350,7 @@ def run_ours(args):
     # each rank draws its own tensors (seed offset by rank): weak scaling, no data exchange
     xs = []
     for k in range(len(inputs.SWEEP_SIGMAS)):
-        x = inputs.normal(SHAPE, inputs.SWEEP_SIGMAS[k], 100 + k + 1000 * rank, device=dev)
+        x = inputs.normal(SHAPE, inputs.SWEEP_SIGMAS[k], rank_seed(k, rank), device=dev)
         xs.append(x)
     sw = Sweep(xs, dev)
     qb, db = step_bytes(sw.pts, numel)
@@ -370,21 +386,15 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     total = sum(ph)
-    if world > 1:
-        t = torch.tensor([total] + ph, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total, ph = float(t[0]), [float(v) for v in t[1:]]
+    comb = max_over_ranks([total] + ph, dev)
+    total, ph = comb[0], comb[1:]
     step_s = total / args.steps
     value = world * (qb + db) / step_s / 1e9
 
     # plain quantize + pack of the same 70 points (not part of the step)
     q_steps = max(3, min(args.steps, 50))
     time_graphs([g_q], 3, stream)
-    t_q = time_graphs([g_q], q_steps, stream)[0] / q_steps
-    if world > 1:
-        t = torch.tensor([t_q], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_q = float(t[0])
+    t_q = max_over_ranks([time_graphs([g_q], q_steps, stream)[0] / q_steps], dev)[0]
 
     # ---- end to end through the public API: pinned H2D of the inputs, eager calls, D2H of stats
     host = [x.cpu().pin_memory() for x in xs]
@@ -405,11 +415,7 @@ def run_ours(args):
     t0 = time.perf_counter()
     for _ in range(args.e2e_steps):
         e2e_step()
-    e2e_s = (time.perf_counter() - t0) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t[0])
+    e2e_s = max_over_ranks([(time.perf_counter() - t0) / args.e2e_steps], dev)[0]
     h2d = sum(x.numel() * x.element_size() for x in xs)
     d2h = stats_host.numel()
 

@@ -1,0 +1,71 @@
+"""Host logic of `bench.py --gpus N` with two ranks on the CPU (gloo backend, world size 2).
+
+The path shards without an exchange step: every rank draws its own seeded tensors and the only
+collective is the max over ranks of the timings.  These tests run that logic in two processes.
+"""
+import io
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from fp4_microscaling_tensor_b200 import inputs
+        # timings: element-wise max over ranks
+        got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5 * rank], "cpu")
+        # each rank draws its own tensors: checksums differ across ranks
+        x = inputs.normal((64, 256), inputs.SWEEP_SIGMAS[2], bench.rank_seed(2, rank))
+        chk = torch.tensor([float(x.float().sum())], dtype=torch.float64)
+        allc = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(allc, chk)
+        # the reference arm: only rank 0 prints
+        buf = io.StringIO()
+        args = bench.parse(["--impl", "reference", "--gpus", str(world), "--steps", "1",
+                            "--warmup", "0"])
+        if rank != 0:
+            with redirect_stdout(buf):
+                bench.run_reference(args)
+        out[rank] = (got, [float(c) for c in allc], buf.getvalue())
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_ranks_gloo():
+    world = 2
+    port = free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for rank in range(world):
+        got, checks, printed = res[rank]
+        assert got == [2.0, 10.0, 0.5]
+        assert checks[0] != checks[1]
+        assert printed == ""
+
+
+def test_single_process_identity():
+    assert bench.max_over_ranks([3.0, 4.0], "cpu") == [3.0, 4.0]
+    assert bench.rank_seed(0, 0) != bench.rank_seed(0, 1)
