@@ -27,7 +27,20 @@ MX_SCALE_E4M3, MX_SCALE_UE5M3 = 0, 1
 EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_error_stats",
            "mx_quantize_stats",
            "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
+           "mx_quantize_group", "mx_dequantize_group", "mx_quantize_stats_group",
            "mx_status_string", "mx_kernel_launches")
+MX_MAX_GROUP = 16
+
+
+class Tensor(ctypes.Structure):
+    """mx_tensor_t (64 bytes): one tensor of a grouped call."""
+    _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("packed", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("global_scale_fp16", ctypes.c_uint16), ("reserved", ctypes.c_uint16 * 3)]
+
+
+assert ctypes.sizeof(Tensor) == 64
 
 _i, _i64, _u16, _vp, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_uint16, ctypes.c_void_p, ctypes.c_size_t
 
@@ -47,6 +60,13 @@ lib.mx_global_scale.restype = _i
 lib.mx_global_scale.argtypes = [_vp, _i, _i64, _i64, _i, _vp, _vp, _sz, _vp]
 lib.mx_error_stats_noalloc.restype = _i
 lib.mx_error_stats_noalloc.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp]
+_tp = ctypes.POINTER(Tensor)
+lib.mx_quantize_group.restype = _i
+lib.mx_quantize_group.argtypes = [_tp, _i, _i, _i, _i, _vp]
+lib.mx_dequantize_group.restype = _i
+lib.mx_dequantize_group.argtypes = [_tp, _i, _i, _i, _i, _vp]
+lib.mx_quantize_stats_group.restype = _i
+lib.mx_quantize_stats_group.argtypes = [_tp, _i, _i, _i, _i, _vp, _sz, _vp]
 lib.mx_status_string.restype = ctypes.c_char_p
 lib.mx_status_string.argtypes = [_i]
 lib.mx_kernel_launches.restype = ctypes.c_longlong

@@ -9,8 +9,8 @@ import struct
 import numpy as np
 import torch
 
-from ._lib import (MX_BF16, MX_F32, MX_SCALE_E4M3, MX_SCALE_UE5M3, MXError, check,  # noqa: F401
-                   lib)
+from ._lib import (MX_BF16, MX_F32, MX_MAX_GROUP, MX_SCALE_E4M3, MX_SCALE_UE5M3,  # noqa: F401
+                   MXError, Tensor, check, lib)
 
 E4M3, UE5M3 = MX_SCALE_E4M3, MX_SCALE_UE5M3
 _FMT = {"e4m3": E4M3, "ue5m3": UE5M3, E4M3: E4M3, UE5M3: UE5M3}
@@ -170,6 +170,113 @@ def global_scale(x, fmt="e4m3", out=None, workspace=None, stream=None):
                               out.data_ptr(), workspace.data_ptr(), workspace.numel(),
                               _stream(stream, x.device)), "mx_global_scale")
     return out[:2].view(torch.uint16)
+
+
+# ---- grouped calls: one launch for up to MX_MAX_GROUP tensors of the same dtype, block, format
+
+def _group(n, what):
+    if not 1 <= n <= MX_MAX_GROUP:
+        raise ValueError(f"{what}: between 1 and {MX_MAX_GROUP} tensors per call")
+    return (Tensor * n)()
+
+
+def _gs(g, n):
+    if isinstance(g, (list, tuple)):
+        if len(g) != n:
+            raise ValueError("one global scale per tensor")
+        return [g_bits(v) for v in g]
+    return [g_bits(g)] * n
+
+
+def quantize_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None, stream=None):
+    """quantize() of every tensor of xs in one launch; g: one value or one per tensor.
+    Returns (list of packed, list of scales)."""
+    xs = list(xs)
+    n = len(xs)
+    desc = _group(n, "quantize_group")
+    dt = {x.dtype for x in xs}
+    if len(dt) != 1 or next(iter(dt)) not in _DT:
+        raise ValueError("all tensors float32 or all bfloat16")
+    gs = _gs(g, n)
+    packed = list(packed) if packed is not None else [None] * n
+    scales = list(scales) if scales is not None else [None] * n
+    for k, x in enumerate(xs):
+        rows, cols = _shape2d(x, "x")
+        lead = tuple(x.shape[:-1])
+        if packed[k] is None:
+            packed[k] = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+        if scales[k] is None:
+            scales[k] = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+                                    device=x.device)
+        desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
+                                                     scales[k].data_ptr())
+        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = rows, cols, gs[k]
+    check(lib.mx_quantize_group(desc, n, _DT[xs[0].dtype], int(block), fmt_code(fmt),
+                                _stream(stream, xs[0].device)), "mx_quantize_group")
+    return packed, scales
+
+
+def dequantize_group(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=torch.bfloat16,
+                     out=None, stream=None):
+    """dequantize() of every (packed, scales) pair in one launch.  Returns the list of outputs."""
+    packed, scales = list(packed), list(scales)
+    n = len(packed)
+    if len(scales) != n:
+        raise ValueError("one scales tensor per packed tensor")
+    if out_dtype not in _DT:
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    desc = _group(n, "dequantize_group")
+    gs = _gs(g, n)
+    out = list(out) if out is not None else [None] * n
+    for k in range(n):
+        prow, pcols = _shape2d(packed[k], "packed")
+        _shape2d(scales[k], "scales")
+        if out[k] is None:
+            out[k] = torch.empty(tuple(packed[k].shape[:-1]) + (2 * pcols,), dtype=out_dtype,
+                                 device=packed[k].device)
+        desc[k].y, desc[k].packed, desc[k].scales = (out[k].data_ptr(), packed[k].data_ptr(),
+                                                     scales[k].data_ptr())
+        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = prow, 2 * pcols, gs[k]
+    check(lib.mx_dequantize_group(desc, n, int(block), fmt_code(fmt), _DT[out_dtype],
+                                  _stream(stream, packed[0].device)), "mx_dequantize_group")
+    return out
+
+
+def quantize_with_stats_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None,
+                              out=None, workspace=None, stream=None):
+    """quantize_with_stats() of every tensor of xs in one launch.  out: a uint8 tensor of
+    len(xs) x 64 bytes for the records (allocated when None).  Returns (packed list, scales list,
+    list of ErrorStats)."""
+    xs = list(xs)
+    n = len(xs)
+    desc = _group(n, "quantize_with_stats_group")
+    dt = {x.dtype for x in xs}
+    if len(dt) != 1 or next(iter(dt)) not in _DT:
+        raise ValueError("all tensors float32 or all bfloat16")
+    gs = _gs(g, n)
+    dev = xs[0].device
+    if out is None:
+        out = torch.empty(n, STATS_BYTES, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = stats_workspace(dev)
+    packed = list(packed) if packed is not None else [None] * n
+    scales = list(scales) if scales is not None else [None] * n
+    for k, x in enumerate(xs):
+        rows, cols = _shape2d(x, "x")
+        lead = tuple(x.shape[:-1])
+        if packed[k] is None:
+            packed[k] = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+        if scales[k] is None:
+            scales[k] = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+                                    device=x.device)
+        desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
+                                                     scales[k].data_ptr())
+        desc[k].stats = out[k].data_ptr()
+        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = rows, cols, gs[k]
+    check(lib.mx_quantize_stats_group(desc, n, _DT[xs[0].dtype], int(block), fmt_code(fmt),
+                                      workspace.data_ptr(), workspace.numel(),
+                                      _stream(stream, dev)), "mx_quantize_stats_group")
+    return packed, scales, [ErrorStats(out[k]) for k in range(n)]
 
 
 def kernel_launches():

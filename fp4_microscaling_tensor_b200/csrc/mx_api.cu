@@ -8,6 +8,8 @@
 #include "mx_launch.h"
 
 static_assert(sizeof(mx_error_stats_t) == 64, "mx_error_stats_t layout");
+static_assert(sizeof(mx_tensor_t) == 64, "mx_tensor_t layout");
+static_assert(MX_MAX_GROUP == mxk::kMaxGroup, "group size");
 
 namespace {
 
@@ -153,6 +155,83 @@ mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols
   int n = 0;
   const cudaError_t e = mxk::run_global_scale(x, xt == MX_BF16, numel, (int)fmt, out_fp16_dev,
                                               workspace, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+namespace {
+
+// Checks shared by the grouped calls: per tensor shape, pointers (`need` says which) and g.
+enum : unsigned { kNeedX = 1, kNeedY = 2, kNeedCodes = 4, kNeedStats = 8 };
+
+mx_status check_group(const mx_tensor_t* t, int count, int block, unsigned need,
+                      mxk::TensorArgs* args) {
+  if (!t || count < 1 || count > MX_MAX_GROUP) return MX_ERR_INVALID_ARG;
+  for (int k = 0; k < count; ++k) {
+    const mx_tensor_t& d = t[k];
+    if (!shape_ok(d.rows, d.cols) || !valid_g(d.global_scale_fp16) || d.reserved[0] ||
+        d.reserved[1] || d.reserved[2])
+      return MX_ERR_INVALID_ARG;
+    if (d.cols % block != 0) return MX_ERR_INVALID_ARG;
+    const int64_t numel = d.rows * d.cols;
+    if ((need & kNeedStats) && !d.stats) return MX_ERR_INVALID_ARG;
+    if ((need & kNeedStats) && !aligned16(d.stats)) return MX_ERR_MISALIGNED;
+    if (numel != 0) {
+      if (((need & kNeedX) && !d.x) || ((need & kNeedY) && !d.y) ||
+          ((need & kNeedCodes) && (!d.packed || !d.scales)))
+        return MX_ERR_INVALID_ARG;
+      if (((need & kNeedX) && !aligned16(d.x)) || ((need & kNeedY) && !aligned16(d.y)) ||
+          ((need & kNeedCodes) && (!aligned16(d.packed) || !aligned16(d.scales))))
+        return MX_ERR_MISALIGNED;
+    }
+    args[k] = {d.x, d.y, d.packed, d.scales, d.stats, numel, d.global_scale_fp16};
+  }
+  return MX_OK;
+}
+
+}  // namespace
+
+mx_status mx_quantize_group(const mx_tensor_t* tensors, int count, mx_dtype xt, int block,
+                            mx_scale_fmt fmt, cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  mxk::TensorArgs args[MX_MAX_GROUP];
+  const mx_status st = check_group(tensors, count, block, kNeedX | kNeedCodes, args);
+  if (st != MX_OK) return st;
+  int n = 0;
+  const cudaError_t e =
+      mxk::run_quantize_group(args, count, xt == MX_BF16, block, (int)fmt, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+mx_status mx_dequantize_group(const mx_tensor_t* tensors, int count, int block, mx_scale_fmt fmt,
+                              mx_dtype yt, cudaStream_t stream) {
+  if (!valid_dtype(yt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  mxk::TensorArgs args[MX_MAX_GROUP];
+  const mx_status st = check_group(tensors, count, block, kNeedY | kNeedCodes, args);
+  if (st != MX_OK) return st;
+  int n = 0;
+  const cudaError_t e =
+      mxk::run_dequantize_group(args, count, yt == MX_BF16, block, (int)fmt, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtype xt, int block,
+                                  mx_scale_fmt fmt, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  mxk::TensorArgs args[MX_MAX_GROUP];
+  const mx_status st = check_group(tensors, count, block, kNeedX | kNeedCodes | kNeedStats, args);
+  if (st != MX_OK) return st;
+  if (!workspace || ws_bytes < stats_ws_bytes()) return MX_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_stats_group(args, count, xt == MX_BF16, block, (int)fmt,
+                                             mxk::kStore, workspace, stream, &n);
   g_launches += n;
   return from_cuda(e);
 }

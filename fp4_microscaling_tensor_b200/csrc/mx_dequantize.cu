@@ -31,22 +31,40 @@ struct DShape {
   static constexpr int U = MX_DQ_U;
 };
 
+// Kernel parameters: up to kMaxGroup tensors and the split of the grid among them.
+struct DTensor {
+  const uint8_t* packed;
+  const uint8_t* scales;
+  void* y;
+  int64_t nitems;
+  uint32_t g_bits;
+};
+struct DGroup {
+  DTensor t[kMaxGroup];
+  CtaSplit split;
+};
+
 template <int N, int FMT, bool BF16OUT>
-__global__ void __launch_bounds__(kThreads) k_dequantize(const uint8_t* __restrict__ packed,
-                                                          const uint8_t* __restrict__ scales,
-                                                          int64_t nitems, uint16_t g_bits,
-                                                          void* __restrict__ y) {
+__global__ void __launch_bounds__(kThreads) k_dequantize(const __grid_constant__ DGroup grp) {
   using S = DShape<N, BF16OUT>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U;
+  const int ti = grp.split.find((int)blockIdx.x);
+  const DTensor tt = grp.t[ti];
+  const int cta = (int)blockIdx.x - grp.split.begin[ti];
+  const int nctas = grp.split.begin[ti + 1] - grp.split.begin[ti];
+  const uint8_t* __restrict__ packed = tt.packed;
+  const uint8_t* __restrict__ scales = tt.scales;
+  void* __restrict__ y = tt.y;
+  const int64_t nitems = tt.nitems;
   __shared__ float s_D[256];
-  const float g = fp16_bits_to_float(g_bits);
+  const float g = fp16_bits_to_float((uint16_t)tt.g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   __syncthreads();
   griddep_wait();  // inputs may come from the previous kernel in the stream
   griddep_launch_next();
 
-  const int64_t T = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t T = (int64_t)nctas * blockDim.x;
+  const int64_t tid = (int64_t)cta * blockDim.x + threadIdx.x;
   for (int64_t base = tid; base < nitems; base += T * U) {
     uint32_t cw[U][EPT / 8];
     uint32_t sc[U];
@@ -121,47 +139,62 @@ __global__ void k_dequantize_tail4(const uint8_t* __restrict__ packed,
 }
 
 template <int N, int FMT, bool BF16OUT>
-static cudaError_t launch_dq(const uint8_t* packed, const uint8_t* scales, int64_t numel,
-                             uint16_t g_bits, void* y, cudaStream_t stream, int* launches) {
+static cudaError_t launch_dq(const TensorArgs* ta, int count, cudaStream_t stream,
+                             int* launches) {
   using S = DShape<N, BF16OUT>;
-  const int64_t nitems = numel / S::EPT;
-  if (nitems > 0) {
-    const int grid = persistent_grid((const void*)k_dequantize<N, FMT, BF16OUT>, nitems, S::U);
-    const cudaError_t e = launch_pdl(k_dequantize<N, FMT, BF16OUT>, grid, kThreads, stream, packed,
-                                     scales, nitems, g_bits, y);
+  DGroup grp = {};
+  int64_t nitems[kMaxGroup];
+  for (int k = 0; k < count; ++k) {
+    nitems[k] = ta[k].numel / S::EPT;
+    grp.t[k] = {ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits};
+  }
+  const int grid = split_grid((const void*)k_dequantize<N, FMT, BF16OUT>, nitems, count, S::U,
+                              1 << 30, &grp.split);
+  if (grid > 0) {
+    const cudaError_t e =
+        launch_pdl(k_dequantize<N, FMT, BF16OUT>, grid, kThreads, stream, grp);
     if (e != cudaSuccess) return e;
     ++*launches;
   }
-  if (numel % S::EPT != 0) {
-    k_dequantize_tail4<FMT, BF16OUT><<<1, 32, 0, stream>>>(packed, scales, nitems * S::EPT,
-                                                            g_bits, y);
-    ++*launches;
+  for (int k = 0; k < count; ++k) {
+    if (ta[k].numel % S::EPT != 0) {
+      k_dequantize_tail4<FMT, BF16OUT><<<1, 32, 0, stream>>>(ta[k].packed, ta[k].scales,
+                                                              nitems[k] * S::EPT, ta[k].g_bits,
+                                                              ta[k].y);
+      ++*launches;
+    }
   }
   return cudaGetLastError();
 }
 
 template <int FMT, bool BF16OUT>
-static cudaError_t dq_block(int block, const uint8_t* p, const uint8_t* s, int64_t numel,
-                            uint16_t g, void* y, cudaStream_t st, int* n) {
+static cudaError_t dq_block(int block, const TensorArgs* t, int count, cudaStream_t st, int* n) {
   switch (block) {
-    case 4: return launch_dq<4, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    case 8: return launch_dq<8, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    case 16: return launch_dq<16, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    case 32: return launch_dq<32, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    case 64: return launch_dq<64, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    case 128: return launch_dq<128, FMT, BF16OUT>(p, s, numel, g, y, st, n);
-    default: return launch_dq<256, FMT, BF16OUT>(p, s, numel, g, y, st, n);
+    case 4: return launch_dq<4, FMT, BF16OUT>(t, count, st, n);
+    case 8: return launch_dq<8, FMT, BF16OUT>(t, count, st, n);
+    case 16: return launch_dq<16, FMT, BF16OUT>(t, count, st, n);
+    case 32: return launch_dq<32, FMT, BF16OUT>(t, count, st, n);
+    case 64: return launch_dq<64, FMT, BF16OUT>(t, count, st, n);
+    case 128: return launch_dq<128, FMT, BF16OUT>(t, count, st, n);
+    default: return launch_dq<256, FMT, BF16OUT>(t, count, st, n);
   }
+}
+
+cudaError_t run_dequantize_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                                 cudaStream_t stream, int* launches) {
+  if (fmt == kUE5M3)
+    return bf16 ? dq_block<kUE5M3, true>(block, t, count, stream, launches)
+                : dq_block<kUE5M3, false>(block, t, count, stream, launches);
+  return bf16 ? dq_block<kE4M3, true>(block, t, count, stream, launches)
+              : dq_block<kE4M3, false>(block, t, count, stream, launches);
 }
 
 cudaError_t run_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t numel, int block,
                            int fmt, uint16_t g_bits, void* y, bool bf16, cudaStream_t stream,
                            int* launches) {
-  if (fmt == kUE5M3)
-    return bf16 ? dq_block<kUE5M3, true>(block, packed, scales, numel, g_bits, y, stream, launches)
-                : dq_block<kUE5M3, false>(block, packed, scales, numel, g_bits, y, stream, launches);
-  return bf16 ? dq_block<kE4M3, true>(block, packed, scales, numel, g_bits, y, stream, launches)
-              : dq_block<kE4M3, false>(block, packed, scales, numel, g_bits, y, stream, launches);
+  const TensorArgs t = {nullptr, y, const_cast<uint8_t*>(packed), const_cast<uint8_t*>(scales),
+                        nullptr, numel, g_bits};
+  return run_dequantize_group(&t, 1, bf16, block, fmt, stream, launches);
 }
 
 }  // namespace mxk

@@ -24,8 +24,6 @@
 // Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
 // in a fixed order, so results are deterministic for a given device and grid; with an N = 4 tail a
 // separate one-CTA pass does it.  No CTA waits on another.
-#include <functional>
-
 #include "mx_device.cuh"
 #include "mx_launch.h"
 
@@ -78,8 +76,8 @@ __device__ __forceinline__ unsigned long long warp_sum(unsigned long long v) {
   return v;
 }
 
-// CTA-wide reduction of the accumulators into part[blockIdx.x] (fixed order).
-__device__ void write_partial(const Acc& acc, StatsPartial* part) {
+// CTA-wide reduction of the accumulators into *slot (fixed order).
+__device__ void write_partial(const Acc& acc, StatsPartial* slot) {
   __shared__ double sd[3][kThreads / 32];
   __shared__ unsigned long long su[3][kThreads / 32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,34 +96,59 @@ __device__ void write_partial(const Acc& acc, StatsPartial* part) {
       p.sse_elem += sd[0][k]; p.sse_max += sd[1][k]; p.sse_zero += sd[2][k];
       p.n_zero_blocks += su[0][k]; p.n_scale_sat += su[1][k]; p.n_elem_sat += su[2][k];
     }
-    part[blockIdx.x] = p;
+    *slot = p;
   }
 }
 
-struct FinalArgs {
-  unsigned int* counter;  // zeroed before the launch; nullptr: a separate pass adds the partials
+// One tensor of a grouped error-reduction launch, and the grid split among the tensors.
+struct STensor {
+  const void* x;
+  const uint8_t* packed;   // stored codes (kGiven)
+  const uint8_t* scales;
+  uint8_t* packed_out;     // codes written (kStore)
+  uint8_t* scales_out;
+  StatsPartial* part;      // this tensor's CTAs' partials: part[0 .. its CTA count)
+  unsigned int* counter;   // last-CTA counter, zeroed before the launch; nullptr: a separate pass
+                           // adds the partials (N = 4 tail)
   StatsOut* out;
-  int64_t numel, nblocks;
+  int64_t nitems, numel, nblocks;
+  uint32_t g_bits;
+};
+struct SGroup {
+  STensor t[kMaxGroup];
+  CtaSplit split;
 };
 
-__device__ void final_reduce(const StatsPartial* part, int nparts, int64_t numel, int64_t nblocks,
-                             StatsOut* out);
+// This CTA's tensor, its index among the tensor's CTAs and their number.
+struct SWork {
+  STensor t;
+  int cta, nctas;
+};
+__device__ __forceinline__ SWork s_work(const SGroup& grp) {
+  const int ti = grp.split.find((int)blockIdx.x);
+  return {grp.t[ti], (int)blockIdx.x - grp.split.begin[ti],
+          grp.split.begin[ti + 1] - grp.split.begin[ti]};
+}
 
-// Writes this CTA's partial; the CTA that finishes last (counted with one atomic per CTA after a
-// fence) then adds all partials in a fixed order and resets the counter.  No CTA waits for another.
-__device__ void finish_cta(const Acc& acc, StatsPartial* part, const FinalArgs& fa) {
-  write_partial(acc, part);
-  if (fa.counter == nullptr) return;
+__device__ void final_reduce(const StatsPartial* part, int nparts, const StatsPartial* extra,
+                             int64_t numel, int64_t nblocks, StatsOut* out);
+
+// Writes this CTA's partial; the tensor's CTA that finishes last (counted with one atomic per CTA
+// after a fence) then adds the tensor's partials in a fixed order and resets the counter.  No CTA
+// waits for another.
+__device__ void finish_cta(const Acc& acc, const SWork& wk) {
+  write_partial(acc, wk.t.part + wk.cta);
+  if (wk.t.counter == nullptr) return;
   __shared__ unsigned int s_last;
   if (threadIdx.x == 0) {
     __threadfence();
-    s_last = atomicAdd(fa.counter, 1u) == gridDim.x - 1;
+    s_last = atomicAdd(wk.t.counter, 1u) == (unsigned)wk.nctas - 1u;
   }
   __syncthreads();
   if (s_last) {
     __threadfence();
-    final_reduce(part, gridDim.x, fa.numel, fa.nblocks, fa.out);
-    if (threadIdx.x == 0) *fa.counter = 0;
+    final_reduce(wk.t.part, wk.nctas, nullptr, wk.t.numel, wk.t.nblocks, wk.t.out);
+    if (threadIdx.x == 0) *wk.t.counter = 0;
   }
 }
 
@@ -417,10 +440,9 @@ __device__ __forceinline__ void block_slice(Acc& acc, int lane, bool ok, float a
 // bf16 input
 // ------------------------------------------------------------------------------------------------
 
-// What the bf16 pass does with the codes: read them (kGiven), recompute them in registers with the
-// quantize kernel's rule (kRecompute), or recompute and also write them to packed_out / scales_out
-// (kStore: the fused quantize + pack + reduction pass).
-enum { kGiven = 0, kRecompute = 1, kStore = 2 };
+// What the bf16 pass does with the codes (StatsMode): read them (kGiven), recompute them in
+// registers with the quantize kernel's rule (kRecompute), or recompute and also write them to
+// packed_out / scales_out (kStore: the fused quantize + pack + reduction pass).
 
 // One thread's item: EPT consecutive elements (NW words), their code words and scale bytes.
 template <int NW, int NCW>
@@ -432,10 +454,15 @@ struct StatsItem {
 
 template <int N, int FMT, int MODE>
 __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
-    const uint16_t* __restrict__ x, int64_t nitems, uint16_t g_bits,
-    const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part, FinalArgs fa, uint8_t* __restrict__ packed_out,
-    uint8_t* __restrict__ scales_out) {
+    const __grid_constant__ SGroup grp) {
+  const SWork wk = s_work(grp);
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
+  const uint8_t* __restrict__ packed = wk.t.packed;
+  const uint8_t* __restrict__ scales = wk.t.scales;
+  uint8_t* __restrict__ packed_out = wk.t.packed_out;
+  uint8_t* __restrict__ scales_out = wk.t.scales_out;
+  const int64_t nitems = wk.t.nitems;
+  const uint16_t g_bits = (uint16_t)wk.t.g_bits;
   constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
   // Recomputed codes: the max-valued elements' error in closed form per block (blocks of 16 and
   // more), or summed like the others (small blocks, where the per-block work would cost more).
@@ -460,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
   griddep_launch_next();
 
   Acc acc;
-  const int64_t T = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t T = (int64_t)wk.nctas * blockDim.x;
+  const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = tid - lane;
 
@@ -608,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
     process(B, i);
     i += T;
   }
-  finish_cta(acc, part, fa);
+  finish_cta(acc, wk);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -616,10 +643,13 @@ __global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
 // ------------------------------------------------------------------------------------------------
 
 template <int N, int FMT, bool RECOMPUTE>
-__global__ void __launch_bounds__(kThreads) k_error_stats_f32(
-    const float* __restrict__ x, int64_t nitems, uint16_t g_bits,
-    const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-    StatsPartial* __restrict__ part, FinalArgs fa) {
+__global__ void __launch_bounds__(kThreads) k_error_stats_f32(const __grid_constant__ SGroup grp) {
+  const SWork wk = s_work(grp);
+  const float* __restrict__ x = static_cast<const float*>(wk.t.x);
+  const uint8_t* __restrict__ packed = wk.t.packed;
+  const uint8_t* __restrict__ scales = wk.t.scales;
+  const int64_t nitems = wk.t.nitems;
+  const uint16_t g_bits = (uint16_t)wk.t.g_bits;
   using S = SShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI;
   constexpr int BE = EPT / BPI;
@@ -633,8 +663,8 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
   griddep_launch_next();
 
   Acc acc;
-  const int64_t T = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t T = (int64_t)wk.nctas * blockDim.x;
+  const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
   const int64_t warp0 = tid - (threadIdx.x & 31);
   const int lane = threadIdx.x & 31;
 
@@ -686,7 +716,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(
       block_slice<BE, L>(acc, lane, ok, a, D, sat_thr, __uint_as_float(mn), xval, code);
     }
   }
-  finish_cta(acc, part, fa);
+  finish_cta(acc, wk);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -737,13 +767,15 @@ __global__ void k_error_stats_tail4(const T* __restrict__ x, int64_t first, uint
 
 // Adds nparts partials in a fixed order (thread t takes t, t + 256, ...; then warps, then the 8
 // warp sums in order) and writes the result record.  Run by all threads of one CTA.
-__device__ void final_reduce(const StatsPartial* part, int nparts, int64_t numel, int64_t nblocks,
-                             StatsOut* out) {
+__device__ void final_reduce(const StatsPartial* part, int nparts, const StatsPartial* extra,
+                             int64_t numel, int64_t nblocks, StatsOut* out) {
   double e = 0.0, m = 0.0, z = 0.0;
   unsigned long long c0 = 0, c1 = 0, c2 = 0;
-  for (int k = threadIdx.x; k < nparts; k += blockDim.x) {
-    const double* pd = reinterpret_cast<const double*>(part + k);
-    const unsigned long long* pu = reinterpret_cast<const unsigned long long*>(part + k);
+  const int n = nparts + (extra != nullptr);
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const StatsPartial* src = k < nparts ? part + k : extra;
+    const double* pd = reinterpret_cast<const double*>(src);
+    const unsigned long long* pu = reinterpret_cast<const unsigned long long*>(src);
     e += __ldcg(pd + 0); m += __ldcg(pd + 1); z += __ldcg(pd + 2);
     c0 += __ldcg(pu + 4); c1 += __ldcg(pu + 5); c2 += __ldcg(pu + 6);
   }
@@ -771,188 +803,167 @@ __device__ void final_reduce(const StatsPartial* part, int nparts, int64_t numel
 }
 
 __global__ void __launch_bounds__(kThreads) k_error_stats_final(const StatsPartial* __restrict__ part,
-                                                                int nparts, int64_t numel,
-                                                                int64_t nblocks,
+                                                                int nparts,
+                                                                const StatsPartial* extra,
+                                                                int64_t numel, int64_t nblocks,
                                                                 StatsOut* __restrict__ out) {
-  final_reduce(part, nparts, numel, nblocks, out);
+  final_reduce(part, nparts, extra, numel, nblocks, out);
 }
 
 // ------------------------------------------------------------------------------------------------
 // launcher
 // ------------------------------------------------------------------------------------------------
 
-// Workspace layout: a 64-byte header (the last-CTA counter) and then one 64-byte partial per CTA.
+// Workspace layout: kMaxGroup 64-byte headers (the last-CTA counter of tensor t of a group in
+// header t), then 64-byte partials: the main pass's CTAs in grid order, then one slot per tensor
+// for an N = 4 tail.
 struct Workspace {
-  unsigned int* counter;
+  unsigned int* counters;
   StatsPartial* part;
   explicit Workspace(void* ws)
-      : counter(reinterpret_cast<unsigned int*>(ws)),
-        part(reinterpret_cast<StatsPartial*>(reinterpret_cast<char*>(ws) + 64)) {}
+      : counters(reinterpret_cast<unsigned int*>(ws)),
+        part(reinterpret_cast<StatsPartial*>(reinterpret_cast<char*>(ws) + 64 * kMaxGroup)) {}
+  unsigned int* counter(int t) const { return counters + 16 * t; }
 };
-constexpr int kMaxStatsGrid = kMaxReduceCtas - 2;  // header + one slot for the N = 4 tail
+constexpr int kMaxStatsGrid = kMaxReduceCtas - 2 * kMaxGroup;  // headers + tail slots
 
-// Zeroes the last-CTA counter once the previous kernel in the stream is done with it (launched
-// with programmatic serialization, so its launch overlaps that kernel's tail and the main pass's
-// launch overlaps it).
-__global__ void k_stats_reset(unsigned int* counter) {
+// Zeroes the last-CTA counters of a group once the previous kernel in the stream is done with
+// them (launched with programmatic serialization, so its launch overlaps that kernel's tail and
+// the main pass's launch overlaps it).
+__global__ void k_stats_reset(unsigned int* counters, int n) {
   griddep_wait();
-  if (threadIdx.x == 0) *counter = 0;
+  if ((int)threadIdx.x < n) counters[16 * threadIdx.x] = 0;
   griddep_launch_next();
 }
 
-// Main pass, then (N = 4 tail) the tail partial and a one-CTA final pass, or (empty) the final
-// pass alone.  Without a tail the main pass adds the partials itself.
-template <typename Launch>
-static cudaError_t stats_passes(int64_t nitems, bool tail, int64_t numel, int block, void* out,
-                                Workspace ws, cudaStream_t stream, int* launches, Launch main,
-                                const std::function<void(StatsPartial*)>& tail_pass) {
-  int nparts = 0;
-  if (nitems > 0) {
-    FinalArgs fa{nullptr, (StatsOut*)out, numel, numel / block};
-    if (!tail) {
-      const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, ws.counter);
+// Main pass over the group; then, for each tensor the main pass does not finish, its N = 4 tail
+// (4 elements after the last full item) and a one-CTA final pass, or (no items) the final pass
+// alone.  Without a tail the main pass adds a tensor's partials itself.
+template <int N, int FMT, typename T, int MODE>
+static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Workspace ws,
+                                cudaStream_t stream, int* launches) {
+  using S = SShape<N, T>;
+  constexpr bool RC = MODE != kGiven;
+  SGroup grp = {};
+  int64_t nitems[kMaxGroup];
+  bool tail[kMaxGroup];
+  for (int k = 0; k < count; ++k) {
+    nitems[k] = ta[k].numel / S::EPT;
+    tail[k] = ta[k].numel % S::EPT != 0;
+  }
+  const void* kern = (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, MODE>
+                                      : (const void*)k_error_stats_f32<N, FMT, RC>;
+  const int grid = split_grid(kern, nitems, count, S::U, kMaxStatsGrid, &grp.split);
+  bool any_counter = false;
+  for (int k = 0; k < count; ++k) {
+    const bool counted = !tail[k] && nitems[k] > 0;
+    any_counter |= counted;
+    grp.t[k] = {ta[k].x,
+                MODE == kGiven ? ta[k].packed : nullptr,
+                MODE == kGiven ? ta[k].scales : nullptr,
+                MODE == kStore ? ta[k].packed : nullptr,
+                MODE == kStore ? ta[k].scales : nullptr,
+                ws.part + grp.split.begin[k],
+                counted ? ws.counter(k) : nullptr,
+                (StatsOut*)ta[k].stats,
+                nitems[k],
+                ta[k].numel,
+                ta[k].numel / block,
+                ta[k].g_bits};
+  }
+  if (grid > 0) {
+    if (any_counter) {
+      const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, ws.counters, count);
       if (e != cudaSuccess) return e;
       ++*launches;
-      fa.counter = ws.counter;
     }
-    nparts = main(fa);
+    const cudaError_t e = (sizeof(T) == 2)
+                              ? launch_pdl(k_error_stats_bf16<N, FMT, MODE>, grid, kThreads,
+                                           stream, grp)
+                              : launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream,
+                                           grp);
+    if (e != cudaSuccess) return e;
     ++*launches;
-    if (!tail) return cudaGetLastError();
   }
-  if (tail) {
-    tail_pass(ws.part + nparts);
-    ++nparts;
+  for (int k = 0; k < count; ++k) {
+    if (!tail[k] && nitems[k] > 0) continue;
+    StatsPartial* extra = nullptr;
+    if (tail[k]) {
+      extra = ws.part + grid + k;
+      const int64_t first = nitems[k] * S::EPT;
+      if (MODE == kStore) {  // quantize the last 4 elements, then reduce them from the codes
+        const cudaError_t e = run_quantize_tail4(ta[k].x, sizeof(T) == 2, first, FMT,
+                                                 ta[k].g_bits, ta[k].packed, ta[k].scales, stream,
+                                                 launches);
+        if (e != cudaSuccess) return e;
+      }
+      k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>(
+          (const T*)ta[k].x, first, ta[k].g_bits, MODE == kRecompute ? nullptr : ta[k].packed,
+          ta[k].scales, extra);
+      ++*launches;
+    }
+    const int nparts = nitems[k] > 0 ? grp.split.begin[k + 1] - grp.split.begin[k] : 0;
+    k_error_stats_final<<<1, kThreads, 0, stream>>>(ws.part + grp.split.begin[k], nparts, extra,
+                                                    ta[k].numel, ta[k].numel / block,
+                                                    (StatsOut*)ta[k].stats);
+    ++*launches;
   }
-  k_error_stats_final<<<1, kThreads, 0, stream>>>(ws.part, nparts, numel, numel / block,
-                                                  (StatsOut*)out);
-  ++*launches;
   return cudaGetLastError();
 }
 
-template <int N, int FMT, typename T, bool RC>
-static cudaError_t launch_st(const void* x, int64_t numel, int block, uint16_t g_bits,
-                             const uint8_t* packed, const uint8_t* scales, void* out, Workspace ws,
-                             cudaStream_t stream, int* launches) {
-  using S = SShape<N, T>;
-  const int64_t nitems = numel / S::EPT;
-  auto main = [&](FinalArgs fa) {
-    const void* kern = (sizeof(T) == 2)
-                           ? (const void*)k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>
-                           : (const void*)k_error_stats_f32<N, FMT, RC>;
-    const int grid = persistent_grid(kern, nitems, S::U, kMaxStatsGrid);
-    if (sizeof(T) == 2)
-      launch_pdl(k_error_stats_bf16<N, FMT, RC ? kRecompute : kGiven>, grid, kThreads, stream,
-                 (const uint16_t*)x, nitems, g_bits, packed, scales, ws.part, fa,
-                 (uint8_t*)nullptr, (uint8_t*)nullptr);
-    else
-      launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream, (const float*)x, nitems,
-                 g_bits, packed, scales, ws.part, fa);
-    return grid;
-  };
-  auto tail = [&](StatsPartial* slot) {
-    k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits,
-                                                      RC ? nullptr : packed, scales, slot);
-    ++*launches;
-  };
-  return stats_passes(nitems, numel % S::EPT != 0, numel, block, out, ws, stream, launches, main,
-                      tail);
-}
-
-template <int FMT, typename T, bool RC>
-static cudaError_t st_block(int block, const void* x, int64_t numel, uint16_t g,
-                            const uint8_t* p, const uint8_t* s, void* out, Workspace part,
-                            cudaStream_t st, int* n) {
+template <int FMT, typename T, int MODE>
+static cudaError_t stats_block(int block, const TensorArgs* t, int count, Workspace ws,
+                               cudaStream_t st, int* n) {
   switch (block) {
-    case 4: return launch_st<4, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    case 8: return launch_st<8, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    case 16: return launch_st<16, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    case 32: return launch_st<32, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    case 64: return launch_st<64, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    case 128: return launch_st<128, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
-    default: return launch_st<256, FMT, T, RC>(x, numel, block, g, p, s, out, part, st, n);
+    case 4: return launch_stats<4, FMT, T, MODE>(t, count, block, ws, st, n);
+    case 8: return launch_stats<8, FMT, T, MODE>(t, count, block, ws, st, n);
+    case 16: return launch_stats<16, FMT, T, MODE>(t, count, block, ws, st, n);
+    case 32: return launch_stats<32, FMT, T, MODE>(t, count, block, ws, st, n);
+    case 64: return launch_stats<64, FMT, T, MODE>(t, count, block, ws, st, n);
+    case 128: return launch_stats<128, FMT, T, MODE>(t, count, block, ws, st, n);
+    default: return launch_stats<256, FMT, T, MODE>(t, count, block, ws, st, n);
   }
 }
 
 template <int FMT, typename T>
-static cudaError_t st_rc(bool rc, int block, const void* x, int64_t numel, uint16_t g,
-                         const uint8_t* p, const uint8_t* s, void* out, Workspace part,
-                         cudaStream_t st, int* n) {
-  return rc ? st_block<FMT, T, true>(block, x, numel, g, p, s, out, part, st, n)
-            : st_block<FMT, T, false>(block, x, numel, g, p, s, out, part, st, n);
-}
-
-// ------------------------------------------------------------------------------------------------
-// fused quantize + pack + error reduction (bf16 input): one pass over x
-// ------------------------------------------------------------------------------------------------
-
-template <int N, int FMT>
-static cudaError_t launch_qs(const uint16_t* x, int64_t numel, int block, uint16_t g_bits,
-                             uint8_t* packed, uint8_t* scales, void* out, Workspace ws,
-                             cudaStream_t stream, int* launches) {
-  using S = SShape<N, uint16_t>;
-  const int64_t nitems = numel / S::EPT;
-  auto main = [&](FinalArgs fa) {
-    const int grid = persistent_grid((const void*)k_error_stats_bf16<N, FMT, kStore>, nitems,
-                                     S::U, kMaxStatsGrid);
-    launch_pdl(k_error_stats_bf16<N, FMT, kStore>, grid, kThreads, stream, x, nitems, g_bits,
-               (const uint8_t*)nullptr, (const uint8_t*)nullptr, ws.part, fa, packed, scales);
-    return grid;
-  };
-  // N = 4 with 4 elements left: quantize them, then reduce them from the stored codes
-  auto tail = [&](StatsPartial* slot) {
-    run_quantize_tail4(x, true, nitems * S::EPT, FMT, g_bits, packed, scales, stream, launches);
-    k_error_stats_tail4<FMT, uint16_t><<<1, 32, 0, stream>>>(x, nitems * S::EPT, g_bits, packed,
-                                                             scales, slot);
-    ++*launches;
-  };
-  return stats_passes(nitems, numel % S::EPT != 0, numel, block, out, ws, stream, launches, main,
-                      tail);
-}
-
-template <int FMT>
-static cudaError_t qs_block(int block, const uint16_t* x, int64_t numel, uint16_t g, uint8_t* p,
-                            uint8_t* s, void* out, Workspace part, cudaStream_t st, int* n) {
-  switch (block) {
-    case 4: return launch_qs<4, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    case 8: return launch_qs<8, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    case 16: return launch_qs<16, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    case 32: return launch_qs<32, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    case 64: return launch_qs<64, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    case 128: return launch_qs<128, FMT>(x, numel, block, g, p, s, out, part, st, n);
-    default: return launch_qs<256, FMT>(x, numel, block, g, p, s, out, part, st, n);
+static cudaError_t stats_mode(StatsMode mode, int block, const TensorArgs* t, int count,
+                              Workspace ws, cudaStream_t st, int* n) {
+  switch (mode) {
+    case kGiven: return stats_block<FMT, T, kGiven>(block, t, count, ws, st, n);
+    case kRecompute: return stats_block<FMT, T, kRecompute>(block, t, count, ws, st, n);
+    default: return stats_block<FMT, T, kStore>(block, t, count, ws, st, n);
   }
+}
+
+cudaError_t run_stats_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                            StatsMode mode, void* workspace, cudaStream_t stream, int* launches) {
+  const Workspace ws(workspace);
+  if (!bf16 && mode == kStore) {  // fp32 input: quantize, then reduce from the stored codes
+    const cudaError_t e = run_quantize_group(t, count, false, block, fmt, stream, launches);
+    if (e != cudaSuccess) return e;
+    mode = kGiven;
+  }
+  if (bf16)
+    return fmt == kUE5M3 ? stats_mode<kUE5M3, uint16_t>(mode, block, t, count, ws, stream, launches)
+                         : stats_mode<kE4M3, uint16_t>(mode, block, t, count, ws, stream, launches);
+  return fmt == kUE5M3 ? stats_mode<kUE5M3, float>(mode, block, t, count, ws, stream, launches)
+                       : stats_mode<kE4M3, float>(mode, block, t, count, ws, stream, launches);
 }
 
 cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                                uint16_t g_bits, uint8_t* packed, uint8_t* scales, void* out,
                                void* workspace, cudaStream_t stream, int* launches) {
-  const Workspace part(workspace);
-  if (!bf16) {  // fp32 input: quantize, then reduce from the stored codes
-    cudaError_t e = run_quantize(x, false, numel, block, fmt, g_bits, packed, scales, stream,
-                                 launches);
-    if (e != cudaSuccess) return e;
-    return run_error_stats(x, false, numel, block, fmt, g_bits, packed, scales, out, workspace,
-                           stream, launches);
-  }
-  const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
-  return fmt == kUE5M3 ? qs_block<kUE5M3>(block, xb, numel, g_bits, packed, scales, out, part,
-                                          stream, launches)
-                       : qs_block<kE4M3>(block, xb, numel, g_bits, packed, scales, out, part,
-                                         stream, launches);
+  const TensorArgs t = {x, nullptr, packed, scales, out, numel, g_bits};
+  return run_stats_group(&t, 1, bf16, block, fmt, kStore, workspace, stream, launches);
 }
 
 cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                             uint16_t g_bits, const uint8_t* packed, const uint8_t* scales,
                             void* out, void* workspace, cudaStream_t stream, int* launches) {
-  const Workspace part(workspace);
-  const bool rc = packed == nullptr;
-  if (bf16)
-    return fmt == kUE5M3
-               ? st_rc<kUE5M3, uint16_t>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches)
-               : st_rc<kE4M3, uint16_t>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches);
-  return fmt == kUE5M3
-             ? st_rc<kUE5M3, float>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches)
-             : st_rc<kE4M3, float>(rc, block, x, numel, g_bits, packed, scales, out, part, stream, launches);
+  const TensorArgs t = {x, nullptr, const_cast<uint8_t*>(packed), const_cast<uint8_t*>(scales),
+                        out, numel, g_bits};
+  return run_stats_group(&t, 1, bf16, block, fmt, packed ? kGiven : kRecompute, workspace, stream,
+                         launches);
 }
 
 }  // namespace mxk

@@ -9,20 +9,84 @@ namespace mxk {
 // Upper bound on the CTAs of any reduction kernel; sizes the workspaces.
 constexpr int kMaxReduceCtas = 4096;
 
-// Persistent grid for a grid-stride kernel with kThreads threads: enough CTAs to fill every SM
-// at the kernel's occupancy, never more than the work needs (items / (threads * items_per_iter)).
-inline int persistent_grid(const void* kern, int64_t nitems, int items_per_iter,
-                           int cap = 1 << 30) {
+// Tensors per grouped launch (one persistent grid split among them).
+constexpr int kMaxGroup = 16;
+
+// Static split of a grid among the tensors of a group: CTAs [begin[t], begin[t + 1]) work on
+// tensor t (an empty range for an empty tensor).  Passed by value in the kernel parameters.
+struct CtaSplit {
+  int count;
+  int begin[kMaxGroup + 1];
+#ifdef __CUDACC__
+  // The tensor of CTA `cta` (a linear scan over at most kMaxGroup entries, once per CTA).
+  __device__ __forceinline__ int find(int cta) const {
+    int t = 0;
+    while (t + 1 < count && cta >= begin[t + 1]) ++t;
+    return t;
+  }
+#endif
+};
+
+// Resident CTAs of 256 threads on the whole device for `kern` (SMs x occupancy).
+inline int64_t resident_ctas(const void* kern) {
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
   if (per_sm < 1) per_sm = 1;
-  const int64_t full = (int64_t)sms * per_sm;
+  return (int64_t)sms * per_sm;
+}
+
+// Persistent grid for a grid-stride kernel with kThreads threads: enough CTAs to fill every SM
+// at the kernel's occupancy, never more than the work needs (items / (threads * items_per_iter)).
+inline int persistent_grid(const void* kern, int64_t nitems, int items_per_iter,
+                           int cap = 1 << 30) {
+  const int64_t full = resident_ctas(kern);
   const int64_t need = (nitems + 256LL * items_per_iter - 1) / (256LL * items_per_iter);
   int64_t g = need < full ? need : full;
   if (g > cap) g = cap;
   return (int)(g < 1 ? 1 : g);
+}
+
+// Split one persistent grid among `count` tensors of nitems[t] items: at most the resident CTAs
+// (and `cap`) in total, each tensor with work at least one CTA and at most what its items need,
+// the rest in proportion to the items.  Returns the total grid (0 when there is no work).
+inline int split_grid(const void* kern, const int64_t* nitems, int count, int items_per_iter,
+                      int cap, CtaSplit* split) {
+  int64_t full = resident_ctas(kern);
+  if (full > cap) full = cap;
+  int64_t need[kMaxGroup], total = 0, nonempty = 0;
+  for (int t = 0; t < count; ++t) {
+    need[t] = (nitems[t] + 256LL * items_per_iter - 1) / (256LL * items_per_iter);
+    total += nitems[t];
+    nonempty += nitems[t] > 0;
+  }
+  if (full < nonempty) full = nonempty;
+  int64_t share[kMaxGroup], used = 0;
+  for (int t = 0; t < count; ++t) {
+    share[t] = nitems[t] > 0 ? (int64_t)((double)full * (double)nitems[t] / (double)total) : 0;
+    if (nitems[t] > 0 && share[t] < 1) share[t] = 1;
+    if (share[t] > need[t]) share[t] = need[t];
+    used += share[t];
+  }
+  // hand out what is left, one CTA at a time, to the tensors with the most items per CTA
+  while (used < full) {
+    int best = -1;
+    double best_load = 0.0;
+    for (int t = 0; t < count; ++t) {
+      if (share[t] >= need[t]) continue;
+      const double load = (double)nitems[t] / (double)share[t];
+      if (best < 0 || load > best_load) { best = t; best_load = load; }
+    }
+    if (best < 0) break;
+    ++share[best];
+    ++used;
+  }
+  split->count = count;
+  split->begin[0] = 0;
+  for (int t = 0; t < count; ++t) split->begin[t + 1] = split->begin[t] + (int)share[t];
+  for (int t = count + 1; t <= kMaxGroup; ++t) split->begin[t] = split->begin[count];
+  return split->begin[count];
 }
 
 // Launch with programmatic stream serialization: the kernel may be scheduled while the previous
@@ -45,6 +109,29 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaS
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
+
+// One tensor of a grouped call (all pointers device memory; numel = rows * cols).
+struct TensorArgs {
+  const void* x;      // input of quantize / the error reduction
+  void* y;            // output of dequantize
+  uint8_t* packed;    // codes: written by quantize, read by dequantize / given-code reduction
+  uint8_t* scales;    // scale codes, likewise
+  void* stats;        // device mx_error_stats_t of the error reduction
+  int64_t numel;
+  uint16_t g_bits;
+};
+
+// What the error-reduction pass does with the codes (see mx_error_stats.cu).
+enum StatsMode { kGiven = 0, kRecompute = 1, kStore = 2 };
+
+// Grouped launches: count <= kMaxGroup tensors sharing block size, format and dtype, one
+// persistent grid split among them.
+cudaError_t run_quantize_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                               cudaStream_t stream, int* launches);
+cudaError_t run_dequantize_group(const TensorArgs* t, int count, bool bf16out, int block, int fmt,
+                                 cudaStream_t stream, int* launches);
+cudaError_t run_stats_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                            StatsMode mode, void* workspace, cudaStream_t stream, int* launches);
 
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
                          uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,

@@ -36,6 +36,31 @@ struct QShape {
   static constexpr int U = (sizeof(T) == 2) ? MX_Q_U : 2;                    // items in flight
 };
 
+// Kernel parameters: up to kMaxGroup tensors and the split of the grid among them.  A CTA works
+// on one tensor with a grid stride of its own range of CTAs.
+struct QTensor {
+  const void* x;
+  uint8_t* packed;
+  uint8_t* scales;
+  int64_t nitems;
+  uint32_t g_bits;
+};
+struct QGroup {
+  QTensor t[kMaxGroup];
+  CtaSplit split;
+};
+
+// This CTA's tensor, its index among the tensor's CTAs and their number.
+struct QWork {
+  QTensor t;
+  int cta, nctas;
+};
+__device__ __forceinline__ QWork q_work(const QGroup& grp) {
+  const int ti = grp.split.find((int)blockIdx.x);
+  return {grp.t[ti], (int)blockIdx.x - grp.split.begin[ti],
+          grp.split.begin[ti + 1] - grp.split.begin[ti]};
+}
+
 // ------------------------------------------------------------------------------------------------
 // bf16 input
 // ------------------------------------------------------------------------------------------------
@@ -52,14 +77,16 @@ __device__ __forceinline__ uint32_t absmax_bits(const uint32_t* w) {
 }
 
 template <int N, int FMT>
-__global__ void __launch_bounds__(kThreads) k_quantize_bf16(const uint16_t* __restrict__ x,
-                                                             int64_t nitems, uint16_t g_bits,
-                                                             uint8_t* __restrict__ packed,
-                                                             uint8_t* __restrict__ scales) {
+__global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constant__ QGroup grp) {
   using S = QShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
+  const QWork wk = q_work(grp);
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
+  uint8_t* __restrict__ packed = wk.t.packed;
+  uint8_t* __restrict__ scales = wk.t.scales;
+  const int64_t nitems = wk.t.nitems;
   __shared__ float s_rcp[256];
-  const float g = fp16_bits_to_float(g_bits);
+  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);  // exact (<= 15 significant bits)
     s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;          // zero scale -> every code is +-0
@@ -69,8 +96,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const uint16_t* __re
   griddep_wait();  // inputs may come from the previous kernel in the stream
   griddep_launch_next();
 
-  const int64_t T = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t T = (int64_t)wk.nctas * blockDim.x;
+  const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
   const int64_t warp0 = tid - (threadIdx.x & 31);
   const int lane = threadIdx.x & 31;
 
@@ -138,22 +165,24 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const uint16_t* __re
 // ------------------------------------------------------------------------------------------------
 
 template <int N, int FMT>
-__global__ void __launch_bounds__(kThreads) k_quantize_f32(const float* __restrict__ x,
-                                                            int64_t nitems, uint16_t g_bits,
-                                                            uint8_t* __restrict__ packed,
-                                                            uint8_t* __restrict__ scales) {
+__global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant__ QGroup grp) {
   using S = QShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U;
+  const QWork wk = q_work(grp);
+  const float* __restrict__ x = static_cast<const float*>(wk.t.x);
+  uint8_t* __restrict__ packed = wk.t.packed;
+  uint8_t* __restrict__ scales = wk.t.scales;
+  const int64_t nitems = wk.t.nitems;
   __shared__ float s_D[256];
-  const float g = fp16_bits_to_float(g_bits);
+  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   const float g6 = __fmul_rn(6.0f, g);
   __syncthreads();
   griddep_wait();  // inputs may come from the previous kernel in the stream
   griddep_launch_next();
 
-  const int64_t T = (int64_t)gridDim.x * blockDim.x;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t T = (int64_t)wk.nctas * blockDim.x;
+  const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
   const int64_t warp0 = tid - (threadIdx.x & 31);
   const int lane = threadIdx.x & 31;
 
@@ -241,41 +270,44 @@ __global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_
 // ------------------------------------------------------------------------------------------------
 
 template <int N, int FMT, typename T>
-static cudaError_t launch_q(const void* x, int64_t numel, uint16_t g_bits, uint8_t* packed,
-                            uint8_t* scales, cudaStream_t stream, int* launches) {
+static cudaError_t launch_q(const TensorArgs* ta, int count, cudaStream_t stream, int* launches) {
   using S = QShape<N, T>;
-  const int64_t nitems = numel / S::EPT;
-  if (nitems > 0) {
-    auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT> : (void*)k_quantize_f32<N, FMT>;
-    const int grid = persistent_grid(kern, nitems, S::U);
-    const cudaError_t e =
-        (sizeof(T) == 2)
-            ? launch_pdl(k_quantize_bf16<N, FMT>, grid, kThreads, stream, (const uint16_t*)x,
-                         nitems, g_bits, packed, scales)
-            : launch_pdl(k_quantize_f32<N, FMT>, grid, kThreads, stream, (const float*)x, nitems,
-                         g_bits, packed, scales);
+  QGroup grp = {};
+  int64_t nitems[kMaxGroup];
+  for (int k = 0; k < count; ++k) {
+    nitems[k] = ta[k].numel / S::EPT;
+    grp.t[k] = {ta[k].x, ta[k].packed, ta[k].scales, nitems[k], ta[k].g_bits};
+  }
+  auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT> : (void*)k_quantize_f32<N, FMT>;
+  const int grid = split_grid(kern, nitems, count, S::U, 1 << 30, &grp.split);
+  if (grid > 0) {
+    const cudaError_t e = (sizeof(T) == 2)
+                              ? launch_pdl(k_quantize_bf16<N, FMT>, grid, kThreads, stream, grp)
+                              : launch_pdl(k_quantize_f32<N, FMT>, grid, kThreads, stream, grp);
     if (e != cudaSuccess) return e;
     ++*launches;
   }
-  if (numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
-    k_quantize_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)x, nitems * S::EPT, g_bits, packed,
-                                                   scales);
-    ++*launches;
+  for (int k = 0; k < count; ++k) {
+    if (ta[k].numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
+      k_quantize_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)ta[k].x, nitems[k] * S::EPT,
+                                                     ta[k].g_bits, ta[k].packed, ta[k].scales);
+      ++*launches;
+    }
   }
   return cudaGetLastError();
 }
 
 template <int FMT, typename T>
-static cudaError_t dispatch_block(int block, const void* x, int64_t numel, uint16_t g,
-                                  uint8_t* p, uint8_t* s, cudaStream_t st, int* n) {
+static cudaError_t dispatch_block(int block, const TensorArgs* t, int count, cudaStream_t st,
+                                  int* n) {
   switch (block) {
-    case 4: return launch_q<4, FMT, T>(x, numel, g, p, s, st, n);
-    case 8: return launch_q<8, FMT, T>(x, numel, g, p, s, st, n);
-    case 16: return launch_q<16, FMT, T>(x, numel, g, p, s, st, n);
-    case 32: return launch_q<32, FMT, T>(x, numel, g, p, s, st, n);
-    case 64: return launch_q<64, FMT, T>(x, numel, g, p, s, st, n);
-    case 128: return launch_q<128, FMT, T>(x, numel, g, p, s, st, n);
-    default: return launch_q<256, FMT, T>(x, numel, g, p, s, st, n);
+    case 4: return launch_q<4, FMT, T>(t, count, st, n);
+    case 8: return launch_q<8, FMT, T>(t, count, st, n);
+    case 16: return launch_q<16, FMT, T>(t, count, st, n);
+    case 32: return launch_q<32, FMT, T>(t, count, st, n);
+    case 64: return launch_q<64, FMT, T>(t, count, st, n);
+    case 128: return launch_q<128, FMT, T>(t, count, st, n);
+    default: return launch_q<256, FMT, T>(t, count, st, n);
   }
 }
 
@@ -301,16 +333,20 @@ cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt,
   return cudaGetLastError();
 }
 
+cudaError_t run_quantize_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                               cudaStream_t stream, int* launches) {
+  if (bf16)
+    return fmt == kUE5M3 ? dispatch_block<kUE5M3, uint16_t>(block, t, count, stream, launches)
+                         : dispatch_block<kE4M3, uint16_t>(block, t, count, stream, launches);
+  return fmt == kUE5M3 ? dispatch_block<kUE5M3, float>(block, t, count, stream, launches)
+                       : dispatch_block<kE4M3, float>(block, t, count, stream, launches);
+}
+
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
                          uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
                          int* launches) {
-  if (bf16)
-    return fmt == kUE5M3
-               ? dispatch_block<kUE5M3, uint16_t>(block, x, numel, g_bits, packed, scales, stream, launches)
-               : dispatch_block<kE4M3, uint16_t>(block, x, numel, g_bits, packed, scales, stream, launches);
-  return fmt == kUE5M3
-             ? dispatch_block<kUE5M3, float>(block, x, numel, g_bits, packed, scales, stream, launches)
-             : dispatch_block<kE4M3, float>(block, x, numel, g_bits, packed, scales, stream, launches);
+  const TensorArgs t = {x, nullptr, packed, scales, nullptr, numel, g_bits};
+  return run_quantize_group(&t, 1, bf16, block, fmt, stream, launches);
 }
 
 }  // namespace mxk

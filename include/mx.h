@@ -152,6 +152,42 @@ MX_API mx_status mx_error_stats_noalloc(const void* x, mx_dtype xt, int64_t rows
                                         const uint8_t* packed, const uint8_t* scales,
                                         mx_error_stats_t* out_dev, cudaStream_t stream);
 
+/* ---- Grouped calls (no counterpart in the pages: a launch-level batching of the calls above).
+ * Up to MX_MAX_GROUP tensors that share dtype, block size and scale format are processed by one
+ * persistent kernel launch whose grid is split among them (in proportion to their sizes), instead
+ * of one launch per tensor -- for example every weight matrix of a transformer layer.  Results are
+ * those of the per-tensor calls, tensor by tensor (the error sums up to the order of the
+ * additions).  The descriptor array is host memory, read during the call only.  Arguments are
+ * checked for every tensor before anything is enqueued; count outside [1, MX_MAX_GROUP] gives
+ * MX_ERR_INVALID_ARG. */
+#define MX_MAX_GROUP 16
+
+/* One tensor of a grouped call: rows x cols, row-major, cols % block == 0. */
+typedef struct {
+  const void* x;              /* input of mx_quantize_group / mx_quantize_stats_group */
+  void* y;                    /* output of mx_dequantize_group */
+  uint8_t* packed;            /* rows*cols/2 codes: written by quantize, read by dequantize */
+  uint8_t* scales;            /* rows*cols/block scale codes, likewise */
+  mx_error_stats_t* stats;    /* mx_quantize_stats_group: this tensor's record (device) */
+  int64_t rows, cols;
+  uint16_t global_scale_fp16; /* per-tensor g, as in mx_quantize */
+  uint16_t reserved[3];       /* must be zero */
+} mx_tensor_t;
+
+/* mx_quantize of every tensor (x -> packed, scales). */
+MX_API mx_status mx_quantize_group(const mx_tensor_t* tensors, int count, mx_dtype xt, int block,
+                                   mx_scale_fmt fmt, cudaStream_t stream);
+
+/* mx_dequantize of every tensor (packed, scales -> y of type yt). */
+MX_API mx_status mx_dequantize_group(const mx_tensor_t* tensors, int count, int block,
+                                     mx_scale_fmt fmt, mx_dtype yt, cudaStream_t stream);
+
+/* mx_quantize_stats of every tensor (x -> packed, scales, stats) with one workspace of
+ * mx_error_stats_workspace_size() bytes for the whole group. */
+MX_API mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtype xt,
+                                         int block, mx_scale_fmt fmt, void* workspace,
+                                         size_t ws_bytes, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 MX_API const char* mx_status_string(mx_status status);
 

@@ -136,3 +136,41 @@ def test_python_binding_marshalling_errors():
     with pytest.raises(ValueError):
         mx.fmt_code("e5m2")
     assert mx.g_bits(None) == 0x3C00 and mx.g_bits(1.0) == 0x3C00 and mx.g_bits(0x1234) == 0x1234
+
+
+def group(n, rows=4, cols=64, x=A, y=A, p=A, s=A, st=A, g=0x3C00, reserved=0):
+    d = (_lib.Tensor * max(n, 1))()
+    for k in range(max(n, 1)):
+        d[k].x, d[k].y, d[k].packed, d[k].scales, d[k].stats = x, y, p, s, st
+        d[k].rows, d[k].cols, d[k].global_scale_fp16 = rows, cols, g
+        d[k].reserved[0] = reserved
+    return d
+
+
+def test_group_calls_reject_bad_arguments():
+    ws = L.mx_error_stats_workspace_size(4, 64, 32)
+    for n in (0, _lib.MX_MAX_GROUP + 1):
+        assert L.mx_quantize_group(group(n), n, BF16, 32, E4, None) == INV
+        assert L.mx_dequantize_group(group(n), n, 32, E4, BF16, None) == INV
+        assert L.mx_quantize_stats_group(group(n), n, BF16, 32, E4, A, ws, None) == INV
+    assert L.mx_quantize_group(None, 1, BF16, 32, E4, None) == INV
+    assert L.mx_quantize_group(group(2), 2, 9, 32, E4, None) == INV           # dtype
+    assert L.mx_quantize_group(group(2), 2, BF16, 12, E4, None) == UNS        # block
+    assert L.mx_quantize_group(group(2, cols=48), 2, BF16, 32, E4, None) == INV
+    assert L.mx_quantize_group(group(2, g=0x7C00), 2, BF16, 32, E4, None) == INV
+    assert L.mx_quantize_group(group(2, reserved=1), 2, BF16, 32, E4, None) == INV
+    assert L.mx_quantize_group(group(2, x=None), 2, BF16, 32, E4, None) == INV
+    assert L.mx_quantize_group(group(2, x=A + 8), 2, BF16, 32, E4, None) == MIS
+    assert L.mx_quantize_group(group(2, s=A + 1), 2, BF16, 32, E4, None) == MIS
+    assert L.mx_dequantize_group(group(2, y=None), 2, 32, E4, BF16, None) == INV
+    assert L.mx_dequantize_group(group(2, y=A + 2), 2, 32, E4, BF16, None) == MIS
+    assert L.mx_dequantize_group(group(2), 2, 32, E4, 7, None) == INV
+    assert L.mx_quantize_stats_group(group(2, st=None), 2, BF16, 32, E4, A, ws, None) == INV
+    assert L.mx_quantize_stats_group(group(2, st=A + 8), 2, BF16, 32, E4, A, ws, None) == MIS
+    assert L.mx_quantize_stats_group(group(2), 2, BF16, 32, E4, None, ws, None) == WS
+    assert L.mx_quantize_stats_group(group(2), 2, BF16, 32, E4, A, ws - 1, None) == WS
+    assert L.mx_quantize_stats_group(group(2), 2, BF16, 32, E4, A + 4, ws, None) == MIS
+    # one bad tensor among good ones rejects the whole call
+    d = group(3)
+    d[2].cols = 40
+    assert L.mx_quantize_group(d, 3, BF16, 32, E4, None) == INV

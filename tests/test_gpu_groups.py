@@ -1,0 +1,85 @@
+"""Grouped calls: one launch over several tensors gives, tensor by tensor, the oracle's codes,
+scales and dequantized bits (bit-exact) and error records (within 1e-5 relative), with tensors of
+different sizes and global scales in one group (an empty tensor, an N = 4 tensor with a 4-element
+tail, and sizes that give a tensor a single CTA among many)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp4_microscaling_tensor_b200 as mx
+from fp4_microscaling_tensor_b200 import inputs
+
+from gpu_helpers import BLOCKS, FMTS, assert_same, assert_stats, bits, u8
+
+pytestmark = pytest.mark.gpu
+
+G_MIX = (0x3C00, 0x3555, 0x0003, 0x5A00, 0x3C00, 0x2E66)
+
+
+def make_group(block, dtype, device, seed):
+    """Tensors of one group: sizes from tiny to a few CTAs' worth, one empty, plus (N = 4) one
+    with rows*cols = 4 mod 8."""
+    rng = np.random.default_rng(seed)
+    shapes = [(3, 8 * block), (64, 4 * block), (1, block), (0, block), (257, 2 * block),
+              (512, 1024)]
+    if block == 4:
+        shapes.append((3, 4))  # 12 elements: one full item of 8 and a 4-element tail
+    xs = []
+    for k, (r, c) in enumerate(shapes):
+        x = rng.standard_normal((r, c)) * np.exp(rng.uniform(-3, 1, (r, 1)))
+        xs.append(torch.from_numpy(x.astype(np.float32)).to(dtype).to(device))
+    return xs
+
+
+def oracle_tensor(x, block, fmt, g):
+    rows, cols = x.shape
+    xo = inputs.to_oracle(x)
+    po, so = oracle.quantize(xo, rows, cols, block, fmt, g)
+    yo = oracle.dequantize(po, so, rows, cols, block, fmt, g,
+                           out_bf16=x.dtype == torch.bfloat16)
+    st = oracle.error_stats(xo, rows, cols, block, fmt, g, packed=po, scales=so)
+    return po, so, yo, st
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_groups_match_oracle(cuda_device, block, fmt, dtype):
+    xs = make_group(block, dtype, cuda_device, seed=block * 7 + fmt)
+    gs = [G_MIX[k % len(G_MIX)] for k in range(len(xs))]
+    p, s = mx.quantize_group(xs, block, fmt, gs)
+    y = mx.dequantize_group(p, s, block, fmt, gs, out_dtype=dtype)
+    p2, s2, st = mx.quantize_with_stats_group(xs, block, fmt, gs)
+    for k, x in enumerate(xs):
+        what = f"group N={block} fmt={fmt} {dtype} tensor {k} {tuple(x.shape)} g={gs[k]:#x}"
+        po, so, yo, sto = oracle_tensor(x, block, fmt, gs[k])
+        assert_same(u8(s[k]), so, what + " scales")
+        assert_same(u8(p[k]), po, what + " packed")
+        assert_same(u8(s2[k]), so, what + " fused scales")
+        assert_same(u8(p2[k]), po, what + " fused packed")
+        ref = yo if dtype == torch.bfloat16 else yo.view(np.uint32)
+        assert_same(bits(y[k]), ref, what + " dequant")
+        assert_stats(st[k].to_dict(), sto, what + " stats")
+
+
+def test_group_of_sixteen_bench_point(cuda_device):
+    """The largest group, 16 tensors of the bench's point shape split among the CTAs."""
+    xs = [inputs.workload2(k % 5, shape=(1024, 4096), device=cuda_device) for k in range(16)]
+    p, s, st = mx.quantize_with_stats_group(xs, 32, mx.E4M3)
+    y = mx.dequantize_group(p, s, 32, mx.E4M3)
+    for k in (0, 7, 15):
+        po, so, yo, sto = oracle_tensor(xs[k], 32, mx.E4M3, 0x3C00)
+        assert_same(u8(p[k]), po, f"tensor {k} packed")
+        assert_same(u8(s[k]), so, f"tensor {k} scales")
+        assert_same(bits(y[k]), yo, f"tensor {k} dequant")
+        assert_stats(st[k].to_dict(), sto, f"tensor {k} stats")
+
+
+def test_group_rejects_mixed_dtypes(cuda_device):
+    a = torch.zeros(4, 64, dtype=torch.bfloat16, device=cuda_device)
+    b = torch.zeros(4, 64, dtype=torch.float32, device=cuda_device)
+    with pytest.raises(ValueError):
+        mx.quantize_group([a, b], 32, mx.E4M3)
+    with pytest.raises(ValueError):
+        mx.quantize_group([a] * (mx.MX_MAX_GROUP + 1), 32, mx.E4M3)
