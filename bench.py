@@ -55,6 +55,7 @@ def parse(argv=None):
     ap.add_argument("--block", type=int, default=32)
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--group", type=int, default=1, help="tensors per grouped launch (--case)")
     return ap.parse_args(argv)
 
 
@@ -259,7 +260,8 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------------------
 
 class Sweep:
-    """Device buffers and the three phases of one sweep step."""
+    """Device buffers and the phases of one sweep step.  The five sigma tensors of one (N, format)
+    point are one grouped launch (14 launches per phase)."""
 
     def __init__(self, xs, device):
         import torch
@@ -275,20 +277,31 @@ class Sweep:
         self.ys = [torch.empty(rows, cols, dtype=torch.bfloat16, device=device) for _ in self.pts]
         self.stats = torch.empty(len(self.pts), 64, dtype=torch.uint8, device=device)
         self.ws = mx.stats_workspace(device)
+        # groups: consecutive points that share (N, format), i.e. the sigma tensors
+        self.groups = []
+        for i, (k, n, fmt) in enumerate(self.pts):
+            if self.groups and self.groups[-1][1:] == (n, fmt):
+                self.groups[-1][0].append(i)
+            else:
+                self.groups.append(([i], n, fmt))
 
     def phase_q(self):
-        for i, (k, n, fmt) in enumerate(self.pts):
-            self.mx.quantize(self.xs[k], n, fmt, packed=self.packed[i], scales=self.scales[i])
+        for idx, n, fmt in self.groups:
+            self.mx.quantize_group([self.xs[self.pts[i][0]] for i in idx], n, fmt,
+                                   packed=[self.packed[i] for i in idx],
+                                   scales=[self.scales[i] for i in idx])
 
     def phase_qs(self):
-        for i, (k, n, fmt) in enumerate(self.pts):
-            self.mx.quantize_with_stats(self.xs[k], n, fmt, packed=self.packed[i],
-                                        scales=self.scales[i], out=self.stats[i],
-                                        workspace=self.ws)
+        for idx, n, fmt in self.groups:
+            self.mx.quantize_with_stats_group(
+                [self.xs[self.pts[i][0]] for i in idx], n, fmt,
+                packed=[self.packed[i] for i in idx], scales=[self.scales[i] for i in idx],
+                out=self.stats[idx[0]:idx[-1] + 1], workspace=self.ws)
 
     def phase_dq(self):
-        for i, (k, n, fmt) in enumerate(self.pts):
-            self.mx.dequantize(self.packed[i], self.scales[i], n, fmt, out=self.ys[i])
+        for idx, n, fmt in self.groups:
+            self.mx.dequantize_group([self.packed[i] for i in idx], [self.scales[i] for i in idx],
+                                     n, fmt, out=[self.ys[i] for i in idx])
 
     def step(self):
         self.phase_qs()
@@ -436,7 +449,8 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "points": len(sw.pts), "elements_per_point": numel,
                    "phases": "quantize+pack+error reduction (fused) all -> dequantize all",
-                   "launch": "one CUDA graph per phase",
+                   "launch": "one CUDA graph per phase; one grouped launch per (N, format) over "
+                             "the 5 sigma tensors (14 per phase)",
                    "l2": "inputs 168 MB > 126 MB L2; sigma innermost, each buffer reused only "
                          "after >= 4 other points (>150 MB) have streamed",
                    "parallelism": f"dp{world} (independent sweeps)"},
@@ -448,7 +462,8 @@ def run_ours(args):
                     "dequantize": elems / per_step[1] / 1e9},
         "roofline": {"bound": "hbm",
                      "kernel": "k_error_stats_bf16<kStore> (fused quantize+pack+error reduction), "
-                               "all 70 points; per launch avg incl. its 4-byte counter reset",
+                               "14 grouped launches of 5 tensors; per launch avg incl. its "
+                               "counter-reset kernel",
                      "achieved": qs_gbs, "peak": peak, "unit": "GB/s", "frac": qs_gbs / peak,
                      "peak_kind": peak_kind + " (burst copy)",
                      "traffic": FUSED_TRAFFIC_BYTES,
@@ -477,34 +492,46 @@ def run_ours(args):
 
 
 def run_case(args):
-    """Time one kernel on one bf16 tensor (N(0, 0.02^2), seed 0): CUDA events around each launch,
-    L2 flushed before each launch by writing a 256 MB buffer; prints one JSON line."""
+    """Time one kernel (or, with --group G, one grouped launch over G tensors) on bf16 tensors
+    N(0, 0.02^2): CUDA events around each launch, L2 flushed before each launch by writing a 256 MB
+    buffer; prints one JSON line."""
     import torch
     import fp4_microscaling_tensor_b200 as mx
     from fp4_microscaling_tensor_b200 import inputs
     dev = torch.device("cuda", 0)
     rows, cols = args.shape
-    n, fmt = args.block, mx.fmt_code(args.fmt)
-    x = inputs.normal((rows, cols), 0.02, 0, device=dev)
-    numel = rows * cols
-    packed, scales = mx.quantize(x, n, fmt)
-    y = torch.empty(rows, cols, dtype=torch.bfloat16, device=dev)
-    out = torch.empty(64, dtype=torch.uint8, device=dev)
+    n, fmt, G = args.block, mx.fmt_code(args.fmt), args.group
+    xs = [inputs.normal((rows, cols), 0.02, k, device=dev) for k in range(G)]
+    numel = rows * cols * G
+    packed, scales = mx.quantize_group(xs, n, fmt)
+    ys = [torch.empty(rows, cols, dtype=torch.bfloat16, device=dev) for _ in range(G)]
+    out = torch.empty(G, 64, dtype=torch.uint8, device=dev)
     ws = mx.stats_workspace(dev)
     flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
-    calls = {
-        "quantize": (lambda: mx.quantize(x, n, fmt, packed=packed, scales=scales),
-                     numel * (2.5 + 1.0 / n)),
-        "dequantize": (lambda: mx.dequantize(packed, scales, n, fmt, out=y), numel * (2.5 + 1.0 / n)),
-        "stats": (lambda: mx.error_stats(x, n, fmt, packed=packed, scales=scales, out=out,
-                                         workspace=ws), numel * (2.5 + 1.0 / n)),
-        "stats-recompute": (lambda: mx.error_stats(x, n, fmt, out=out, workspace=ws), numel * 2.0),
-        "quantize-stats": (lambda: mx.quantize_with_stats(x, n, fmt, packed=packed, scales=scales,
-                                                          out=out, workspace=ws),
-                           numel * (2.5 + 1.0 / n)),
-        "global-scale": (lambda: mx.global_scale(x, fmt), numel * 2.0),
-    }
-    fn, nbytes = calls[args.case]
+    if G == 1:
+        x, p, sc, y = xs[0], packed[0], scales[0], ys[0]
+        calls = {
+            "quantize": lambda: mx.quantize(x, n, fmt, packed=p, scales=sc),
+            "dequantize": lambda: mx.dequantize(p, sc, n, fmt, out=y),
+            "stats": lambda: mx.error_stats(x, n, fmt, packed=p, scales=sc, out=out[0],
+                                            workspace=ws),
+            "stats-recompute": lambda: mx.error_stats(x, n, fmt, out=out[0], workspace=ws),
+            "quantize-stats": lambda: mx.quantize_with_stats(x, n, fmt, packed=p, scales=sc,
+                                                             out=out[0], workspace=ws),
+            "global-scale": lambda: mx.global_scale(x, fmt),
+        }
+    else:
+        calls = {
+            "quantize": lambda: mx.quantize_group(xs, n, fmt, packed=packed, scales=scales),
+            "dequantize": lambda: mx.dequantize_group(packed, scales, n, fmt, out=ys),
+            "quantize-stats": lambda: mx.quantize_with_stats_group(
+                xs, n, fmt, packed=packed, scales=scales, out=out, workspace=ws),
+        }
+        if args.case not in calls:
+            raise SystemExit(f"--group applies to {sorted(calls)}")
+    nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0}.get(
+        args.case, numel * (2.5 + 1.0 / n))
+    fn = calls[args.case]
     fn()
     torch.cuda.synchronize()
     times = []
@@ -518,9 +545,10 @@ def run_case(args):
         times.append(e0.elapsed_time(e1) / 1e3)
     t = statistics.median(times)
     peak, kind = measured_peak()
-    print(json.dumps({"case": args.case, "shape": [rows, cols], "block": n, "fmt": args.fmt,
-                      "median_us": t * 1e6, "gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
-                      "peak": peak, "peak_kind": kind, "reps": args.reps}), flush=True)
+    print(json.dumps({"case": args.case, "shape": [rows, cols], "group": G, "block": n,
+                      "fmt": args.fmt, "median_us": t * 1e6, "gbs": nbytes / t / 1e9,
+                      "frac": nbytes / t / 1e9 / peak, "peak": peak, "peak_kind": kind,
+                      "reps": args.reps}), flush=True)
 
 
 def main():
