@@ -50,7 +50,7 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     # single-kernel timing / profiling case (not the benchmark line)
     ap.add_argument("--case", choices=["quantize", "dequantize", "stats", "stats-recompute",
-                                       "quantize-stats", "global-scale"])
+                                       "quantize-stats", "global-scale", "fake-quantize"])
     ap.add_argument("--shape", type=int, nargs=2, default=[16384, 8192])
     ap.add_argument("--block", type=int, default=32)
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
@@ -519,6 +519,7 @@ def run_case(args):
             "quantize-stats": lambda: mx.quantize_with_stats(x, n, fmt, packed=p, scales=sc,
                                                              out=out[0], workspace=ws),
             "global-scale": lambda: mx.global_scale(x, fmt),
+            "fake-quantize": lambda: mx.fake_quantize(x, n, fmt, out=y),
         }
     else:
         calls = {
@@ -529,7 +530,8 @@ def run_case(args):
         }
         if args.case not in calls:
             raise SystemExit(f"--group applies to {sorted(calls)}")
-    nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0}.get(
+    nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0,
+              "fake-quantize": numel * 4.0}.get(
         args.case, numel * (2.5 + 1.0 / n))
     fn = calls[args.case]
     fn()

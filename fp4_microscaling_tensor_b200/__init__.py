@@ -4,7 +4,8 @@ The CUDA library (libmxfp4_b200.so, C ABI in include/mx.h) does the work: quanti
 dequantize, the three-term block-error reduction and the per-tensor FP16 scale.  This package is a
 thin binding over it; importing it fails when the library is missing.
 """
-from .api import (E4M3, MX_MAX_GROUP, UE5M3, ErrorStats, MXError, dequantize,  # noqa: F401
-                  dequantize_group, error_stats, fmt_code, g_bits, global_scale, kernel_launches,
+from .api import (E4M3, MX_MAX_GROUP, UE5M3, ErrorStats, FakeQuantize, MXError,  # noqa: F401
+                  dequantize, dequantize_group, error_stats, fake_quantize, fmt_code, g_bits,
+                  global_scale, kernel_launches,
                   quantize, quantize_group, quantize_with_stats, quantize_with_stats_group,
                   stats_workspace)

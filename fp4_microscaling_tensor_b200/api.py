@@ -91,6 +91,37 @@ def dequantize(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=torch.bfl
     return out
 
 
+def fake_quantize(x, block=32, fmt="e4m3", g=None, out_dtype=None, out=None, stream=None):
+    """dequantize(quantize(x)) in one pass (x read once, only y written); out_dtype defaults to
+    x's dtype.  No gradient: see FakeQuantize for the autograd version."""
+    rows, cols = _shape2d(x, "x")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    out_dtype = out_dtype or x.dtype
+    if out_dtype not in _DT:
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+    check(lib.mx_fake_quantize(x.data_ptr(), _DT[x.dtype], rows, cols, int(block), fmt_code(fmt),
+                               g_bits(g), out.data_ptr(), _DT[out.dtype],
+                               _stream(stream, x.device)), "mx_fake_quantize")
+    return out
+
+
+class FakeQuantize(torch.autograd.Function):
+    """Quantization-aware training op: forward y = dequant(quant(x)) (one kernel pass), backward
+    the straight-through estimator (the incoming gradient passes unchanged to x).  The pages give
+    the forward only; straight-through is the plain reading for the backward."""
+
+    @staticmethod
+    def forward(ctx, x, block=32, fmt="e4m3", g=None):
+        return fake_quantize(x.contiguous(), block, fmt, g)
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        return grad_y, None, None, None
+
+
 class ErrorStats:
     """Device-resident mx_error_stats_t (64 bytes); to_dict() copies it to the host."""
 

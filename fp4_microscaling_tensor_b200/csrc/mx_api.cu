@@ -83,6 +83,25 @@ mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t ro
   return from_cuda(e);
 }
 
+mx_status mx_fake_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
+                           mx_scale_fmt fmt, uint16_t global_scale_fp16, void* y, mx_dtype yt,
+                           cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_dtype(yt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) ||
+      !shape_ok(rows, cols))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
+  if (cols % block != 0) return MX_ERR_INVALID_ARG;
+  const int64_t numel = rows * cols;
+  if (numel == 0) return MX_OK;
+  if (!x || !y) return MX_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return MX_ERR_MISALIGNED;
+  int n = 0;
+  const cudaError_t e = mxk::run_fake_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
+                                               global_scale_fp16, y, yt == MX_BF16, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
 size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int block) {
   (void)rows;
   (void)cols;

@@ -133,6 +133,12 @@ cudaError_t run_dequantize_group(const TensorArgs* t, int count, bool bf16out, i
 cudaError_t run_stats_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
                             StatsMode mode, void* workspace, cudaStream_t stream, int* launches);
 
+// Fake quantization (the round trip quantize -> dequantize in one pass): y = E2M1 * S * g of the
+// codes mx_quantize would store, as bf16 (ybf16) or fp32; nothing else is written.
+cudaError_t run_fake_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                              uint16_t g_bits, void* y, bool ybf16, cudaStream_t stream,
+                              int* launches);
+
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
                          uint16_t g_bits, uint8_t* packed, uint8_t* scales, cudaStream_t stream,
                          int* launches);

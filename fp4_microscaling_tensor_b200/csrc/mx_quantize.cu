@@ -42,9 +42,47 @@ struct QTensor {
   const void* x;
   uint8_t* packed;
   uint8_t* scales;
+  void* y;  // round trip (OUT != kCodes): the dequantized output instead of codes and scales
   int64_t nitems;
   uint32_t g_bits;
 };
+
+// What a quantize kernel writes: codes and scales, or (the fake-quantize round trip) the
+// dequantized value E2M1(code) * S * g of every element, as bf16 (round to nearest even of the
+// exact product) or fp32 (exact).
+enum QOut { kCodes = 0, kRoundTripBf16 = 1, kRoundTripF32 = 2 };
+
+// Round trip: the 8 codes of each code word times the scale of its block, stored to y at item i.
+template <int EPT, int BPI, int OUT>
+__device__ __forceinline__ void store_round_trip(void* y, int64_t i, const uint32_t* codes,
+                                                 uint32_t sc, const float* s_D) {
+  constexpr int BE = EPT / BPI;
+  float out[EPT];
+#pragma unroll
+  for (int b = 0; b < BPI; ++b) {
+    const float D = s_D[(sc >> (8 * b)) & 0xFF];
+#pragma unroll
+    for (int k = 0; k < BE; ++k) {
+      const int e = b * BE + k;  // nibble e % 8 of code word e / 8
+      const float f = __uint_as_float(e2m1_scaled_bits_at(codes[e / 8], 4 * (e % 8)));
+      out[e] = __fmul_rn(__fmul_rn(f, 0x1p126f), D);  // exact
+    }
+  }
+  if constexpr (OUT == kRoundTripBf16) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + i * EPT);
+#pragma unroll
+    for (int h = 0; h < EPT / 8; ++h)
+      __stcs(dst + h, make_uint4(pack_bf16x2(out[8 * h], out[8 * h + 1]),
+                                 pack_bf16x2(out[8 * h + 2], out[8 * h + 3]),
+                                 pack_bf16x2(out[8 * h + 4], out[8 * h + 5]),
+                                 pack_bf16x2(out[8 * h + 6], out[8 * h + 7])));
+  } else {
+    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + i * EPT);
+#pragma unroll
+    for (int h = 0; h < EPT / 4; ++h)
+      __stcs(dst + h, make_float4(out[4 * h], out[4 * h + 1], out[4 * h + 2], out[4 * h + 3]));
+  }
+}
 struct QGroup {
   QTensor t[kMaxGroup];
   CtaSplit split;
@@ -76,7 +114,7 @@ __device__ __forceinline__ uint32_t absmax_bits(const uint32_t* w) {
   return max(t & 0xFFFFu, t >> 16);
 }
 
-template <int N, int FMT>
+template <int N, int FMT, int OUT = kCodes>
 __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constant__ QGroup grp) {
   using S = QShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
@@ -86,10 +124,12 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
   uint8_t* __restrict__ scales = wk.t.scales;
   const int64_t nitems = wk.t.nitems;
   __shared__ float s_rcp[256];
+  __shared__ float s_D[OUT == kCodes ? 1 : 256];
   const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);  // exact (<= 15 significant bits)
     s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;          // zero scale -> every code is +-0
+    if constexpr (OUT != kCodes) s_D[c] = D;
   }
   const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
   __syncthreads();
@@ -146,6 +186,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
         codes[j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3], qv[8 * j + 4],
                               qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
       if (!ok[u]) continue;
+      if constexpr (OUT != kCodes) {
+        store_round_trip<EPT, BPI, OUT>(wk.t.y, i, codes, sc, s_D);
+        continue;
+      }
       if constexpr (NW == 8) {
         *reinterpret_cast<uint2*>(packed + i * 8) = make_uint2(codes[0], codes[1]);
       } else {
@@ -164,7 +208,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
 // fp32 input: IEEE division (see mx_device.cuh for why the multiply shortcut is not used here)
 // ------------------------------------------------------------------------------------------------
 
-template <int N, int FMT>
+template <int N, int FMT, int OUT = kCodes>
 __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant__ QGroup grp) {
   using S = QShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U;
@@ -226,8 +270,12 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant
         }
       }
       if (!ok[u]) continue;
-      *reinterpret_cast<uint32_t*>(packed + i * 4) =
-          cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      const uint32_t code = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      if constexpr (OUT != kCodes) {
+        store_round_trip<EPT, BPI, OUT>(wk.t.y, i, &code, sc, s_D);
+        continue;
+      }
+      *reinterpret_cast<uint32_t*>(packed + i * 4) = code;
       if constexpr (BPI == 1) {
         if ((lane & (L - 1)) == 0) scales[i / L] = (uint8_t)sc;
       } else {
@@ -242,9 +290,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant
 // do not fill an item.  One warp finishes that block with plain per-element code.
 // ------------------------------------------------------------------------------------------------
 
-template <int FMT, typename T>
+template <int FMT, typename T, int OUT = kCodes>
 __global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_t g_bits,
-                                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scales) {
+                                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                                 void* __restrict__ y = nullptr) {
   if (threadIdx.x != 0) return;
   const float g = fp16_bits_to_float(g_bits);
   float v[4], a = 0.0f;
@@ -260,6 +309,16 @@ __global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_
   float q[4];
   for (int k = 0; k < 4; ++k) q[k] = D > 0.0f ? __fdiv_rn(v[k], D) : __fmul_rn(v[k], 0.0f);
   const uint32_t c = cvt_e2m1x8(q[0], q[1], q[2], q[3], 0.f, 0.f, 0.f, 0.f);
+  if constexpr (OUT != kCodes) {
+    for (int k = 0; k < 4; ++k) {
+      const float v = __fmul_rn(e2m1_to_float(c >> (4 * k)), D);  // exact
+      if constexpr (OUT == kRoundTripBf16)
+        reinterpret_cast<__nv_bfloat16*>(y)[first + k] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<float*>(y)[first + k] = v;
+    }
+    return;
+  }
   packed[first / 2] = (uint8_t)(c & 0xFF);
   packed[first / 2 + 1] = (uint8_t)((c >> 8) & 0xFF);
   scales[first / 4] = (uint8_t)s;
@@ -269,45 +328,47 @@ __global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_
 // launcher
 // ------------------------------------------------------------------------------------------------
 
-template <int N, int FMT, typename T>
+template <int N, int FMT, typename T, int OUT>
 static cudaError_t launch_q(const TensorArgs* ta, int count, cudaStream_t stream, int* launches) {
   using S = QShape<N, T>;
   QGroup grp = {};
   int64_t nitems[kMaxGroup];
   for (int k = 0; k < count; ++k) {
     nitems[k] = ta[k].numel / S::EPT;
-    grp.t[k] = {ta[k].x, ta[k].packed, ta[k].scales, nitems[k], ta[k].g_bits};
+    grp.t[k] = {ta[k].x, ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits};
   }
-  auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT> : (void*)k_quantize_f32<N, FMT>;
+  auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT, OUT>
+                               : (void*)k_quantize_f32<N, FMT, OUT>;
   const int grid = split_grid(kern, nitems, count, S::U, 1 << 30, &grp.split);
   if (grid > 0) {
-    const cudaError_t e = (sizeof(T) == 2)
-                              ? launch_pdl(k_quantize_bf16<N, FMT>, grid, kThreads, stream, grp)
-                              : launch_pdl(k_quantize_f32<N, FMT>, grid, kThreads, stream, grp);
+    const cudaError_t e =
+        (sizeof(T) == 2) ? launch_pdl(k_quantize_bf16<N, FMT, OUT>, grid, kThreads, stream, grp)
+                         : launch_pdl(k_quantize_f32<N, FMT, OUT>, grid, kThreads, stream, grp);
     if (e != cudaSuccess) return e;
     ++*launches;
   }
   for (int k = 0; k < count; ++k) {
     if (ta[k].numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
-      k_quantize_tail4<FMT, T><<<1, 32, 0, stream>>>((const T*)ta[k].x, nitems[k] * S::EPT,
-                                                     ta[k].g_bits, ta[k].packed, ta[k].scales);
+      k_quantize_tail4<FMT, T, OUT><<<1, 32, 0, stream>>>(
+          (const T*)ta[k].x, nitems[k] * S::EPT, ta[k].g_bits, ta[k].packed, ta[k].scales,
+          ta[k].y);
       ++*launches;
     }
   }
   return cudaGetLastError();
 }
 
-template <int FMT, typename T>
+template <int FMT, typename T, int OUT>
 static cudaError_t dispatch_block(int block, const TensorArgs* t, int count, cudaStream_t st,
                                   int* n) {
   switch (block) {
-    case 4: return launch_q<4, FMT, T>(t, count, st, n);
-    case 8: return launch_q<8, FMT, T>(t, count, st, n);
-    case 16: return launch_q<16, FMT, T>(t, count, st, n);
-    case 32: return launch_q<32, FMT, T>(t, count, st, n);
-    case 64: return launch_q<64, FMT, T>(t, count, st, n);
-    case 128: return launch_q<128, FMT, T>(t, count, st, n);
-    default: return launch_q<256, FMT, T>(t, count, st, n);
+    case 4: return launch_q<4, FMT, T, OUT>(t, count, st, n);
+    case 8: return launch_q<8, FMT, T, OUT>(t, count, st, n);
+    case 16: return launch_q<16, FMT, T, OUT>(t, count, st, n);
+    case 32: return launch_q<32, FMT, T, OUT>(t, count, st, n);
+    case 64: return launch_q<64, FMT, T, OUT>(t, count, st, n);
+    case 128: return launch_q<128, FMT, T, OUT>(t, count, st, n);
+    default: return launch_q<256, FMT, T, OUT>(t, count, st, n);
   }
 }
 
@@ -333,13 +394,28 @@ cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt,
   return cudaGetLastError();
 }
 
+template <int OUT>
+static cudaError_t quantize_out(const TensorArgs* t, int count, bool bf16, int block, int fmt,
+                                cudaStream_t stream, int* launches) {
+  if (bf16)
+    return fmt == kUE5M3
+               ? dispatch_block<kUE5M3, uint16_t, OUT>(block, t, count, stream, launches)
+               : dispatch_block<kE4M3, uint16_t, OUT>(block, t, count, stream, launches);
+  return fmt == kUE5M3 ? dispatch_block<kUE5M3, float, OUT>(block, t, count, stream, launches)
+                       : dispatch_block<kE4M3, float, OUT>(block, t, count, stream, launches);
+}
+
 cudaError_t run_quantize_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,
                                cudaStream_t stream, int* launches) {
-  if (bf16)
-    return fmt == kUE5M3 ? dispatch_block<kUE5M3, uint16_t>(block, t, count, stream, launches)
-                         : dispatch_block<kE4M3, uint16_t>(block, t, count, stream, launches);
-  return fmt == kUE5M3 ? dispatch_block<kUE5M3, float>(block, t, count, stream, launches)
-                       : dispatch_block<kE4M3, float>(block, t, count, stream, launches);
+  return quantize_out<kCodes>(t, count, bf16, block, fmt, stream, launches);
+}
+
+cudaError_t run_fake_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,
+                              uint16_t g_bits, void* y, bool ybf16, cudaStream_t stream,
+                              int* launches) {
+  const TensorArgs t = {x, y, nullptr, nullptr, nullptr, numel, g_bits};
+  return ybf16 ? quantize_out<kRoundTripBf16>(&t, 1, bf16, block, fmt, stream, launches)
+               : quantize_out<kRoundTripF32>(&t, 1, bf16, block, fmt, stream, launches);
 }
 
 cudaError_t run_quantize(const void* x, bool bf16, int64_t numel, int block, int fmt,

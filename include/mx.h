@@ -95,6 +95,16 @@ MX_API mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int
                         int block, mx_scale_fmt fmt, uint16_t global_scale_fp16, void* y,
                         mx_dtype yt, cudaStream_t stream);
 
+/* Fake quantization for quantization-aware training ([MX] §5.2 item 1: the forward pass injects
+ * the quantization noise, x -> dequant(quant(x))): y is, bit for bit, what mx_dequantize writes
+ * for the codes and scales mx_quantize would store, computed in one pass that reads x and writes
+ * only y (4 bytes per element for bf16 -> bf16).  Arguments as mx_quantize (x, xt, rows, cols,
+ * block, fmt, global scale) and mx_dequantize (y, yt).  The gradient (straight-through) belongs to
+ * the caller's autograd; the Python binding provides it. */
+MX_API mx_status mx_fake_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
+                                  int block, mx_scale_fmt fmt, uint16_t global_scale_fp16, void* y,
+                                  mx_dtype yt, cudaStream_t stream);
+
 /* Bytes of device workspace mx_error_stats needs (a bound that holds for any device). */
 MX_API size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int block);
 

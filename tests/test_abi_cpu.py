@@ -174,3 +174,18 @@ def test_group_calls_reject_bad_arguments():
     d = group(3)
     d[2].cols = 40
     assert L.mx_quantize_group(d, 3, BF16, 32, E4, None) == INV
+
+
+def test_fake_quantize_rejects_bad_arguments():
+    def fq(x=A, xt=BF16, rows=4, cols=64, block=32, fmt=E4, g=0x3C00, y=A, yt=BF16):
+        return L.mx_fake_quantize(x, xt, rows, cols, block, fmt, g, y, yt, None)
+    assert fq(x=None) == INV
+    assert fq(y=None) == INV
+    assert fq(yt=3) == INV
+    assert fq(xt=3) == INV
+    assert fq(cols=40) == INV
+    assert fq(block=24) == UNS
+    assert fq(g=0xFC00) == INV
+    assert fq(x=A + 2) == MIS
+    assert fq(y=A + 8) == MIS
+    assert fq(rows=0, x=None, y=None) == OK      # empty: nothing to do
