@@ -33,10 +33,10 @@ METRIC = "quantize+pack / dequant GB/s and Gelem/s on 1 B200; fraction of HBM pe
 WORKLOAD = "bf16-4096x4096 x5 sigma sweep, blocks 4..256 x {E4M3,UE5M3} (70 points)"
 SHAPE = (4096, 4096)
 L2_BYTES = 126 * 2 ** 20
-# DRAM bytes (read + write) of one fused-pass launch at the bench point shape (N = 32, E4M3), from
-# the ncu capture summarised in profiles/k_error_stats_bf16_fused_4096x4096_n32.md: x is read once,
-# the codes and scales stay in L2 at the end of the launch.
-FUSED_TRAFFIC_BYTES = 33607424 + 7168
+# DRAM bytes (read + write) of one grouped fused-pass launch (5 tensors, N = 32, E4M3), from the
+# ncu capture summarised in profiles/k_error_stats_bf16_fused_group5_4096x4096_n32.md: every x is
+# read once, most of the codes and scales are still in L2 when the launch ends.
+FUSED_TRAFFIC_BYTES = 167830272 + 7129600
 
 
 def parse(argv=None):
@@ -467,8 +467,9 @@ def run_ours(args):
                      "achieved": qs_gbs, "peak": peak, "unit": "GB/s", "frac": qs_gbs / peak,
                      "peak_kind": peak_kind + " (burst copy)",
                      "traffic": FUSED_TRAFFIC_BYTES,
-                     "traffic_note": "bytes per launch, ncu dram__bytes_read+write, N=32 point; "
-                                     "algorithmic bytes per launch " + str(int(q_bytes(numel, 32)))},
+                     "traffic_note": "bytes per grouped launch (5 tensors, N=32), ncu "
+                                     "dram__bytes_read+write; algorithmic bytes per such launch "
+                                     + str(int(5 * q_bytes(numel, 32)))},
         "e2e": {"value": world * (qb + db) / e2e_s / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
