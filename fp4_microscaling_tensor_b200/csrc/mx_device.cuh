@@ -58,6 +58,23 @@ __device__ __forceinline__ float snap21(float v) {
 }
 
 // FP8 code of u >= 0 (already exact or snapped), nearest-even, saturating.
+// Quotients x / (S g) of two elements (lo / hi: their fp32 bits) for the E2M1 conversion, on the
+// FMA pipe.  r = RN(1 / (S g)), so x r is within 2^-21 of the true quotient t when |t| <= 8.
+// Adding 48 (whose binade [32, 64) has spacing 2^-18) and subtracting it again rounds x r onto that
+// grid exactly (Sterbenz for the subtraction).  A midpoint of the E2M1 grid (a multiple of 1/4) is
+// then hit exactly when t is one; otherwise t is at least 2^-17 away from every midpoint (x is
+// bf16, 8 significant bits, and S g has at most 15), and the rounded value stays on t's side.  Larger |t| only has to stay above 6, which it does.
+// Signs: the subtraction rounds toward -inf, so a quotient that cancels to zero is -0; the final
+// FMA adds x 2^-60, which leaves any non-zero quotient unchanged (|x| 2^-60 is below a quarter of
+// its unit in the last place, since r >= 2^-33) and gives a zero quotient the sign of x (+0 + -0 is
+// +0, -0 + -0 is -0): the E2M1 code's sign bit always follows x.
+__device__ __forceinline__ float2 snap_quotient2(uint32_t lo, uint32_t hi, float r) {
+  const float2 x = make_float2(__uint_as_float(lo), __uint_as_float(hi));
+  const float2 y = __ffma2_rn(x, make_float2(r, r), make_float2(48.0f, 48.0f));
+  const float2 q = __fadd2_rd(y, make_float2(-48.0f, -48.0f));
+  return __ffma2_rn(x, make_float2(0x1p-60f, 0x1p-60f), q);
+}
+
 template <int FMT>
 __device__ __forceinline__ uint32_t encode_scale(float u) {
   if constexpr (FMT == kE4M3) {

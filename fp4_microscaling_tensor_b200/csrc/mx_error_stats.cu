@@ -162,22 +162,6 @@ __device__ __forceinline__ double scaled_to_double(float v, int E) {
   return b ? __hiloint2double((int)hi, (int)lo) : 0.0;
 }
 
-// Quotients x / (S g) of two bf16 elements (lo / hi: their fp32 bits), rounded to multiples of
-// 2^-18 on the FMA pipe, for the E2M1 conversion.  r = RN(1 / (S g)), so x r is within 2^-21 of the
-// true quotient t when |t| <= 8.  Adding and subtracting 48 (whose binade [32, 64) has spacing
-// 2^-18) rounds x r to that grid exactly (Sterbenz for the subtraction).  A midpoint of the E2M1
-// grid (a multiple of 1/4) is then hit exactly when t is one; otherwise t is at least 2^-17 away
-// from every midpoint (x has 8 significant bits, S g at most 15), and the rounded value stays on
-// t's side.  Larger |t| only has to stay above 6, which it does.  The sign is copied from x, so that
-// quotients rounding to zero keep the sign of x (the code's sign bit always follows x).
-__device__ __forceinline__ float2 snap_quotient2(uint32_t lo, uint32_t hi, float r) {
-  const float2 q = __fadd2_rn(__ffma2_rn(make_float2(__uint_as_float(lo), __uint_as_float(hi)),
-                                         make_float2(r, r), make_float2(48.0f, 48.0f)),
-                              make_float2(-48.0f, -48.0f));
-  return make_float2(__uint_as_float((__float_as_uint(q.x) & 0x7FFFFFFFu) | (lo & 0x80000000u)),
-                     __uint_as_float((__float_as_uint(q.y) & 0x7FFFFFFFu) | (hi & 0x80000000u)));
-}
-
 // Per-block constants of one block slice (see the file comment for the scaling).
 struct SliceSetup {
   int E;           // biased exponent of the block maximum a (at least 1)

@@ -176,8 +176,9 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
 #pragma unroll
         for (int k = 0; k < BW; ++k) {
           const uint32_t wk = w[u][b * BW + k];
-          qv[2 * (b * BW + k)] = snap21(__fmul_rn(bf16lo(wk), r));
-          qv[2 * (b * BW + k) + 1] = snap21(__fmul_rn(bf16hi(wk), r));
+          const float2 q = snap_quotient2(wk << 16, wk & 0xFFFF0000u, r);
+          qv[2 * (b * BW + k)] = q.x;
+          qv[2 * (b * BW + k) + 1] = q.y;
         }
       }
       uint32_t codes[EPT / 8];
