@@ -10,6 +10,8 @@
 // codes, multiplies by the per-code constant S g from a
 // shared-memory table and writes 16-byte vectors.  Codes are decoded with exact bit arithmetic
 // (e2m1_scaled_bits_at), not with a conversion instruction.
+#include <cuda_fp16.h>
+
 #include "mx_device.cuh"
 #include "mx_launch.h"
 
@@ -22,6 +24,24 @@ namespace mxk {
 #ifndef MX_DQ_U
 #define MX_DQ_U 2
 #endif
+
+#ifndef MX_DQ_HWDEC
+#define MX_DQ_HWDEC 1
+#endif
+
+// The eight codes of a loaded word w (code k in nibble k) decoded to f16x2 values h[0..3] (word k:
+// codes 2k, 2k+1) by the E2M1x2 -> f16x2 conversion; exact (E2M1 values are f16 values).  The word
+// comes from memory and is split into its bytes inside the same asm block.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t* h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
 
 template <int N, bool BF16OUT>
 struct DShape {
@@ -93,6 +113,24 @@ __global__ void __launch_bounds__(kThreads) k_dequantize(const __grid_constant__
       const int64_t i = base + (int64_t)u * T;
       if (i >= nitems) continue;
       float out[EPT];
+#if MX_DQ_HWDEC
+      uint32_t hv[EPT / 2];
+#pragma unroll
+      for (int j = 0; j < EPT / 8; ++j) e2m1x8_to_f16x2(cw[u][j], &hv[4 * j]);
+#pragma unroll
+      for (int b = 0; b < BPI; ++b) {
+        const float D = s_D[(sc[u] >> (8 * b)) & 0xFF];
+        constexpr int BE = EPT / BPI;
+#pragma unroll
+        for (int k = 0; k < BE / 2; ++k) {
+          const int e = b * BE + 2 * k;  // elements e, e + 1: word e / 2 of hv
+          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&hv[e / 2]));
+          const float2 y2 = __fmul2_rn(v, make_float2(D, D));  // exact
+          out[e] = y2.x;
+          out[e + 1] = y2.y;
+        }
+      }
+#else
 #pragma unroll
       for (int b = 0; b < BPI; ++b) {
         const float D = s_D[(sc[u] >> (8 * b)) & 0xFF];
@@ -104,6 +142,7 @@ __global__ void __launch_bounds__(kThreads) k_dequantize(const __grid_constant__
           out[e] = __fmul_rn(__fmul_rn(f, 0x1p126f), D);
         }
       }
+#endif
       if constexpr (BF16OUT) {
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + i * EPT);
 #pragma unroll
