@@ -324,6 +324,44 @@ def time_graphs(graphs, steps, stream):
             for j in range(len(graphs))]
 
 
+def small_tensor_latency(dev, stream, calls=1000):
+    """Microseconds per call for the fp32 256 x 256 tensor (N = 32, E4M3): quantize, dequantize
+    (fp32 out), error reduction from the stored codes, each replayed as one graph of `calls`."""
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    from fp4_microscaling_tensor_b200 import inputs
+    x = inputs.workload1(device=dev)
+    p, s = mx.quantize(x, 32, mx.E4M3)
+    y = torch.empty_like(x)
+    out = torch.empty(64, dtype=torch.uint8, device=dev)
+    ws = mx.stats_workspace(dev)
+    fns = {"quantize": lambda: mx.quantize(x, 32, mx.E4M3, packed=p, scales=s),
+           "dequantize": lambda: mx.dequantize(p, s, 32, mx.E4M3, out_dtype=torch.float32, out=y),
+           "error_stats": lambda: mx.error_stats(x, 32, mx.E4M3, packed=p, scales=s, out=out,
+                                                 workspace=ws)}
+    res = {}
+    for name, fn in fns.items():
+        with torch.cuda.stream(stream):
+            fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(calls):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / calls
+        del g
+    return res
+
+
 def rank_seed(k, rank):
     """Seed of sigma index k on a rank: every rank draws its own tensors (weak scaling)."""
     return 100 + k + 1000 * rank
@@ -409,6 +447,10 @@ def run_ours(args):
     time_graphs([g_q], 3, stream)
     t_q = max_over_ranks([time_graphs([g_q], q_steps, stream)[0] / q_steps], dev)[0]
 
+    # ---- the small fp32 tensor (256 x 256, N = 32, E4M3): latency per call, one graph of 1000
+    #      calls per kernel (launch-bound; reported beside the throughput, no roofline claim)
+    small = small_tensor_latency(dev, stream)
+
     # ---- end to end through the public API: pinned H2D of the inputs, eager calls, D2H of stats
     host = [x.cpu().pin_memory() for x in xs]
     dxs = [torch.empty_like(x) for x in xs]
@@ -474,6 +516,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "deterministic_stats": deterministic,
+        "small_tensor_latency_us": small,
         "wall_s_timed": t_wall,
     }
     result["clocks"] = clk.summary()

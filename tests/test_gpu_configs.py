@@ -18,7 +18,8 @@ Configurations (sizes as the workloads state them):
      scale: layer 0 whole, every layer sampled.
   4  activations bf16 16384x8192 with outlier channels, N = 16, E4M3: whole.
   5  Llama-2-70B-shaped layer (2 x 8192^2, 2 x 1024x8192, 3 x 8192x28672), N = 32, UE5M3 + global
-     scale, with the error record: layer 0 whole, layers 1 and 79 sampled + properties.
+     scale, with the error record: layer 0 whole; layers 1, 13, 27, 40, 53, 66, 79 sampled +
+     properties.
 """
 import numpy as np
 import pytest
@@ -137,7 +138,7 @@ def test_config4_activations(cuda_device):
     assert_same(bits(y), yo, "config 4 dequant")
 
 
-@pytest.mark.parametrize("layer", [0, 1, 79])
+@pytest.mark.parametrize("layer", [0, 1, 13, 27, 40, 53, 66, 79])
 def test_config5_llama70b_layer(cuda_device, layer):
     for j in range(len(inputs.LLAMA70B_SHAPES)):
         x = inputs.workload5_tensor(layer, j, device=cuda_device)
