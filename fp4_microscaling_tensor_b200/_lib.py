@@ -28,7 +28,7 @@ EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_
            "mx_quantize_stats",
            "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
            "mx_quantize_group", "mx_dequantize_group", "mx_quantize_stats_group",
-           "mx_fake_quantize",
+           "mx_fake_quantize", "mx_test_fail_next_calls",
            "mx_status_string", "mx_kernel_launches")
 MX_MAX_GROUP = 16
 
@@ -61,6 +61,8 @@ lib.mx_global_scale.restype = _i
 lib.mx_global_scale.argtypes = [_vp, _i, _i64, _i64, _i, _vp, _vp, _sz, _vp]
 lib.mx_error_stats_noalloc.restype = _i
 lib.mx_error_stats_noalloc.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _vp, _vp, _vp]
+lib.mx_test_fail_next_calls.restype = _i
+lib.mx_test_fail_next_calls.argtypes = [_i]
 lib.mx_fake_quantize.restype = _i
 lib.mx_fake_quantize.argtypes = [_vp, _i, _i64, _i64, _i, _i, _u16, _vp, _i, _vp]
 _tp = ctypes.POINTER(Tensor)

@@ -14,6 +14,16 @@ static_assert(MX_MAX_GROUP == mxk::kMaxGroup, "group size");
 namespace {
 
 std::atomic<long long> g_launches{0};  // diagnostic: kernels enqueued by this library
+std::atomic<int> g_fail_next{0};       // test hook: calls still to fail with MX_ERR_CUDA
+
+// True when an armed test failure is consumed by this call (nothing is enqueued then).
+bool injected_failure() {
+  int n = g_fail_next.load();
+  while (n > 0) {
+    if (g_fail_next.compare_exchange_weak(n, n - 1)) return true;
+  }
+  return false;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -58,6 +68,7 @@ mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, in
   if (numel == 0) return MX_OK;
   if (!x || !packed || !scales) return MX_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
                                           global_scale_fp16, packed, scales, stream, &n);
@@ -76,6 +87,7 @@ mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t ro
   if (numel == 0) return MX_OK;
   if (!packed || !scales || !y) return MX_ERR_INVALID_ARG;
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(y)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_dequantize(packed, scales, numel, block, (int)fmt,
                                             global_scale_fp16, y, yt == MX_BF16, stream, &n);
@@ -95,6 +107,7 @@ mx_status mx_fake_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t col
   if (numel == 0) return MX_OK;
   if (!x || !y) return MX_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_fake_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
                                                global_scale_fp16, y, yt == MX_BF16, stream, &n);
@@ -125,6 +138,7 @@ mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
   if ((numel != 0 && !aligned16(x)) || !aligned16(out_dev) || !aligned16(workspace) ||
       (packed && (!aligned16(packed) || !aligned16(scales))))
     return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e =
       mxk::run_error_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
@@ -148,6 +162,7 @@ mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t co
   if ((numel != 0 && (!aligned16(x) || !aligned16(packed) || !aligned16(scales))) ||
       !aligned16(out_dev) || !aligned16(workspace))
     return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_quantize_stats(numel ? x : nullptr, xt == MX_BF16, numel, block,
                                                 (int)fmt, global_scale_fp16, packed, scales,
@@ -171,6 +186,7 @@ mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols
   if (numel != 0 && !x) return MX_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < amax_ws_bytes()) return MX_ERR_WORKSPACE;
   if ((numel != 0 && !aligned16(x)) || !aligned16(workspace)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_global_scale(x, xt == MX_BF16, numel, (int)fmt, out_fp16_dev,
                                               workspace, stream, &n);
@@ -217,6 +233,7 @@ mx_status mx_quantize_group(const mx_tensor_t* tensors, int count, mx_dtype xt, 
   mxk::TensorArgs args[MX_MAX_GROUP];
   const mx_status st = check_group(tensors, count, block, kNeedX | kNeedCodes, args);
   if (st != MX_OK) return st;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e =
       mxk::run_quantize_group(args, count, xt == MX_BF16, block, (int)fmt, stream, &n);
@@ -231,6 +248,7 @@ mx_status mx_dequantize_group(const mx_tensor_t* tensors, int count, int block, 
   mxk::TensorArgs args[MX_MAX_GROUP];
   const mx_status st = check_group(tensors, count, block, kNeedY | kNeedCodes, args);
   if (st != MX_OK) return st;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e =
       mxk::run_dequantize_group(args, count, yt == MX_BF16, block, (int)fmt, stream, &n);
@@ -248,6 +266,7 @@ mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtyp
   if (st != MX_OK) return st;
   if (!workspace || ws_bytes < stats_ws_bytes()) return MX_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e = mxk::run_stats_group(args, count, xt == MX_BF16, block, (int)fmt,
                                              mxk::kStore, workspace, stream, &n);
@@ -268,5 +287,7 @@ const char* mx_status_string(mx_status status) {
 }
 
 long long mx_kernel_launches(void) { return g_launches.load(); }
+
+int mx_test_fail_next_calls(int count) { return g_fail_next.exchange(count > 0 ? count : 0); }
 
 }  // extern "C"

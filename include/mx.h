@@ -198,6 +198,12 @@ MX_API mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, 
                                          int block, mx_scale_fmt fmt, void* workspace,
                                          size_t ws_bytes, cudaStream_t stream);
 
+/* Test hook for error paths (no counterpart in the pages).  The next `count` calls that pass
+ * their argument checks and would enqueue work return MX_ERR_CUDA instead, as a failed launch is
+ * reported, without enqueueing anything or touching any buffer.  count <= 0 disarms the hook.
+ * Returns the number of armed failures that were still pending. */
+MX_API int mx_test_fail_next_calls(int count);
+
 /* Static description of a status code (never NULL). */
 MX_API const char* mx_status_string(mx_status status);
 

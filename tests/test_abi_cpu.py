@@ -189,3 +189,18 @@ def test_fake_quantize_rejects_bad_arguments():
     assert fq(x=A + 2) == MIS
     assert fq(y=A + 8) == MIS
     assert fq(rows=0, x=None, y=None) == OK      # empty: nothing to do
+
+
+def test_injected_cuda_failure_is_reported_before_any_launch():
+    # valid arguments on fake pointers: the armed failures are consumed before anything is
+    # enqueued, so nothing touches the (fake) buffers; the status is MX_ERR_CUDA
+    assert L.mx_test_fail_next_calls(2) == 0
+    assert q() == _lib.MX_ERR_CUDA
+    ws = L.mx_error_stats_workspace_size(4, 64, 32)
+    assert L.mx_quantize_stats(A, BF16, 4, 64, 32, E4, 0x3C00, A, A, A, A, ws, None) == \
+        _lib.MX_ERR_CUDA
+    assert L.mx_test_fail_next_calls(0) == 0           # both consumed
+    # argument checks come first: an invalid call does not consume an armed failure
+    assert L.mx_test_fail_next_calls(1) == 0
+    assert q(block=12) == UNS
+    assert L.mx_test_fail_next_calls(0) == 1           # still pending, now disarmed
