@@ -69,3 +69,45 @@ def test_two_ranks_gloo():
 def test_single_process_identity():
     assert bench.max_over_ranks([3.0, 4.0], "cpu") == [3.0, 4.0]
     assert bench.rank_seed(0, 0) != bench.rank_seed(0, 1)
+
+
+def shard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        import oracle
+        from fp4_microscaling_tensor_b200 import dist as mxdist, inputs
+        # one tensor, split by rows: each rank reduces its shard with the oracle, then combines
+        x = inputs.student_t4_rowgain((64, 512), 5)
+        shard = x[rank * 32:(rank + 1) * 32]
+        xo = inputs.to_oracle(shard)
+        g_local = oracle.global_scale(xo, oracle.UE5M3)
+        g = mxdist.combine_g_bits(g_local)
+        st = oracle.error_stats(xo, 32, 512, 32, oracle.UE5M3, g)
+        out[rank] = (g, mxdist.combine_stats(st))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_row_sharded_tensor_combines_to_whole():
+    import oracle
+    from fp4_microscaling_tensor_b200 import inputs
+    world = 2
+    port = free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(shard_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    x = inputs.student_t4_rowgain((64, 512), 5)
+    xo = inputs.to_oracle(x)
+    g_whole = oracle.global_scale(xo, oracle.UE5M3)
+    whole = oracle.error_stats(xo, 64, 512, 32, oracle.UE5M3, g_whole)
+    for rank in range(world):
+        g, st = res[rank]
+        assert g == g_whole
+        for k in ("numel", "n_blocks", "n_zero_blocks", "n_scale_sat", "n_elem_sat"):
+            assert st[k] == whole[k], k
+        for k in ("sse_elem", "sse_max", "sse_zero"):
+            assert abs(st[k] - whole[k]) <= 1e-12 * max(abs(whole[k]), 1e-300), k
