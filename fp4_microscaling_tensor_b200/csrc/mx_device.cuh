@@ -132,18 +132,6 @@ __device__ __forceinline__ float e2m1_to_float(uint32_t nib) {
   return __fmul_rn(__uint_as_float(e2m1_scaled_bits<0>(nib)), 0x1p126f);
 }
 
-// The 8 codes of w (code k at bits 4k..4k+3) times D, exact in fp32 (<= 17 significant bits).
-__device__ __forceinline__ void e2m1x8_times(uint32_t w, float D, float* out) {
-  out[0] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<0>(w)), 0x1p126f), D);
-  out[1] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<4>(w)), 0x1p126f), D);
-  out[2] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<8>(w)), 0x1p126f), D);
-  out[3] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<12>(w)), 0x1p126f), D);
-  out[4] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<16>(w)), 0x1p126f), D);
-  out[5] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<20>(w)), 0x1p126f), D);
-  out[6] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<24>(w)), 0x1p126f), D);
-  out[7] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits<28>(w)), 0x1p126f), D);
-}
-
 // max(|a|, |b|) per bf16 half (the sign of the result is meaningless; callers mask it).
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -151,14 +139,6 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
   return d;
 }
 
-// min(|a|, |b|) per bf16 half (sign meaningless, as above).
-__device__ __forceinline__ uint32_t bf16x2_absmin(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// Streaming 16-byte load of read-only data (not kept in L1).
 // Programmatic dependent launch: wait until the previous grid in the stream has completed and its
 // memory is visible (a no-op without such a dependency); then allow the next grid to be scheduled.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -166,6 +146,7 @@ __device__ __forceinline__ void griddep_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Streaming 16-byte load of read-only data (not kept in L1).
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;
   asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
