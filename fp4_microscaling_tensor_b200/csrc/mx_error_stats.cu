@@ -820,6 +820,12 @@ __global__ void k_stats_reset(unsigned int* counters, int n) {
   griddep_launch_next();
 }
 
+cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches) {
+  const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, counter, 1);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
 // Main pass over the group; then, for each tensor the main pass does not finish, its N = 4 tail
 // (4 elements after the last full item) and a one-CTA final pass, or (no items) the final pass
 // alone.  Without a tail the main pass adds a tensor's partials itself.

@@ -158,6 +158,10 @@ cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int bloc
 cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt, uint16_t g_bits,
                                uint8_t* packed, uint8_t* scales, cudaStream_t stream,
                                int* launches);
+// Zeroes one last-CTA counter once the previous kernel in the stream is done with it (a one-thread
+// kernel launched with programmatic serialization).
+cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches);
+
 cudaError_t run_global_scale(const void* x, bool bf16, int64_t numel, int fmt, uint16_t* out,
                              void* workspace, cudaStream_t stream, int* launches);
 
