@@ -110,6 +110,37 @@ def model(sigma, N, fmt, g=1.0):
     return out
 
 
+def adaptive_block_size(sigma):
+    """The pages' dynamic block-size rule (microscaling article §6 item 2): 128 below sigma =
+    0.01, 64 below 0.1, else 32."""
+    if sigma < 0.01:
+        return 128
+    if sigma < 0.1:
+        return 64
+    return 32
+
+
+def bits_per_element(N):
+    """Storage per element: a 4-bit code plus an 8-bit scale per block of N."""
+    return 4.0 + 8.0 / N
+
+
+def model_block_size(sigma, fmt, g=1.0, max_bits=None, blocks=BLOCKS):
+    """The block size with the smallest modelled total MSE for N(0, sigma^2) data, among those
+    whose storage (4 + 8/N bits per element) is at most max_bits (all when None); ties go to the
+    larger block (less storage)."""
+    best = None
+    for n in sorted(blocks, reverse=True):
+        if max_bits is not None and bits_per_element(n) > max_bits:
+            continue
+        tot = sum(model(sigma, n, fmt, g).values())
+        if best is None or tot < best[1]:
+            best = (n, tot)
+    if best is None:
+        raise ValueError("no block size fits the storage budget")
+    return best[0]
+
+
 def measure_sweep(shape=(4096, 4096)):
     """The sweep on the GPU: {(sigma, N, fmt): {'elem', 'max', 'zero'}} measured by the fused
     quantize + error-reduction pass on bf16 N(0, sigma^2) tensors (one grouped launch per point

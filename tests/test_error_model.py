@@ -51,3 +51,21 @@ def test_measured_terms_match_model(cuda_device, sigma, N, fmt):
             assert abs(got[k] - mod[k]) <= 0.05 * mod[k], (k, got[k], mod[k])
         else:
             assert got[k] <= 0.02 * tot, (k, got[k], mod[k])
+
+
+def test_adaptive_block_size_rule():
+    assert [em.adaptive_block_size(s) for s in (0.001, 0.0099, 0.01, 0.05, 0.0999, 0.1, 1.0)] == \
+        [128, 128, 64, 64, 64, 32, 32]
+
+
+def test_model_block_size():
+    # wide tensors: smaller blocks are more accurate; narrow E4M3 tensors: the zero-scale term
+    # makes the smallest blocks worst (the pages' anomaly), UE5M3 removes it
+    assert em.model_block_size(0.1, em.E4M3) == 4
+    assert em.model_block_size(0.005, em.E4M3) > 4
+    assert em.model_block_size(0.005, em.UE5M3) == 4
+    # a storage budget of 4.25 bits per element allows N >= 32 only
+    n = em.model_block_size(0.1, em.E4M3, max_bits=4.25)
+    assert n == 32 and em.bits_per_element(n) <= 4.25
+    with pytest.raises(ValueError):
+        em.model_block_size(0.1, em.E4M3, max_bits=4.0)
