@@ -37,6 +37,9 @@
 #ifndef MX_ST_MINB  // minimum resident CTAs per SM for the bf16 pass (register cap)
 #define MX_ST_MINB 2
 #endif
+#ifndef MX_ST_MINB_SMALL  // the same for N <= 8 (8-element items: more warps hide the latency)
+#define MX_ST_MINB_SMALL 3
+#endif
 
 namespace mxk {
 
@@ -437,7 +440,8 @@ struct StatsItem {
 };
 
 template <int N, int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, MX_ST_MINB) k_error_stats_bf16(
+__global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MINB)
+    k_error_stats_bf16(
     const __grid_constant__ SGroup grp) {
   const SWork wk = s_work(grp);
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
