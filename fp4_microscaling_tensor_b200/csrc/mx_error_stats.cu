@@ -22,7 +22,7 @@
 //   * Underflow.  A slice whose scaled non-max sum is below 2^-80 (squares below 2^-126 could be
 //     lost), or whose stored scale is far from a, redoes its slice in double.
 // Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
-// in a fixed order, so results are deterministic for a given device and grid; with an N = 4 tail a
+// in a fixed order, so results are deterministic for a given device and grid; with a tail (N <= 8) a
 // separate one-CTA pass does it.  No CTA waits on another.
 #include "mx_device.cuh"
 #include "mx_launch.h"
@@ -37,7 +37,10 @@
 #ifndef MX_ST_MINB  // minimum resident CTAs per SM for the bf16 pass (register cap)
 #define MX_ST_MINB 2
 #endif
-#ifndef MX_ST_MINB_SMALL  // the same for N <= 8 (8-element items: more warps hide the latency)
+#ifndef MX_ST_EPT_SMALL  // elements per item of the bf16 pass for N <= 8 (a multiple of 8)
+#define MX_ST_EPT_SMALL 16
+#endif
+#ifndef MX_ST_MINB_SMALL  // the same for N <= 8 (short per-block work: more warps hide the latency)
 #define MX_ST_MINB_SMALL 3
 #endif
 
@@ -55,8 +58,9 @@ struct StatsOut {  // layout of mx_error_stats_t
 
 template <int N, typename T>
 struct SShape {
-  static constexpr int EPT = (sizeof(T) == 2 && N >= 16) ? (N < MX_ST_EPT_BF16 ? N : MX_ST_EPT_BF16)
-                                                         : 8;
+  static constexpr int EPT = sizeof(T) != 2 ? 8
+                             : N >= 16 ? (N < MX_ST_EPT_BF16 ? N : MX_ST_EPT_BF16)
+                                       : MX_ST_EPT_SMALL;
   static constexpr int L = (N >= EPT) ? N / EPT : 1;
   static constexpr int BPI = (N >= EPT) ? 1 : EPT / N;
   static constexpr int U = (sizeof(T) == 2) ? MX_ST_U : 1;
@@ -112,7 +116,7 @@ struct STensor {
   uint8_t* scales_out;
   StatsPartial* part;      // this tensor's CTAs' partials: part[0 .. its CTA count)
   unsigned int* counter;   // last-CTA counter, zeroed before the launch; nullptr: a separate pass
-                           // adds the partials (N = 4 tail)
+                           // adds the partials (a tail, N <= 8)
   StatsOut* out;
   int64_t nitems, numel, nblocks;
   uint32_t g_bits;
@@ -504,7 +508,8 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
           it.cw[0] = __ldcs(reinterpret_cast<const unsigned int*>(packed) + i);
         }
         if constexpr (BPI == 1) it.scw = __ldg(scales + i / L);
-        else it.scw = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
+        else if constexpr (BPI == 2) it.scw = __ldg(reinterpret_cast<const unsigned short*>(scales) + i);
+        else it.scw = __ldg(reinterpret_cast<const unsigned int*>(scales) + i);
       }
     }
   };
@@ -711,45 +716,50 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(const __grid_const
 // N = 4 tail (4 elements) and the final reduction
 // ------------------------------------------------------------------------------------------------
 
+// The elements after the last whole item (count of them, a multiple of the block size N <= 8):
+// one thread, block by block, in double; codes recomputed (packed == nullptr) or read.
 template <int FMT, typename T>
-__global__ void k_error_stats_tail4(const T* __restrict__ x, int64_t first, uint16_t g_bits,
-                                    const uint8_t* __restrict__ packed,
-                                    const uint8_t* __restrict__ scales, StatsPartial* part) {
+__global__ void k_error_stats_tail(const T* __restrict__ x, int64_t first, int count, int N,
+                                   uint16_t g_bits, const uint8_t* __restrict__ packed,
+                                   const uint8_t* __restrict__ scales, StatsPartial* part) {
   if (threadIdx.x != 0) return;
   const float g = fp16_bits_to_float(g_bits);
-  float v[4], a = 0.0f;
-  int imax = 0;
-  for (int k = 0; k < 4; ++k) {
-    if constexpr (sizeof(T) == 2)
-      v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[first + k] << 16);
-    else
-      v[k] = reinterpret_cast<const float*>(x)[first + k];
-    if (fabsf(v[k]) > a) { a = fabsf(v[k]); imax = k; }
-  }
-  uint32_t s, codes[4];
-  if (packed == nullptr) {
-    s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
-    const float D0 = __fmul_rn(scale_value((int)s, FMT), g);
-    for (int k = 0; k < 4; ++k) {
-      const float q = D0 > 0.0f ? __fdiv_rn(v[k], D0) : __fmul_rn(v[k], 0.0f);
-      codes[k] = cvt_e2m1x8(q, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xF;
-    }
-  } else {
-    s = scales[first / 4];
-    for (int k = 0; k < 4; ++k) codes[k] = (packed[(first + k) / 2] >> (4 * ((first + k) & 1))) & 0xF;
-  }
-  const float D = __fmul_rn(scale_value((int)s, FMT), g);
   StatsPartial p{};
-  for (int k = 0; k < 4; ++k) {
-    const double y = (double)__fmul_rn(e2m1_to_float(codes[k]), D);
-    const double d = (double)v[k] - y;
-    if (!(D > 0.0f)) p.sse_zero += (double)v[k] * (double)v[k];
-    else if (k == imax) p.sse_max += d * d;
-    else p.sse_elem += d * d;
-    if (D > 0.0f && fabsf(v[k]) > __fmul_rn(6.0f, D)) p.n_elem_sat += 1;
+  for (int b0 = 0; b0 < count; b0 += N) {
+    const int64_t f = first + b0;
+    float v[8], a = 0.0f;
+    int imax = 0;
+    for (int k = 0; k < N; ++k) {
+      if constexpr (sizeof(T) == 2)
+        v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[f + k] << 16);
+      else
+        v[k] = reinterpret_cast<const float*>(x)[f + k];
+      if (fabsf(v[k]) > a) { a = fabsf(v[k]); imax = k; }
+    }
+    uint32_t s, codes[8];
+    if (packed == nullptr) {
+      s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
+      const float D0 = __fmul_rn(scale_value((int)s, FMT), g);
+      for (int k = 0; k < N; ++k) {
+        const float q = D0 > 0.0f ? __fdiv_rn(v[k], D0) : __fmul_rn(v[k], 0.0f);
+        codes[k] = cvt_e2m1x8(q, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xF;
+      }
+    } else {
+      s = scales[f / N];
+      for (int k = 0; k < N; ++k) codes[k] = (packed[(f + k) / 2] >> (4 * ((f + k) & 1))) & 0xF;
+    }
+    const float D = __fmul_rn(scale_value((int)s, FMT), g);
+    for (int k = 0; k < N; ++k) {
+      const double y = (double)__fmul_rn(e2m1_to_float(codes[k]), D);
+      const double d = (double)v[k] - y;
+      if (!(D > 0.0f)) p.sse_zero += (double)v[k] * (double)v[k];
+      else if (k == imax) p.sse_max += d * d;
+      else p.sse_elem += d * d;
+      if (D > 0.0f && fabsf(v[k]) > __fmul_rn(6.0f, D)) p.n_elem_sat += 1;
+    }
+    p.n_zero_blocks += (D > 0.0f) ? 0 : 1;
+    p.n_scale_sat += (a > __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>())) ? 1 : 0;
   }
-  p.n_zero_blocks = (D > 0.0f) ? 0 : 1;
-  p.n_scale_sat = (a > __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>())) ? 1 : 0;
   part[0] = p;
 }
 
@@ -830,9 +840,9 @@ cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int
   return e;
 }
 
-// Main pass over the group; then, for each tensor the main pass does not finish, its N = 4 tail
-// (4 elements after the last full item) and a one-CTA final pass, or (no items) the final pass
-// alone.  Without a tail the main pass adds a tensor's partials itself.
+// Main pass over the group; then, for each tensor the main pass does not finish, its tail (the
+// elements after the last whole item: N <= 8 only) and a one-CTA final pass, or (no items) the
+// final pass alone.  Without a tail the main pass adds a tensor's partials itself.
 template <int N, int FMT, typename T, int MODE>
 static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Workspace ws,
                                 cudaStream_t stream, int* launches) {
@@ -885,15 +895,16 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
     if (tail[k]) {
       extra = ws.part + grid + k;
       const int64_t first = nitems[k] * S::EPT;
-      if (MODE == kStore) {  // quantize the last 4 elements, then reduce them from the codes
-        const cudaError_t e = run_quantize_tail4(ta[k].x, sizeof(T) == 2, first, FMT,
-                                                 ta[k].g_bits, ta[k].packed, ta[k].scales, stream,
-                                                 launches);
+      const int count = (int)(ta[k].numel - first);  // < EPT, a multiple of N <= 8
+      if (MODE == kStore) {  // quantize the last elements, then reduce them from the codes
+        const cudaError_t e = run_quantize_tail(ta[k].x, sizeof(T) == 2, first, count, N, FMT,
+                                                ta[k].g_bits, ta[k].packed, ta[k].scales, stream,
+                                                launches);
         if (e != cudaSuccess) return e;
       }
-      k_error_stats_tail4<FMT, T><<<1, 32, 0, stream>>>(
-          (const T*)ta[k].x, first, ta[k].g_bits, MODE == kRecompute ? nullptr : ta[k].packed,
-          ta[k].scales, extra);
+      k_error_stats_tail<FMT, T><<<1, 32, 0, stream>>>(
+          (const T*)ta[k].x, first, count, N, ta[k].g_bits,
+          MODE == kRecompute ? nullptr : ta[k].packed, ta[k].scales, extra);
       ++*launches;
     }
     const int nparts = nitems[k] > 0 ? grp.split.begin[k + 1] - grp.split.begin[k] : 0;

@@ -154,10 +154,11 @@ cudaError_t run_error_stats(const void* x, bool bf16, int64_t numel, int block, 
 cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int block, int fmt,
                                uint16_t g_bits, uint8_t* packed, uint8_t* scales, void* out,
                                void* workspace, cudaStream_t stream, int* launches);
-// The last 4 elements of an N = 4 tensor whose size is not a multiple of 8 (from element `first`).
-cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt, uint16_t g_bits,
-                               uint8_t* packed, uint8_t* scales, cudaStream_t stream,
-                               int* launches);
+// The `count` elements from `first` on (a multiple of the block size N <= 8, fewer than an item of
+// the calling kernel): quantize + pack them with plain per-element code.
+cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,
+                              uint16_t g_bits, uint8_t* packed, uint8_t* scales,
+                              cudaStream_t stream, int* launches);
 // Zeroes one last-CTA counter once the previous kernel in the stream is done with it (a one-thread
 // kernel launched with programmatic serialization).
 cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches);

@@ -287,42 +287,47 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------------------------
-// tail: when N = 4 and the element count is not a multiple of 8, the last 4 elements (one block)
-// do not fill an item.  One warp finishes that block with plain per-element code.
+// tail: the elements after the last whole item (a multiple of N <= 8, fewer than an item).  One
+// thread finishes them block by block with plain per-element code (IEEE division).
 // ------------------------------------------------------------------------------------------------
 
 template <int FMT, typename T, int OUT = kCodes>
-__global__ void k_quantize_tail4(const T* __restrict__ x, int64_t first, uint16_t g_bits,
-                                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
-                                 void* __restrict__ y = nullptr) {
+__global__ void k_quantize_tail(const T* __restrict__ x, int64_t first, int count, int N,
+                                uint16_t g_bits, uint8_t* __restrict__ packed,
+                                uint8_t* __restrict__ scales, void* __restrict__ y = nullptr) {
   if (threadIdx.x != 0) return;
   const float g = fp16_bits_to_float(g_bits);
-  float v[4], a = 0.0f;
-  for (int k = 0; k < 4; ++k) {
-    if constexpr (sizeof(T) == 2)
-      v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[first + k] << 16);
-    else
-      v[k] = reinterpret_cast<const float*>(x)[first + k];
-    a = fmaxf(a, fabsf(v[k]));
-  }
-  const uint32_t s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
-  const float D = __fmul_rn(scale_value((int)s, FMT), g);
-  float q[4];
-  for (int k = 0; k < 4; ++k) q[k] = D > 0.0f ? __fdiv_rn(v[k], D) : __fmul_rn(v[k], 0.0f);
-  const uint32_t c = cvt_e2m1x8(q[0], q[1], q[2], q[3], 0.f, 0.f, 0.f, 0.f);
-  if constexpr (OUT != kCodes) {
-    for (int k = 0; k < 4; ++k) {
-      const float v = __fmul_rn(e2m1_to_float(c >> (4 * k)), D);  // exact
-      if constexpr (OUT == kRoundTripBf16)
-        reinterpret_cast<__nv_bfloat16*>(y)[first + k] = __float2bfloat16_rn(v);
+  for (int b0 = 0; b0 < count; b0 += N) {
+    const int64_t f = first + b0;
+    float v[8], a = 0.0f;
+    for (int k = 0; k < N; ++k) {
+      if constexpr (sizeof(T) == 2)
+        v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[f + k] << 16);
       else
-        reinterpret_cast<float*>(y)[first + k] = v;
+        v[k] = reinterpret_cast<const float*>(x)[f + k];
+      a = fmaxf(a, fabsf(v[k]));
     }
-    return;
+    const uint32_t s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
+    const float D = __fmul_rn(scale_value((int)s, FMT), g);
+    for (int k0 = 0; k0 < N; k0 += 2) {  // one byte (two codes) at a time
+      float q[2];
+      for (int k = 0; k < 2; ++k)
+        q[k] = D > 0.0f ? __fdiv_rn(v[k0 + k], D) : __fmul_rn(v[k0 + k], 0.0f);
+      const uint32_t c = cvt_e2m1x8(q[0], q[1], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xFF;
+      if constexpr (OUT != kCodes) {
+        for (int k = 0; k < 2; ++k) {
+          const float yv = __fmul_rn(e2m1_to_float(c >> (4 * k)), D);  // exact
+          if constexpr (OUT == kRoundTripBf16)
+            reinterpret_cast<__nv_bfloat16*>(y)[f + k0 + k] = __float2bfloat16_rn(yv);
+          else
+            reinterpret_cast<float*>(y)[f + k0 + k] = yv;
+        }
+      } else {
+        packed[(f + k0) / 2] = (uint8_t)c;
+      }
+    }
+    if constexpr (OUT == kCodes) scales[f / N] = (uint8_t)s;
   }
-  packed[first / 2] = (uint8_t)(c & 0xFF);
-  packed[first / 2 + 1] = (uint8_t)((c >> 8) & 0xFF);
-  scales[first / 4] = (uint8_t)s;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -350,9 +355,9 @@ static cudaError_t launch_q(const TensorArgs* ta, int count, cudaStream_t stream
   }
   for (int k = 0; k < count; ++k) {
     if (ta[k].numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
-      k_quantize_tail4<FMT, T, OUT><<<1, 32, 0, stream>>>(
-          (const T*)ta[k].x, nitems[k] * S::EPT, ta[k].g_bits, ta[k].packed, ta[k].scales,
-          ta[k].y);
+      k_quantize_tail<FMT, T, OUT><<<1, 32, 0, stream>>>(
+          (const T*)ta[k].x, nitems[k] * S::EPT, (int)(ta[k].numel % S::EPT), N, ta[k].g_bits,
+          ta[k].packed, ta[k].scales, ta[k].y);
       ++*launches;
     }
   }
@@ -373,23 +378,23 @@ static cudaError_t dispatch_block(int block, const TensorArgs* t, int count, cud
   }
 }
 
-cudaError_t run_quantize_tail4(const void* x, bool bf16, int64_t first, int fmt, uint16_t g_bits,
-                               uint8_t* packed, uint8_t* scales, cudaStream_t stream,
-                               int* launches) {
+cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,
+                              uint16_t g_bits, uint8_t* packed, uint8_t* scales,
+                              cudaStream_t stream, int* launches) {
   if (bf16) {
     if (fmt == kUE5M3)
-      k_quantize_tail4<kUE5M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, g_bits,
-                                                               packed, scales);
+      k_quantize_tail<kUE5M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, count, N,
+                                                              g_bits, packed, scales);
     else
-      k_quantize_tail4<kE4M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, g_bits,
-                                                              packed, scales);
+      k_quantize_tail<kE4M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, count, N,
+                                                             g_bits, packed, scales);
   } else {
     if (fmt == kUE5M3)
-      k_quantize_tail4<kUE5M3, float><<<1, 32, 0, stream>>>((const float*)x, first, g_bits, packed,
-                                                            scales);
+      k_quantize_tail<kUE5M3, float><<<1, 32, 0, stream>>>((const float*)x, first, count, N,
+                                                           g_bits, packed, scales);
     else
-      k_quantize_tail4<kE4M3, float><<<1, 32, 0, stream>>>((const float*)x, first, g_bits, packed,
-                                                           scales);
+      k_quantize_tail<kE4M3, float><<<1, 32, 0, stream>>>((const float*)x, first, count, N,
+                                                          g_bits, packed, scales);
   }
   ++*launches;
   return cudaGetLastError();

@@ -30,9 +30,9 @@ def test_workload1_fp32_full(cuda_device):
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_ragged_shapes_special_values(cuda_device, block, fmt, dtype):
-    # rows x cols chosen so the item count is not a multiple of a warp and, for N = 4, the element
-    # count is not a multiple of 8 (the tail path)
-    for i, (rows, k) in enumerate(((37, 5), (1, 1), (129, 3))):
+    # rows x cols chosen so the item count is not a multiple of a warp and, for N <= 8, the element
+    # count leaves 4, 8 or 12 elements after the last 16-element item (the tail paths)
+    for i, (rows, k) in enumerate(((37, 5), (1, 1), (129, 3), (5, 2))):
         cols = block * k
         g = G_CASES[i % len(G_CASES)]
         x = special_values_bf16(fmt, g, rows * cols, seed=block * 7 + fmt + i).to(dtype)
