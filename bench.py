@@ -36,7 +36,7 @@ L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) of one grouped fused-pass launch (5 tensors, N = 32, E4M3), from the
 # ncu capture summarised in profiles/k_error_stats_bf16_fused_group5_4096x4096_n32.md: every x is
 # read once, most of the codes and scales are still in L2 when the launch ends.
-FUSED_TRAFFIC_BYTES = 167830272 + 7129600
+FUSED_TRAFFIC_BYTES = 167829760 + 8332032
 
 
 def parse(argv=None):
