@@ -125,3 +125,20 @@ def global_scale(x, fmt):
     """Per-tensor FP16 scale bit pattern."""
     x, xt = _xarg(x)
     return lib.orc_global_scale(_ptr(x), xt, x.size, fmt)
+
+
+def matmul(a_packed, a_scales, a_g_bits, b_packed, b_scales, b_g_bits, m, n, k, block, fmt):
+    """C = dequant(A) dequant(B)^T in float64 (m x n), A m x k and B n x k in the library's layout.
+
+    The 4-bit float quantization article (gtnt.cn/news/16247, §3.1, the inference step that
+    dequantizes the stored weights before the matrix multiply) dequantizes, then multiplies.  Here both operands are stored block-quantized along k (the reduction dimension);
+    each is dequantized exactly (E2M1 x scale x g fits float32 exactly) and the product is one
+    float64 matrix multiply, whose rounding error (at most k 2^-53 relative to sum |a b|) is far
+    below any float32 accumulation.
+    """
+    ya = dequantize(a_packed, a_scales, m, k, block, fmt, a_g_bits, out_bf16=False)
+    yb = dequantize(b_packed, b_scales, n, k, block, fmt, b_g_bits, out_bf16=False)
+    A = ya.astype(np.float64).reshape(m, k)
+    B = yb.astype(np.float64).reshape(n, k)
+    return A @ B.T
+

@@ -1,0 +1,110 @@
+"""Pins of the oracle's block-scaled matrix product (dequantize both operands, then multiply).
+
+The oracle's product is tied to decoders outside it: E2M1 codes through ml_dtypes, E4M3 scales
+through torch.float8_e4m3fn, the global scales through numpy binary16, the nibble order and the
+scale indexing written out here, and exact rational sums on tiny cases.  Special cases reduce the
+product to a column selection and to a transpose.
+"""
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+E2M1 = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+E4M3 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def fp16(bits):
+    return float(np.array([bits], np.uint16).view(np.float16)[0])
+
+
+def decode(packed, scales, rows, cols, block, g_bits):
+    """Values of a stored operand: element 2i is the low nibble of byte i, element 2i+1 the
+    high nibble; block b of row r takes scales[r * cols / block + b]; everything times g."""
+    codes = np.empty(rows * cols, np.uint8)
+    codes[0::2] = packed & 0xF
+    codes[1::2] = packed >> 4
+    v = E2M1[codes].reshape(rows, cols)
+    s = E4M3[scales].reshape(rows, cols // block)
+    return v * np.repeat(s, block, axis=1) * fp16(g_bits)
+
+
+def random_operand(rng, rows, cols, block):
+    packed = rng.integers(0, 256, rows * cols // 2, dtype=np.uint8)
+    scales = rng.integers(0, 0x7F, rows * cols // block, dtype=np.uint8)  # every finite E4M3 code
+    return packed, scales
+
+
+def test_brute_force_exact_sums():
+    rng = np.random.default_rng(7)
+    m, n, k, block = 3, 2, 32, 16
+    ga, gb = 0x3C00, 0x3800  # 1.0 and 0.5
+    pa, sa = random_operand(rng, m, k, block)
+    pb, sb = random_operand(rng, n, k, block)
+    A = decode(pa, sa, m, k, block, ga)
+    B = decode(pb, sb, n, k, block, gb)
+    C = oracle.matmul(pa, sa, ga, pb, sb, gb, m, n, k, block, oracle.E4M3)
+    for i in range(m):
+        for j in range(n):
+            exact = sum(Fraction(float(A[i, t])) * Fraction(float(B[j, t])) for t in range(k))
+            mag = sum(abs(Fraction(float(A[i, t])) * Fraction(float(B[j, t]))) for t in range(k))
+            assert abs(Fraction(float(C[i, j])) - exact) <= mag * Fraction(1, 2 ** 48)
+
+
+@pytest.mark.parametrize("shape", [(17, 9, 64), (5, 33, 256)])
+def test_matches_independent_decode(shape):
+    rng = np.random.default_rng(sum(shape))
+    m, n, k = shape
+    pa, sa = random_operand(rng, m, k, 16)
+    pb, sb = random_operand(rng, n, k, 16)
+    ga, gb = 0x3C00, 0x4400  # 1.0, 4.0
+    C = oracle.matmul(pa, sa, ga, pb, sb, gb, m, n, k, 16, oracle.E4M3)
+    ref = decode(pa, sa, m, k, 16, ga) @ decode(pb, sb, n, k, 16, gb).T
+    mag = np.abs(decode(pa, sa, m, k, 16, ga)) @ np.abs(decode(pb, sb, n, k, 16, gb)).T
+    assert np.all(np.abs(C - ref) <= mag * 2.0 ** -45)
+
+
+def test_one_hot_columns_select_a():
+    # row j of B holds 1.0 (code 0x2, scale 0x38 = 1.0) at column j and +0 elsewhere, so column
+    # j of the product is column j of dequant(A)
+    rng = np.random.default_rng(3)
+    m, n, k = 9, 32, 64
+    pa, sa = random_operand(rng, m, k, 16)
+    codes = np.zeros((n, k), np.uint8)
+    codes[np.arange(n), np.arange(n)] = 0x2
+    flat = codes.reshape(-1)
+    pb = (flat[0::2] | (flat[1::2] << 4)).astype(np.uint8)
+    sb = np.full(n * k // 16, 0x38, np.uint8)
+    C = oracle.matmul(pa, sa, 0x3C00, pb, sb, 0x3C00, m, n, k, 16, oracle.E4M3)
+    A = decode(pa, sa, m, k, 16, 0x3C00)
+    assert np.array_equal(C, A[:, :n])
+
+
+def test_transpose_symmetry():
+    rng = np.random.default_rng(11)
+    m, n, k = 7, 12, 48
+    pa, sa = random_operand(rng, m, k, 16)
+    pb, sb = random_operand(rng, n, k, 16)
+    C = oracle.matmul(pa, sa, 0x3C00, pb, sb, 0x3A00, m, n, k, 16, oracle.E4M3)
+    Ct = oracle.matmul(pb, sb, 0x3A00, pa, sa, 0x3C00, n, m, k, 16, oracle.E4M3)
+    assert np.array_equal(C, Ct.T)
+
+
+def test_integer_sums_are_exact():
+    # scales 1.0 and g = 1: every value is a multiple of 0.5 with |v| <= 6, so every partial sum
+    # is a multiple of 0.25 below 2^24 and the product is exact in any order
+    rng = np.random.default_rng(5)
+    m, n, k = 8, 8, 256
+    pa = rng.integers(0, 256, m * k // 2, dtype=np.uint8)
+    pb = rng.integers(0, 256, n * k // 2, dtype=np.uint8)
+    s1 = np.full(m * k // 16, 0x38, np.uint8)
+    C = oracle.matmul(pa, s1, 0x3C00, pb, s1[: n * k // 16], 0x3C00, m, n, k, 16, oracle.E4M3)
+    A = decode(pa, s1, m, k, 16, 0x3C00)
+    B = decode(pb, s1[: n * k // 16], n, k, 16, 0x3C00)
+    exact = [[sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(A[i], B[j]))
+              for j in range(n)] for i in range(m)]
+    assert all(Fraction(float(C[i, j])) == exact[i][j] for i in range(m) for j in range(n))
