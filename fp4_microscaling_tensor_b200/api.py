@@ -1,9 +1,10 @@
-"""Python API over the C ABI: quantize, dequantize, error_stats, global_scale.
+"""Python API over the C ABI: quantize, dequantize, error_stats, global_scale, matmul.
 
 Tensors are CUDA tensors, contiguous, row-major, with blocks along the last dimension.  Outputs are
 allocated with torch on the tensor's device unless given.  Calls are asynchronous on the current
 torch stream (or `stream=`); nothing here synchronizes except ErrorStats.to_dict().
 """
+import ctypes
 import struct
 
 import numpy as np
@@ -308,6 +309,37 @@ def quantize_with_stats_group(xs, block=32, fmt="e4m3", g=None, packed=None, sca
                                       workspace.data_ptr(), workspace.numel(),
                                       _stream(stream, dev)), "mx_quantize_stats_group")
     return packed, scales, [ErrorStats(out[k]) for k in range(n)]
+
+
+def matmul(a_packed, a_scales, b_packed, b_scales, a_g=None, b_g=None, out_dtype=torch.bfloat16,
+           out=None, stream=None):
+    """C = dequant(A) dequant(B)^T on the tensor cores (block 16, E4M3 scales, as quantize writes
+    them): a_packed [m, k/2] / a_scales [m, k/16] of an m x k tensor, b_packed [n, k/2] /
+    b_scales [n, k/16] of an n x k tensor; returns C [m, n] of out_dtype."""
+    if out_dtype not in _DT:
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    for t, what in ((a_packed, "a_packed"), (a_scales, "a_scales"), (b_packed, "b_packed"),
+                    (b_scales, "b_scales")):
+        if t.dim() != 2:
+            raise ValueError(f"{what} must be 2-D")
+        _shape2d(t, what)
+    m, n, k = a_packed.shape[0], b_packed.shape[0], 2 * a_packed.shape[1]
+    if 2 * b_packed.shape[1] != k:
+        raise ValueError("A and B must have the same k")
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=a_packed.device)
+    check(lib.mx_matmul(a_packed.data_ptr(), a_scales.data_ptr(), g_bits(a_g), b_packed.data_ptr(),
+                        b_scales.data_ptr(), g_bits(b_g), m, n, k, 16, E4M3, out.data_ptr(),
+                        _DT[out.dtype], _stream(stream, a_packed.device)), "mx_matmul")
+    return out
+
+
+def matmul_gave_up():
+    """Number of matmul thread blocks whose bounded waits ran out since the last call (0 normally);
+    synchronizes the device."""
+    c = ctypes.c_uint(0)
+    check(lib.mx_matmul_gave_up(ctypes.byref(c)), "mx_matmul_gave_up")
+    return int(c.value)
 
 
 def kernel_launches():

@@ -2,6 +2,7 @@
 // launches of mx_quantize.cu, mx_dequantize.cu, mx_error_stats.cu and mx_global_scale.cu on the
 // caller's stream.  Nothing is allocated and nothing is synchronized here.
 #include <atomic>
+#include <cmath>
 
 #include "../../include/mx.h"
 #include "mx_device.cuh"
@@ -192,6 +193,45 @@ mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols
                                               workspace, stream, &n);
   g_launches += n;
   return from_cuda(e);
+}
+
+namespace {
+
+// Value of a finite binary16 bit pattern (exact in float).
+float half_value(uint16_t h) {
+  const int e = (h >> 10) & 31, m = h & 1023;
+  const float v = e == 0 ? std::ldexp((float)m, -24) : std::ldexp((float)(1024 + m), e - 25);
+  return (h & 0x8000u) ? -v : v;
+}
+
+}  // namespace
+
+mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
+                    const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g, int64_t m,
+                    int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c, mx_dtype ct,
+                    cudaStream_t stream) {
+  if (!valid_fmt(fmt) || !valid_dtype(ct) || !valid_g(a_g) || !valid_g(b_g)) return MX_ERR_INVALID_ARG;
+  if (m < 0 || n < 0 || k < 0 || m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) ||
+      k > (int64_t(1) << 40))
+    return MX_ERR_INVALID_ARG;
+  if (block != 16 || fmt != MX_SCALE_E4M3 || k == 0 || k % 256 != 0) return MX_ERR_UNSUPPORTED;
+  if (m == 0 || n == 0) return MX_OK;
+  if (!a_packed || !a_scales || !b_packed || !b_scales || !c) return MX_ERR_INVALID_ARG;
+  if (!aligned16(a_packed) || !aligned16(a_scales) || !aligned16(b_packed) ||
+      !aligned16(b_scales) || !aligned16(c))
+    return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
+  int launches = 0;
+  const cudaError_t e = mxk::run_matmul_nvfp4(a_packed, a_scales, b_packed, b_scales, m, n, k,
+                                              half_value(a_g) * half_value(b_g), c, ct == MX_BF16,
+                                              stream, &launches);
+  g_launches += launches;
+  return from_cuda(e);
+}
+
+mx_status mx_matmul_gave_up(unsigned int* count) {
+  if (!count) return MX_ERR_INVALID_ARG;
+  return from_cuda(mxk::matmul_gave_up(count));
 }
 
 namespace {

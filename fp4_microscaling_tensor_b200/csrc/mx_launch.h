@@ -163,6 +163,15 @@ cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count
 // kernel launched with programmatic serialization).
 cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches);
 
+// C (m x n, fp32 or bf16) = alpha * dequant(A) dequant(B)^T for A (m x k) and B (n x k) stored
+// with blocks of 16 along k and E4M3 scales; k a positive multiple of 256.
+cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
+                             const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
+                             int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
+                             cudaStream_t stream, int* launches);
+// Reads and clears the count of matmul CTAs whose bounded waits ran out (synchronizes).
+cudaError_t matmul_gave_up(unsigned int* count);
+
 cudaError_t run_global_scale(const void* x, bool bf16, int64_t numel, int fmt, uint16_t* out,
                              void* workspace, cudaStream_t stream, int* launches);
 

@@ -1,0 +1,411 @@
+// mx_matmul.cu -- C = gA gB * dequant(A) dequant(B)^T on the fifth-generation tensor cores.
+//
+// Method: the 4-bit float quantization article (gtnt.cn/news/16247) §3.1 runs inference by
+// dequantizing stored FP4 weights and multiplying; here both operands are stored by this library
+// (E2M1 codes, two per byte, low nibble first; one E4M3 scale per block of 16 along the reduction
+// dimension k; an FP16 global scale per operand) and the tensor core applies the block scales
+// inside the multiply (tcgen05.mma kind::mxf4nvf4, block16, E4M3 scales), so nothing is
+// dequantized to memory.  A is m x k and B is n x k, both row-major with k contiguous ("K-major"),
+// which is the layout the quantizer writes; C is m x n row-major, float32 or bfloat16.
+//
+// One CTA per 128 x 128 tile of C, 4 warps:
+//   * warp 0 produces: for each 256-element step of k, one TMA load per operand (128 rows x 128
+//     bytes, 128-byte swizzle) and the 128 x 16 scale bytes of each operand, which the 32 lanes
+//     load with plain 16-byte loads and store into the 512-byte scale atoms the scale-copy
+//     instruction expects (row r of a 128-row tile at byte 16 (r % 32) + 4 (r / 32) + j for the
+//     four scales j of one 64-element MMA step);
+//   * warp 1, one thread, issues per step 8 tcgen05.cp (scale atoms -> TMEM) and 4 tcgen05.mma
+//     (128 x 128 x 64 each, fp32 accumulator in TMEM), then a tcgen05.commit that frees the stage;
+//   * all 4 warps then read the accumulator (tcgen05.ld, one row per thread), multiply by gA gB
+//     and store C.
+// Stages are handed over with mbarriers (full: TMA bytes + 32 producer arrivals; empty: the
+// commit).  Every wait is bounded: a CTA that gives up records it in a device counter, lets its
+// issued copies and MMAs finish (bounded again), frees its TMEM and returns.
+#include <cuda.h>
+
+#include "mx_device.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+namespace {
+
+constexpr int kBM = 128, kBN = 128;   // C tile
+constexpr int kBK = 256;              // k elements per stage (128 bytes of codes per row)
+constexpr int kRowBytes = kBK / 2;
+constexpr int kStages = 5;
+constexpr int kABytes = kBM * kRowBytes;          // 16 KiB
+constexpr int kBBytes = kBN * kRowBytes;          // 16 KiB
+constexpr int kSfBytes = kBM * (kBK / 16);        // 2 KiB: four 512-byte atoms
+constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;  // + barriers, + alignment slack
+constexpr uint32_t kTmemCols = 256;   // accumulator 128 columns, scales 2 x 16 columns
+constexpr uint32_t kSfaCol = 128, kSfbCol = 144;
+constexpr uint32_t kWaitLimit = 1u << 20;  // polls of one mbarrier before a CTA gives up
+
+// Instruction descriptor of kind::mxf4nvf4 (block-scaled): A and B E2M1 (format 1), K-major,
+// E4M3 scales (scale format 0), N = 128 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16),
+// scale-factor ids 0, dense, K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+__device__ unsigned int g_mm_gave_up;     // CTAs that stopped waiting (bounded waits ran out)
+__device__ volatile int g_mm_abandon;     // set by a CTA that gave up: the others stop waiting too
+
+struct MmArgs {
+  const uint8_t* a_scales;
+  const uint8_t* b_scales;
+  void* c;
+  int64_t m, n, k;
+  float alpha;
+  int c_bf16;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// True once the phase with the given parity has completed; false after kWaitLimit polls, or
+// earlier once another CTA has given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if ((i & 1023u) == 1023u && g_mm_abandon) return false;
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand with 128-byte swizzle: rows of 128 bytes,
+// 8-row groups 1024 bytes apart (stride byte offset), version 1, layout type 2.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Descriptor of one 512-byte scale atom for tcgen05.cp: 32 rows of 16 bytes, no swizzle, 8-row
+// groups 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(128 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+
+__device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// 32 consecutive accumulator columns of this warp's 32 lanes (one row per thread).
+__device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// The 128 x 16 scale bytes of one stage (rows r0 .. r0 + 127, k step kt) into four atoms:
+// lane l loads rows r0 + l + 32 q (q = 0..3) and writes, for each MMA step j, the 16 bytes
+// {row l word j, row l + 32 word j, row l + 64 word j, row l + 96 word j} at atom j + 16 l.
+// Rows past the end give zero scales.
+__device__ __forceinline__ void stage_scales(const uint8_t* __restrict__ scales, int64_t rows,
+                                             int64_t r0, int64_t pitch, int kt, uint8_t* atoms,
+                                             int lane) {
+  uint4 v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int64_t r = r0 + 32 * q + lane;
+    v[q] = r < rows ? __ldg(reinterpret_cast<const uint4*>(scales + r * pitch + (int64_t)kt * 16))
+                    : make_uint4(0, 0, 0, 0);
+  }
+  const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w},
+                            {v[1].x, v[1].y, v[1].z, v[1].w},
+                            {v[2].x, v[2].y, v[2].z, v[2].w},
+                            {v[3].x, v[3].y, v[3].z, v[3].w}};
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(atoms + 512 * j + 16 * lane) =
+        make_uint4(w[0][j], w[1][j], w[2][j], w[3][j]);
+}
+
+__global__ void __launch_bounds__(128, 1)
+    k_matmul_nvfp4(const __grid_constant__ CUtensorMap tma_a,
+                   const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ MmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* gave_up = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * kBN;
+  const int KT = (int)(args.k / kBK);
+  const int64_t pitch = args.k / 16;  // scale bytes per row
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(full + s), 32);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *gave_up = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    int issued = 0;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % kStages;
+      bool ok = true;  // lane 0 waits; the warp follows its answer
+      if (lane == 0) {
+        ok = !*gave_up &&
+             (kt < kStages || mbar_wait(smem_u32(empty + s), ((kt / kStages) + 1) & 1));
+        if (!ok) *gave_up = 1;
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      uint8_t* st = smem + s * kStageBytes;
+      const uint32_t bar = smem_u32(full + s);
+      if (lane == 0) {
+        mbar_expect_tx(bar, kABytes + kBBytes);
+        tma_load_2d(smem_u32(st), &tma_a, kt * kRowBytes, (int)m0, bar);
+        tma_load_2d(smem_u32(st + kABytes), &tma_b, kt * kRowBytes, (int)n0, bar);
+      }
+      stage_scales(args.a_scales, args.m, m0, pitch, kt, st + kABytes + kBBytes, lane);
+      stage_scales(args.b_scales, args.n, n0, pitch, kt, st + kABytes + kBBytes + kSfBytes, lane);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar);
+      issued = kt + 1;
+    }
+    if (lane == 0 && *gave_up) {
+      // let the loads already issued land before the CTA can exit (bounded)
+      for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt)
+        mbar_wait(smem_u32(full + kt % kStages), (kt / kStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1)) {
+          *gave_up = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes);
+        const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfBytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tc_copy_sf(tmem + kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
+          tc_copy_sf(tmem + kSfbCol + 4 * j, desc_sf(sfb + 512 * j));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j),
+                 tmem + kSfaCol + 4 * j, tmem + kSfbCol + 4 * j, (kt | j) != 0);
+        tc_commit(smem_u32(empty + s));
+      }
+      tc_commit(smem_u32(done));  // also after giving up: the epilogue waits for issued MMAs
+    }
+    __syncwarp();
+  }
+
+  // ---------------- epilogue: all 4 warps, one accumulator row per thread ----------------
+  __syncwarp();
+  bool ok = true;
+  if (lane == 0) {
+    ok = mbar_wait(smem_u32(done), 0);
+    if (!ok) *gave_up = 1;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  tc_fence_after();
+  if (__all_sync(0xffffffffu, ok && !*gave_up)) {
+    const int64_t row = m0 + 32 * warp + lane;
+    const bool row_ok = row < args.m;
+#pragma unroll 1
+    for (int cb = 0; cb < kBN / 32; ++cb) {
+      uint32_t r[32];
+      tc_load32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cb, r);
+      const int64_t col = n0 + 32 * cb;
+      if (!row_ok || col >= args.n) continue;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), args.alpha);
+      const bool whole = col + 32 <= args.n;
+      if (args.c_bf16) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + row * args.n + col;
+        if (whole && (args.n % 8) == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(v[i], v[i + 1]);
+            pk.y = pack_bf16x2(v[i + 2], v[i + 3]);
+            pk.z = pack_bf16x2(v[i + 4], v[i + 5]);
+            pk.w = pack_bf16x2(v[i + 6], v[i + 7]);
+            *reinterpret_cast<uint4*>(out + i) = pk;
+          }
+        } else {
+          for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = __float2bfloat16_rn(v[i]);
+        }
+      } else {
+        float* out = static_cast<float*>(args.c) + row * args.n + col;
+        if (whole && (args.n % 4) == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+          for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = v[i];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *gave_up) {
+    atomicAdd(&g_mm_gave_up, 1u);
+    g_mm_abandon = 1;
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiled>(nullptr);
+    return reinterpret_cast<EncodeTiled>(p);
+  }();
+  return fn;
+}
+
+// Map of one operand's codes: rows x (k / 2) bytes, row pitch k / 2, boxes of 128 x 128 bytes
+// loaded with the 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k) {
+  const EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)kBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
+                             const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
+                             int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
+                             cudaStream_t stream, int* launches) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        k_matmul_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a_packed, m, k) || !make_map(&mb, b_packed, n, k))
+    return cudaErrorInvalidValue;
+  MmArgs args{a_scales, b_scales, c, m, n, k, alpha, c_bf16 ? 1 : 0};
+  const dim3 grid((unsigned)((n + kBN - 1) / kBN), (unsigned)((m + kBM - 1) / kBM));
+  k_matmul_nvfp4<<<grid, 128, kSmemBytes, stream>>>(ma, mb, args);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t matmul_gave_up(unsigned int* count) {
+  const unsigned int zero = 0;
+  const int izero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_mm_gave_up, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_mm_gave_up, &zero, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_mm_abandon, &izero, sizeof(int));
+  return e;
+}
+
+}  // namespace mxk

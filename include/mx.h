@@ -198,6 +198,30 @@ MX_API mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, 
                                          int block, mx_scale_fmt fmt, void* workspace,
                                          size_t ws_bytes, cudaStream_t stream);
 
+/* ---- Block-scaled matrix product on the tensor cores.
+ * C = dequant(A) * dequant(B)^T, the dequantize-then-multiply step of inference in the 4-bit float
+ * quantization article (gtnt.cn/news/16247, §3.1), with both operands stored by mx_quantize and
+ * the block scales applied inside the tensor-core multiply (nothing is dequantized to memory):
+ *   - A is m x k (a_packed: m*k/2 bytes, a_scales: m*k/16 bytes), B is n x k (likewise), both
+ *     quantized with block = 16 along k and fmt = MX_SCALE_E4M3, exactly as mx_quantize writes
+ *     a row-major m x k (n x k) tensor; a_g / b_g are the global scales they were quantized with;
+ *   - C is m x n, row-major, float32 (ct = MX_F32) or bfloat16 (MX_BF16, rounded to nearest even):
+ *     C[i][j] = a_g b_g sum_t E2M1(A[i][t]) S(A)[i][t/16] E2M1(B[j][t]) S(B)[j][t/16], accumulated
+ *     in float32 by the tensor core (any order), then multiplied by a_g b_g (one rounding);
+ *   - block != 16 or fmt != MX_SCALE_E4M3 (no native tensor-core form), k == 0 or k % 256 != 0:
+ *     MX_ERR_UNSUPPORTED; m, n or k negative, or m, n >= 2^31: MX_ERR_INVALID_ARG; m == 0 or
+ *     n == 0: nothing is enqueued.
+ * Every wait inside the kernel is bounded; a launch whose waits ran out leaves C unspecified and
+ * is counted by mx_matmul_gave_up. */
+MX_API mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
+                           const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g,
+                           int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c,
+                           mx_dtype ct, cudaStream_t stream);
+
+/* Number of mx_matmul thread blocks that stopped waiting since the previous call (0 in normal
+ * operation), written to *count (host memory); clears the count.  Synchronizes the device. */
+MX_API mx_status mx_matmul_gave_up(unsigned int* count);
+
 /* Test hook for error paths (no counterpart in the pages).  The next `count` calls that pass
  * their argument checks and would enqueue work return MX_ERR_CUDA instead, as a failed launch is
  * reported, without enqueueing anything or touching any buffer.  count <= 0 disarms the hook.

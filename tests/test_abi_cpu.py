@@ -191,6 +191,31 @@ def test_fake_quantize_rejects_bad_arguments():
     assert fq(rows=0, x=None, y=None) == OK      # empty: nothing to do
 
 
+def test_matmul_rejects_bad_arguments():
+    def mm(ap=A, as_=A, ag=0x3C00, bp=A, bs=A, bg=0x3C00, m=128, n=64, k=256, block=16, fmt=E4,
+           c=A, ct=BF16):
+        return L.mx_matmul(ap, as_, ag, bp, bs, bg, m, n, k, block, fmt, c, ct, None)
+    assert mm(block=32) == UNS                   # no native tensor-core form
+    assert mm(fmt=1) == UNS                      # UE5M3 scales
+    assert mm(k=128) == UNS                      # k % 256 != 0
+    assert mm(k=0) == UNS
+    assert mm(fmt=5) == INV
+    assert mm(ct=4) == INV
+    assert mm(ag=0x7C00) == INV                  # g must be finite and positive
+    assert mm(bg=0x8000) == INV
+    assert mm(m=-1) == INV
+    assert mm(n=1 << 31) == INV
+    assert mm(ap=None) == INV
+    assert mm(bs=None) == INV
+    assert mm(c=None) == INV
+    assert mm(ap=A + 8) == MIS
+    assert mm(bs=A + 4) == MIS
+    assert mm(c=A + 2) == MIS
+    assert mm(m=0, ap=None, as_=None, c=None) == OK   # empty product: nothing to do
+    assert mm(n=0) == OK
+    assert L.mx_matmul_gave_up(None) == INV
+
+
 def test_injected_cuda_failure_is_reported_before_any_launch():
     # valid arguments on fake pointers: the armed failures are consumed before anything is
     # enqueued, so nothing touches the (fake) buffers; the status is MX_ERR_CUDA
