@@ -50,7 +50,10 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     # single-kernel timing / profiling case (not the benchmark line)
     ap.add_argument("--case", choices=["quantize", "dequantize", "stats", "stats-recompute",
-                                       "quantize-stats", "global-scale", "fake-quantize"])
+                                       "quantize-stats", "global-scale", "fake-quantize",
+                                       "matmul"])
+    ap.add_argument("--mnk", type=int, nargs=3, default=[8192, 8192, 8192],
+                    help="m n k of --case matmul")
     ap.add_argument("--shape", type=int, nargs=2, default=[16384, 8192])
     ap.add_argument("--block", type=int, default=32)
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
@@ -535,6 +538,63 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+def measured_tensor_peak():
+    """Dense FP4 tensor-core peak in TFLOP/s: the measured bf16 GEMM burst figure times the nominal
+    FP4 : BF16 ratio of B200 (9 : 2.25)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]) * 4.0, "measured bf16 x 4 (nominal ratio)"
+    except Exception:
+        return 1590.0 * 4.0, "fallback bf16 x 4 (nominal ratio)"
+
+
+def run_matmul_case(args):
+    """Time mx_matmul (C = dequant(A) dequant(B)^T, block 16, E4M3 scales, bf16 out) on random
+    codes and scales, L2 flushed before each launch; TFLOP/s = 2 m n k / median time."""
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    m, n, k = args.mnk
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(4096)
+    a = torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device=dev, generator=g)
+    b = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=g)
+    sa = torch.randint(0x28, 0x48, (m, k // 16), dtype=torch.uint8, device=dev, generator=g)
+    sb = torch.randint(0x28, 0x48, (n, k // 16), dtype=torch.uint8, device=dev, generator=g)
+    c = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    pa, pb = mx.prepare_scales(sa, k), mx.prepare_scales(sb, k)
+    fn = lambda: mx.matmul(a, pa, b, pb, out=c, prepared=True)  # noqa: E731
+    fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    prep = []  # the activation's scale reordering, timed alone (weights are prepared once)
+    for _ in range(args.reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mx.prepare_scales(sa, k, out=pa)
+        e1.record()
+        torch.cuda.synchronize()
+        prep.append(e0.elapsed_time(e1) / 1e3)
+    peak, kind = measured_tensor_peak()
+    tflops = 2.0 * m * n * k / t / 1e12
+    print(json.dumps({"case": "matmul", "mnk": [m, n, k], "median_us": t * 1e6, "tflops": tflops,
+                      "prepare_a_scales_us": statistics.median(prep) * 1e6,
+                      "frac": tflops / peak, "peak_tflops": peak, "peak_kind": kind,
+                      "gave_up": mx.matmul_gave_up(), "reps": args.reps}), flush=True)
+
+
 def run_case(args):
     """Time one kernel (or, with --group G, one grouped launch over G tensors) on bf16 tensors
     N(0, 0.02^2): CUDA events around each launch, L2 flushed before each launch by writing a 256 MB
@@ -599,6 +659,9 @@ def run_case(args):
 
 def main():
     args = parse()
+    if args.case == "matmul":
+        run_matmul_case(args)
+        return
     if args.case:
         run_case(args)
         return

@@ -7,6 +7,6 @@ thin binding over it; importing it fails when the library is missing.
 """
 from .api import (E4M3, MX_MAX_GROUP, UE5M3, ErrorStats, FakeQuantize, MXError,  # noqa: F401
                   dequantize, dequantize_group, error_stats, fake_quantize, fmt_code, g_bits,
-                  global_scale, kernel_launches, matmul, matmul_gave_up,
+                  global_scale, kernel_launches, matmul, matmul_gave_up, prepare_scales,
                   quantize, quantize_group, quantize_with_stats, quantize_with_stats_group,
                   stats_workspace)

@@ -28,7 +28,8 @@ EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_
            "mx_quantize_stats",
            "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
            "mx_quantize_group", "mx_dequantize_group", "mx_quantize_stats_group",
-           "mx_fake_quantize", "mx_matmul", "mx_matmul_gave_up", "mx_test_fail_next_calls",
+           "mx_fake_quantize", "mx_matmul_scales_size", "mx_matmul_prepare_scales",
+           "mx_matmul", "mx_matmul_gave_up", "mx_test_fail_next_calls",
            "mx_status_string", "mx_kernel_launches")
 MX_MAX_GROUP = 16
 
@@ -74,6 +75,10 @@ lib.mx_quantize_stats_group.restype = _i
 lib.mx_quantize_stats_group.argtypes = [_tp, _i, _i, _i, _i, _vp, _sz, _vp]
 lib.mx_matmul.restype = _i
 lib.mx_matmul.argtypes = [_vp, _vp, _u16, _vp, _vp, _u16, _i64, _i64, _i64, _i, _i, _vp, _i, _vp]
+lib.mx_matmul_scales_size.restype = _sz
+lib.mx_matmul_scales_size.argtypes = [_i64, _i64]
+lib.mx_matmul_prepare_scales.restype = _i
+lib.mx_matmul_prepare_scales.argtypes = [_vp, _i64, _i64, _vp, _sz, _vp]
 lib.mx_matmul_gave_up.restype = _i
 lib.mx_matmul_gave_up.argtypes = [ctypes.POINTER(ctypes.c_uint)]
 lib.mx_status_string.restype = ctypes.c_char_p

@@ -311,21 +311,39 @@ def quantize_with_stats_group(xs, block=32, fmt="e4m3", g=None, packed=None, sca
     return packed, scales, [ErrorStats(out[k]) for k in range(n)]
 
 
+def prepare_scales(scales, k, out=None, stream=None):
+    """Scales of a rows x k operand (uint8 [rows, k/16], block 16) in tensor-core order for
+    matmul; returns a uint8 tensor of mx_matmul_scales_size(rows, k) bytes."""
+    rows = scales.shape[0] if scales.dim() == 2 else 0
+    _shape2d(scales, "scales")
+    size = int(lib.mx_matmul_scales_size(rows, int(k)))
+    if size == 0 and rows:
+        raise ValueError("k must be a positive multiple of 256")
+    if out is None:
+        out = torch.empty(max(size, 16), dtype=torch.uint8, device=scales.device)
+    check(lib.mx_matmul_prepare_scales(scales.data_ptr(), rows, int(k), out.data_ptr(), out.numel(),
+                                       _stream(stream, scales.device)), "mx_matmul_prepare_scales")
+    return out
+
+
 def matmul(a_packed, a_scales, b_packed, b_scales, a_g=None, b_g=None, out_dtype=torch.bfloat16,
-           out=None, stream=None):
+           out=None, prepared=False, stream=None):
     """C = dequant(A) dequant(B)^T on the tensor cores (block 16, E4M3 scales, as quantize writes
-    them): a_packed [m, k/2] / a_scales [m, k/16] of an m x k tensor, b_packed [n, k/2] /
-    b_scales [n, k/16] of an n x k tensor; returns C [m, n] of out_dtype."""
+    them): a_packed [m, k/2] of an m x k tensor, b_packed [n, k/2] of an n x k tensor; a_scales /
+    b_scales are the quantizer's [rows, k/16] arrays, or (prepared=True) the outputs of
+    prepare_scales.  Returns C [m, n] of out_dtype."""
     if out_dtype not in _DT:
         raise ValueError("out_dtype must be float32 or bfloat16")
-    for t, what in ((a_packed, "a_packed"), (a_scales, "a_scales"), (b_packed, "b_packed"),
-                    (b_scales, "b_scales")):
+    for t, what in ((a_packed, "a_packed"), (b_packed, "b_packed")):
         if t.dim() != 2:
             raise ValueError(f"{what} must be 2-D")
         _shape2d(t, what)
     m, n, k = a_packed.shape[0], b_packed.shape[0], 2 * a_packed.shape[1]
     if 2 * b_packed.shape[1] != k:
         raise ValueError("A and B must have the same k")
+    if not prepared and m and n:
+        a_scales = prepare_scales(a_scales, k, stream=stream)
+        b_scales = prepare_scales(b_scales, k, stream=stream)
     if out is None:
         out = torch.empty((m, n), dtype=out_dtype, device=a_packed.device)
     check(lib.mx_matmul(a_packed.data_ptr(), a_scales.data_ptr(), g_bits(a_g), b_packed.data_ptr(),

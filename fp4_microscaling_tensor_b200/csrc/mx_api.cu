@@ -229,6 +229,28 @@ mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a
   return from_cuda(e);
 }
 
+size_t mx_matmul_scales_size(int64_t rows, int64_t k) {
+  if (rows < 0 || rows >= (int64_t(1) << 31) || k <= 0 || k % 256 != 0 || k > (int64_t(1) << 40))
+    return 0;
+  return (size_t)mxk::mma_scales_bytes(rows, k);
+}
+
+mx_status mx_matmul_prepare_scales(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out,
+                                   size_t out_bytes, cudaStream_t stream) {
+  if (rows < 0 || rows >= (int64_t(1) << 31) || k < 0 || k > (int64_t(1) << 40))
+    return MX_ERR_INVALID_ARG;
+  if (k == 0 || k % 256 != 0) return MX_ERR_UNSUPPORTED;
+  if (rows == 0) return MX_OK;
+  if (!scales || !out) return MX_ERR_INVALID_ARG;
+  if (out_bytes < mx_matmul_scales_size(rows, k)) return MX_ERR_WORKSPACE;
+  if (!aligned16(scales) || !aligned16(out)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
+  int launches = 0;
+  const cudaError_t e = mxk::run_scales_to_mma(scales, rows, k, out, stream, &launches);
+  g_launches += launches;
+  return from_cuda(e);
+}
+
 mx_status mx_matmul_gave_up(unsigned int* count) {
   if (!count) return MX_ERR_INVALID_ARG;
   return from_cuda(mxk::matmul_gave_up(count));

@@ -164,11 +164,16 @@ cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count
 cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches);
 
 // C (m x n, fp32 or bf16) = alpha * dequant(A) dequant(B)^T for A (m x k) and B (n x k) stored
-// with blocks of 16 along k and E4M3 scales; k a positive multiple of 256.
+// with blocks of 16 along k and E4M3 scales; k a positive multiple of 256; scales in the
+// tensor-core order written by run_scales_to_mma.
 cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
                              cudaStream_t stream, int* launches);
+// Bytes of an operand's scales in tensor-core order, and the reordering kernel.
+int64_t mma_scales_bytes(int64_t rows, int64_t k);
+cudaError_t run_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out,
+                              cudaStream_t stream, int* launches);
 // Reads and clears the count of matmul CTAs whose bounded waits ran out (synchronizes).
 cudaError_t matmul_gave_up(unsigned int* count);
 

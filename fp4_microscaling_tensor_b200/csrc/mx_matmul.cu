@@ -8,18 +8,18 @@
 // dequantized to memory.  A is m x k and B is n x k, both row-major with k contiguous ("K-major"),
 // which is the layout the quantizer writes; C is m x n row-major, float32 or bfloat16.
 //
-// One CTA per 128 x 128 tile of C, 4 warps:
+// One CTA per 128 x BN tile of C (BN = 256 by default, MMA N = BN), 4 warps:
 //   * warp 0 produces: for each 256-element step of k, one TMA load per operand (128 rows x 128
 //     bytes, 128-byte swizzle) and the 128 x 16 scale bytes of each operand, which the 32 lanes
-//     load with plain 16-byte loads and store into the 512-byte scale atoms the scale-copy
+//     copy asynchronously (cp.async, 4 bytes each) into the 512-byte scale atoms the scale-copy
 //     instruction expects (row r of a 128-row tile at byte 16 (r % 32) + 4 (r / 32) + j for the
 //     four scales j of one 64-element MMA step);
 //   * warp 1, one thread, issues per step 8 tcgen05.cp (scale atoms -> TMEM) and 4 tcgen05.mma
-//     (128 x 128 x 64 each, fp32 accumulator in TMEM), then a tcgen05.commit that frees the stage;
+//     (128 x BN x 64 each, fp32 accumulator in TMEM), then a tcgen05.commit that frees the stage;
 //   * all 4 warps then read the accumulator (tcgen05.ld, one row per thread), multiply by gA gB
 //     and store C.
-// Stages are handed over with mbarriers (full: TMA bytes + 32 producer arrivals; empty: the
-// commit).  Every wait is bounded: a CTA that gives up records it in a device counter, lets its
+// Stages are handed over with mbarriers (full: TMA bytes + one arrival per producer lane when its
+// scale copies land; empty: the commit).  Every wait is bounded: a CTA that gives up records it in a device counter, lets its
 // issued copies and MMAs finish (bounded again), frees its TMEM and returns.
 #include <cuda.h>
 
@@ -29,25 +29,38 @@
 namespace mxk {
 namespace {
 
-constexpr int kBM = 128, kBN = 128;   // C tile
+#ifndef MX_MM_BN  // columns of C per CTA: 128 or 256 (MMA N)
+#define MX_MM_BN 256
+#endif
+
+constexpr int kBM = 128;              // rows of C per CTA (MMA M)
 constexpr int kBK = 256;              // k elements per stage (128 bytes of codes per row)
 constexpr int kRowBytes = kBK / 2;
-constexpr int kStages = 5;
-constexpr int kABytes = kBM * kRowBytes;          // 16 KiB
-constexpr int kBBytes = kBN * kRowBytes;          // 16 KiB
-constexpr int kSfBytes = kBM * (kBK / 16);        // 2 KiB: four 512-byte atoms
-constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
-static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
-constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t kTmemCols = 256;   // accumulator 128 columns, scales 2 x 16 columns
-constexpr uint32_t kSfaCol = 128, kSfbCol = 144;
 constexpr uint32_t kWaitLimit = 1u << 20;  // polls of one mbarrier before a CTA gives up
 
-// Instruction descriptor of kind::mxf4nvf4 (block-scaled): A and B E2M1 (format 1), K-major,
-// E4M3 scales (scale format 0), N = 128 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16),
-// scale-factor ids 0, dense, K = 64.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+// Tile geometry for BN columns of C per CTA.
+template <int BN>
+struct Tile {
+  static constexpr int kHalves = BN / 128;                     // 128-row scale atoms of B per step
+  static constexpr int kStages = BN == 256 ? 4 : 5;
+  static constexpr int kABytes = kBM * kRowBytes;             // 16 KiB
+  static constexpr int kBBytes = BN * kRowBytes;              // 16 or 32 KiB
+  static constexpr int kSfaBytes = kBM * (kBK / 16);          // four 512-byte atoms
+  static constexpr int kSfbBytes = BN * (kBK / 16);           // 4 x kHalves atoms
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;  // + barriers, alignment
+  // TMEM: accumulator BN columns, then A's scales (4 per MMA step), then B's (4 kHalves per step);
+  // column w of a step's scales serves rows 32 w .. 32 w + 31 of its operand tile.
+  static constexpr uint32_t kSfaCol = BN, kSfbCol = BN + 16;
+  static constexpr uint32_t kTmemCols = BN == 256 ? 512 : 256;
+  static_assert(kSfbCol + 16 * kHalves <= kTmemCols, "TMEM columns");
+  // Instruction descriptor of kind::mxf4nvf4 (block-scaled): A and B E2M1 (format 1), K-major,
+  // E4M3 scales (scale format 0), N = BN (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16),
+  // scale-factor ids 0, dense, K = 64.
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((uint32_t)(kBM >> 4) << 24);
+};
 
 __device__ unsigned int g_mm_gave_up;     // CTAs that stopped waiting (bounded waits ran out)
 __device__ volatile int g_mm_abandon;     // set by a CTA that gave up: the others stop waiting too
@@ -68,18 +81,21 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 // True once the phase with the given parity has completed; false after kWaitLimit polls, or
-// earlier once another CTA has given up.
+// earlier once another CTA has given up.  SLEEP_NS > 0 sleeps between polls: waits off the
+// critical path must not flood the shared-memory pipe that the TMA and the tensor core use.
+template <int SLEEP_NS = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
     if ((i & 1023u) == 1023u && g_mm_abandon) return false;
+    if (SLEEP_NS > 0 && i > 0) __nanosleep(SLEEP_NS);
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -126,14 +142,14 @@ __device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t desc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
                : "memory");
 }
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
-                                       uint32_t sfb, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
       "p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -158,33 +174,55 @@ __device__ __forceinline__ void tc_load32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// The 128 x 16 scale bytes of one stage (rows r0 .. r0 + 127, k step kt) into four atoms:
-// lane l loads rows r0 + l + 32 q (q = 0..3) and writes, for each MMA step j, the 16 bytes
-// {row l word j, row l + 32 word j, row l + 64 word j, row l + 96 word j} at atom j + 16 l.
-// Rows past the end give zero scales.
-__device__ __forceinline__ void stage_scales(const uint8_t* __restrict__ scales, int64_t rows,
-                                             int64_t r0, int64_t pitch, int kt, uint8_t* atoms,
-                                             int lane) {
-  uint4 v[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t r = r0 + 32 * q + lane;
-    v[q] = r < rows ? __ldg(reinterpret_cast<const uint4*>(scales + r * pitch + (int64_t)kt * 16))
-                    : make_uint4(0, 0, 0, 0);
-  }
-  const uint32_t w[4][4] = {{v[0].x, v[0].y, v[0].z, v[0].w},
-                            {v[1].x, v[1].y, v[1].z, v[1].w},
-                            {v[2].x, v[2].y, v[2].z, v[2].w},
-                            {v[3].x, v[3].y, v[3].z, v[3].w}};
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4*>(atoms + 512 * j + 16 * lane) =
-        make_uint4(w[0][j], w[1][j], w[2][j], w[3][j]);
+// One contiguous block of global memory into shared memory (bulk copy engine), completing on bar.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
+// Scale bytes in tensor-core order: for each 128-row tile t of an operand and each 256-element
+// step kt of k, 2048 contiguous bytes = four 512-byte atoms (one per 64-element MMA step j); in
+// atom j, row 32 q + r of the tile has its four scales at byte 16 r + 4 q.  The tile count is
+// rounded up to even (a 256-column tile of C reads two), and rows past the end of the operand
+// give zero scales.  One thread per (t, kt, r) reads the 16 scale bytes of rows 32 q + r
+// (q = 0..3) and writes 16 bytes to each atom.
+__global__ void k_scales_to_mma(const uint8_t* __restrict__ scales, int64_t rows, int64_t k,
+                                uint8_t* __restrict__ out) {
+  const int64_t KT = k / kBK, pitch = k / 16;
+  const int64_t tiles = 2 * ((rows + 2 * kBM - 1) / (2 * kBM));
+  const int64_t total = tiles * KT * 32;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i & 31);
+    const int64_t tk = i >> 5, t = tk / KT, kt = tk - t * KT;
+    uint4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t row = t * kBM + 32 * q + r;
+      v[q] = row < rows ? __ldg(reinterpret_cast<const uint4*>(scales + row * pitch + kt * 16))
+                        : make_uint4(0, 0, 0, 0);
+    }
+    uint8_t* dst = out + tk * 2048 + 16 * r;
+    *reinterpret_cast<uint4*>(dst + 0) = make_uint4(v[0].x, v[1].x, v[2].x, v[3].x);
+    *reinterpret_cast<uint4*>(dst + 512) = make_uint4(v[0].y, v[1].y, v[2].y, v[3].y);
+    *reinterpret_cast<uint4*>(dst + 1024) = make_uint4(v[0].z, v[1].z, v[2].z, v[3].z);
+    *reinterpret_cast<uint4*>(dst + 1536) = make_uint4(v[0].w, v[1].w, v[2].w, v[3].w);
+  }
+}
+
+template <int BN>
 __global__ void __launch_bounds__(128, 1)
     k_matmul_nvfp4(const __grid_constant__ CUtensorMap tma_a,
                    const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ MmArgs args) {
+  using T = Tile<BN>;
+  constexpr int kStages = T::kStages, kStageBytes = T::kStageBytes, kABytes = T::kABytes,
+                kBBytes = T::kBBytes, kSfaBytes = T::kSfaBytes, kSfbBytes = T::kSfbBytes,
+                kH = T::kHalves;
+  constexpr uint32_t kTmemCols = T::kTmemCols, kSfaCol = T::kSfaCol, kSfbCol = T::kSfbCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -195,13 +233,12 @@ __global__ void __launch_bounds__(128, 1)
   volatile int* gave_up = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * kBN;
+  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * BN;
   const int KT = (int)(args.k / kBK);
-  const int64_t pitch = args.k / 16;  // scale bytes per row
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(full + s), 32);
+      mbar_init(smem_u32(full + s), 1);
       mbar_init(smem_u32(empty + s), 1);
     }
     mbar_init(smem_u32(done), 1);
@@ -222,34 +259,37 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
-    int issued = 0;
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % kStages;
-      bool ok = true;  // lane 0 waits; the warp follows its answer
-      if (lane == 0) {
-        ok = !*gave_up &&
-             (kt < kStages || mbar_wait(smem_u32(empty + s), ((kt / kStages) + 1) & 1));
-        if (!ok) *gave_up = 1;
+    // ---------------- producer (one thread) ----------------
+    if (lane == 0) {
+      const int64_t KTl = KT;
+      const uint8_t* sfa_src = args.a_scales + (m0 / kBM) * KTl * 2048;
+      const uint8_t* sfb_src = args.b_scales + (n0 / kBM) * KTl * 2048;
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (*gave_up ||
+            (kt >= kStages && !mbar_wait<20>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
+          *gave_up = 1;
+          break;
+        }
+        const uint32_t st = smem_u32(smem + s * kStageBytes), bar = smem_u32(full + s);
+        mbar_expect_tx(bar, kABytes + kBBytes + kSfaBytes + kSfbBytes);  // OOB rows included
+        tma_load_2d(st, &tma_a, kt * kRowBytes, (int)m0, bar);
+        tma_load_2d(st + kABytes, &tma_b, kt * kRowBytes, (int)n0, bar);
+        // scales: A's tile, then each 128-row half of B's (2048 bytes per tile and step)
+        bulk_load(st + kABytes + kBBytes, sfa_src + (int64_t)kt * 2048, 2048, bar);
+#pragma unroll
+        for (int h = 0; h < kH; ++h)
+          bulk_load(st + kABytes + kBBytes + kSfaBytes + 2048 * h,
+                    sfb_src + ((int64_t)h * KTl + kt) * 2048, 2048, bar);
+        mbar_arrive(bar);
+        issued = kt + 1;
       }
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      uint8_t* st = smem + s * kStageBytes;
-      const uint32_t bar = smem_u32(full + s);
-      if (lane == 0) {
-        mbar_expect_tx(bar, kABytes + kBBytes);
-        tma_load_2d(smem_u32(st), &tma_a, kt * kRowBytes, (int)m0, bar);
-        tma_load_2d(smem_u32(st + kABytes), &tma_b, kt * kRowBytes, (int)n0, bar);
+      if (*gave_up) {
+        // let the copies already issued land before the CTA can exit (bounded)
+        for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt)
+          mbar_wait<100>(smem_u32(full + kt % kStages), (kt / kStages) & 1);
       }
-      stage_scales(args.a_scales, args.m, m0, pitch, kt, st + kABytes + kBBytes, lane);
-      stage_scales(args.b_scales, args.n, n0, pitch, kt, st + kABytes + kBBytes + kSfBytes, lane);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bar);
-      issued = kt + 1;
-    }
-    if (lane == 0 && *gave_up) {
-      // let the loads already issued land before the CTA can exit (bounded)
-      for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt)
-        mbar_wait(smem_u32(full + kt % kStages), (kt / kStages) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -263,16 +303,18 @@ __global__ void __launch_bounds__(128, 1)
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
-        const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfBytes;
+        const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfaBytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           tc_copy_sf(tmem + kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
-          tc_copy_sf(tmem + kSfbCol + 4 * j, desc_sf(sfb + 512 * j));
+#pragma unroll
+          for (int h = 0; h < kH; ++h)
+            tc_copy_sf(tmem + kSfbCol + 4 * (kH * j + h), desc_sf(sfb + 2048 * h + 512 * j));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          tc_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j),
-                 tmem + kSfaCol + 4 * j, tmem + kSfbCol + 4 * j, (kt | j) != 0);
+          tc_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j), T::kIdesc,
+                 tmem + kSfaCol + 4 * j, tmem + kSfbCol + 4 * kH * j, (kt | j) != 0);
         tc_commit(smem_u32(empty + s));
       }
       tc_commit(smem_u32(done));  // also after giving up: the epilogue waits for issued MMAs
@@ -284,7 +326,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncwarp();
   bool ok = true;
   if (lane == 0) {
-    ok = mbar_wait(smem_u32(done), 0);
+    ok = mbar_wait<200>(smem_u32(done), 0);  // sleeps through the main loop
     if (!ok) *gave_up = 1;
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -293,7 +335,7 @@ __global__ void __launch_bounds__(128, 1)
     const int64_t row = m0 + 32 * warp + lane;
     const bool row_ok = row < args.m;
 #pragma unroll 1
-    for (int cb = 0; cb < kBN / 32; ++cb) {
+    for (int cb = 0; cb < BN / 32; ++cb) {
       uint32_t r[32];
       tc_load32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cb, r);
       const int64_t col = n0 + 32 * cb;
@@ -362,14 +404,14 @@ EncodeTiled encode_fn() {
   return fn;
 }
 
-// Map of one operand's codes: rows x (k / 2) bytes, row pitch k / 2, boxes of 128 x 128 bytes
-// loaded with the 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k) {
+// Map of one operand's codes: rows x (k / 2) bytes, row pitch k / 2, boxes of box_rows x 128
+// bytes loaded with the 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k, int box_rows) {
   const EncodeTiled enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)kBM};
+  const cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -382,19 +424,36 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
                              cudaStream_t stream, int* launches) {
+  constexpr int BN = MX_MM_BN;
+  static_assert(BN == 128 || BN == 256, "tile width");
+  using T = Tile<BN>;
   static bool attr_set = false;
   if (!attr_set) {
     const cudaError_t e = cudaFuncSetAttribute(
-        k_matmul_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        k_matmul_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   CUtensorMap ma, mb;
-  if (!make_map(&ma, a_packed, m, k) || !make_map(&mb, b_packed, n, k))
+  if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, BN))
     return cudaErrorInvalidValue;
   MmArgs args{a_scales, b_scales, c, m, n, k, alpha, c_bf16 ? 1 : 0};
-  const dim3 grid((unsigned)((n + kBN - 1) / kBN), (unsigned)((m + kBM - 1) / kBM));
-  k_matmul_nvfp4<<<grid, 128, kSmemBytes, stream>>>(ma, mb, args);
+  const dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)((m + kBM - 1) / kBM));
+  k_matmul_nvfp4<BN><<<grid, 128, T::kSmemBytes, stream>>>(ma, mb, args);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+int64_t mma_scales_bytes(int64_t rows, int64_t k) {
+  return 2 * ((rows + 2 * kBM - 1) / (2 * kBM)) * kBM * (k / 16);
+}
+
+cudaError_t run_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out,
+                              cudaStream_t stream, int* launches) {
+  const int64_t threads = mma_scales_bytes(rows, k) / 64;  // 64 bytes written per thread
+  const int64_t blocks = (threads + 255) / 256;
+  k_scales_to_mma<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(scales, rows, k,
+                                                                                  out);
   ++*launches;
   return cudaGetLastError();
 }

@@ -201,20 +201,37 @@ MX_API mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, 
 /* ---- Block-scaled matrix product on the tensor cores.
  * C = dequant(A) * dequant(B)^T, the dequantize-then-multiply step of inference in the 4-bit float
  * quantization article (gtnt.cn/news/16247, §3.1), with both operands stored by mx_quantize and
- * the block scales applied inside the tensor-core multiply (nothing is dequantized to memory):
- *   - A is m x k (a_packed: m*k/2 bytes, a_scales: m*k/16 bytes), B is n x k (likewise), both
- *     quantized with block = 16 along k and fmt = MX_SCALE_E4M3, exactly as mx_quantize writes
- *     a row-major m x k (n x k) tensor; a_g / b_g are the global scales they were quantized with;
- *   - C is m x n, row-major, float32 (ct = MX_F32) or bfloat16 (MX_BF16, rounded to nearest even):
- *     C[i][j] = a_g b_g sum_t E2M1(A[i][t]) S(A)[i][t/16] E2M1(B[j][t]) S(B)[j][t/16], accumulated
- *     in float32 by the tensor core (any order), then multiplied by a_g b_g (one rounding);
- *   - block != 16 or fmt != MX_SCALE_E4M3 (no native tensor-core form), k == 0 or k % 256 != 0:
- *     MX_ERR_UNSUPPORTED; m, n or k negative, or m, n >= 2^31: MX_ERR_INVALID_ARG; m == 0 or
- *     n == 0: nothing is enqueued.
- * Every wait inside the kernel is bounded; a launch whose waits ran out leaves C unspecified and
- * is counted by mx_matmul_gave_up. */
-MX_API mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
-                           const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g,
+ * the block scales applied inside the tensor-core multiply (nothing is dequantized to memory).
+ *
+ * Operands: A is m x k (a_packed: m*k/2 bytes, as mx_quantize writes a row-major m x k tensor with
+ * block = 16 and MX_SCALE_E4M3), B is n x k (b_packed: n*k/2 bytes, likewise); a_g / b_g are the
+ * global scales they were quantized with.  Their scale arrays are first put into tensor-core
+ * order by mx_matmul_prepare_scales (for weights, once), and mx_matmul reads the prepared arrays.
+ *
+ * mx_matmul_scales_size(rows, k): bytes of a prepared scale array for a rows x k operand,
+ * 2 * ceil(rows / 256) * 128 * k / 16 (rows padded with zero scales); 0 when rows < 0 or k is not
+ * a positive multiple of 256. */
+MX_API size_t mx_matmul_scales_size(int64_t rows, int64_t k);
+
+/* scales (rows * k / 16 bytes, the mx_quantize layout, block 16) -> out (out_bytes >=
+ * mx_matmul_scales_size(rows, k), device memory): for each 128-row tile and each 256-element step
+ * of k, 2048 contiguous bytes holding four 512-byte groups (one per 64-element tensor-core step);
+ * in group j, row 32 q + r of the tile has its four scales at byte 16 r + 4 q.  Errors: k not a
+ * positive multiple of 256 -> MX_ERR_UNSUPPORTED; rows < 0 -> MX_ERR_INVALID_ARG; out_bytes too
+ * small -> MX_ERR_WORKSPACE; rows == 0 enqueues nothing. */
+MX_API mx_status mx_matmul_prepare_scales(const uint8_t* scales, int64_t rows, int64_t k,
+                                          uint8_t* out, size_t out_bytes, cudaStream_t stream);
+
+/* C (m x n, row-major, float32 for ct = MX_F32 or bfloat16 rounded to nearest even for MX_BF16)
+ *   C[i][j] = a_g b_g sum_t E2M1(A[i][t]) S(A)[i][t/16] E2M1(B[j][t]) S(B)[j][t/16],
+ * accumulated in float32 by the tensor core (order unspecified), then multiplied by a_g b_g (one
+ * rounding).  a_scales_mma / b_scales_mma are the prepared arrays of A (m rows) and B (n rows).
+ * block != 16 or fmt != MX_SCALE_E4M3 (no native tensor-core form), k == 0 or k % 256 != 0:
+ * MX_ERR_UNSUPPORTED; m, n or k negative, or m, n >= 2^31: MX_ERR_INVALID_ARG; m == 0 or n == 0:
+ * nothing is enqueued.  Every wait inside the kernel is bounded; a launch whose waits ran out
+ * leaves C unspecified and is counted by mx_matmul_gave_up. */
+MX_API mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales_mma, uint16_t a_g,
+                           const uint8_t* b_packed, const uint8_t* b_scales_mma, uint16_t b_g,
                            int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c,
                            mx_dtype ct, cudaStream_t stream);
 

@@ -216,6 +216,26 @@ def test_matmul_rejects_bad_arguments():
     assert L.mx_matmul_gave_up(None) == INV
 
 
+def test_matmul_scale_preparation_arguments():
+    assert L.mx_matmul_scales_size(128, 256) == 256 * 16        # rows padded to 256
+    assert L.mx_matmul_scales_size(300, 512) == 512 * 32
+    assert L.mx_matmul_scales_size(0, 256) == 0
+    assert L.mx_matmul_scales_size(128, 128) == 0               # k not a multiple of 256
+    assert L.mx_matmul_scales_size(-1, 256) == 0
+    size = L.mx_matmul_scales_size(128, 256)
+    def prep(s=A, rows=128, k=256, out=A, nbytes=size):
+        return L.mx_matmul_prepare_scales(s, rows, k, out, nbytes, None)
+    assert prep(k=128) == UNS
+    assert prep(k=0) == UNS
+    assert prep(rows=-1) == INV
+    assert prep(s=None) == INV
+    assert prep(out=None) == INV
+    assert prep(nbytes=size - 1) == WS
+    assert prep(s=A + 4) == MIS
+    assert prep(out=A + 8) == MIS
+    assert prep(rows=0, s=None, out=None) == OK
+
+
 def test_injected_cuda_failure_is_reported_before_any_launch():
     # valid arguments on fake pointers: the armed failures are consumed before anything is
     # enqueued, so nothing touches the (fake) buffers; the status is MX_ERR_CUDA

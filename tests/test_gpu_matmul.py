@@ -154,5 +154,28 @@ def test_empty_and_unsupported():
     assert mx.matmul(a, s, b, bs).shape == (0, 8)
     b2 = torch.zeros((8, 64), dtype=torch.uint8, device="cuda")
     s2 = torch.zeros((8, 8), dtype=torch.uint8, device="cuda")
-    with pytest.raises(mx.MXError):
+    with pytest.raises((mx.MXError, ValueError)):
         mx.matmul(b2, s2, b2, s2)  # k = 128: not a multiple of 256
+    with pytest.raises(mx.MXError):
+        mx.matmul(b2, s2, b2, s2, prepared=True)
+
+
+@pytest.mark.parametrize("rows,k", [(128, 256), (300, 768), (1, 512)])
+def test_prepared_scale_layout(rows, k):
+    # tensor-core order, written out here: tile t (256-row padded), step kt, group j, then
+    # row 32 q + r of the tile at byte 16 r + 4 q, its 4 scales of group j in order
+    rng = np.random.default_rng(rows + k)
+    sc = rng.integers(0, 0x7F, (rows, k // 16), dtype=np.uint8)
+    got = mx.prepare_scales(dev(sc), k).cpu().numpy()
+    tiles = 2 * ((rows + 255) // 256)
+    pad = np.zeros((tiles * 128, k // 16), np.uint8)
+    pad[:rows] = sc
+    ref = np.zeros((tiles, k // 256, 4, 32, 4, 4), np.uint8)
+    for t in range(tiles):
+        for kt in range(k // 256):
+            for j in range(4):
+                for q in range(4):
+                    ref[t, kt, j, :, q, :] = pad[t * 128 + 32 * q: t * 128 + 32 * q + 32,
+                                                 16 * kt + 4 * j: 16 * kt + 4 * j + 4]
+    assert got.size == ref.size
+    assert np.array_equal(got, ref.reshape(-1))
