@@ -216,6 +216,10 @@ mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a
     return MX_ERR_INVALID_ARG;
   if (block != 16 || fmt != MX_SCALE_E4M3 || k == 0 || k % 256 != 0) return MX_ERR_UNSUPPORTED;
   if (m == 0 || n == 0) return MX_OK;
+  // TMA coordinates are 32-bit: k / 2 bytes per row and the prepared scales as 256-byte rows
+  if (k >= (int64_t(1) << 31) || mxk::mma_scales_bytes(m, k) / 256 >= (int64_t(1) << 31) ||
+      mxk::mma_scales_bytes(n, k) / 256 >= (int64_t(1) << 31))
+    return MX_ERR_UNSUPPORTED;
   if (!a_packed || !a_scales || !b_packed || !b_scales || !c) return MX_ERR_INVALID_ARG;
   if (!aligned16(a_packed) || !aligned16(a_scales) || !aligned16(b_packed) ||
       !aligned16(b_scales) || !aligned16(c))

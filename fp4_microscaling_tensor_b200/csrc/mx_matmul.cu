@@ -22,6 +22,7 @@
 // scale copies land; empty: the commit).  Every wait is bounded: a CTA that gives up records it in a device counter, lets its
 // issued copies and MMAs finish (bounded again), frees its TMEM and returns.
 #include <cuda.h>
+#include <stdlib.h>
 
 #include "mx_device.cuh"
 #include "mx_launch.h"
@@ -29,7 +30,17 @@
 namespace mxk {
 namespace {
 
-#ifndef MX_MM_BN  // columns of C per CTA: 128 or 256 (MMA N)
+#ifndef MX_MM_PAIR_STAGES  // pipeline stages of the CTA-pair kernel
+#define MX_MM_PAIR_STAGES 5
+#endif
+#ifndef MX_MM_PROD_SLEEP  // ns slept between polls of an empty barrier by a producer
+#define MX_MM_PROD_SLEEP 20
+#endif
+
+#ifndef MX_MM_SFBUF  // TMEM copies of the scales in rotation: a step's scale copies never wait
+#define MX_MM_SFBUF 2  // for the previous step's MMAs to finish reading the same columns
+#endif
+#ifndef MX_MM_BN  // columns of C per CTA in the one-CTA kernel: 128 or 256 (MMA N)
 #define MX_MM_BN 256
 #endif
 
@@ -50,11 +61,13 @@ struct Tile {
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;  // + barriers, alignment
-  // TMEM: accumulator BN columns, then A's scales (4 per MMA step), then B's (4 kHalves per step);
-  // column w of a step's scales serves rows 32 w .. 32 w + 31 of its operand tile.
+  // TMEM: accumulator BN columns, then MX_MM_SFBUF scale buffers of kSfCols columns each: A's
+  // scales (4 per MMA step), then B's (4 kHalves per step); column w of a step's scales serves
+  // rows 32 w .. 32 w + 31 of its operand tile.
+  static constexpr uint32_t kSfCols = 16 + 16 * kHalves;
   static constexpr uint32_t kSfaCol = BN, kSfbCol = BN + 16;
   static constexpr uint32_t kTmemCols = BN == 256 ? 512 : 256;
-  static_assert(kSfbCol + 16 * kHalves <= kTmemCols, "TMEM columns");
+  static_assert(BN + MX_MM_SFBUF * kSfCols <= kTmemCols, "TMEM columns");
   // Instruction descriptor of kind::mxf4nvf4 (block-scaled): A and B E2M1 (format 1), K-major,
   // E4M3 scales (scale format 0), N = BN (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16),
   // scale-factor ids 0, dense, K = 64.
@@ -91,19 +104,29 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 // True once the phase with the given parity has completed; false after kWaitLimit polls, or
 // earlier once another CTA has given up.  SLEEP_NS > 0 sleeps between polls: waits off the
 // critical path must not flood the shared-memory pipe that the TMA and the tensor core use.
-template <int SLEEP_NS = 0>
+// CLUSTER: acquire at cluster scope (the phase was completed by the other CTA of a pair).
+template <int SLEEP_NS = 0, bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
     if ((i & 1023u) == 1023u && g_mm_abandon) return false;
     if (SLEEP_NS > 0 && i > 0) __nanosleep(SLEEP_NS);
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+    if constexpr (CLUSTER)
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    else
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
     if (ok) return true;
   }
   return false;
@@ -214,6 +237,51 @@ __global__ void k_scales_to_mma(const uint8_t* __restrict__ scales, int64_t rows
   }
 }
 
+// Epilogue of one CTA: accumulator rows row0 + 32 w + lane (one per thread; warp w reads TMEM
+// lanes 32 w ..), NC columns from n0, times alpha, stored to C as float32 or bfloat16.
+template <int NC>
+__device__ __forceinline__ void store_rows(uint32_t tmem, int warp, int lane, int64_t row0,
+                                           int64_t n0, const MmArgs& args) {
+  const int64_t row = row0 + 32 * warp + lane;
+  const bool row_ok = row < args.m;
+#pragma unroll 1
+  for (int cb = 0; cb < NC / 32; ++cb) {
+    uint32_t r[32];
+    tc_load32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cb, r);
+    const int64_t col = n0 + 32 * cb;
+    if (!row_ok || col >= args.n) continue;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), args.alpha);
+    const bool whole = col + 32 <= args.n;
+    if (args.c_bf16) {
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + row * args.n + col;
+      if (whole && (args.n % 8) == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 pk;
+          pk.x = pack_bf16x2(v[i], v[i + 1]);
+          pk.y = pack_bf16x2(v[i + 2], v[i + 3]);
+          pk.z = pack_bf16x2(v[i + 4], v[i + 5]);
+          pk.w = pack_bf16x2(v[i + 6], v[i + 7]);
+          *reinterpret_cast<uint4*>(out + i) = pk;
+        }
+      } else {
+        for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = __float2bfloat16_rn(v[i]);
+      }
+    } else {
+      float* out = static_cast<float*>(args.c) + row * args.n + col;
+      if (whole && (args.n % 4) == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+        for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = v[i];
+      }
+    }
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(128, 1)
     k_matmul_nvfp4(const __grid_constant__ CUtensorMap tma_a,
@@ -268,7 +336,7 @@ __global__ void __launch_bounds__(128, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % kStages;
         if (*gave_up ||
-            (kt >= kStages && !mbar_wait<20>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
+            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
           *gave_up = 1;
           break;
         }
@@ -304,17 +372,18 @@ __global__ void __launch_bounds__(128, 1)
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
         const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfaBytes;
+        const uint32_t tsf = tmem + (kt % MX_MM_SFBUF) * T::kSfCols;  // this step's buffer
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          tc_copy_sf(tmem + kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
+          tc_copy_sf(tsf + kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
 #pragma unroll
           for (int h = 0; h < kH; ++h)
-            tc_copy_sf(tmem + kSfbCol + 4 * (kH * j + h), desc_sf(sfb + 2048 * h + 512 * j));
+            tc_copy_sf(tsf + kSfbCol + 4 * (kH * j + h), desc_sf(sfb + 2048 * h + 512 * j));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           tc_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j), T::kIdesc,
-                 tmem + kSfaCol + 4 * j, tmem + kSfbCol + 4 * kH * j, (kt | j) != 0);
+                 tsf + kSfaCol + 4 * j, tsf + kSfbCol + 4 * kH * j, (kt | j) != 0);
         tc_commit(smem_u32(empty + s));
       }
       tc_commit(smem_u32(done));  // also after giving up: the epilogue waits for issued MMAs
@@ -331,46 +400,7 @@ __global__ void __launch_bounds__(128, 1)
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   tc_fence_after();
-  if (__all_sync(0xffffffffu, ok && !*gave_up)) {
-    const int64_t row = m0 + 32 * warp + lane;
-    const bool row_ok = row < args.m;
-#pragma unroll 1
-    for (int cb = 0; cb < BN / 32; ++cb) {
-      uint32_t r[32];
-      tc_load32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * cb, r);
-      const int64_t col = n0 + 32 * cb;
-      if (!row_ok || col >= args.n) continue;
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), args.alpha);
-      const bool whole = col + 32 <= args.n;
-      if (args.c_bf16) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + row * args.n + col;
-        if (whole && (args.n % 8) == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(v[i], v[i + 1]);
-            pk.y = pack_bf16x2(v[i + 2], v[i + 3]);
-            pk.z = pack_bf16x2(v[i + 4], v[i + 5]);
-            pk.w = pack_bf16x2(v[i + 6], v[i + 7]);
-            *reinterpret_cast<uint4*>(out + i) = pk;
-          }
-        } else {
-          for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = __float2bfloat16_rn(v[i]);
-        }
-      } else {
-        float* out = static_cast<float*>(args.c) + row * args.n + col;
-        if (whole && (args.n % 4) == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        } else {
-          for (int i = 0; i < 32 && col + i < args.n; ++i) out[i] = v[i];
-        }
-      }
-    }
-  }
+  if (__all_sync(0xffffffffu, ok && !*gave_up)) store_rows<BN>(tmem, warp, lane, m0, n0, args);
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *gave_up) {
@@ -381,6 +411,221 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+
+// ------------------------------------------------------------------------------------------------
+// CTA pair (tcgen05 cta_group::2): a cluster of two CTAs on one TPC computes a 256 x 256 tile of
+// C with 256 x 256 x 64 MMAs issued by the even CTA (the leader).  CTA r holds rows 128 r .. of
+// the tile's A rows and rows 128 r .. of its 256 B rows (the MMA reads both CTAs' shared memory
+// at the same offsets), A's scales for its own rows and B's scales for all 256 rows; the
+// accumulator of CTA r (its 128 rows x 256 columns) is in its own TMEM.  Per SM that is 32 KiB
+// of codes per 256-element step for 128 x 256 outputs, against 48 KiB in the one-CTA kernel.
+// Both CTAs' tile and scale copies (TMA, cta_group::2 form, no multicast) complete on the
+// leader's full barrier, which expects the bytes of both; the leader commits its MMAs to its own
+// and to the peer's empty / done barriers with separate single-target commits.
+// ------------------------------------------------------------------------------------------------
+struct Pair {
+  static constexpr int kStages = MX_MM_PAIR_STAGES;
+  static constexpr int kABytes = kBM * kRowBytes;   // this CTA's 128 rows of A
+  static constexpr int kBBytes = kBM * kRowBytes;   // this CTA's 128 of the 256 B rows
+  static constexpr int kSfaBytes = 2048;            // A's scales, this CTA's rows
+  static constexpr int kSfbBytes = 4096;            // B's scales, all 256 rows
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
+  static constexpr uint32_t kTmemCols = 512, kSfaCol = 256, kSfbCol = 272, kSfCols = 48;
+  static_assert(256 + MX_MM_SFBUF * kSfCols <= kTmemCols, "TMEM columns");
+  // M = 256 (bits 24..28: 16), N = 256 (bits 17..22: 32), otherwise as the one-CTA descriptor
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (32u << 17) | (16u << 24);
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// TMA 2-D load into this CTA's shared memory whose completion is counted on an mbarrier of
+// either CTA of the pair (here: the leader's).
+__device__ __forceinline__ void tma2_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                             uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc2_copy_sf(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+__device__ __forceinline__ void tc2_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Arrive on one mbarrier (this CTA's or the peer's, shared::cluster address) when the pair's
+// MMAs issued so far are complete.
+__device__ __forceinline__ void tc2_commit(uint32_t cluster_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   cluster_addr)
+               : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+    k_matmul_nvfp4_pair(const __grid_constant__ CUtensorMap tma_a,
+                        const __grid_constant__ CUtensorMap tma_b,
+                        const __grid_constant__ CUtensorMap tma_sfa,
+                        const __grid_constant__ CUtensorMap tma_sfb,
+                        const __grid_constant__ MmArgs args) {
+  using P = Pair;
+  constexpr int kStages = P::kStages, kStageBytes = P::kStageBytes, kABytes = P::kABytes,
+                kBBytes = P::kBBytes, kSfaBytes = P::kSfaBytes, kSfbBytes = P::kSfbBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* gave_up = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int64_t pair = blockIdx.x >> 1, NT = (args.n + 255) / 256;
+  const int64_t mt = pair / NT, nt = pair - mt * NT;
+  const int64_t m0 = mt * 256 + 128 * rank;  // this CTA's rows of A and of C
+  const int64_t n0 = nt * 256;               // the pair's columns of C
+  const int KT = (int)(args.k / kBK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *gave_up = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(P::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialized and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- producer (one thread per CTA) ----------------
+    // Both CTAs' copies complete on the leader's full barrier; the leader expects both.
+    if (lane == 0) {
+      const uint32_t full0 = map_to(smem_u32(full), 0);
+      const int sfa_row = (int)((m0 / kBM) * KT * 8), sfb_row = (int)((n0 / kBM) * KT * 8);
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (*gave_up ||
+            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
+          *gave_up = 1;
+          break;
+        }
+        const uint32_t st = smem_u32(smem + s * kStageBytes), bar = full0 + 8 * s;
+        if (rank == 0)
+          mbar_expect_tx(smem_u32(full + s), 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
+        tma2_load_2d(st, &tma_a, kt * kRowBytes, (int)m0, bar);
+        tma2_load_2d(st + kABytes, &tma_b, kt * kRowBytes, (int)(n0 + 128 * rank), bar);
+        // scale groups: 2048 bytes = 8 rows of 256 in the scale maps
+        tma2_load_2d(st + kABytes + kBBytes, &tma_sfa, 0, sfa_row + 8 * kt, bar);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma2_load_2d(st + kABytes + kBBytes + kSfaBytes + 2048 * h, &tma_sfb, 0,
+                       sfb_row + 8 * (h * KT + kt), bar);
+        if (rank == 0) mbar_arrive(smem_u32(full + s));
+        issued = kt + 1;
+      }
+      if (*gave_up && issued > 0) {
+        // this CTA cannot see its copies complete (they count on the leader's barrier): give
+        // them time to land before the CTA may exit (bounded)
+        for (int i = 0; i < 4096; ++i) __nanosleep(1000);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader, one thread) ----------------
+      const uint32_t empty1 = map_to(smem_u32(empty), 1), done1 = map_to(smem_u32(done), 1);
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1)) {
+          *gave_up = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes);
+        const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfaBytes;
+        const uint32_t tsf = tmem + (kt % MX_MM_SFBUF) * P::kSfCols;  // this step's buffer
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tc2_copy_sf(tsf + P::kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tc2_copy_sf(tsf + P::kSfbCol + 4 * (2 * j + h), desc_sf(sfb + 2048 * h + 512 * j));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc2_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j), P::kIdesc,
+                  tsf + P::kSfaCol + 4 * j, tsf + P::kSfbCol + 8 * j, (kt | j) != 0);
+        tc2_commit(smem_u32(empty + s));
+        tc2_commit(empty1 + 8 * s);
+      }
+      tc2_commit(smem_u32(done));  // also after giving up: both epilogues wait for issued MMAs
+      tc2_commit(done1);
+    }
+    __syncwarp();
+  }
+
+  // ---------------- epilogue: this CTA's 128 rows x 256 columns ----------------
+  __syncwarp();
+  bool ok = true;
+  if (lane == 0) {
+    ok = mbar_wait<200>(smem_u32(done), 0);
+    if (!ok) *gave_up = 1;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  tc_fence_after();
+  if (__all_sync(0xffffffffu, ok && !*gave_up)) store_rows<256>(tmem, warp, lane, m0, n0, args);
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *gave_up) {
+    atomicAdd(&g_mm_gave_up, 1u);
+    g_mm_abandon = 1;
+  }
+  cluster_sync();  // neither CTA releases TMEM or exits while the pair still signals it
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(P::kTmemCols)
                  : "memory");
   }
 }
@@ -418,28 +663,66 @@ bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k, i
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map of a prepared scale array seen as rows of 256 bytes, boxes of 8 rows (one 2048-byte group).
+bool make_rows_map(CUtensorMap* map, const uint8_t* scales, int64_t rows) {
+  const EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {256, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, 8};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(scales), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
+
+int64_t mma_scales_bytes(int64_t rows, int64_t k);
 
 cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
                              cudaStream_t stream, int* launches) {
-  constexpr int BN = MX_MM_BN;
-  static_assert(BN == 128 || BN == 256, "tile width");
-  using T = Tile<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        k_matmul_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, BN))
-    return cudaErrorInvalidValue;
   MmArgs args{a_scales, b_scales, c, m, n, k, alpha, c_bf16 ? 1 : 0};
-  const dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)((m + kBM - 1) / kBM));
-  k_matmul_nvfp4<BN><<<grid, 128, T::kSmemBytes, stream>>>(ma, mb, args);
+  CUtensorMap ma, mb;
+  // The CTA-pair kernel is correct but, with its per-step scale copies, not yet faster than the
+  // one-CTA kernel on B200; MXFP4_MATMUL_PAIRS=1 selects it (for m > 128).
+  const char* env = getenv("MXFP4_MATMUL_PAIRS");
+  const bool pairs_on = env != nullptr && env[0] == '1';
+  if (m > kBM && pairs_on) {
+    // CTA pairs: 256 x 256 tiles of C
+    static bool attr_set = false;
+    if (!attr_set) {
+      const cudaError_t e = cudaFuncSetAttribute(
+          k_matmul_nvfp4_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, Pair::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    CUtensorMap msa, msb;
+    if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, kBM) ||
+        !make_rows_map(&msa, a_scales, mma_scales_bytes(m, k) / 256) ||
+        !make_rows_map(&msb, b_scales, mma_scales_bytes(n, k) / 256))
+      return cudaErrorInvalidValue;
+    const int64_t pairs = ((m + 255) / 256) * ((n + 255) / 256);
+    k_matmul_nvfp4_pair<<<(unsigned)(2 * pairs), 128, Pair::kSmemBytes, stream>>>(ma, mb, msa, msb,
+                                                                                 args);
+  } else {
+    constexpr int BN = MX_MM_BN;
+    static_assert(BN == 128 || BN == 256, "tile width");
+    using T = Tile<BN>;
+    static bool attr_set = false;
+    if (!attr_set) {
+      const cudaError_t e = cudaFuncSetAttribute(
+          k_matmul_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, BN))
+      return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)((m + kBM - 1) / kBM));
+    k_matmul_nvfp4<BN><<<grid, 128, T::kSmemBytes, stream>>>(ma, mb, args);
+  }
   ++*launches;
   return cudaGetLastError();
 }

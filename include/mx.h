@@ -229,7 +229,9 @@ MX_API mx_status mx_matmul_prepare_scales(const uint8_t* scales, int64_t rows, i
  * block != 16 or fmt != MX_SCALE_E4M3 (no native tensor-core form), k == 0 or k % 256 != 0:
  * MX_ERR_UNSUPPORTED; m, n or k negative, or m, n >= 2^31: MX_ERR_INVALID_ARG; m == 0 or n == 0:
  * nothing is enqueued.  Every wait inside the kernel is bounded; a launch whose waits ran out
- * leaves C unspecified and is counted by mx_matmul_gave_up. */
+ * leaves C unspecified and is counted by mx_matmul_gave_up.  Kernel: one CTA per 128 x 256 tile
+ * of C; with the environment variable MXFP4_MATMUL_PAIRS=1 (read at each call) and m > 128, CTA
+ * pairs (tcgen05 cta_group::2) per 256 x 256 tile instead, with the same results. */
 MX_API mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales_mma, uint16_t a_g,
                            const uint8_t* b_packed, const uint8_t* b_scales_mma, uint16_t b_g,
                            int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c,

@@ -22,6 +22,13 @@ from fp4_microscaling_tensor_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
+
+@pytest.fixture(params=["one_cta", "cta_pairs"], autouse=True)
+def kernel(request, monkeypatch):
+    """Every test runs with both kernels (the CTA-pair kernel is used for m > 128)."""
+    monkeypatch.setenv("MXFP4_MATMUL_PAIRS", "1" if request.param == "cta_pairs" else "0")
+    return request.param
+
 ONE = 0x38  # E4M3 code of 1.0
 
 
