@@ -122,9 +122,15 @@ int orc_round_e2m1_mag(double v) {
 static int bad_shape(int64_t rows, int64_t cols, int block) {
   if (rows < 0 || cols < 0) return 1;
   if (block < 4 || block > 256 || (block & (block - 1)) != 0) return 1; /* [MX] §1: 4..256 */
-  if (cols % block != 0) return 1;
   return 0;
 }
+
+/* Row layout (any cols): a row is cut into blocks of N from its first element, the last block
+ * holding cols mod N elements when N does not divide cols; a row's codes take ceil(cols / 2)
+ * bytes (element 2k low nibble, 2k + 1 high nibble of byte k; an odd last element leaves the high
+ * nibble 0) and its scales ceil(cols / N) bytes. */
+static int64_t row_bytes(int64_t cols) { return (cols + 1) / 2; }
+static int64_t row_blocks(int64_t cols, int block) { return (cols + block - 1) / block; }
 
 static int bad_g(uint16_t g_bits) {
   double g = orc_fp16_value(g_bits);
@@ -195,9 +201,10 @@ static int quantize_block(const double* xs, int n, int fmt, double g, uint8_t* c
   return s;
 }
 
-static int get_code(const uint8_t* packed, int64_t idx) {
-  uint8_t b = packed[idx >> 1];
-  return (idx & 1) ? (b >> 4) : (b & 15); /* even element in the low nibble */
+/* code of element j of row r */
+static int get_code(const uint8_t* packed, int64_t cols, int64_t r, int64_t j) {
+  uint8_t b = packed[r * row_bytes(cols) + (j >> 1)];
+  return (j & 1) ? (b >> 4) : (b & 15); /* even element in the low nibble */
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -216,16 +223,18 @@ static void q_rows(void* p, int64_t r0, int64_t r1, int tid) {
   q_ctx* c = (q_ctx*)p;
   double xs[256];
   uint8_t codes[256];
-  int64_t r, b, nb = c->cols / c->block;
+  int64_t r, b, nb = row_blocks(c->cols, c->block), pb = row_bytes(c->cols);
   int i;
   (void)tid;
   for (r = r0; r < r1; ++r) {
     for (b = 0; b < nb; ++b) {
-      int64_t base = r * c->cols + b * c->block;
-      for (i = 0; i < c->block; ++i) xs[i] = load_x(c->x, c->xdtype, base + i);
-      c->scales[r * nb + b] = (uint8_t)quantize_block(xs, c->block, c->fmt, c->g, codes);
-      for (i = 0; i < c->block; i += 2)
-        c->packed[(base + i) >> 1] = (uint8_t)(codes[i] | (codes[i + 1] << 4));
+      const int64_t j0 = b * c->block; /* even: blocks start on byte boundaries */
+      const int len = (int)(c->cols - j0 < c->block ? c->cols - j0 : c->block);
+      for (i = 0; i < len; ++i) xs[i] = load_x(c->x, c->xdtype, r * c->cols + j0 + i);
+      c->scales[r * nb + b] = (uint8_t)quantize_block(xs, len, c->fmt, c->g, codes);
+      for (i = 0; i < len; i += 2)
+        c->packed[r * pb + ((j0 + i) >> 1)] =
+            (uint8_t)(codes[i] | (i + 1 < len ? codes[i + 1] << 4 : 0));
     }
   }
 }
@@ -279,13 +288,13 @@ typedef struct {
 
 static void dq_rows(void* p, int64_t r0, int64_t r1, int tid) {
   dq_ctx* c = (dq_ctx*)p;
-  int64_t r, j, nb = c->cols / c->block;
+  int64_t r, j, nb = row_blocks(c->cols, c->block);
   (void)tid;
   for (r = r0; r < r1; ++r) {
     for (j = 0; j < c->cols; ++j) {
       int64_t idx = r * c->cols + j;
       double S = orc_scale_value(c->scales[r * nb + j / c->block], c->fmt);
-      double v = orc_e2m1_value(get_code(c->packed, idx)) * S * c->g;
+      double v = orc_e2m1_value(get_code(c->packed, c->cols, r, j)) * S * c->g;
       if (c->ydtype == ORC_BF16)
         ((uint16_t*)c->y)[idx] = to_bf16_bits(v);
       else
@@ -330,17 +339,18 @@ static void st_rows(void* p, int64_t r0, int64_t r1, int tid) {
   orc_stats* o = &c->part[tid];
   double xs[256];
   uint8_t codes[256];
-  int64_t r, b, nb = c->cols / c->block;
+  int64_t r, b, nb = row_blocks(c->cols, c->block);
   double smax = orc_scale_max(c->fmt);
   int i;
   memset(o, 0, sizeof(*o));
   for (r = r0; r < r1; ++r) {
     for (b = 0; b < nb; ++b) {
-      int64_t base = r * c->cols + b * c->block;
+      const int64_t j0 = b * c->block;
+      const int len = (int)(c->cols - j0 < c->block ? c->cols - j0 : c->block);
       double a = 0.0, S;
       int s, imax = 0;
-      for (i = 0; i < c->block; ++i) {
-        xs[i] = load_x(c->x, c->xdtype, base + i);
+      for (i = 0; i < len; ++i) {
+        xs[i] = load_x(c->x, c->xdtype, r * c->cols + j0 + i);
         if (fabs(xs[i]) > a) { /* strict: the first index of the largest |x| is "the max element" */
           a = fabs(xs[i]);
           imax = i;
@@ -348,9 +358,9 @@ static void st_rows(void* p, int64_t r0, int64_t r1, int tid) {
       }
       if (c->packed) {
         s = c->scales[r * nb + b];
-        for (i = 0; i < c->block; ++i) codes[i] = (uint8_t)get_code(c->packed, base + i);
+        for (i = 0; i < len; ++i) codes[i] = (uint8_t)get_code(c->packed, c->cols, r, j0 + i);
       } else {
-        s = quantize_block(xs, c->block, c->fmt, c->g, codes);
+        s = quantize_block(xs, len, c->fmt, c->g, codes);
       }
       S = orc_scale_value(s, c->fmt);
       o->n_blocks += 1;
@@ -358,10 +368,10 @@ static void st_rows(void* p, int64_t r0, int64_t r1, int tid) {
       if (S == 0.0) {
         /* item 3: the whole block is stored as zero; its error is sum x^2 */
         o->n_zero_blocks += 1;
-        for (i = 0; i < c->block; ++i) o->sse_zero += xs[i] * xs[i];
+        for (i = 0; i < len; ++i) o->sse_zero += xs[i] * xs[i];
         continue;
       }
-      for (i = 0; i < c->block; ++i) {
+      for (i = 0; i < len; ++i) {
         double y = orc_e2m1_value(codes[i]) * S * c->g;
         double d = xs[i] - y;
         if (i == imax)

@@ -22,8 +22,12 @@
  *   - E2M1 has no inf/NaN (all 16 codes finite); E4M3 is the OCP "FN" variant (bias 7, max 448,
  *     0x7F/0xFF NaN, never produced); UE5M3 is unsigned, bias 15, subnormals, every code finite,
  *     max 122880;
- *   - blocks are N consecutive elements of a row; cols % N == 0;
- *   - element 2k of a row goes to the low nibble of byte k, element 2k+1 to the high nibble;
+ *   - blocks are N consecutive elements of a row, from its first element; when N does not divide
+ *     cols the last block of each row holds the cols mod N remaining elements (its own absmax and
+ *     scale, the same element rule);
+ *   - element 2k of a row goes to the low nibble of byte k, element 2k+1 to the high nibble; a
+ *     row's codes take ceil(cols/2) bytes (an odd last element leaves the high nibble 0) and its
+ *     scales ceil(cols/N) bytes;
  *   - the code's sign bit is the sign bit of x, also in zero-scale blocks and for -0.0;
  *   - the error terms are sums over the tensor; each MSE is its sum divided by rows*cols;
  *   - the per-tensor FP16 scale chosen by orc_global_scale is the smallest FP16 value g with

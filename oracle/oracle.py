@@ -83,11 +83,13 @@ def _ptr(a):
 
 
 def quantize(x, rows, cols, block, fmt, g_bits=0x3C00, threads=None):
-    """Return (packed uint8[rows*cols/2], scales uint8[rows*cols/block])."""
+    """Return (packed uint8[rows*ceil(cols/2)], scales uint8[rows*ceil(cols/block)]): rows of
+    ceil(cols/2) code bytes and ceil(cols/block) scale bytes (the last block of a row holds
+    cols mod block elements when block does not divide cols)."""
     x, xt = _xarg(x)
     assert x.size == rows * cols
-    packed = np.zeros(rows * cols // 2, np.uint8)
-    scales = np.zeros(rows * cols // block, np.uint8)
+    packed = np.zeros(rows * ((cols + 1) // 2), np.uint8)
+    scales = np.zeros(rows * (-(-cols // block) if block > 0 else 0), np.uint8)
     rc = lib.orc_quantize(_ptr(x), xt, rows, cols, block, fmt, g_bits, _ptr(packed), _ptr(scales),
                           threads or _THREADS)
     if rc != 0:
