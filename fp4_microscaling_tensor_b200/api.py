@@ -66,9 +66,9 @@ def quantize(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, stream=N
         raise ValueError("x must be float32 or bfloat16")
     lead = tuple(x.shape[:-1])
     if packed is None:
-        packed = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+        packed = torch.empty(lead + ((cols + 1) // 2,), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+        scales = torch.empty(lead + (-(-cols // block) if block else 0,), dtype=torch.uint8,
                              device=x.device)
     check(lib.mx_quantize(x.data_ptr(), _DT[x.dtype], rows, cols, int(block), fmt_code(fmt),
                           g_bits(g), packed.data_ptr(), scales.data_ptr(),
@@ -77,13 +77,17 @@ def quantize(x, block=32, fmt="e4m3", g=None, packed=None, scales=None, stream=N
 
 
 def dequantize(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=torch.bfloat16, out=None,
-               stream=None):
-    """Dequantize packed codes and block scales into a [..., cols] tensor of out_dtype."""
+               stream=None, cols=None):
+    """Dequantize packed codes and block scales into a [..., cols] tensor of out_dtype.  cols
+    defaults to 2 * packed.shape[-1]; give it for rows of odd length (ragged last blocks)."""
     if out_dtype not in _DT:
         raise ValueError("out_dtype must be float32 or bfloat16")
     prow, pcols = _shape2d(packed, "packed")
     _shape2d(scales, "scales")
-    cols = 2 * pcols
+    if cols is None:
+        cols = 2 * pcols
+    elif (cols + 1) // 2 != pcols:
+        raise ValueError("cols does not match packed.shape[-1]")
     if out is None:
         out = torch.empty(tuple(packed.shape[:-1]) + (cols,), dtype=out_dtype, device=packed.device)
     check(lib.mx_dequantize(packed.data_ptr(), scales.data_ptr(), prow, cols, int(block),
@@ -173,9 +177,9 @@ def quantize_with_stats(x, block=32, fmt="e4m3", g=None, packed=None, scales=Non
         raise ValueError("x must be float32 or bfloat16")
     lead = tuple(x.shape[:-1])
     if packed is None:
-        packed = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
+        packed = torch.empty(lead + ((cols + 1) // 2,), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+        scales = torch.empty(lead + (-(-cols // block) if block else 0,), dtype=torch.uint8,
                              device=x.device)
     if out is None:
         out = torch.empty(STATS_BYTES, dtype=torch.uint8, device=x.device)

@@ -64,15 +64,19 @@ mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, in
   if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
     return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  if (cols % block != 0) return MX_ERR_INVALID_ARG;
   const int64_t numel = rows * cols;
   if (numel == 0) return MX_OK;
   if (!x || !packed || !scales) return MX_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales)) return MX_ERR_MISALIGNED;
   if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
-  const cudaError_t e = mxk::run_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
-                                          global_scale_fp16, packed, scales, stream, &n);
+  const cudaError_t e =
+      cols % block != 0
+          ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
+                            nullptr, nullptr, packed, scales, nullptr, false, nullptr, nullptr,
+                            stream, &n)
+          : mxk::run_quantize(x, xt == MX_BF16, numel, block, (int)fmt, global_scale_fp16, packed,
+                              scales, stream, &n);
   g_launches += n;
   return from_cuda(e);
 }
@@ -83,15 +87,18 @@ mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t ro
   if (!valid_dtype(yt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
     return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  if (cols % block != 0) return MX_ERR_INVALID_ARG;
   const int64_t numel = rows * cols;
   if (numel == 0) return MX_OK;
   if (!packed || !scales || !y) return MX_ERR_INVALID_ARG;
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(y)) return MX_ERR_MISALIGNED;
   if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
-  const cudaError_t e = mxk::run_dequantize(packed, scales, numel, block, (int)fmt,
-                                            global_scale_fp16, y, yt == MX_BF16, stream, &n);
+  const cudaError_t e =
+      cols % block != 0
+          ? mxk::run_ragged_dequantize(packed, scales, rows, cols, block, (int)fmt,
+                                       global_scale_fp16, y, yt == MX_BF16, stream, &n)
+          : mxk::run_dequantize(packed, scales, numel, block, (int)fmt, global_scale_fp16, y,
+                                yt == MX_BF16, stream, &n);
   g_launches += n;
   return from_cuda(e);
 }
@@ -103,15 +110,19 @@ mx_status mx_fake_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t col
       !shape_ok(rows, cols))
     return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  if (cols % block != 0) return MX_ERR_INVALID_ARG;
   const int64_t numel = rows * cols;
   if (numel == 0) return MX_OK;
   if (!x || !y) return MX_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return MX_ERR_MISALIGNED;
   if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
-  const cudaError_t e = mxk::run_fake_quantize(x, xt == MX_BF16, numel, block, (int)fmt,
-                                               global_scale_fp16, y, yt == MX_BF16, stream, &n);
+  const cudaError_t e =
+      cols % block != 0
+          ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
+                            nullptr, nullptr, nullptr, nullptr, y, yt == MX_BF16, nullptr,
+                            nullptr, stream, &n)
+          : mxk::run_fake_quantize(x, xt == MX_BF16, numel, block, (int)fmt, global_scale_fp16,
+                                   y, yt == MX_BF16, stream, &n);
   g_launches += n;
   return from_cuda(e);
 }
@@ -130,7 +141,6 @@ mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
   if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
     return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  if (cols % block != 0) return MX_ERR_INVALID_ARG;
   if ((packed == nullptr) != (scales == nullptr)) return MX_ERR_INVALID_ARG;
   if (!out_dev) return MX_ERR_INVALID_ARG;
   const int64_t numel = rows * cols;
@@ -142,8 +152,13 @@ mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
   if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
   const cudaError_t e =
-      mxk::run_error_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
-                           global_scale_fp16, packed, scales, out_dev, workspace, stream, &n);
+      numel != 0 && cols % block != 0
+          ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
+                            packed, scales, nullptr, nullptr, nullptr, false, out_dev, workspace,
+                            stream, &n)
+          : mxk::run_error_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
+                                 global_scale_fp16, packed, scales, out_dev, workspace, stream,
+                                 &n);
   g_launches += n;
   return from_cuda(e);
 }
@@ -155,7 +170,6 @@ mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t co
   if (!valid_dtype(xt) || !valid_fmt(fmt) || !valid_g(global_scale_fp16) || !shape_ok(rows, cols))
     return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  if (cols % block != 0) return MX_ERR_INVALID_ARG;
   if (!out_dev) return MX_ERR_INVALID_ARG;
   const int64_t numel = rows * cols;
   if (numel != 0 && (!x || !packed || !scales)) return MX_ERR_INVALID_ARG;
@@ -165,9 +179,14 @@ mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t co
     return MX_ERR_MISALIGNED;
   if (injected_failure()) return MX_ERR_CUDA;
   int n = 0;
-  const cudaError_t e = mxk::run_quantize_stats(numel ? x : nullptr, xt == MX_BF16, numel, block,
-                                                (int)fmt, global_scale_fp16, packed, scales,
-                                                out_dev, workspace, stream, &n);
+  const cudaError_t e =
+      numel != 0 && cols % block != 0
+          ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
+                            nullptr, nullptr, packed, scales, nullptr, false, out_dev, workspace,
+                            stream, &n)
+          : mxk::run_quantize_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
+                                    global_scale_fp16, packed, scales, out_dev, workspace, stream,
+                                    &n);
   g_launches += n;
   return from_cuda(e);
 }

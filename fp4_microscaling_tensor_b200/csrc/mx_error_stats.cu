@@ -46,11 +46,6 @@
 
 namespace mxk {
 
-struct StatsPartial {  // 64 bytes
-  double sse_elem, sse_max, sse_zero, pad;
-  unsigned long long n_zero_blocks, n_scale_sat, n_elem_sat, pad2;
-};
-
 struct StatsOut {  // layout of mx_error_stats_t
   double sse_elem, sse_max, sse_zero;
   long long numel, n_blocks, n_zero_blocks, n_scale_sat, n_elem_sat;
@@ -824,6 +819,14 @@ struct Workspace {
   unsigned int* counter(int t) const { return counters + 16 * t; }
 };
 constexpr int kMaxStatsGrid = kMaxReduceCtas - 2 * kMaxGroup;  // headers + tail slots
+
+cudaError_t launch_stats_final(const StatsPartial* part, int nparts, int64_t numel,
+                               int64_t nblocks, void* out, cudaStream_t stream, int* launches) {
+  k_error_stats_final<<<1, kThreads, 0, stream>>>(part, nparts, nullptr, numel, nblocks,
+                                                  static_cast<StatsOut*>(out));
+  ++*launches;
+  return cudaGetLastError();
+}
 
 // Zeroes the last-CTA counters of a group once the previous kernel in the stream is done with
 // them (launched with programmatic serialization, so its launch overlaps that kernel's tail and

@@ -159,6 +159,27 @@ cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int bloc
 cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,
                               uint16_t g_bits, uint8_t* packed, uint8_t* scales,
                               cudaStream_t stream, int* launches);
+// One CTA's partial sums of the error reduction (64 bytes; the workspace holds one per CTA after
+// a header of kMaxGroup 64-byte counters).
+struct StatsPartial {
+  double sse_elem, sse_max, sse_zero, pad;
+  unsigned long long n_zero_blocks, n_scale_sat, n_elem_sat, pad2;
+};
+// One CTA adds nparts partials in a fixed order and writes the mx_error_stats_t record.
+cudaError_t launch_stats_final(const StatsPartial* part, int nparts, int64_t numel,
+                               int64_t nblocks, void* out, cudaStream_t stream, int* launches);
+
+// Ragged tensors (cols % block != 0): one thread per block with plain per-element code.  Outputs
+// that are null are not produced: codes + scales (packed / scales), the round trip (y), the error
+// record (out, with workspace; from stored codes when packed_in is given).
+cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int block, int fmt,
+                       uint16_t g_bits, const uint8_t* packed_in, const uint8_t* scales_in,
+                       uint8_t* packed, uint8_t* scales, void* y, bool y_bf16, void* out,
+                       void* workspace, cudaStream_t stream, int* launches);
+cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
+                                  int64_t cols, int block, int fmt, uint16_t g_bits, void* y,
+                                  bool y_bf16, cudaStream_t stream, int* launches);
+
 // Zeroes one last-CTA counter once the previous kernel in the stream is done with it (a one-thread
 // kernel launched with programmatic serialization).
 cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches);

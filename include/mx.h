@@ -4,7 +4,8 @@
  * The method (microscaling article, hotelren.com/news/2192771, page titled "企业官网建设流程全解析";
  * cited below as [MX]):
  *   - a tensor is cut into blocks of N consecutive values, N in 4..256 ([MX] §1); here a block is
- *     N consecutive columns of one row, so cols must be a multiple of N;
+ *     N consecutive columns of one row; when N does not divide cols, the last block of every row
+ *     holds the cols mod N remaining values (its own absmax and scale, the same rule);
  *   - each block gets one FP8 scale s = Q_fp8(absmax / (6 g)) in E4M3 or UE5M3 ([MX] §3.1 items 1-2);
  *   - each value becomes the FP4 E2M1 code q = Q_fp4(x / (s g)) ([MX] §1, §3.1 item 2);
  *   - g is an optional per-tensor FP16 factor, value = FP4 x FP8_scale x FP16_scale ([MX] §3.1 item 3);
@@ -22,6 +23,11 @@
  *     was launched.  MX_ERR_CUDA reports a launch error (cudaGetLastError); faults that happen while
  *     a kernel runs surface at the caller's next synchronization, as usual in CUDA.
  *   - Every pointer argument must be 16-byte aligned (MX_ERR_MISALIGNED otherwise).
+ *   - Layout of codes and scales: row-major, a row's codes in ceil(cols/2) bytes (element 2k in
+ *     the low nibble of byte k, 2k+1 in the high nibble; an odd last element leaves the high
+ *     nibble 0) and its scales in ceil(cols/N) bytes.  For cols % N == 0 that is rows*cols/2 and
+ *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged") run on a one-thread-per-block
+ *     path; the grouped calls accept whole blocks only (cols % N != 0: MX_ERR_INVALID_ARG).
  *   - rows == 0 or cols == 0 is an empty tensor: quantize / dequantize enqueue nothing,
  *     mx_error_stats writes an all-zero result and mx_global_scale writes 1.0.
  *   - x must be finite: NaN or Inf in x gives unspecified codes (no kernel faults or hangs).
@@ -48,7 +54,7 @@ extern "C" {
 
 typedef enum {
   MX_OK = 0,
-  MX_ERR_INVALID_ARG = 1, /* null pointer, negative size, cols % block != 0, bad enum, bad g */
+  MX_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, bad g */
   MX_ERR_UNSUPPORTED = 2, /* block not one of 4, 8, 16, 32, 64, 128, 256 */
   MX_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
   MX_ERR_WORKSPACE = 4,   /* workspace pointer NULL or smaller than the *_workspace_size() value */
@@ -75,12 +81,13 @@ typedef struct {
 /* Quantize + pack ([MX] §3.1 item 2, with g from §3.1 item 3; packing from the 4-bit float
  * article, gtnt.cn/news/16247, §4.3, two FP4 values per byte).
  *   x       rows x cols values of type xt (MX_BF16 or MX_F32), device.
- *   block   N, one of 4, 8, 16, 32, 64, 128, 256; cols % block == 0.
+ *   block   N, one of 4, 8, 16, 32, 64, 128, 256 (any cols: a ragged last block per row when N
+ *           does not divide cols).
  *   fmt     scale format of the block scales.
- *   packed  OUT rows*cols/2 bytes, device: element 2k of the flattened tensor in the low nibble of
+ *   packed  OUT rows*ceil(cols/2) bytes, device: element 2k of a row in the low nibble of the row's
  *           byte k, element 2k+1 in the high nibble.  Nibble = sign<<3 | E2M1 magnitude code; the
  *           sign bit is x's sign bit (also for -0.0 and in zero-scale blocks).
- *   scales  OUT rows*cols/block bytes, device: the FP8 code of each block, row-major.
+ *   scales  OUT rows*ceil(cols/block) bytes, device: the FP8 code of each block, row-major.
  * A block whose scale rounds to zero (absmax <= 3 g smin) stores magnitude 0 in every element. */
 MX_API mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
                       mx_scale_fmt fmt, uint16_t global_scale_fp16, uint8_t* packed,

@@ -50,7 +50,7 @@ def test_quantize_rejects_bad_arguments():
     assert q(p=None) == INV
     assert q(s=None) == INV
     assert q(rows=-1) == INV
-    assert q(cols=48) == INV                      # 48 % 32 != 0
+    assert q(cols=-8) == INV                      # negative size
     assert q(block=12) == UNS
     assert q(block=512) == UNS
     assert q(block=2) == UNS
@@ -69,7 +69,7 @@ def test_dequantize_rejects_bad_arguments():
         return L.mx_dequantize(p, s, rows, cols, block, fmt, g, y, yt, None)
     assert dq(p=None) == INV
     assert dq(y=None) == INV
-    assert dq(cols=40) == INV
+    assert dq(cols=-40) == INV
     assert dq(block=24) == UNS
     assert dq(yt=2) == INV
     assert dq(g=0) == INV
@@ -88,7 +88,7 @@ def test_error_stats_rejects_bad_arguments():
     assert st(p=None, s=A) == INV
     assert st(w=None) == WS
     assert st(n=ws - 1) == WS
-    assert st(cols=50) == INV
+    assert st(cols=-50) == INV
     assert st(block=3) == UNS
     assert st(g=0xFFFF) == INV
     assert st(out=A + 8) == MIS
@@ -107,7 +107,7 @@ def test_quantize_stats_rejects_bad_arguments():
     assert qs(out=None) == INV
     assert qs(w=None) == WS
     assert qs(n=ws - 1) == WS
-    assert qs(cols=48) == INV
+    assert qs(cols=-48) == INV
     assert qs(block=64 * 8) == UNS
     assert qs(g=0x7C00) == INV
     assert qs(xt=5) == INV
@@ -183,7 +183,7 @@ def test_fake_quantize_rejects_bad_arguments():
     assert fq(y=None) == INV
     assert fq(yt=3) == INV
     assert fq(xt=3) == INV
-    assert fq(cols=40) == INV
+    assert fq(cols=-40) == INV
     assert fq(block=24) == UNS
     assert fq(g=0xFC00) == INV
     assert fq(x=A + 2) == MIS

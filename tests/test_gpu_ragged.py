@@ -1,0 +1,103 @@
+"""Parity of ragged tensors (cols not a multiple of the block size N) with the oracle.
+
+Rows of cols values end in a block of cols mod N values; codes take ceil(cols/2) bytes per row and
+scales ceil(cols/N).  Every output is written into a buffer with a guard band of 0xA5 bytes after
+it, which must stay untouched.  Codes, scales and dequantized values are bit-exact; error sums
+within 1e-5 relative, counts exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp4_microscaling_tensor_b200 as mx
+import oracle
+from fp4_microscaling_tensor_b200 import inputs
+from gpu_helpers import FMTS, assert_same, assert_stats, bits, special_values_bf16, u8
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 64
+SHAPES = [(5, 7, 4), (3, 13, 8), (17, 45, 32), (2, 300, 256), (9, 100, 64), (33, 129, 128),
+          (4, 3, 32), (7, 1, 4), (64, 1000, 16), (300, 33, 32)]
+G_CASES = (0x3C00, 0x2E66)
+
+
+def guarded(n, dtype=torch.uint8):
+    t = torch.full((n * torch.empty((), dtype=dtype).element_size() + GUARD,), 0xA5,
+                   dtype=torch.uint8, device="cuda")
+    return t, t[: n * torch.empty((), dtype=dtype).element_size()].view(dtype)
+
+
+def guard_ok(t, n_bytes, what):
+    tail = t[n_bytes:].cpu().numpy()
+    assert np.all(tail == 0xA5), f"{what}: write past the end"
+
+
+@pytest.mark.parametrize("rows,cols,block", SHAPES)
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ragged_parity(rows, cols, block, fmt, dtype):
+    g = G_CASES[(rows + cols) % 2]
+    x = special_values_bf16(fmt, g, rows * cols, seed=rows * 31 + cols).to(dtype)
+    x = x.reshape(rows, cols).cuda()
+    xo = inputs.to_oracle(x)
+    pb, nb = (cols + 1) // 2, -(-cols // block)
+    po, so = oracle.quantize(xo, rows, cols, block, fmt, g)
+
+    # quantize
+    pbuf, p = guarded(rows * pb)
+    sbuf, s = guarded(rows * nb)
+    mx.quantize(x, block, fmt, g, packed=p.view(rows, pb), scales=s.view(rows, nb))
+    torch.cuda.synchronize()
+    assert_same(u8(s), so, "ragged scales")
+    assert_same(u8(p), po, "ragged packed")
+    guard_ok(pbuf, rows * pb, "packed")
+    guard_ok(sbuf, rows * nb, "scales")
+
+    # dequantize, both output types
+    pd, sd = p.view(rows, pb), s.view(rows, nb)
+    for dt, bf in ((torch.bfloat16, True), (torch.float32, False)):
+        ybuf, y = guarded(rows * cols, dt)
+        mx.dequantize(pd, sd, block, fmt, g, out=y.view(rows, cols), cols=cols)
+        torch.cuda.synchronize()
+        yo = oracle.dequantize(po, so, rows, cols, block, fmt, g, out_bf16=bf)
+        assert_same(bits(y), yo if bf else yo.view(np.uint32), f"ragged dequant {dt}")
+        guard_ok(ybuf, rows * cols * (2 if bf else 4), "y")
+        # fake quantize = dequantize(quantize(x)) in one pass
+        fbuf, yf = guarded(rows * cols, dt)
+        mx.fake_quantize(x, block, fmt, g, out_dtype=dt, out=yf.view(rows, cols))
+        torch.cuda.synchronize()
+        assert_same(bits(yf), yo if bf else yo.view(np.uint32), f"ragged fake quantize {dt}")
+        guard_ok(fbuf, rows * cols * (2 if bf else 4), "fake y")
+
+    # error reduction: recomputed codes, stored codes, fused with quantize
+    ref = oracle.error_stats(xo, rows, cols, block, fmt, g)
+    got = mx.error_stats(x, block, fmt, g).to_dict()
+    assert_stats(got, ref, "ragged stats (recomputed)")
+    got = mx.error_stats(x, block, fmt, g, packed=pd, scales=sd).to_dict()
+    assert_stats(got, ref, "ragged stats (stored codes)")
+    p2buf, p2 = guarded(rows * pb)
+    s2buf, s2 = guarded(rows * nb)
+    _, _, st = mx.quantize_with_stats(x, block, fmt, g, packed=p2.view(rows, pb),
+                                      scales=s2.view(rows, nb))
+    assert_stats(st.to_dict(), ref, "ragged fused")
+    assert_same(u8(p2), po, "ragged fused packed")
+    assert_same(u8(s2), so, "ragged fused scales")
+    guard_ok(p2buf, rows * pb, "fused packed")
+    guard_ok(s2buf, rows * nb, "fused scales")
+
+
+def test_ragged_large_sampled_rows():
+    # 4096 x 4100 (N = 32: 128 whole blocks and a block of 4 per row), N(0, 0.02^2): whole tensor
+    # quantized on the GPU, 256 seeded rows compared with the oracle, the error record whole
+    rows, cols, block = 4096, 4100, 32
+    x = inputs.normal((rows, cols), 0.02, seed=4100).cuda()
+    p, s, st = mx.quantize_with_stats(x, block, "e4m3")
+    xo = inputs.to_oracle(x)
+    ref = oracle.error_stats(xo, rows, cols, block, mx.E4M3)
+    assert_stats(st.to_dict(), ref, "ragged 4096x4100")
+    sel = np.sort(np.random.default_rng(7).choice(rows, 256, replace=False))
+    xs = xo.reshape(rows, cols)[sel].reshape(-1)
+    po, so = oracle.quantize(xs, len(sel), cols, block, mx.E4M3)
+    assert_same(u8(p.view(rows, -1)[torch.from_numpy(sel).cuda()]), po, "sampled packed")
+    assert_same(u8(s.view(rows, -1)[torch.from_numpy(sel).cuda()]), so, "sampled scales")
