@@ -607,7 +607,11 @@ def run_case(args):
     n, fmt, G = args.block, mx.fmt_code(args.fmt), args.group
     xs = [inputs.normal((rows, cols), 0.02, k, device=dev) for k in range(G)]
     numel = rows * cols * G
-    packed, scales = mx.quantize_group(xs, n, fmt)
+    if G == 1:  # (also ragged shapes, which grouped calls do not take)
+        p0, s0 = mx.quantize(xs[0], n, fmt)
+        packed, scales = [p0], [s0]
+    else:
+        packed, scales = mx.quantize_group(xs, n, fmt)
     ys = [torch.empty(rows, cols, dtype=torch.bfloat16, device=dev) for _ in range(G)]
     out = torch.empty(G, 64, dtype=torch.uint8, device=dev)
     ws = mx.stats_workspace(dev)
@@ -616,7 +620,7 @@ def run_case(args):
         x, p, sc, y = xs[0], packed[0], scales[0], ys[0]
         calls = {
             "quantize": lambda: mx.quantize(x, n, fmt, packed=p, scales=sc),
-            "dequantize": lambda: mx.dequantize(p, sc, n, fmt, out=y),
+            "dequantize": lambda: mx.dequantize(p, sc, n, fmt, out=y, cols=cols),
             "stats": lambda: mx.error_stats(x, n, fmt, packed=p, scales=sc, out=out[0],
                                             workspace=ws),
             "stats-recompute": lambda: mx.error_stats(x, n, fmt, out=out[0], workspace=ws),
@@ -634,9 +638,9 @@ def run_case(args):
         }
         if args.case not in calls:
             raise SystemExit(f"--group applies to {sorted(calls)}")
+    code_bytes = G * rows * (((cols + 1) // 2) + -(-cols // n))  # codes + scales (any cols)
     nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0,
-              "fake-quantize": numel * 4.0}.get(
-        args.case, numel * (2.5 + 1.0 / n))
+              "fake-quantize": numel * 4.0}.get(args.case, numel * 2.0 + code_bytes)
     fn = calls[args.case]
     fn()
     torch.cuda.synchronize()

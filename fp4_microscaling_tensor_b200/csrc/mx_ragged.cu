@@ -8,11 +8,11 @@
 // another.  For cols % N == 0 this is the layout of the whole-block kernels, which handle that
 // case; these kernels cover the rest.
 //
-// One thread per block, grid-stride, with plain per-element code: absmax (first index of the
-// largest |x|), scale s = RNE_fmt(a / (6 g)) and quotients x / (S g) by IEEE division (a correctly
-// rounded quotient lands on a rounding midpoint only when the exact quotient does), E2M1 codes by
-// the hardware RNE-saturating conversion.  Errors are formed and summed in double; each CTA
-// writes one partial and one CTA adds the partials in a fixed order.
+// One warp per row, lanes over consecutive element pairs (coalesced loads and byte stores), block
+// maxima by segmented warp reductions; scale s = RNE_fmt(a / (6 g)) and quotients x / (S g) by
+// IEEE division (a correctly rounded quotient lands on a rounding midpoint only when the exact
+// quotient does), E2M1 codes by the hardware RNE-saturating conversion.  Errors are formed and
+// summed in double; each CTA writes one partial and one CTA adds the partials in a fixed order.
 #include "mx_device.cuh"
 #include "mx_launch.h"
 
@@ -59,70 +59,151 @@ __device__ __forceinline__ unsigned long long warp_sum_u(unsigned long long v) {
   return v;
 }
 
-template <typename T, int FMT>
-__global__ void __launch_bounds__(kThreads) k_ragged_blocks(const __grid_constant__ RaggedArgs a) {
+// One warp per row (grid-stride over rows).  A warp step covers 256 elements of the row: lane l
+// holds the 8 consecutive elements 8 l .. 8 l + 7 of the step (one 16-byte load when the row
+// start allows it, else element loads), i.e. two blocks of 4, one block of 8, or 1 / G of a block
+// of N = 8 G; a block's absmax and first max index are in-lane or segmented warp reductions over
+// G lanes.  Elements past the row end are absent (zero for the absmax, nothing stored or summed).
+// bf16 inputs use the exact reciprocal-multiply quotients of the whole-block kernels (snap21 for
+// the scale, snap_quotient2 for the elements); fp32 inputs the IEEE division.
+template <typename T, int FMT, int N>
+__global__ void __launch_bounds__(kThreads) k_ragged_rows(const __grid_constant__ RaggedArgs a) {
+  constexpr bool BF16 = sizeof(T) == 2;
+  constexpr int BPL = N == 4 ? 2 : 1;          // blocks per lane
+  constexpr int G = N <= 8 ? 1 : N / 8;        // lanes per block
+  constexpr int EB = N == 4 ? 4 : 8;           // elements of a lane in one block
   const float g = fp16_bits_to_float((uint16_t)a.g_bits);
   const float g6 = __fmul_rn(6.0f, g);                   // exact
+  const float r6 = __frcp_rn(g6);
   const float sat_thr = __fmul_rn(g6, scale_max<FMT>());  // exact
-  const int64_t nb = (a.cols + a.N - 1) / a.N, pb = (a.cols + 1) / 2;
-  const int64_t total = a.rows * nb;
+  const int cols = (int)a.cols;
+  const int nb = (cols + N - 1) / N, pb = (cols + 1) / 2;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   double e_elem = 0.0, e_max = 0.0, e_zero = 0.0;
   unsigned long long c_zero = 0, c_ssat = 0, c_esat = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / nb, b = i - r * nb, j0 = b * a.N;  // j0 even: whole bytes
-    const int len = (int)(a.cols - j0 < a.N ? a.cols - j0 : a.N);
-    const T* xr = static_cast<const T*>(a.x) + r * a.cols + j0;
-    float amax = 0.0f;
-    int imax = 0;
-    for (int k = 0; k < len; ++k) {
-      const float v = fabsf(load_x(xr + k));
-      if (v > amax) { amax = v; imax = k; }
-    }
-    const uint32_t s = a.packed_in ? (uint32_t)a.scales_in[r * nb + b]
-                                   : encode_scale<FMT>(__fdiv_rn(amax, g6));
-    const float D = __fmul_rn(scale_value((int)s, FMT), g);  // exact
-    if (a.scales) a.scales[r * nb + b] = (uint8_t)s;
-    const int64_t byte0 = r * pb + j0 / 2;
-    for (int k = 0; k < len; k += 2) {
-      const bool two = k + 1 < len;
-      const float v0 = load_x(xr + k), v1 = two ? load_x(xr + k + 1) : 0.0f;
-      uint32_t c;
-      if (a.packed_in) {
-        c = a.packed_in[byte0 + k / 2];
+  for (int64_t r = warp; r < a.rows; r += nwarps) {
+    const T* xr = static_cast<const T*>(a.x) + r * a.cols;
+    const bool x_aligned = ((r * a.cols) & (BF16 ? 7 : 3)) == 0;  // 16-byte row start
+    const int64_t prow = r * pb, srow = r * nb;
+    for (int e0 = 0; e0 < cols; e0 += 256) {
+      const int j0 = e0 + 8 * lane;  // this lane's first element
+      const int nv = max(0, min(8, cols - j0));
+      float v[8];
+      if (nv == 8 && x_aligned) {
+        if constexpr (BF16) {
+          const uint4 w = *reinterpret_cast<const uint4*>(xr + j0);
+          v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+          v[4] = bf16lo(w.z); v[5] = bf16hi(w.z); v[6] = bf16lo(w.w); v[7] = bf16hi(w.w);
+        } else {
+          const float4 u0 = *reinterpret_cast<const float4*>(xr + j0);
+          const float4 u1 = *reinterpret_cast<const float4*>(xr + j0 + 4);
+          v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+          v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+        }
       } else {
-        const float q0 = D > 0.0f ? __fdiv_rn(v0, D) : __fmul_rn(v0, 0.0f);
-        const float q1 = D > 0.0f ? __fdiv_rn(v1, D) : __fmul_rn(v1, 0.0f);
-        c = cvt_e2m1x8(q0, q1, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & (two ? 0xFFu : 0xFu);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = k < nv ? load_x(xr + j0 + k) : 0.0f;
       }
-      if (a.packed) a.packed[byte0 + k / 2] = (uint8_t)c;
-      if (a.y) {
-        store_y(a.y, r * a.cols + j0 + k, __fmul_rn(e2m1_to_float(c & 0xF), D), a.y_bf16);
-        if (two) store_y(a.y, r * a.cols + j0 + k + 1, __fmul_rn(e2m1_to_float(c >> 4), D),
-                         a.y_bf16);
-      }
-      if (a.part) {
-        for (int t = 0; t < 1 + (int)two; ++t) {
-          const float v = t ? v1 : v0;
-          const double yv = (double)__fmul_rn(e2m1_to_float((c >> (4 * t)) & 0xF), D);  // exact
-          const double d = (double)v - yv;                                           // exact
-          if (!(D > 0.0f)) e_zero += (double)v * (double)v;
-          else if (k + t == imax) e_max += d * d;
-          else e_elem += d * d;
-          if (D > 0.0f && fabsf(v) > __fmul_rn(6.0f, D)) ++c_esat;
+      uint32_t codes = 0;  // 8 codes, element k in nibble k
+#pragma unroll
+      for (int h = 0; h < BPL; ++h) {
+        const float* vb = v + EB * h;
+        const int jb0 = j0 + EB * h;           // this lane's first element of the block
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < EB; ++k) m = fmaxf(m, fabsf(vb[k]));
+#pragma unroll
+        for (int off = 1; off < G; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const int jb = N >= 16 ? jb0 - EB * (lane & (G - 1)) : jb0;  // first element of the block
+        const int b = jb / N;
+        const bool block_here = jb < cols;
+        const bool leader = (lane & (G - 1)) == 0;
+        uint32_t s = 0;
+        if (a.packed_in) {
+          if (block_here) s = a.scales_in[srow + b];
+        } else {
+          s = BF16 ? encode_scale<FMT>(snap21(__fmul_rn(m, r6)))
+                   : encode_scale<FMT>(__fdiv_rn(m, g6));
+        }
+        const float D = __fmul_rn(scale_value((int)s, FMT), g);  // exact
+        if (a.scales && leader && block_here) a.scales[srow + b] = (uint8_t)s;
+        uint32_t cb;  // this block's codes of this lane (EB nibbles)
+        if (a.packed_in) {
+          cb = 0;
+#pragma unroll
+          for (int k = 0; k < EB; k += 2)
+            if (k < nv - EB * h) cb |= (uint32_t)a.packed_in[prow + (jb0 + k) / 2] << (4 * k);
+        } else {
+          float q[8];
+          if constexpr (BF16) {
+            const float rD = D > 0.0f ? __frcp_rn(D) : 0.0f;
+#pragma unroll
+            for (int k = 0; k < EB; k += 2) {
+              const float2 qq =
+                  snap_quotient2(__float_as_uint(vb[k]), __float_as_uint(vb[k + 1]), rD);
+              q[k] = qq.x;
+              q[k + 1] = qq.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < EB; ++k)
+              q[k] = D > 0.0f ? __fdiv_rn(vb[k], D) : __fmul_rn(vb[k], 0.0f);
+          }
+          if constexpr (EB == 8) cb = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+          else cb = cvt_e2m1x8(q[0], q[1], q[2], q[3], 0.f, 0.f, 0.f, 0.f) & 0xFFFFu;
+        }
+        codes |= cb << (4 * EB * h);
+        if (a.part) {
+          // first index of the block maximum: in-lane, then over the block's lanes
+          int imax = INT_MAX;
+#pragma unroll
+          for (int k = EB - 1; k >= 0; --k)
+            if (k < nv - EB * h && fabsf(vb[k]) == m) imax = jb0 + k;
+#pragma unroll
+          for (int off = 1; off < G; off <<= 1) imax = min(imax, __shfl_xor_sync(0xffffffffu, imax, off));
+#pragma unroll
+          for (int k = 0; k < EB; ++k) {
+            if (k >= nv - EB * h) break;
+            const float xv = vb[k];
+            const double yv = (double)__fmul_rn(e2m1_to_float((cb >> (4 * k)) & 0xF), D);
+            const double d = (double)xv - yv;  // exact
+            if (!(D > 0.0f)) e_zero += (double)xv * (double)xv;
+            else if (jb0 + k == imax) e_max += d * d;
+            else e_elem += d * d;
+            if (D > 0.0f && fabsf(xv) > __fmul_rn(6.0f, D)) ++c_esat;
+          }
+          if (leader && block_here) {
+            c_zero += D > 0.0f ? 0 : 1;
+            c_ssat += m > sat_thr ? 1 : 0;
+          }
+        }
+        if (a.y) {
+#pragma unroll
+          for (int k = 0; k < EB; ++k)
+            if (k < nv - EB * h)
+              store_y(a.y, r * a.cols + jb0 + k,
+                      __fmul_rn(e2m1_to_float((cb >> (4 * k)) & 0xF), D), a.y_bf16);
         }
       }
-    }
-    if (a.part) {
-      c_zero += D > 0.0f ? 0 : 1;
-      c_ssat += amax > sat_thr ? 1 : 0;
+      if (a.packed && nv > 0) {
+        if (nv & 1) codes &= ~(0xFu << (4 * nv));  // an odd row end leaves the high nibble 0
+        if (nv == 8 && ((prow + j0 / 2) & 3) == 0) {
+          *reinterpret_cast<uint32_t*>(a.packed + prow + j0 / 2) = codes;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (2 * k < nv) a.packed[prow + j0 / 2 + k] = (uint8_t)(codes >> (8 * k));
+        }
+      }
     }
   }
   if (!a.part) return;
   // CTA partial, fixed order (lanes, then warps)
   __shared__ double sd[3][kThreads / 32];
   __shared__ unsigned long long su[3][kThreads / 32];
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
   e_elem = warp_sum_d(e_elem); e_max = warp_sum_d(e_max); e_zero = warp_sum_d(e_zero);
   c_zero = warp_sum_u(c_zero); c_ssat = warp_sum_u(c_ssat); c_esat = warp_sum_u(c_esat);
   if (lane == 0) {
@@ -140,36 +221,82 @@ __global__ void __launch_bounds__(kThreads) k_ragged_blocks(const __grid_constan
   }
 }
 
-// One thread per code byte: y = E2M1 x S x g (exact), bf16 = its round to nearest even.
-template <int FMT>
+// One warp per row: lane l takes code bytes l, l + 32, ... of the row; y = E2M1 x S x g (exact),
+// bf16 = its round to nearest even.  Both elements of a byte are in one block (blocks start at
+// even columns).
+template <int FMT, int LOGN>
 __global__ void __launch_bounds__(kThreads)
     k_ragged_dequantize(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-                        int64_t rows, int64_t cols, int N, uint16_t g_bits, void* y, int y_bf16) {
+                        int64_t rows, int64_t cols, uint16_t g_bits, void* y, int y_bf16) {
   const float g = fp16_bits_to_float(g_bits);
-  const int64_t nb = (cols + N - 1) / N, pb = (cols + 1) / 2, total = rows * pb;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / pb, j = 2 * (i - r * pb);
-    const uint32_t c = packed[i];
-    const float D = __fmul_rn(scale_value((int)scales[r * nb + j / N], FMT), g);  // one block
-    store_y(y, r * cols + j, __fmul_rn(e2m1_to_float(c & 0xF), D), y_bf16);
-    if (j + 1 < cols) store_y(y, r * cols + j + 1, __fmul_rn(e2m1_to_float(c >> 4), D), y_bf16);
+  const int64_t nb = (cols + (1 << LOGN) - 1) >> LOGN, pb = (cols + 1) / 2;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp; r < rows; r += nwarps) {
+    for (int64_t k = lane; k < pb; k += 32) {
+      const int64_t j = 2 * k;
+      const uint32_t c = packed[r * pb + k];
+      const float D = __fmul_rn(scale_value((int)scales[r * nb + (j >> LOGN)], FMT), g);
+      store_y(y, r * cols + j, __fmul_rn(e2m1_to_float(c & 0xF), D), y_bf16);
+      if (j + 1 < cols)
+        store_y(y, r * cols + j + 1, __fmul_rn(e2m1_to_float(c >> 4), D), y_bf16);
+    }
   }
 }
 
 constexpr int kMaxRaggedGrid = kMaxReduceCtas - 2 * kMaxGroup;  // partials after the header
 
-template <typename T, int FMT>
-cudaError_t launch_ragged(const RaggedArgs& args, int64_t nblocks, void* out, cudaStream_t stream,
-                          int* launches) {
-  const int grid = persistent_grid((const void*)k_ragged_blocks<T, FMT>, nblocks, 1,
+template <typename T, int FMT, int N>
+cudaError_t launch_rows(const RaggedArgs& args, int64_t nblocks, void* out, cudaStream_t stream,
+                        int* launches) {
+  // one warp per row: rows / 8 CTAs, at most the resident CTAs (and the partial slots)
+  const int grid = persistent_grid((const void*)k_ragged_rows<T, FMT, N>, args.rows * 32, 1,
                                    kMaxRaggedGrid);
-  k_ragged_blocks<T, FMT><<<grid, kThreads, 0, stream>>>(args);
+  k_ragged_rows<T, FMT, N><<<grid, kThreads, 0, stream>>>(args);
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && args.part)
     e = launch_stats_final(args.part, grid, args.rows * args.cols, nblocks, out, stream, launches);
   return e;
+}
+
+template <typename T, int FMT>
+cudaError_t launch_ragged(const RaggedArgs& args, int64_t nblocks, void* out, cudaStream_t stream,
+                          int* launches) {
+  switch (args.N) {
+    case 4: return launch_rows<T, FMT, 4>(args, nblocks, out, stream, launches);
+    case 8: return launch_rows<T, FMT, 8>(args, nblocks, out, stream, launches);
+    case 16: return launch_rows<T, FMT, 16>(args, nblocks, out, stream, launches);
+    case 32: return launch_rows<T, FMT, 32>(args, nblocks, out, stream, launches);
+    case 64: return launch_rows<T, FMT, 64>(args, nblocks, out, stream, launches);
+    case 128: return launch_rows<T, FMT, 128>(args, nblocks, out, stream, launches);
+    default: return launch_rows<T, FMT, 256>(args, nblocks, out, stream, launches);
+  }
+}
+
+template <int FMT, int LOGN>
+cudaError_t launch_dq(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t cols,
+                      uint16_t g_bits, void* y, bool y_bf16, cudaStream_t stream) {
+  const int grid = persistent_grid((const void*)k_ragged_dequantize<FMT, LOGN>, rows * 32, 1);
+  k_ragged_dequantize<FMT, LOGN><<<grid, kThreads, 0, stream>>>(packed, scales, rows, cols,
+                                                                 g_bits, y, y_bf16 ? 1 : 0);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_dq_fmt(const uint8_t* packed, const uint8_t* scales, int64_t rows,
+                          int64_t cols, int block, uint16_t g_bits, void* y, bool y_bf16,
+                          cudaStream_t stream) {
+  switch (block) {
+    case 4: return launch_dq<FMT, 2>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 8: return launch_dq<FMT, 3>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 16: return launch_dq<FMT, 4>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 32: return launch_dq<FMT, 5>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 64: return launch_dq<FMT, 6>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 128: return launch_dq<FMT, 7>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    default: return launch_dq<FMT, 8>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+  }
 }
 
 }  // namespace
@@ -178,6 +305,7 @@ cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int
                        uint16_t g_bits, const uint8_t* packed_in, const uint8_t* scales_in,
                        uint8_t* packed, uint8_t* scales, void* y, bool y_bf16, void* out,
                        void* workspace, cudaStream_t stream, int* launches) {
+  if (cols > (int64_t(1) << 30)) return cudaErrorInvalidValue;  // in-row indices are 32-bit
   RaggedArgs args{x, rows, cols, block, g_bits, packed_in, scales_in, packed, scales, y,
                   y_bf16 ? 1 : 0, nullptr};
   if (out)  // partials after the workspace's 64-byte counter headers
@@ -193,18 +321,10 @@ cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int
 cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
                                   int64_t cols, int block, int fmt, uint16_t g_bits, void* y,
                                   bool y_bf16, cudaStream_t stream, int* launches) {
-  const int64_t bytes = rows * ((cols + 1) / 2);
-  if (fmt == kUE5M3) {
-    const int grid = persistent_grid((const void*)k_ragged_dequantize<kUE5M3>, bytes, 1);
-    k_ragged_dequantize<kUE5M3><<<grid, kThreads, 0, stream>>>(packed, scales, rows, cols, block,
-                                                               g_bits, y, y_bf16 ? 1 : 0);
-  } else {
-    const int grid = persistent_grid((const void*)k_ragged_dequantize<kE4M3>, bytes, 1);
-    k_ragged_dequantize<kE4M3><<<grid, kThreads, 0, stream>>>(packed, scales, rows, cols, block,
-                                                              g_bits, y, y_bf16 ? 1 : 0);
-  }
   ++*launches;
-  return cudaGetLastError();
+  return fmt == kUE5M3
+             ? launch_dq_fmt<kUE5M3>(packed, scales, rows, cols, block, g_bits, y, y_bf16, stream)
+             : launch_dq_fmt<kE4M3>(packed, scales, rows, cols, block, g_bits, y, y_bf16, stream);
 }
 
 }  // namespace mxk

@@ -26,8 +26,9 @@
  *   - Layout of codes and scales: row-major, a row's codes in ceil(cols/2) bytes (element 2k in
  *     the low nibble of byte k, 2k+1 in the high nibble; an odd last element leaves the high
  *     nibble 0) and its scales in ceil(cols/N) bytes.  For cols % N == 0 that is rows*cols/2 and
- *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged") run on a one-thread-per-block
- *     path; the grouped calls accept whole blocks only (cols % N != 0: MX_ERR_INVALID_ARG).
+ *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged") run on a row-wise path (one
+ *     warp per row; cols up to 2^30, else MX_ERR_CUDA); the grouped calls accept whole blocks
+ *     only (cols % N != 0: MX_ERR_INVALID_ARG).
  *   - rows == 0 or cols == 0 is an empty tensor: quantize / dequantize enqueue nothing,
  *     mx_error_stats writes an all-zero result and mx_global_scale writes 1.0.
  *   - x must be finite: NaN or Inf in x gives unspecified codes (no kernel faults or hangs).
