@@ -43,6 +43,9 @@
 #ifndef MX_ST_MINB_SMALL  // the same for N <= 8 (short per-block work: more warps hide the latency)
 #define MX_ST_MINB_SMALL 3
 #endif
+#ifndef MX_QS_MINB  // the same for the small-block kernel with recomputed codes
+#define MX_QS_MINB 2
+#endif
 
 namespace mxk {
 
@@ -65,6 +68,7 @@ struct Acc {
   double elem = 0.0, mx = 0.0, zero = 0.0;
   unsigned n_zero = 0, n_ssat = 0;
   float n_esat = 0.0f;  // clipped elements (exact: a thread sees far fewer than 2^24)
+  float n_zero_f = 0.0f, n_ssat_f = 0.0f;  // the same counts kept in fp32 (small-block kernel)
 };
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -84,8 +88,10 @@ __device__ void write_partial(const Acc& acc, StatsPartial* slot) {
   __shared__ unsigned long long su[3][kThreads / 32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double a0 = warp_sum(acc.elem), a1 = warp_sum(acc.mx), a2 = warp_sum(acc.zero);
-  const unsigned long long c0 = warp_sum((unsigned long long)acc.n_zero);
-  const unsigned long long c1 = warp_sum((unsigned long long)acc.n_ssat);
+  const unsigned long long c0 = warp_sum((unsigned long long)acc.n_zero +
+                                         (unsigned long long)acc.n_zero_f);
+  const unsigned long long c1 = warp_sum((unsigned long long)acc.n_ssat +
+                                         (unsigned long long)acc.n_ssat_f);
   const unsigned long long c2 = warp_sum((unsigned long long)acc.n_esat);
   if (lane == 0) {
     sd[0][w] = a0; sd[1][w] = a1; sd[2][w] = a2;
@@ -253,6 +259,41 @@ __device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, 
 #undef MX_PAIR_TAIL
 }
 
+// Core of a bf16 block slice with recomputed codes (blocks of 16 and more), one word at a time:
+// every element's scaled error d goes into the f32x2 sum of squares lt2 -- the max-valued ones
+// included, the first of them is taken out per block, see slice_finish_closed -- and the clipped
+// elements (|x| > 6 S g, i.e. |x| above S2 = RD_bf16(6 S g)) are counted per half in nsat2 as
+// bf16x2 integers (exact: a half sees at most 128 of them).
+template <int J>
+__device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
+                                              float sc, float nDq, uint32_t S2,
+                                              unsigned long long& lt2, uint32_t& nsat2) {
+  static_assert(J >= 0 && J < 4, "byte index");
+  asm("{\n\t"
+      ".reg .b32 blo, bhi, aw, t, m;\n\t"
+      ".reg .b64 x2, s2, b2, q2, d2;\n\t"
+      "mov.b64 x2, {%8, %9};\n\t"
+      "mov.b64 s2, {%3, %3};\n\t"
+      "mul.rn.f32x2 x2, x2, s2;\n\t"
+      "mul.lo.u32 t, %2, %6;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 blo, t, 0x81c00000;\n\t"
+      "mul.lo.u32 t, %2, %7;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 bhi, t, 0x81c00000;\n\t"
+      "mov.b64 b2, {blo, bhi};\n\t"
+      "mov.b64 q2, {%4, %4};\n\t"
+      "fma.rn.f32x2 d2, b2, q2, x2;\n\t"
+      "fma.rn.f32x2 %0, d2, d2, %0;\n\t"
+      "and.b32 aw, %10, 0x7fff7fff;\n\t"
+      "set.gt.bf16x2.bf16x2 m, aw, %5;\n\t"
+      "add.rn.bf16x2 %1, %1, m;\n\t"
+      "}"
+      : "+l"(lt2), "+r"(nsat2)
+      : "r"(cw), "f"(sc), "f"(nDq), "r"(S2), "n"(1u << (28 - 8 * J)), "n"(1u << (24 - 8 * J)),
+        "r"(lo), "r"(hi), "r"(w));
+}
+
 // Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
 // cnt the number of max-valued elements, nsat the clipped elements.  xval(k) / code(k) (k a
 // compile-time constant) serve the exact path: ties of the maximum in this lane, or a slice that
@@ -389,6 +430,63 @@ __device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, f
   }
 }
 
+// Tail of a bf16 block slice with recomputed codes (blocks of 16 and more).  lt2 sums the scaled
+// squares of all the slice's elements; every max-valued element has the error dmax (scaled), so
+// the lane holding the block's first max element moves dmax^2 (exact in double) from that sum to
+// SSE_max and the rest stays in SSE_elem (other max-valued elements included, as they should).
+// The subtraction only loses digits when dmax^2 dominates the slice's sum; a slice whose remainder
+// is below dmax^2 / 8, or whose sum is below 2^-80 (squares below 2^-126 could be lost), is redone
+// exactly in double.  has_max: this lane holds a max-valued element.
+template <int NE, int L, typename XF, typename CF>
+__device__ __forceinline__ void slice_finish_closed(Acc& acc, int lane, bool ok, bool has_max,
+                                                    float a, float D, float sat_thr,
+                                                    const SliceSetup& st,
+                                                    unsigned long long lt2, float dmax,
+                                                    uint32_t nsat2, XF xval, CF code) {
+  bool is_first_lane = has_max;
+  if constexpr (L > 1) {
+    const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
+    const unsigned has = __ballot_sync(0xffffffffu, has_max) & gmask;
+    is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
+  }
+  float l0, l1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lt2));
+  const float lt = __fadd_rn(l0, l1);
+  double rest = 0.0, first = 0.0, others = 0.0;
+  bool exact = lt < 0x1p-80f;
+  if (!exact) {
+    rest = (double)lt * unscale_sq(st.E);
+    if (is_first_lane && !st.zero_blk) {
+      first = (double)dmax * (double)dmax * unscale_sq(st.E);  // exact
+      rest -= first;
+      exact = rest < 0.125 * first;
+    }
+  }
+  if (exact) {
+    rest = first = others = 0.0;
+    exact_slice<NE, false>(a, D, xval, code, rest, first, others);
+    rest += others;
+    if (!is_first_lane) rest += first, first = 0.0;
+  }
+  if (st.zero_blk) {
+    acc.zero += rest + first;
+  } else {
+    acc.elem += rest;
+    acc.mx += first;
+    float c0, c1;
+    asm("{\n\t.reg .b16 h0, h1;\n\t"
+        "mov.b32 {h0, h1}, %2;\n\t"
+        "cvt.f32.bf16 %0, h0;\n\t"
+        "cvt.f32.bf16 %1, h1;\n\t}"
+        : "=f"(c0), "=f"(c1) : "r"(nsat2));
+    acc.n_esat += c0 + c1;
+  }
+  if (ok && (lane & (L - 1)) == 0) {
+    acc.n_zero += st.zero_blk ? 1u : 0u;
+    acc.n_ssat += (a > sat_thr) ? 1u : 0u;
+  }
+}
+
 // Generic block slice of NE elements (fp32 input): xval(k) value, code(k) a word whose low nibble
 // is element k's code (k a compile-time constant after unrolling).  min_abs: the slice's min|x|
 // (zeros included); a nonzero value below 2^-30 a could lose digits to fp32 underflow.
@@ -513,6 +611,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
     const bool ok = i < nitems;
     float a_b[BPI], D_b[BPI], r_b[BPI];
     uint32_t m_b[BPI];
+    bool own_b[BPI];      // this lane holds a max-valued element of block b
     uint32_t sc_all = 0;  // scale codes of the item's blocks, byte b = block b
 #pragma unroll
     for (int b = 0; b < BPI; ++b) {
@@ -522,6 +621,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       for (int k = 1; k < BW; ++k) t = bf16x2_absmax(t, wb[k]);
       t &= 0x7FFF7FFFu;
       uint32_t m = max(t & 0xFFFFu, t >> 16);
+      const uint32_t m_lane = m;
 #pragma unroll
       for (int off = 1; off < L; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
       const float a = __uint_as_float(m << 16);
@@ -534,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       }
       a_b[b] = a;
       m_b[b] = m;
+      own_b[b] = m_lane == m;
       D_b[b] = s_D[s];
       sc_all |= s << (8 * b);
     }
@@ -579,8 +680,21 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       const uint32_t A2 = m_b[b] * 0x10001u, S2 = sb * 0x10001u;
       float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f, dmax = 0.0f;
       const float nD = st.nDq;
+      unsigned long long lt2 = 0ull;
+      uint32_t nsat2 = 0u;
 #pragma unroll
-      for (int k = 0; k < BW; ++k) {
+      for (int k = 0; k < BW && CLOSED; ++k) {
+        const int wi = b * BW + k;
+        const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
+        switch (wi & 3) {
+          case 0: pair_step_all<0>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
+          case 1: pair_step_all<1>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
+          case 2: pair_step_all<2>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
+          default: pair_step_all<3>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < BW && !CLOSED; ++k) {
         const int wi = b * BW + k;
         const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
         constexpr bool MS = !CLOSED;
@@ -604,8 +718,12 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
         return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
       };
       auto code = [&](int k) { return it.cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
-      slice_finish_bf16<BE, L, RECOMPUTE, CLOSED>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax, cnt,
-                                          nsat, xval, code);
+      if constexpr (CLOSED)
+        slice_finish_closed<BE, L>(acc, lane, ok, own_b[b], a, D, sat_thr, st, lt2, dmax, nsat2,
+                                   xval, code);
+      else
+        slice_finish_bf16<BE, L, RECOMPUTE, false>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax,
+                                                   cnt, nsat, xval, code);
     }
   };
 
@@ -619,6 +737,296 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
     process(A, i);
     i += T;
     if (!(warp0 + (i - tid) < nitems)) break;
+    load(A, i + T);
+    process(B, i);
+    i += T;
+  }
+  finish_cta(acc, wk);
+}
+
+// ------------------------------------------------------------------------------------------------
+// bf16 input, small blocks (N = 4, 8) with recomputed codes
+// ------------------------------------------------------------------------------------------------
+// The per-block work dominates at these sizes, so it is done for two blocks at once where the
+// hardware has paired forms: block maxima as one bf16x2 word per block pair, two scale quotients
+// per f32x2 multiply, two E4M3 codes per conversion, the max elements' errors per f32x2 FMA.  The
+// whole item (16 elements) shares one scaling s = 2^(127 - E), E the exponent of the item's
+// largest block maximum, so the three sums are kept in fp32 per item and turned into double once
+// per item.  Every element's square goes into its block's sum; each non-zero block then moves its
+// first max element's square (dmax^2: all max-valued elements of a block share that error) to
+// SSE_max.  Where dmax^2 dominates a block so much (remainder below dmax^2 / 64) that the
+// subtraction would cost digits, that block's elements below the maximum are summed apart.  An
+// item is redone exactly in double when squares could have been lost to fp32 underflow: a non-zero
+// block maximum with a sum below 2^-80, or (in a block summed apart) a non-zero scaled error below
+// 2^-63.
+
+// Quotients of two elements with their own reciprocals (see snap_quotient2).
+__device__ __forceinline__ float2 snap_quotient2v(float2 x, float2 r) {
+  const float2 y = __ffma2_rn(x, r, make_float2(48.0f, 48.0f));
+  const float2 q = __fadd2_rd(y, make_float2(-48.0f, -48.0f));
+  return __ffma2_rn(x, make_float2(0x1p-60f, 0x1p-60f), q);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_set_gt(uint32_t a, uint32_t b) {  // 1.0 where a > b
+  uint32_t d;
+  asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_set_eq(uint32_t a, uint32_t b) {  // 1.0 where a == b
+  uint32_t d;
+  asm("set.eq.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// Sum of the two halves of a bf16x2 word of small integers, as fp32.
+__device__ __forceinline__ float bf16x2_hsum(uint32_t v) {
+  return __fadd_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+template <int N, int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads, MX_QS_MINB)
+    k_qstats_small(const __grid_constant__ SGroup grp) {
+  static_assert(N == 4 || N == 8, "small blocks only");
+  static_assert(MODE != kGiven, "codes are recomputed");
+  const SWork wk = s_work(grp);
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
+  uint8_t* __restrict__ packed_out = wk.t.packed_out;
+  uint8_t* __restrict__ scales_out = wk.t.scales_out;
+  const int64_t nitems = wk.t.nitems;
+  constexpr bool STORE = MODE == kStore;
+  using S = SShape<N, uint16_t>;
+  constexpr int EPT = S::EPT, NW = EPT / 2, NCW = EPT / 8, NB = EPT / N, BW = N / 2, NP = NB / 2;
+  static_assert(NB % 2 == 0 && NB <= 4 && (NCW == 2 || NCW == 4), "2 or 4 blocks per item");
+  __shared__ float s_rcp[256], s_D[256];
+  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+    const float D = __fmul_rn(scale_value(c, FMT), g);
+    s_D[c] = D;
+    s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;
+  }
+  const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
+  const float sat_thr = __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>());  // exact
+  const uint32_t SAT2 = (__float_as_uint(sat_thr) >> 16) * 0x10001u;      // RD to bf16, twice
+  __syncthreads();
+  griddep_wait();  // inputs may come from the previous kernel in the stream
+  griddep_launch_next();
+
+  Acc acc;
+  const int64_t T = (int64_t)wk.nctas * blockDim.x;
+  const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
+  using Item = StatsItem<NW, NCW>;
+
+  auto load = [&](Item& it, int64_t i) {
+    const bool ok = i < nitems;
+#pragma unroll
+    for (int h = 0; h < NW / 4; ++h) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (ok) v = ld_stream16(x + i * EPT + h * 8);
+      it.w[4 * h + 0] = v.x; it.w[4 * h + 1] = v.y; it.w[4 * h + 2] = v.z; it.w[4 * h + 3] = v.w;
+    }
+  };
+
+  auto process = [&](Item& it, int64_t i) {
+    const bool ok = i < nitems;
+    // block maxima, two blocks per bf16x2 word: M[j] = {a_2j, a_2j+1}
+    uint32_t M[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      uint32_t t0 = it.w[2 * j * BW], t1 = it.w[(2 * j + 1) * BW];
+#pragma unroll
+      for (int k = 1; k < BW; ++k) {
+        t0 = bf16x2_absmax(t0, it.w[2 * j * BW + k]);
+        t1 = bf16x2_absmax(t1, it.w[(2 * j + 1) * BW + k]);
+      }
+      M[j] = bf16x2_absmax(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632)) & 0x7FFF7FFFu;
+    }
+    // the item's scaling
+    uint32_t mm = M[0];
+#pragma unroll
+    for (int j = 1; j < NP; ++j) mm = bf16x2_absmax(mm, M[j]);
+    const int E = max((int)(max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu) >> 7), 1);
+    const float sc = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);
+    // scale codes, reciprocals and per-block constants, two blocks at a time
+    float r_b[NB], D_b[NB], nDq_b[NB];
+    uint32_t S2_b[NB];
+    uint32_t sc_all = 0, zc2 = 0, ss2 = 0;  // scale bytes; zero-block and saturated-scale counts
+    float2 af[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      af[j] = make_float2(__uint_as_float(M[j] << 16), __uint_as_float(M[j] & 0xFFFF0000u));
+      const float2 u = __fmul2_rn(af[j], make_float2(r6, r6));
+      uint32_t s0, s1;
+      if constexpr (FMT == kE4M3) {
+        unsigned short h;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(h) : "f"(snap21(u.y)), "f"(snap21(u.x)));
+        s0 = h & 0xFFu;
+        s1 = (uint32_t)h >> 8;
+      } else {
+        s0 = encode_scale<FMT>(snap21(u.x));
+        s1 = encode_scale<FMT>(snap21(u.y));
+      }
+      sc_all |= (s0 | (s1 << 8)) << (16 * j);
+      r_b[2 * j] = s_rcp[s0];
+      r_b[2 * j + 1] = s_rcp[s1];
+      const float2 D2 = make_float2(s_D[s0], s_D[s1]);
+      D_b[2 * j] = D2.x;
+      D_b[2 * j + 1] = D2.y;
+      const float2 nDq = __fmul2_rn(__fmul2_rn(D2, make_float2(sc, sc)),
+                                    make_float2(-0x1p126f, -0x1p126f));
+      nDq_b[2 * j] = nDq.x;
+      nDq_b[2 * j + 1] = nDq.y;
+      // clip levels RD_bf16(6 S g) (exact products, truncated); a zero block gets the largest
+      // finite bf16, which no finite |x| exceeds
+      const float2 six = __fmul2_rn(D2, make_float2(6.0f, 6.0f));
+      uint32_t thr = __byte_perm(__float_as_uint(six.x), __float_as_uint(six.y), 0x7632);
+      const uint32_t z2 = bf16x2_set_eq(thr, 0u);
+      thr = bf16x2_fma(z2, 0x7F7F7F7Fu, thr);
+      S2_b[2 * j] = __byte_perm(thr, thr, 0x1010);
+      S2_b[2 * j + 1] = __byte_perm(thr, thr, 0x3232);
+      zc2 = bf16x2_add(zc2, z2);
+      ss2 = bf16x2_add(ss2, bf16x2_set_gt(M[j], SAT2));
+    }
+    // codes: eight quotients per code word
+    uint32_t cw[NCW];
+#pragma unroll
+    for (int c = 0; c < NCW; ++c) {
+      float q[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int wi = 4 * c + k;
+        const uint32_t w = it.w[wi];
+        const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
+        q[2 * k] = qq.x;
+        q[2 * k + 1] = qq.y;
+      }
+      cw[c] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    }
+    if constexpr (STORE) {
+      if (ok) {
+        if constexpr (NCW == 4)
+          *reinterpret_cast<uint4*>(packed_out + i * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        else
+          *reinterpret_cast<uint2*>(packed_out + i * 8) = make_uint2(cw[0], cw[1]);
+        if constexpr (NB == 2) *reinterpret_cast<uint16_t*>(scales_out + i * 2) = (uint16_t)sc_all;
+        else *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
+      }
+    }
+    // errors: every element's scaled square into its block's sum, clipped elements counted
+    float ae = 0.0f, am = 0.0f, az = 0.0f;
+    uint32_t nsat2 = 0u;
+    bool exact = false;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      unsigned long long lt2[2] = {0ull, 0ull};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = 2 * j + h;
+#pragma unroll
+        for (int k = 0; k < BW; ++k) {
+          const int wi = b * BW + k;
+          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, c = cw[wi >> 2];
+          switch (wi & 3) {
+            case 0: pair_step_all<0>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
+            case 1: pair_step_all<1>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
+            case 2: pair_step_all<2>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
+            default: pair_step_all<3>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
+          }
+        }
+      }
+      // the two blocks' max elements: code of a / (S g), scaled error, square
+      const float2 qa = snap_quotient2v(af[j], make_float2(r_b[2 * j], r_b[2 * j + 1]));
+      const uint32_t ca = cvt_e2m1x8(qa.x, qa.y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+      const float2 dec = make_float2(__uint_as_float(e2m1_scaled_bits_at(ca, 0)),
+                                     __uint_as_float(e2m1_scaled_bits_at(ca, 4)));
+      const float2 dm = __ffma2_rn(dec, make_float2(nDq_b[2 * j], nDq_b[2 * j + 1]),
+                                   __fmul2_rn(af[j], make_float2(sc, sc)));
+      const float2 f2 = __fmul2_rn(dm, dm);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = 2 * j + h;
+        float l0, l1;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lt2[h]));
+        const float tb = __fadd_rn(l0, l1);
+        const float first = h ? f2.y : f2.x;
+        const float ab = h ? af[j].y : af[j].x;
+        exact |= ab > 0.0f && tb < 0x1p-80f;
+        if (D_b[b] > 0.0f) {
+          float rest = __fsub_rn(tb, first);
+          if (rest < __fmul_rn(first, 0x1p-6f)) {
+            // dmax^2 dominates the block: sum the elements below the maximum apart (no
+            // cancellation) and add the other max-valued elements' copies of dmax^2
+            float rs = 0.0f, nt = 0.0f;
+#pragma unroll
+            for (int k = 0; k < N; ++k) {
+              const int e = b * N + k;
+              const uint32_t wd = it.w[e >> 1];
+              const float xv = (e & 1) ? bf16hi(wd) : bf16lo(wd);
+              const float dq = __uint_as_float(e2m1_scaled_bits_at(cw[e >> 3], 4 * (e & 7)));
+              const float d = __fmaf_rn(dq, nDq_b[b], __fmul_rn(xv, sc));
+              if (fabsf(xv) != ab) rs = __fmaf_rn(d, d, rs);
+              else nt += 1.0f;
+              exact |= d != 0.0f && fabsf(d) < 0x1p-63f;  // its square would be lost
+            }
+            rest = __fmaf_rn(nt - 1.0f, first, rs);
+          }
+          ae = __fadd_rn(ae, rest);
+          am = __fadd_rn(am, first);
+        } else {
+          az = __fadd_rn(az, tb);
+        }
+      }
+    }
+    if (!exact) {
+      const double us = unscale_sq(E);
+      acc.elem += (double)ae * us;
+      acc.mx += (double)am * us;
+      acc.zero += (double)az * us;
+    } else {
+      // exact in double, block by block (first max element by index)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int e0 = b * N;
+        auto xval = [&](int k) {
+          const uint32_t wd = it.w[(e0 + k) >> 1];
+          return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
+        };
+        auto code = [&](int k) { return cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
+        const float ab = (b & 1) ? af[b >> 1].y : af[b >> 1].x;
+        double rest = 0.0, first = 0.0, others = 0.0;
+        exact_slice<N, false>(ab, D_b[b], xval, code, rest, first, others);
+        if (D_b[b] > 0.0f) {
+          acc.elem += rest + others;
+          acc.mx += first;
+        } else {
+          acc.zero += rest + first + others;
+        }
+      }
+    }
+    if (ok) {
+      acc.n_esat += bf16x2_hsum(nsat2);
+      acc.n_zero_f += bf16x2_hsum(zc2);
+      acc.n_ssat_f += bf16x2_hsum(ss2);
+    }
+  };
+
+  Item A, B;
+  int64_t i = tid;
+  load(A, i);
+  while (i < nitems) {
+    load(B, i + T);
+    process(A, i);
+    i += T;
+    if (!(i < nitems)) break;
     load(A, i + T);
     process(B, i);
     i += T;
@@ -858,8 +1266,11 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
     nitems[k] = ta[k].numel / S::EPT;
     tail[k] = ta[k].numel % S::EPT != 0;
   }
-  const void* kern = (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, MODE>
-                                      : (const void*)k_error_stats_f32<N, FMT, RC>;
+  // bf16 with recomputed codes and N <= 8: the small-block kernel
+  constexpr bool SMALL = sizeof(T) == 2 && RC && N <= 8;
+  const void* kern = SMALL ? (const void*)k_qstats_small<(N <= 8 ? N : 4), FMT, (RC ? MODE : kStore)>
+                     : (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, MODE>
+                                        : (const void*)k_error_stats_f32<N, FMT, RC>;
   const int grid = split_grid(kern, nitems, count, S::U, kMaxStatsGrid, &grp.split);
   bool any_counter = false;
   for (int k = 0; k < count; ++k) {
@@ -884,7 +1295,10 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
       if (e != cudaSuccess) return e;
       ++*launches;
     }
-    const cudaError_t e = (sizeof(T) == 2)
+    const cudaError_t e = SMALL ? launch_pdl(k_qstats_small<(N <= 8 ? N : 4), FMT,
+                                                             (RC ? MODE : kStore)>,
+                                             grid, kThreads, stream, grp)
+                          : (sizeof(T) == 2)
                               ? launch_pdl(k_error_stats_bf16<N, FMT, MODE>, grid, kThreads,
                                            stream, grp)
                               : launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream,
