@@ -22,7 +22,7 @@
 //   * Underflow.  A slice whose scaled non-max sum is below 2^-80 (squares below 2^-126 could be
 //     lost), or whose stored scale is far from a, redoes its slice in double.
 // Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
-// in a fixed order, so results are deterministic for a given device and grid; with a tail (N <= 8) a
+// in a fixed order, so results are deterministic for a given device and grid; with a tail (N <= 16) a
 // separate one-CTA pass does it.  No CTA waits on another.
 #include "mx_device.cuh"
 #include "mx_launch.h"
@@ -117,7 +117,7 @@ struct STensor {
   uint8_t* scales_out;
   StatsPartial* part;      // this tensor's CTAs' partials: part[0 .. its CTA count)
   unsigned int* counter;   // last-CTA counter, zeroed before the launch; nullptr: a separate pass
-                           // adds the partials (a tail, N <= 8)
+                           // adds the partials (a tail, N <= 16)
   StatsOut* out;
   int64_t nitems, numel, nblocks;
   uint32_t g_bits;
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
 }
 
 // ------------------------------------------------------------------------------------------------
-// bf16 input, small blocks (N = 4, 8) with recomputed codes
+// bf16 input, small blocks (N = 4, 8, 16) with recomputed codes
 // ------------------------------------------------------------------------------------------------
 // The per-block work dominates at these sizes, so it is done for two blocks at once where the
 // hardware has paired forms: block maxima as one bf16x2 word per block pair, two scale quotients
@@ -792,10 +792,17 @@ __device__ __forceinline__ float bf16x2_hsum(uint32_t v) {
   return __fadd_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
+// Item shape of the small-block kernel: 16 elements for N = 4, 8 (four or two blocks), 32 for
+// N = 16 (two blocks), so that blocks always come in pairs.
+template <int N>
+struct QSShape {
+  static constexpr int EPT = N == 16 ? 32 : MX_ST_EPT_SMALL;
+};
+
 template <int N, int FMT, int MODE>
 __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     k_qstats_small(const __grid_constant__ SGroup grp) {
-  static_assert(N == 4 || N == 8, "small blocks only");
+  static_assert(N == 4 || N == 8 || N == 16, "small blocks only");
   static_assert(MODE != kGiven, "codes are recomputed");
   const SWork wk = s_work(grp);
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
@@ -803,8 +810,8 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
   uint8_t* __restrict__ scales_out = wk.t.scales_out;
   const int64_t nitems = wk.t.nitems;
   constexpr bool STORE = MODE == kStore;
-  using S = SShape<N, uint16_t>;
-  constexpr int EPT = S::EPT, NW = EPT / 2, NCW = EPT / 8, NB = EPT / N, BW = N / 2, NP = NB / 2;
+  constexpr int EPT = QSShape<N>::EPT, NW = EPT / 2, NCW = EPT / 8, NB = EPT / N, BW = N / 2;
+  constexpr int NP = NB / 2;
   static_assert(NB % 2 == 0 && NB <= 4 && (NCW == 2 || NCW == 4), "2 or 4 blocks per item");
   __shared__ float s_rcp[256], s_D[256];
   const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
@@ -1119,7 +1126,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(const __grid_const
 // N = 4 tail (4 elements) and the final reduction
 // ------------------------------------------------------------------------------------------------
 
-// The elements after the last whole item (count of them, a multiple of the block size N <= 8):
+// The elements after the last whole item (count of them, a multiple of the block size N <= 16):
 // one thread, block by block, in double; codes recomputed (packed == nullptr) or read.
 template <int FMT, typename T>
 __global__ void k_error_stats_tail(const T* __restrict__ x, int64_t first, int count, int N,
@@ -1130,7 +1137,7 @@ __global__ void k_error_stats_tail(const T* __restrict__ x, int64_t first, int c
   StatsPartial p{};
   for (int b0 = 0; b0 < count; b0 += N) {
     const int64_t f = first + b0;
-    float v[8], a = 0.0f;
+    float v[16], a = 0.0f;
     int imax = 0;
     for (int k = 0; k < N; ++k) {
       if constexpr (sizeof(T) == 2)
@@ -1139,7 +1146,7 @@ __global__ void k_error_stats_tail(const T* __restrict__ x, int64_t first, int c
         v[k] = reinterpret_cast<const float*>(x)[f + k];
       if (fabsf(v[k]) > a) { a = fabsf(v[k]); imax = k; }
     }
-    uint32_t s, codes[8];
+    uint32_t s, codes[16];
     if (packed == nullptr) {
       s = encode_scale<FMT>(__fdiv_rn(a, __fmul_rn(6.0f, g)));
       const float D0 = __fmul_rn(scale_value((int)s, FMT), g);
@@ -1252,23 +1259,24 @@ cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int
 }
 
 // Main pass over the group; then, for each tensor the main pass does not finish, its tail (the
-// elements after the last whole item: N <= 8 only) and a one-CTA final pass, or (no items) the
+// elements after the last whole item: N <= 16 only) and a one-CTA final pass, or (no items) the
 // final pass alone.  Without a tail the main pass adds a tensor's partials itself.
 template <int N, int FMT, typename T, int MODE>
 static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Workspace ws,
                                 cudaStream_t stream, int* launches) {
   using S = SShape<N, T>;
   constexpr bool RC = MODE != kGiven;
+  // bf16 with recomputed codes and N <= 16: the small-block kernel
+  constexpr bool SMALL = sizeof(T) == 2 && RC && N <= 16;
+  constexpr int EPT = SMALL ? QSShape<N>::EPT : S::EPT;
   SGroup grp = {};
   int64_t nitems[kMaxGroup];
   bool tail[kMaxGroup];
   for (int k = 0; k < count; ++k) {
-    nitems[k] = ta[k].numel / S::EPT;
-    tail[k] = ta[k].numel % S::EPT != 0;
+    nitems[k] = ta[k].numel / EPT;
+    tail[k] = ta[k].numel % EPT != 0;
   }
-  // bf16 with recomputed codes and N <= 8: the small-block kernel
-  constexpr bool SMALL = sizeof(T) == 2 && RC && N <= 8;
-  const void* kern = SMALL ? (const void*)k_qstats_small<(N <= 8 ? N : 4), FMT, (RC ? MODE : kStore)>
+  const void* kern = SMALL ? (const void*)k_qstats_small<(N <= 16 ? N : 4), FMT, (RC ? MODE : kStore)>
                      : (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, MODE>
                                         : (const void*)k_error_stats_f32<N, FMT, RC>;
   const int grid = split_grid(kern, nitems, count, S::U, kMaxStatsGrid, &grp.split);
@@ -1295,7 +1303,7 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
       if (e != cudaSuccess) return e;
       ++*launches;
     }
-    const cudaError_t e = SMALL ? launch_pdl(k_qstats_small<(N <= 8 ? N : 4), FMT,
+    const cudaError_t e = SMALL ? launch_pdl(k_qstats_small<(N <= 16 ? N : 4), FMT,
                                                              (RC ? MODE : kStore)>,
                                              grid, kThreads, stream, grp)
                           : (sizeof(T) == 2)
@@ -1311,8 +1319,8 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
     StatsPartial* extra = nullptr;
     if (tail[k]) {
       extra = ws.part + grid + k;
-      const int64_t first = nitems[k] * S::EPT;
-      const int count = (int)(ta[k].numel - first);  // < EPT, a multiple of N <= 8
+      const int64_t first = nitems[k] * EPT;
+      const int count = (int)(ta[k].numel - first);  // < EPT, a multiple of N <= 16
       if (MODE == kStore) {  // quantize the last elements, then reduce them from the codes
         const cudaError_t e = run_quantize_tail(ta[k].x, sizeof(T) == 2, first, count, N, FMT,
                                                 ta[k].g_bits, ta[k].packed, ta[k].scales, stream,

@@ -299,7 +299,7 @@ __global__ void k_quantize_tail(const T* __restrict__ x, int64_t first, int coun
   const float g = fp16_bits_to_float(g_bits);
   for (int b0 = 0; b0 < count; b0 += N) {
     const int64_t f = first + b0;
-    float v[8], a = 0.0f;
+    float v[16], a = 0.0f;  // N <= 16
     for (int k = 0; k < N; ++k) {
       if constexpr (sizeof(T) == 2)
         v[k] = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[f + k] << 16);
