@@ -37,7 +37,7 @@ L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) of one grouped fused-pass launch (5 tensors, N = 32, E4M3), from the
 # ncu capture summarised in profiles/k_error_stats_bf16_fused_group5_4096x4096_n32.md: every x is
 # read once, most of the codes and scales are still in L2 when the launch ends.
-FUSED_TRAFFIC_BYTES = 167829760 + 8332032
+FUSED_TRAFFIC_BYTES = 167834368 + 8116736
 
 
 def parse(argv=None):
@@ -60,6 +60,10 @@ def parse(argv=None):
     ap.add_argument("--fmt", choices=["e4m3", "ue5m3"], default="e4m3")
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--group", type=int, default=1, help="tensors per grouped launch (--case)")
+    ap.add_argument("--rotate", type=int, default=1,
+                    help="--case: cycle R independent input sets, 4R launches between two events "
+                         "(no flush: each set is evicted by the others), instead of one flushed "
+                         "launch per event pair")
     return ap.parse_args(argv)
 
 
@@ -621,8 +625,63 @@ def run_case(args):
     dev = torch.device("cuda", 0)
     rows, cols = args.shape
     n, fmt, G = args.block, mx.fmt_code(args.fmt), args.group
-    xs = [inputs.normal((rows, cols), 0.02, k, device=dev) for k in range(G)]
     numel = rows * cols * G
+    sets = [case_calls(args, mx, inputs, dev, r) for r in range(max(1, args.rotate))]
+    code_bytes = G * rows * (((cols + 1) // 2) + -(-cols // n))  # codes + scales (any cols)
+    nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0,
+              "fake-quantize": numel * 4.0}.get(args.case, numel * 2.0 + code_bytes)
+    fns = [c[args.case] for c in sets]
+    for fn in fns:
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    if args.rotate > 1:
+        # one CUDA graph of 4R launches (no host gaps between them), replayed between two events
+        k = 4 * len(fns)
+        graph = torch.cuda.CUDAGraph()
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            for fn in fns:  # warm-up on the capture stream
+                fn()
+            stream.synchronize()
+            with torch.cuda.graph(graph, stream=stream):
+                for j in range(k):
+                    fns[j % len(fns)]()
+        torch.cuda.current_stream().wait_stream(stream)
+        graph.replay()
+        torch.cuda.synchronize()
+        for _ in range(args.reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3 / k)
+    else:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+        for _ in range(args.reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fns[0]()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    peak, kind = measured_peak()
+    print(json.dumps({"case": args.case, "shape": [rows, cols], "group": G, "block": n,
+                      "fmt": args.fmt, "median_us": t * 1e6, "gbs": nbytes / t / 1e9,
+                      "frac": nbytes / t / 1e9 / peak, "peak": peak, "peak_kind": kind,
+                      "reps": args.reps, "rotate": args.rotate}), flush=True)
+
+
+def case_calls(args, mx, inputs, dev, r):
+    """The calls of one input set of run_case (set r draws its tensors from seeds 100 r + k)."""
+    import torch
+    rows, cols = args.shape
+    n, fmt, G = args.block, mx.fmt_code(args.fmt), args.group
+    xs = [inputs.normal((rows, cols), 0.02, 100 * r + k, device=dev) for k in range(G)]
     if G == 1:  # (also ragged shapes, which grouped calls do not take)
         p0, s0 = mx.quantize(xs[0], n, fmt)
         packed, scales = [p0], [s0]
@@ -631,7 +690,6 @@ def run_case(args):
     ys = [torch.empty(rows, cols, dtype=torch.bfloat16, device=dev) for _ in range(G)]
     out = torch.empty(G, 64, dtype=torch.uint8, device=dev)
     ws = mx.stats_workspace(dev)
-    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
     if G == 1:
         x, p, sc, y = xs[0], packed[0], scales[0], ys[0]
         calls = {
@@ -654,27 +712,7 @@ def run_case(args):
         }
         if args.case not in calls:
             raise SystemExit(f"--group applies to {sorted(calls)}")
-    code_bytes = G * rows * (((cols + 1) // 2) + -(-cols // n))  # codes + scales (any cols)
-    nbytes = {"stats-recompute": numel * 2.0, "global-scale": numel * 2.0,
-              "fake-quantize": numel * 4.0}.get(args.case, numel * 2.0 + code_bytes)
-    fn = calls[args.case]
-    fn()
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(args.reps):
-        flush.fill_(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        fn()
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1) / 1e3)
-    t = statistics.median(times)
-    peak, kind = measured_peak()
-    print(json.dumps({"case": args.case, "shape": [rows, cols], "group": G, "block": n,
-                      "fmt": args.fmt, "median_us": t * 1e6, "gbs": nbytes / t / 1e9,
-                      "frac": nbytes / t / 1e9 / peak, "peak": peak, "peak_kind": kind,
-                      "reps": args.reps}), flush=True)
+    return calls
 
 
 def main():

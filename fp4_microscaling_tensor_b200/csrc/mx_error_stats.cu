@@ -259,11 +259,11 @@ __device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, 
 #undef MX_PAIR_TAIL
 }
 
-// Core of a bf16 block slice with recomputed codes (blocks of 16 and more), one word at a time:
-// every element's scaled error d goes into the f32x2 sum of squares lt2 -- the max-valued ones
-// included, the first of them is taken out per block, see slice_finish_closed -- and the clipped
-// elements (|x| > 6 S g, i.e. |x| above S2 = RD_bf16(6 S g)) are counted per half in nsat2 as
-// bf16x2 integers (exact: a half sees at most 128 of them).
+// Error step of one word (two elements) whose codes were computed beforehand (the signed form of
+// qs_word8's error part, used where the codes of a whole item are converted first): every
+// element's scaled error d goes into the f32x2 sum of squares lt2 -- the max-valued ones included,
+// the first of them is taken out per block, see slice_finish_closed -- and the clipped elements
+// (|x| above S2 = RD_bf16(6 S g)) are counted per half in nsat2 as bf16x2 integers.
 template <int J>
 __device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
                                               float sc, float nDq, uint32_t S2,
@@ -292,6 +292,57 @@ __device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t 
       : "+l"(lt2), "+r"(nsat2)
       : "r"(cw), "f"(sc), "f"(nDq), "r"(S2), "n"(1u << (28 - 8 * J)), "n"(1u << (24 - 8 * J)),
         "r"(lo), "r"(hi), "r"(w));
+}
+
+// One code word's eight elements (words w[0..3]) with recomputed codes, quantized and reduced in
+// one go.  The quotients are taken of the magnitudes (x r + 48 - 48 rounds |x| r exactly onto the
+// 2^-18 grid, see snap_quotient2; a magnitude needs no sign fix for zero), so the E2M1 conversion
+// gives magnitude codes whose decode is one shift and one mask; x's sign bits are put into the
+// codes afterwards (byte permutes that replicate each half's sign, two masked ORs).  Errors use the
+// magnitudes too: (|x| s - |q| S g s)^2 is the element's scaled square.  Per pair k the block
+// constants are those of block k / PB (PB = pairs per block inside the word: 2 for N = 4, else 4);
+// lt2[k / PB] collects the squares, nsat2 the clipped elements (|x| > RD_bf16(6 S g) = S2).
+template <int PB>
+__device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, const float* nDq,
+                                              const uint32_t* S2, float sc, float2* lt2,
+                                              uint32_t& nsat2) {
+  uint32_t aw[4];
+  float2 xa[4];
+  float q[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    aw[k] = w[k] & 0x7FFF7FFFu;
+    xa[k] = make_float2(__uint_as_float(aw[k] << 16), __uint_as_float(aw[k] & 0xFFFF0000u));
+    const float rk = r[k / PB];
+    const float2 y = __ffma2_rn(xa[k], make_float2(rk, rk), make_float2(48.0f, 48.0f));
+    const float2 qq = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
+    q[2 * k] = qq.x;
+    q[2 * k + 1] = qq.y;
+  }
+  const uint32_t cm = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // magnitude bits of byte k's two codes moved to bits 22..24: the value times 2^-126
+    const uint32_t blo = (k < 3 ? cm << (22 - 8 * k) : cm >> 2) & 0x01C00000u;
+    const uint32_t bhi = (k < 3 ? cm << (18 - 8 * k) : cm >> 6) & 0x01C00000u;
+    const float nd = nDq[k / PB];
+    const float2 xs = __fmul2_rn(xa[k], make_float2(sc, sc));
+    const float2 d = __ffma2_rn(make_float2(__uint_as_float(blo), __uint_as_float(bhi)),
+                                make_float2(nd, nd), xs);
+    lt2[k / PB] = __ffma2_rn(d, d, lt2[k / PB]);
+    uint32_t m;
+    asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(aw[k]), "r"(S2[k / PB]));
+    asm("add.rn.bf16x2 %0, %0, %1;" : "+r"(nsat2) : "r"(m));
+  }
+  // sign bits: per word, bytes 1 and 3 (the halves' high bytes) with their sign bit replicated
+  // over the byte (prmt selector nibbles with the top bit set), then regrouped so that byte k of
+  // hs / ls holds the sign of word k's high / low half
+  uint32_t x01, x23, hs, ls;
+  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x01) : "r"(w[0]), "r"(w[1]));
+  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x23) : "r"(w[2]), "r"(w[3]));
+  asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(hs) : "r"(x01), "r"(x23));
+  asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(ls) : "r"(x01), "r"(x23));
+  return (cm | (hs & 0x80808080u)) | (ls & 0x08080808u);
 }
 
 // Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
@@ -440,18 +491,16 @@ __device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, f
 template <int NE, int L, typename XF, typename CF>
 __device__ __forceinline__ void slice_finish_closed(Acc& acc, int lane, bool ok, bool has_max,
                                                     float a, float D, float sat_thr,
-                                                    const SliceSetup& st,
-                                                    unsigned long long lt2, float dmax,
-                                                    uint32_t nsat2, XF xval, CF code) {
+                                                    const SliceSetup& st, float2 lt2,
+                                                    float dmax, uint32_t nsat2, XF xval,
+                                                    CF code) {
   bool is_first_lane = has_max;
   if constexpr (L > 1) {
     const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
     const unsigned has = __ballot_sync(0xffffffffu, has_max) & gmask;
     is_first_lane = has != 0 && (__ffs(has) - 1) == lane;
   }
-  float l0, l1;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lt2));
-  const float lt = __fadd_rn(l0, l1);
+  const float lt = __fadd_rn(lt2.x, lt2.y);
   double rest = 0.0, first = 0.0, others = 0.0;
   bool exact = lt < 0x1p-80f;
   if (!exact) {
@@ -638,7 +687,21 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       D_b[b] = s_D[s];
       sc_all |= s << (8 * b);
     }
-    if constexpr (RECOMPUTE) {
+    // closed form (one block slice per item): codes and squares together, per code word
+    SliceSetup st0;
+    float2 lt0 = make_float2(0.0f, 0.0f);
+    uint32_t nsat0 = 0u;
+    // (measured: the per-code-word form is faster when a lane holds a whole block, L == 1; with
+    // blocks spread over lanes, converting the item's codes first and then reducing is faster)
+    constexpr bool W8 = CLOSED && L == 1;
+    if constexpr (W8) {
+      static_assert(!CLOSED || BPI == 1, "one block slice per item");
+      st0 = slice_setup(a_b[0], D_b[0]);
+      const uint32_t S2 = (__float_as_uint(__fmul_rn(6.0f, D_b[0])) >> 16) * 0x10001u;
+#pragma unroll
+      for (int j = 0; j < NCW; ++j)
+        it.cw[j] = qs_word8<4>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0, nsat0);
+    } else if constexpr (RECOMPUTE) {
       // codes: eight quotients per code word, converted right away
 #pragma unroll
       for (int j = 0; j < NCW; ++j) {
@@ -675,23 +738,25 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
 #pragma unroll
     for (int b = 0; b < BPI; ++b) {
       const float a = a_b[b], D = D_b[b];
-      const SliceSetup st = slice_setup(a, D);
+      const SliceSetup st = W8 ? st0 : slice_setup(a, D);
       const uint32_t sb = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // 6 S g rounded down
       const uint32_t A2 = m_b[b] * 0x10001u, S2 = sb * 0x10001u;
       float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f, dmax = 0.0f;
       const float nD = st.nDq;
-      unsigned long long lt2 = 0ull;
-      uint32_t nsat2 = 0u;
+      if constexpr (CLOSED && !W8) {
+        unsigned long long l2 = 0ull;
 #pragma unroll
-      for (int k = 0; k < BW && CLOSED; ++k) {
-        const int wi = b * BW + k;
-        const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
-        switch (wi & 3) {
-          case 0: pair_step_all<0>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
-          case 1: pair_step_all<1>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
-          case 2: pair_step_all<2>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
-          default: pair_step_all<3>(w, lo, hi, cw, st.sc, nD, S2, lt2, nsat2); break;
+        for (int k = 0; k < BW; ++k) {
+          const int wi = b * BW + k;
+          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
+          switch (wi & 3) {
+            case 0: pair_step_all<0>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
+            case 1: pair_step_all<1>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
+            case 2: pair_step_all<2>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
+            default: pair_step_all<3>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
+          }
         }
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lt0.x), "=f"(lt0.y) : "l"(l2));
       }
 #pragma unroll
       for (int k = 0; k < BW && !CLOSED; ++k) {
@@ -719,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       };
       auto code = [&](int k) { return it.cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
       if constexpr (CLOSED)
-        slice_finish_closed<BE, L>(acc, lane, ok, own_b[b], a, D, sat_thr, st, lt2, dmax, nsat2,
+        slice_finish_closed<BE, L>(acc, lane, ok, own_b[b], a, D, sat_thr, st, lt0, dmax, nsat0,
                                    xval, code);
       else
         slice_finish_bf16<BE, L, RECOMPUTE, false>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax,
@@ -903,20 +968,51 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
       zc2 = bf16x2_add(zc2, z2);
       ss2 = bf16x2_add(ss2, bf16x2_set_gt(M[j], SAT2));
     }
-    // codes: eight quotients per code word
+    // codes and every element's scaled square (into its block's sum), one code word at a time;
+    // clipped elements counted
+    // (measured: for N = 4, converting the item's codes first and then reducing is faster)
+    constexpr int PB = BW < 4 ? BW : 4;  // pairs per block inside a code word
     uint32_t cw[NCW];
+    float2 lt[NB];
+    uint32_t nsat2 = 0u;
 #pragma unroll
-    for (int c = 0; c < NCW; ++c) {
-      float q[8];
+    for (int b = 0; b < NB; ++b) lt[b] = make_float2(0.0f, 0.0f);
+    if constexpr (N >= 8) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int wi = 4 * c + k;
-        const uint32_t w = it.w[wi];
-        const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
-        q[2 * k] = qq.x;
-        q[2 * k + 1] = qq.y;
+      for (int c = 0; c < NCW; ++c) {
+        const int b0 = (4 * c) / BW;  // block of the code word's first pair
+        cw[c] = qs_word8<PB>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0], nsat2);
       }
-      cw[c] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < NCW; ++c) {
+        float q[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int wi = 4 * c + k;
+          const uint32_t w = it.w[wi];
+          const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
+          q[2 * k] = qq.x;
+          q[2 * k + 1] = qq.y;
+        }
+        cw[c] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        unsigned long long l2 = 0ull;
+#pragma unroll
+        for (int k = 0; k < BW; ++k) {
+          const int wi = b * BW + k;
+          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, c = cw[wi >> 2];
+          switch (wi & 3) {
+            case 0: pair_step_all<0>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            case 1: pair_step_all<1>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            case 2: pair_step_all<2>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            default: pair_step_all<3>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+          }
+        }
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lt[b].x), "=f"(lt[b].y) : "l"(l2));
+      }
     }
     if constexpr (STORE) {
       if (ok) {
@@ -928,28 +1024,11 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
         else *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
       }
     }
-    // errors: every element's scaled square into its block's sum, clipped elements counted
+    // per block pair: the max elements' errors, then each block's split of its sum
     float ae = 0.0f, am = 0.0f, az = 0.0f;
-    uint32_t nsat2 = 0u;
     bool exact = false;
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-      unsigned long long lt2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int b = 2 * j + h;
-#pragma unroll
-        for (int k = 0; k < BW; ++k) {
-          const int wi = b * BW + k;
-          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, c = cw[wi >> 2];
-          switch (wi & 3) {
-            case 0: pair_step_all<0>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
-            case 1: pair_step_all<1>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
-            case 2: pair_step_all<2>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
-            default: pair_step_all<3>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], lt2[h], nsat2); break;
-          }
-        }
-      }
       // the two blocks' max elements: code of a / (S g), scaled error, square
       const float2 qa = snap_quotient2v(af[j], make_float2(r_b[2 * j], r_b[2 * j + 1]));
       const uint32_t ca = cvt_e2m1x8(qa.x, qa.y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
@@ -961,9 +1040,7 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int b = 2 * j + h;
-        float l0, l1;
-        asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lt2[h]));
-        const float tb = __fadd_rn(l0, l1);
+        const float tb = __fadd_rn(lt[b].x, lt[b].y);
         const float first = h ? f2.y : f2.x;
         const float ab = h ? af[j].y : af[j].x;
         exact |= ab > 0.0f && tb < 0x1p-80f;
