@@ -524,9 +524,9 @@ def run_ours(args):
                     "quantize_pack": elems / t_q / 1e9,
                     "dequantize": elems / per_step[1] / 1e9},
         "roofline": {"bound": "hbm",
-                     "kernel": "k_error_stats_bf16<kStore> (fused quantize+pack+error reduction), "
-                               "14 grouped launches of 5 tensors; per launch avg incl. its "
-                               "counter-reset kernel",
+                     "kernel": "fused quantize+pack+error reduction (k_qstats_small for N <= 16, "
+                               "k_error_stats_bf16 for N >= 32, kStore), 14 grouped launches of 5 "
+                               "tensors; per launch avg incl. its counter-reset kernel",
                      "achieved": qs_gbs, "peak": peak, "unit": "GB/s", "frac": qs_gbs / peak,
                      "peak_kind": peak_kind + " (burst copy)",
                      "traffic": FUSED_TRAFFIC_BYTES,
