@@ -5,22 +5,25 @@
 // scale-rounding error of item 2), every other element to SSE_elem (item 1).  A block whose scale
 // is zero contributes sum x^2 to SSE_zero (item 3).  y is the exact E2M1 * S * g.
 //
-// Main pass (k_error_stats_*): persistent grid; each thread walks items of 8, 16 or 32 elements
-// with the next item's loads issued before the current item's arithmetic.  The codes are read
-// (kGiven), recomputed in registers with the quantize rule (kRecompute), or recomputed and stored
-// (kStore: the fused quantize + pack + reduction pass, x read once).  Per block slice held by a
-// lane:
+// Main pass: persistent grid; each thread walks items of 8, 16 or 32 elements with the next item's
+// loads issued before the current item's arithmetic.  The codes are read (kGiven), recomputed in
+// registers with the quantize rule (kRecompute), or recomputed and stored (kStore: the fused
+// quantize + pack + reduction pass, x read once).  Blocks of 4, 8 and 16 with recomputed codes run
+// on k_qstats_small (block pairs, per-item sums; see there), everything else on k_error_stats_bf16
+// (bf16) or k_error_stats_f32.  Per block slice held by a lane of k_error_stats_bf16:
 //   * Scaling.  s = 2^k brings the block maximum a into [1, 2).  d' = x s - code * (S g s) is one
 //     FMA (the code's bits are its value times 2^-126; S g s 2^126 is a per-block constant) and
 //     exact; squares are summed in fp32 (at most 32 terms) and scaled back exactly in double.
-//   * Two bf16x2 compares per word: |x| >= a (the max-valued elements) and |x| > 6 S g (clipped
-//     elements, counted).  The max-valued elements stay out of the per-element sum: with
-//     recomputed codes (N >= 16) they all share one error, computed once per block; otherwise
-//     their squares are summed apart, and a lane holding a tie of the maximum redoes them in
-//     double.  The block's first max element (lowest lane, lowest index) goes to SSE_max,
-//     everything else to SSE_elem.  All added terms are non-negative, so exact zeros stay exact.
-//   * Underflow.  A slice whose scaled non-max sum is below 2^-80 (squares below 2^-126 could be
-//     lost), or whose stored scale is far from a, redoes its slice in double.
+//   * Recomputed codes (blocks of 32 and more): every element's square goes into the slice sum;
+//     all max-valued elements of a block share one error dmax, computed once per block, and the
+//     lane holding the block's first max element moves dmax^2 to SSE_max (slice_finish_closed).
+//     Clipped elements (|x| > 6 S g) are counted with one bf16x2 compare per word.
+//   * Stored codes: two bf16x2 compares per word, |x| >= a (the max-valued elements, whose codes
+//     may differ) and |x| > 6 S g; the max-valued squares are summed apart, and a lane holding a
+//     tie of the maximum redoes them in double.  The block's first max element (lowest lane,
+//     lowest index) goes to SSE_max, everything else to SSE_elem.
+//   * Underflow.  A slice whose scaled sum is below 2^-80 (squares below 2^-126 could be lost),
+//     or whose stored scale is far from a, redoes its slice in double.
 // Final sum: the CTA that finishes last (one atomic counter per launch) adds the per-CTA partials
 // in a fixed order, so results are deterministic for a given device and grid; with a tail (N <= 16) a
 // separate one-CTA pass does it.  No CTA waits on another.
@@ -598,9 +601,10 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
   const int64_t nitems = wk.t.nitems;
   const uint16_t g_bits = (uint16_t)wk.t.g_bits;
   constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
-  // Recomputed codes: the max-valued elements' error in closed form per block (blocks of 16 and
-  // more), or summed like the others (small blocks, where the per-block work would cost more).
-  constexpr bool CLOSED = RECOMPUTE && N >= 16;
+  // Recomputed codes (blocks of 32 and more; smaller blocks run on k_qstats_small): the
+  // max-valued elements' error in closed form per block.
+  static_assert(!RECOMPUTE || N >= 32, "recomputed codes with N <= 16 run on k_qstats_small");
+  constexpr bool CLOSED = RECOMPUTE;
   using S = SShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, NW = EPT / 2, NCW = EPT / 8;
   constexpr int BW = NW / BPI;  // words per block inside an item
@@ -1353,9 +1357,10 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
     nitems[k] = ta[k].numel / EPT;
     tail[k] = ta[k].numel % EPT != 0;
   }
-  const void* kern = SMALL ? (const void*)k_qstats_small<(N <= 16 ? N : 4), FMT, (RC ? MODE : kStore)>
-                     : (sizeof(T) == 2) ? (const void*)k_error_stats_bf16<N, FMT, MODE>
-                                        : (const void*)k_error_stats_f32<N, FMT, RC>;
+  const void* kern;
+  if constexpr (SMALL) kern = (const void*)k_qstats_small<N, FMT, MODE>;
+  else if constexpr (sizeof(T) == 2) kern = (const void*)k_error_stats_bf16<N, FMT, MODE>;
+  else kern = (const void*)k_error_stats_f32<N, FMT, RC>;
   const int grid = split_grid(kern, nitems, count, S::U, kMaxStatsGrid, &grp.split);
   bool any_counter = false;
   for (int k = 0; k < count; ++k) {
@@ -1380,14 +1385,13 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
       if (e != cudaSuccess) return e;
       ++*launches;
     }
-    const cudaError_t e = SMALL ? launch_pdl(k_qstats_small<(N <= 16 ? N : 4), FMT,
-                                                             (RC ? MODE : kStore)>,
-                                             grid, kThreads, stream, grp)
-                          : (sizeof(T) == 2)
-                              ? launch_pdl(k_error_stats_bf16<N, FMT, MODE>, grid, kThreads,
-                                           stream, grp)
-                              : launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream,
-                                           grp);
+    cudaError_t e;
+    if constexpr (SMALL)
+      e = launch_pdl(k_qstats_small<N, FMT, MODE>, grid, kThreads, stream, grp);
+    else if constexpr (sizeof(T) == 2)
+      e = launch_pdl(k_error_stats_bf16<N, FMT, MODE>, grid, kThreads, stream, grp);
+    else
+      e = launch_pdl(k_error_stats_f32<N, FMT, RC>, grid, kThreads, stream, grp);
     if (e != cudaSuccess) return e;
     ++*launches;
   }
