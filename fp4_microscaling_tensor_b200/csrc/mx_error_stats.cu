@@ -861,11 +861,14 @@ __device__ __forceinline__ float bf16x2_hsum(uint32_t v) {
   return __fadd_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
-// Item shape of the small-block kernel: 16 elements for N = 4, 8 (four or two blocks), 32 for
-// N = 16 (two blocks), so that blocks always come in pairs.
+// Item shape of the small-block kernel: 16 elements for N = 4 (four blocks), 32 for N = 8 and 16
+// (four or two blocks), so that blocks always come in pairs.
+#ifndef MX_QS_EPT8  // elements per item of the small-block kernel for N = 8 (16 or 32)
+#define MX_QS_EPT8 32
+#endif
 template <int N>
 struct QSShape {
-  static constexpr int EPT = N == 16 ? 32 : MX_ST_EPT_SMALL;
+  static constexpr int EPT = N == 16 ? 32 : N == 8 ? MX_QS_EPT8 : MX_ST_EPT_SMALL;
 };
 
 template <int N, int FMT, int MODE>
