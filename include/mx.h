@@ -128,8 +128,7 @@ MX_API size_t mx_error_stats_workspace_size(int64_t rows, int64_t cols, int bloc
  * The reconstruction used for the errors is the exact E2M1 * S * g.  Each thread sums the squared
  * errors of at most 32 elements in fp32 and adds those partial sums in double; the partials are
  * combined in a fixed order for a given device, so repeated calls give identical results.  The
- * three sums are within 1e-5 relative of the exact sums (in practice about 1e-7); the counts are
- * exact. */
+ * three sums are within 1e-5 relative of the exact sums; the counts are exact. */
 MX_API mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols, int block,
                          mx_scale_fmt fmt, uint16_t global_scale_fp16, const uint8_t* packed,
                          const uint8_t* scales, mx_error_stats_t* out_dev, void* workspace,
