@@ -819,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
 // The per-block work dominates at these sizes, so it is done for two blocks at once where the
 // hardware has paired forms: block maxima as one bf16x2 word per block pair, two scale quotients
 // per f32x2 multiply, two E4M3 codes per conversion, the max elements' errors per f32x2 FMA.  The
-// whole item (16 elements) shares one scaling s = 2^(127 - E), E the exponent of the item's
+// whole item (16 or 32 elements) shares one scaling s = 2^(127 - E), E the exponent of the item's
 // largest block maximum, so the three sums are kept in fp32 per item and turned into double once
 // per item.  Every element's square goes into its block's sum; each non-zero block then moves its
 // first max element's square (dmax^2: all max-valued elements of a block share that error) to
