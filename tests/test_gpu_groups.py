@@ -1,7 +1,8 @@
 """Grouped calls: one launch over several tensors gives, tensor by tensor, the oracle's codes,
 scales and dequantized bits (bit-exact) and error records (within 1e-5 relative), with tensors of
-different sizes and global scales in one group (an empty tensor, an N = 4 tensor with a 4-element
-tail, and sizes that give a tensor a single CTA among many)."""
+different sizes and global scales in one group (an empty tensor, tensors whose size is not a
+multiple of the kernels' item (tails, N <= 16), and sizes that give a tensor a single CTA among
+many)."""
 import numpy as np
 import pytest
 import torch
@@ -19,12 +20,12 @@ G_MIX = (0x3C00, 0x3555, 0x0003, 0x5A00, 0x3C00, 0x2E66)
 
 def make_group(block, dtype, device, seed):
     """Tensors of one group: sizes from tiny to a few CTAs' worth, one empty, plus (N = 4) one
-    with rows*cols = 4 mod 8."""
+    of 12 elements (shorter than an item: all tail)."""
     rng = np.random.default_rng(seed)
     shapes = [(3, 8 * block), (64, 4 * block), (1, block), (0, block), (257, 2 * block),
               (512, 1024)]
     if block == 4:
-        shapes.append((3, 4))  # 12 elements: one full item of 8 and a 4-element tail
+        shapes.append((3, 4))  # 12 elements: less than one item, handled by the tail pass
     xs = []
     for k, (r, c) in enumerate(shapes):
         x = rng.standard_normal((r, c)) * np.exp(rng.uniform(-3, 1, (r, 1)))
