@@ -20,12 +20,13 @@ G_MIX = (0x3C00, 0x3555, 0x0003, 0x5A00, 0x3C00, 0x2E66)
 
 def make_group(block, dtype, device, seed):
     """Tensors of one group: sizes from tiny to a few CTAs' worth, one empty, plus (N = 4) one
-    of 12 elements (shorter than an item: all tail)."""
+    of 12 elements."""
     rng = np.random.default_rng(seed)
     shapes = [(3, 8 * block), (64, 4 * block), (1, block), (0, block), (257, 2 * block),
               (512, 1024)]
     if block == 4:
-        shapes.append((3, 4))  # 12 elements: less than one item, handled by the tail pass
+        shapes.append((3, 4))  # 12 elements: a tail after the last whole item (one item of 8 in
+        #                        the quantize kernel, none in the error kernels' items of 16)
     xs = []
     for k, (r, c) in enumerate(shapes):
         x = rng.standard_normal((r, c)) * np.exp(rng.uniform(-3, 1, (r, 1)))
