@@ -7,9 +7,7 @@ been built; there is no fallback.
 import ctypes
 import os
 
-# MXFP4_B200_LIB may name another build of the same library (e.g. a tuning variant).
-LIB_PATH = os.environ.get("MXFP4_B200_LIB") or os.path.join(
-    os.path.dirname(os.path.abspath(__file__)), "libmxfp4_b200.so")
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxfp4_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -28,21 +26,23 @@ EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_
            "mx_quantize_stats",
            "mx_global_scale_workspace_size", "mx_global_scale", "mx_error_stats_noalloc",
            "mx_quantize_group", "mx_dequantize_group", "mx_quantize_stats_group",
+           "mx_global_scale_group", "mx_error_stats_means",
            "mx_fake_quantize", "mx_matmul_scales_size", "mx_matmul_prepare_scales",
-           "mx_matmul", "mx_matmul_gave_up", "mx_test_fail_next_calls",
-           "mx_status_string", "mx_kernel_launches")
+           "mx_matmul", "mx_matmul_pair", "mx_matmul_gave_up", "mx_test_matmul_abandon_last",
+           "mx_test_fail_next_calls", "mx_status_string", "mx_kernel_launches")
 MX_MAX_GROUP = 16
 
 
 class Tensor(ctypes.Structure):
-    """mx_tensor_t (64 bytes): one tensor of a grouped call."""
+    """mx_tensor_t (72 bytes): one tensor of a grouped call."""
     _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("packed", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+                ("global_scale_dev", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("global_scale_fp16", ctypes.c_uint16), ("reserved", ctypes.c_uint16 * 3)]
 
 
-assert ctypes.sizeof(Tensor) == 64
+assert ctypes.sizeof(Tensor) == 72
 
 _i, _i64, _u16, _vp, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_uint16, ctypes.c_void_p, ctypes.c_size_t
 
@@ -73,8 +73,16 @@ lib.mx_dequantize_group.restype = _i
 lib.mx_dequantize_group.argtypes = [_tp, _i, _i, _i, _i, _vp]
 lib.mx_quantize_stats_group.restype = _i
 lib.mx_quantize_stats_group.argtypes = [_tp, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.mx_global_scale_group.restype = _i
+lib.mx_global_scale_group.argtypes = [_tp, _i, _i, _i, _vp, _sz, _vp]
+lib.mx_error_stats_means.restype = _i
+lib.mx_error_stats_means.argtypes = [_vp, ctypes.POINTER(ctypes.c_double)]
 lib.mx_matmul.restype = _i
 lib.mx_matmul.argtypes = [_vp, _vp, _u16, _vp, _vp, _u16, _i64, _i64, _i64, _i, _i, _vp, _i, _vp]
+lib.mx_matmul_pair.restype = _i
+lib.mx_matmul_pair.argtypes = lib.mx_matmul.argtypes
+lib.mx_test_matmul_abandon_last.restype = _i
+lib.mx_test_matmul_abandon_last.argtypes = []
 lib.mx_matmul_scales_size.restype = _sz
 lib.mx_matmul_scales_size.argtypes = [_i64, _i64]
 lib.mx_matmul_prepare_scales.restype = _i

@@ -127,6 +127,25 @@ class FakeQuantize(torch.autograd.Function):
         return grad_y, None, None, None
 
 
+def record_dict(raw):
+    """An mx_error_stats_t record (64 bytes, host) as a dict of its fields plus the pages' mean
+    squared errors (mse_elem, mse_max, mse_zero, mse_total), which the library computes from the
+    sums (mx_error_stats_means)."""
+    raw = bytes(raw)
+    d = dict(zip(STATS_FIELDS, struct.unpack("<3d5q", raw)))
+    buf = ctypes.create_string_buffer(raw, STATS_BYTES)
+    mse = (ctypes.c_double * 4)()
+    check(lib.mx_error_stats_means(ctypes.addressof(buf), mse), "mx_error_stats_means")
+    d.update(mse_elem=mse[0], mse_max=mse[1], mse_zero=mse[2], mse_total=mse[3])
+    return d
+
+
+def record_bytes(d):
+    """The 64-byte mx_error_stats_t of a dict with the record's fields."""
+    return struct.pack("<3d5q", *(float(d[k]) for k in STATS_FIELDS[:3]),
+                       *(int(d[k]) for k in STATS_FIELDS[3:]))
+
+
 class ErrorStats:
     """Device-resident mx_error_stats_t (64 bytes); to_dict() copies it to the host."""
 
@@ -134,13 +153,7 @@ class ErrorStats:
         self.tensor = tensor
 
     def to_dict(self):
-        raw = self.tensor.cpu().numpy().tobytes()
-        vals = struct.unpack("<3d5q", raw)
-        d = dict(zip(STATS_FIELDS, vals))
-        n = d["numel"] or 1
-        d.update(mse_elem=d["sse_elem"] / n, mse_max=d["sse_max"] / n, mse_zero=d["sse_zero"] / n)
-        d["mse_total"] = d["mse_elem"] + d["mse_max"] + d["mse_zero"]
-        return d
+        return record_dict(self.tensor.cpu().numpy().tobytes())
 
 
 def stats_workspace(device, rows=0, cols=0, block=32):
@@ -210,6 +223,32 @@ def global_scale(x, fmt="e4m3", out=None, workspace=None, stream=None):
 
 # ---- grouped calls: one launch for up to MX_MAX_GROUP tensors of the same dtype, block, format
 
+def global_scale_group(xs, fmt="e4m3", out=None, workspace=None, stream=None):
+    """global_scale() of every tensor of xs in one launch.  Returns a CUDA int16 tensor of
+    len(xs) binary16 bit patterns, which the other grouped calls accept as g (read on the
+    device)."""
+    xs = list(xs)
+    n = len(xs)
+    desc = _group(n, "global_scale_group")
+    dt = {x.dtype for x in xs}
+    if len(dt) != 1 or next(iter(dt)) not in _DT:
+        raise ValueError("all tensors float32 or all bfloat16")
+    dev = xs[0].device
+    if out is None:
+        out = torch.empty(n, dtype=torch.int16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib.mx_global_scale_workspace_size(0, 0), dtype=torch.uint8,
+                                device=dev)
+    for k, x in enumerate(xs):
+        rows, cols = _shape2d(x, "x")
+        desc[k].x, desc[k].rows, desc[k].cols = x.data_ptr(), rows, cols
+        desc[k].global_scale_dev = out.data_ptr() + 2 * k
+    check(lib.mx_global_scale_group(desc, n, _DT[xs[0].dtype], fmt_code(fmt), workspace.data_ptr(),
+                                    workspace.numel(), _stream(stream, dev)),
+          "mx_global_scale_group")
+    return out
+
+
 def _group(n, what):
     if not 1 <= n <= MX_MAX_GROUP:
         raise ValueError(f"{what}: between 1 and {MX_MAX_GROUP} tensors per call")
@@ -217,11 +256,23 @@ def _group(n, what):
 
 
 def _gs(g, n):
+    """Per-tensor g of a grouped call: (bit patterns, device addresses).  g may be one value, one
+    value per tensor, or a CUDA tensor of n 16-bit elements (e.g. from global_scale_group), whose
+    values the kernels read on the device (they never visit the host)."""
+    if isinstance(g, torch.Tensor):
+        if not g.is_cuda or g.numel() != n or g.element_size() != 2 or not g.is_contiguous():
+            raise ValueError("device global scales: a contiguous CUDA tensor of n 16-bit values")
+        return [0] * n, [g.data_ptr() + 2 * k for k in range(n)]
     if isinstance(g, (list, tuple)):
         if len(g) != n:
             raise ValueError("one global scale per tensor")
-        return [g_bits(v) for v in g]
-    return [g_bits(g)] * n
+        return [g_bits(v) for v in g], [None] * n
+    return [g_bits(g)] * n, [None] * n
+
+
+def _set_g(desc, gs, k):
+    desc.global_scale_fp16 = gs[0][k]
+    desc.global_scale_dev = gs[1][k]
 
 
 def quantize_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None, stream=None):
@@ -246,7 +297,8 @@ def quantize_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None, s
                                     device=x.device)
         desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
-        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = rows, cols, gs[k]
+        desc[k].rows, desc[k].cols = rows, cols
+        _set_g(desc[k], gs, k)
     check(lib.mx_quantize_group(desc, n, _DT[xs[0].dtype], int(block), fmt_code(fmt),
                                 _stream(stream, xs[0].device)), "mx_quantize_group")
     return packed, scales
@@ -272,7 +324,8 @@ def dequantize_group(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=tor
                                  device=packed[k].device)
         desc[k].y, desc[k].packed, desc[k].scales = (out[k].data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
-        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = prow, 2 * pcols, gs[k]
+        desc[k].rows, desc[k].cols = prow, 2 * pcols
+        _set_g(desc[k], gs, k)
     check(lib.mx_dequantize_group(desc, n, int(block), fmt_code(fmt), _DT[out_dtype],
                                   _stream(stream, packed[0].device)), "mx_dequantize_group")
     return out
@@ -308,7 +361,8 @@ def quantize_with_stats_group(xs, block=32, fmt="e4m3", g=None, packed=None, sca
         desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
         desc[k].stats = out[k].data_ptr()
-        desc[k].rows, desc[k].cols, desc[k].global_scale_fp16 = rows, cols, gs[k]
+        desc[k].rows, desc[k].cols = rows, cols
+        _set_g(desc[k], gs, k)
     check(lib.mx_quantize_stats_group(desc, n, _DT[xs[0].dtype], int(block), fmt_code(fmt),
                                       workspace.data_ptr(), workspace.numel(),
                                       _stream(stream, dev)), "mx_quantize_stats_group")
@@ -331,11 +385,12 @@ def prepare_scales(scales, k, out=None, stream=None):
 
 
 def matmul(a_packed, a_scales, b_packed, b_scales, a_g=None, b_g=None, out_dtype=torch.bfloat16,
-           out=None, prepared=False, stream=None):
+           out=None, prepared=False, stream=None, cta_pairs=False):
     """C = dequant(A) dequant(B)^T on the tensor cores (block 16, E4M3 scales, as quantize writes
     them): a_packed [m, k/2] of an m x k tensor, b_packed [n, k/2] of an n x k tensor; a_scales /
     b_scales are the quantizer's [rows, k/16] arrays, or (prepared=True) the outputs of
-    prepare_scales.  Returns C [m, n] of out_dtype."""
+    prepare_scales.  cta_pairs: the CTA-pair kernel (mx_matmul_pair).  Returns C [m, n] of
+    out_dtype."""
     if out_dtype not in _DT:
         raise ValueError("out_dtype must be float32 or bfloat16")
     for t, what in ((a_packed, "a_packed"), (b_packed, "b_packed")):
@@ -350,9 +405,10 @@ def matmul(a_packed, a_scales, b_packed, b_scales, a_g=None, b_g=None, out_dtype
         b_scales = prepare_scales(b_scales, k, stream=stream)
     if out is None:
         out = torch.empty((m, n), dtype=out_dtype, device=a_packed.device)
-    check(lib.mx_matmul(a_packed.data_ptr(), a_scales.data_ptr(), g_bits(a_g), b_packed.data_ptr(),
-                        b_scales.data_ptr(), g_bits(b_g), m, n, k, 16, E4M3, out.data_ptr(),
-                        _DT[out.dtype], _stream(stream, a_packed.device)), "mx_matmul")
+    fn = lib.mx_matmul_pair if cta_pairs else lib.mx_matmul
+    check(fn(a_packed.data_ptr(), a_scales.data_ptr(), g_bits(a_g), b_packed.data_ptr(),
+             b_scales.data_ptr(), g_bits(b_g), m, n, k, 16, E4M3, out.data_ptr(), _DT[out.dtype],
+             _stream(stream, a_packed.device)), "mx_matmul")
     return out
 
 

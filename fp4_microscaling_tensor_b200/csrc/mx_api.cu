@@ -9,7 +9,7 @@
 #include "mx_launch.h"
 
 static_assert(sizeof(mx_error_stats_t) == 64, "mx_error_stats_t layout");
-static_assert(sizeof(mx_tensor_t) == 64, "mx_tensor_t layout");
+static_assert(sizeof(mx_tensor_t) == 72, "mx_tensor_t layout");
 static_assert(MX_MAX_GROUP == mxk::kMaxGroup, "group size");
 
 namespace {
@@ -191,6 +191,20 @@ mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t co
   return from_cuda(e);
 }
 
+mx_status mx_error_stats_means(const mx_error_stats_t* record, double* mse4) {
+  if (!record || !mse4) return MX_ERR_INVALID_ARG;
+  if (record->numel <= 0) {
+    mse4[0] = mse4[1] = mse4[2] = mse4[3] = 0.0;
+    return MX_OK;
+  }
+  const double n = (double)record->numel;
+  mse4[0] = record->sse_elem / n;
+  mse4[1] = record->sse_max / n;
+  mse4[2] = record->sse_zero / n;
+  mse4[3] = mse4[0] + mse4[1] + mse4[2];
+  return MX_OK;
+}
+
 size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols) {
   (void)rows;
   (void)cols;
@@ -214,6 +228,8 @@ mx_status mx_global_scale(const void* x, mx_dtype xt, int64_t rows, int64_t cols
   return from_cuda(e);
 }
 
+}  // extern "C"
+
 namespace {
 
 // Value of a finite binary16 bit pattern (exact in float).
@@ -223,12 +239,10 @@ float half_value(uint16_t h) {
   return (h & 0x8000u) ? -v : v;
 }
 
-}  // namespace
-
-mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
-                    const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g, int64_t m,
-                    int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c, mx_dtype ct,
-                    cudaStream_t stream) {
+mx_status matmul_impl(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
+                      const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g, int64_t m,
+                      int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c, mx_dtype ct,
+                      bool cta_pairs, cudaStream_t stream) {
   if (!valid_fmt(fmt) || !valid_dtype(ct) || !valid_g(a_g) || !valid_g(b_g)) return MX_ERR_INVALID_ARG;
   if (m < 0 || n < 0 || k < 0 || m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) ||
       k > (int64_t(1) << 40))
@@ -247,9 +261,29 @@ mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a
   int launches = 0;
   const cudaError_t e = mxk::run_matmul_nvfp4(a_packed, a_scales, b_packed, b_scales, m, n, k,
                                               half_value(a_g) * half_value(b_g), c, ct == MX_BF16,
-                                              stream, &launches);
+                                              cta_pairs, stream, &launches);
   g_launches += launches;
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
+                    const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g, int64_t m,
+                    int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c, mx_dtype ct,
+                    cudaStream_t stream) {
+  return matmul_impl(a_packed, a_scales, a_g, b_packed, b_scales, b_g, m, n, k, block, fmt, c, ct,
+                     false, stream);
+}
+
+mx_status mx_matmul_pair(const uint8_t* a_packed, const uint8_t* a_scales, uint16_t a_g,
+                         const uint8_t* b_packed, const uint8_t* b_scales, uint16_t b_g,
+                         int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c,
+                         mx_dtype ct, cudaStream_t stream) {
+  return matmul_impl(a_packed, a_scales, a_g, b_packed, b_scales, b_g, m, n, k, block, fmt, c, ct,
+                     true, stream);
 }
 
 size_t mx_matmul_scales_size(int64_t rows, int64_t k) {
@@ -279,19 +313,25 @@ mx_status mx_matmul_gave_up(unsigned int* count) {
   return from_cuda(mxk::matmul_gave_up(count));
 }
 
+mx_status mx_test_matmul_abandon_last(void) { return from_cuda(mxk::matmul_abandon_last()); }
+
 namespace {
 
 // Checks shared by the grouped calls: per tensor shape, pointers (`need` says which) and g.
-enum : unsigned { kNeedX = 1, kNeedY = 2, kNeedCodes = 4, kNeedStats = 8 };
+enum : unsigned { kNeedX = 1, kNeedY = 2, kNeedCodes = 4, kNeedStats = 8, kNeedGOut = 16 };
 
 mx_status check_group(const mx_tensor_t* t, int count, int block, unsigned need,
                       mxk::TensorArgs* args) {
   if (!t || count < 1 || count > MX_MAX_GROUP) return MX_ERR_INVALID_ARG;
   for (int k = 0; k < count; ++k) {
     const mx_tensor_t& d = t[k];
-    if (!shape_ok(d.rows, d.cols) || !valid_g(d.global_scale_fp16) || d.reserved[0] ||
-        d.reserved[1] || d.reserved[2])
+    // g: an output (kNeedGOut), read from device memory (global_scale_dev), or the bit pattern
+    const bool g_ok = (need & kNeedGOut) ? d.global_scale_dev != nullptr
+                                         : (d.global_scale_dev != nullptr ||
+                                            valid_g(d.global_scale_fp16));
+    if (!shape_ok(d.rows, d.cols) || !g_ok || d.reserved[0] || d.reserved[1] || d.reserved[2])
       return MX_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(d.global_scale_dev) & 1u) != 0) return MX_ERR_MISALIGNED;
     if (d.cols % block != 0) return MX_ERR_INVALID_ARG;
     const int64_t numel = d.rows * d.cols;
     if ((need & kNeedStats) && !d.stats) return MX_ERR_INVALID_ARG;
@@ -304,7 +344,8 @@ mx_status check_group(const mx_tensor_t* t, int count, int block, unsigned need,
           ((need & kNeedCodes) && (!aligned16(d.packed) || !aligned16(d.scales))))
         return MX_ERR_MISALIGNED;
     }
-    args[k] = {d.x, d.y, d.packed, d.scales, d.stats, numel, d.global_scale_fp16};
+    args[k] = {d.x, d.y, d.packed, d.scales, d.stats, numel, d.global_scale_fp16,
+               d.global_scale_dev};
   }
   return MX_OK;
 }
@@ -355,6 +396,23 @@ mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtyp
   int n = 0;
   const cudaError_t e = mxk::run_stats_group(args, count, xt == MX_BF16, block, (int)fmt,
                                              mxk::kStore, workspace, stream, &n);
+  g_launches += n;
+  return from_cuda(e);
+}
+
+mx_status mx_global_scale_group(const mx_tensor_t* tensors, int count, mx_dtype xt,
+                                 mx_scale_fmt fmt, void* workspace, size_t ws_bytes,
+                                 cudaStream_t stream) {
+  if (!valid_dtype(xt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
+  mxk::TensorArgs args[MX_MAX_GROUP];
+  const mx_status st = check_group(tensors, count, 1, kNeedX | kNeedGOut, args);
+  if (st != MX_OK) return st;
+  if (!workspace || ws_bytes < amax_ws_bytes()) return MX_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
+  int n = 0;
+  const cudaError_t e =
+      mxk::run_global_scale_group(args, count, xt == MX_BF16, (int)fmt, workspace, stream, &n);
   g_launches += n;
   return from_cuda(e);
 }

@@ -58,6 +58,7 @@ struct DTensor {
   void* y;
   int64_t nitems;
   uint32_t g_bits;
+  const uint16_t* g_dev;  // g in device memory (written by the previous kernel) when set
 };
 struct DGroup {
   DTensor t[kMaxGroup];
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kThreads) k_dequantize(const __grid_constant__
   void* __restrict__ y = tt.y;
   const int64_t nitems = tt.nitems;
   __shared__ float s_D[256];
-  const float g = fp16_bits_to_float((uint16_t)tt.g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(tt.g_bits, tt.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   __syncthreads();
   griddep_wait();  // inputs may come from the previous kernel in the stream
@@ -165,10 +166,11 @@ __global__ void __launch_bounds__(kThreads) k_dequantize(const __grid_constant__
 template <int FMT, bool BF16OUT>
 __global__ void k_dequantize_tail4(const uint8_t* __restrict__ packed,
                                    const uint8_t* __restrict__ scales, int64_t first,
-                                   uint16_t g_bits, void* __restrict__ y) {
+                                   uint16_t g_bits, const uint16_t* g_dev, void* __restrict__ y) {
   if (threadIdx.x >= 4) return;
   const int64_t e = first + threadIdx.x;
-  const float D = __fmul_rn(scale_value(scales[first / 4], FMT), fp16_bits_to_float(g_bits));
+  const float D = __fmul_rn(scale_value(scales[first / 4], FMT),
+                            fp16_bits_to_float(tensor_g_bits(g_bits, g_dev)));
   const uint32_t nib = (uint32_t)(packed[e / 2] >> (4 * (e & 1))) & 0xFu;
   const float v = __fmul_rn(e2m1_to_float(nib), D);
   if (BF16OUT)
@@ -185,7 +187,7 @@ static cudaError_t launch_dq(const TensorArgs* ta, int count, cudaStream_t strea
   int64_t nitems[kMaxGroup];
   for (int k = 0; k < count; ++k) {
     nitems[k] = ta[k].numel / S::EPT;
-    grp.t[k] = {ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits};
+    grp.t[k] = {ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits, ta[k].g_dev};
   }
   const int grid = split_grid((const void*)k_dequantize<N, FMT, BF16OUT>, nitems, count, S::U,
                               1 << 30, &grp.split);
@@ -199,7 +201,7 @@ static cudaError_t launch_dq(const TensorArgs* ta, int count, cudaStream_t strea
     if (ta[k].numel % S::EPT != 0) {
       k_dequantize_tail4<FMT, BF16OUT><<<1, 32, 0, stream>>>(ta[k].packed, ta[k].scales,
                                                               nitems[k] * S::EPT, ta[k].g_bits,
-                                                              ta[k].y);
+                                                              ta[k].g_dev, ta[k].y);
       ++*launches;
     }
   }

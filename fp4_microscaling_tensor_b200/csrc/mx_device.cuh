@@ -57,13 +57,15 @@ __device__ __forceinline__ float snap21(float v) {
   return __uint_as_float((__float_as_uint(v) + 4u) & ~7u);
 }
 
-// FP8 code of u >= 0 (already exact or snapped), nearest-even, saturating.
 // Quotients x / (S g) of two elements (lo / hi: their fp32 bits) for the E2M1 conversion, on the
 // FMA pipe.  r = RN(1 / (S g)), so x r is within 2^-21 of the true quotient t when |t| <= 8.
 // Adding 48 (whose binade [32, 64) has spacing 2^-18) and subtracting it again rounds x r onto that
 // grid exactly (Sterbenz for the subtraction).  A midpoint of the E2M1 grid (a multiple of 1/4) is
-// then hit exactly when t is one; otherwise t is at least 2^-17 away from every midpoint (x is
-// bf16, 8 significant bits, and S g has at most 15), and the rounded value stays on t's side.  Larger |t| only has to stay above 6, which it does.
+// then hit exactly when t is one.  Otherwise (x is bf16 with 8 significant bits, S g has at most
+// 15) t lies more than 2^-18 from every midpoint: at least 1.25 * 2^-18 from the 3-significant-bit
+// midpoints 1.25, 1.75, 2.5, 3.5 and 5, at least 2^-17 from the others.  That margin exceeds half
+// the grid spacing (2^-19) plus the product error (2^-21), so the rounded value stays on t's side.
+// Larger |t| only has to stay above 6, which it does.
 // Signs: the subtraction rounds toward -inf, so a quotient that cancels to zero is -0; the final
 // FMA adds x 2^-60, which leaves any non-zero quotient unchanged (|x| 2^-60 is below a quarter of
 // its unit in the last place, since r >= 2^-33) and gives a zero quotient the sign of x (+0 + -0 is
@@ -75,6 +77,7 @@ __device__ __forceinline__ float2 snap_quotient2(uint32_t lo, uint32_t hi, float
   return __ffma2_rn(x, make_float2(0x1p-60f, 0x1p-60f), q);
 }
 
+// FP8 code of u >= 0 (already exact or snapped), nearest-even, saturating.
 template <int FMT>
 __device__ __forceinline__ uint32_t encode_scale(float u) {
   if constexpr (FMT == kE4M3) {
@@ -144,6 +147,14 @@ __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// g of one tensor: its binary16 bit pattern, or, when g_dev is set, the value the previous kernel
+// in the stream wrote there (the global-scale launch); that read first waits for that kernel.
+__device__ __forceinline__ uint16_t tensor_g_bits(uint32_t g_bits, const uint16_t* g_dev) {
+  if (g_dev == nullptr) return (uint16_t)g_bits;
+  griddep_wait();
+  return __ldcg(g_dev);
 }
 
 // Streaming 16-byte load of read-only data (not kept in L1).

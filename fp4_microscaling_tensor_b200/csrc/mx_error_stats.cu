@@ -124,6 +124,7 @@ struct STensor {
   StatsOut* out;
   int64_t nitems, numel, nblocks;
   uint32_t g_bits;
+  const uint16_t* g_dev;   // g in device memory (written by the previous kernel) when set
 };
 struct SGroup {
   STensor t[kMaxGroup];
@@ -599,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
   uint8_t* __restrict__ packed_out = wk.t.packed_out;
   uint8_t* __restrict__ scales_out = wk.t.scales_out;
   const int64_t nitems = wk.t.nitems;
-  const uint16_t g_bits = (uint16_t)wk.t.g_bits;
+  const uint16_t g_bits = tensor_g_bits(wk.t.g_bits, wk.t.g_dev);
   constexpr bool RECOMPUTE = MODE != kGiven, STORE = MODE == kStore;
   // Recomputed codes (blocks of 32 and more; smaller blocks run on k_qstats_small): the
   // max-valued elements' error in closed form per block.
@@ -886,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
   constexpr int NP = NB / 2;
   static_assert(NB % 2 == 0 && NB <= 4 && (NCW == 2 || NCW == 4), "2 or 4 blocks per item");
   __shared__ float s_rcp[256], s_D[256];
-  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(wk.t.g_bits, wk.t.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);
     s_D[c] = D;
@@ -1136,7 +1137,7 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(const __grid_const
   const uint8_t* __restrict__ packed = wk.t.packed;
   const uint8_t* __restrict__ scales = wk.t.scales;
   const int64_t nitems = wk.t.nitems;
-  const uint16_t g_bits = (uint16_t)wk.t.g_bits;
+  const uint16_t g_bits = tensor_g_bits(wk.t.g_bits, wk.t.g_dev);
   using S = SShape<N, float>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI;
   constexpr int BE = EPT / BPI;
@@ -1214,10 +1215,11 @@ __global__ void __launch_bounds__(kThreads) k_error_stats_f32(const __grid_const
 // one thread, block by block, in double; codes recomputed (packed == nullptr) or read.
 template <int FMT, typename T>
 __global__ void k_error_stats_tail(const T* __restrict__ x, int64_t first, int count, int N,
-                                   uint16_t g_bits, const uint8_t* __restrict__ packed,
+                                   uint16_t g_bits, const uint16_t* g_dev,
+                                   const uint8_t* __restrict__ packed,
                                    const uint8_t* __restrict__ scales, StatsPartial* part) {
   if (threadIdx.x != 0) return;
-  const float g = fp16_bits_to_float(g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(g_bits, g_dev));
   StatsPartial p{};
   for (int b0 = 0; b0 < count; b0 += N) {
     const int64_t f = first + b0;
@@ -1337,7 +1339,12 @@ __global__ void k_stats_reset(unsigned int* counters, int n) {
 }
 
 cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int* launches) {
-  const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, counter, 1);
+  return launch_counters_reset(counter, 1, stream, launches);
+}
+
+cudaError_t launch_counters_reset(unsigned int* counters, int n, cudaStream_t stream,
+                                  int* launches) {
+  const cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, counters, n);
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -1380,7 +1387,8 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
                 nitems[k],
                 ta[k].numel,
                 ta[k].numel / block,
-                ta[k].g_bits};
+                ta[k].g_bits,
+                ta[k].g_dev};
   }
   if (grid > 0) {
     if (any_counter) {
@@ -1407,12 +1415,12 @@ static cudaError_t launch_stats(const TensorArgs* ta, int count, int block, Work
       const int count = (int)(ta[k].numel - first);  // < EPT, a multiple of N <= 16
       if (MODE == kStore) {  // quantize the last elements, then reduce them from the codes
         const cudaError_t e = run_quantize_tail(ta[k].x, sizeof(T) == 2, first, count, N, FMT,
-                                                ta[k].g_bits, ta[k].packed, ta[k].scales, stream,
-                                                launches);
+                                                ta[k].g_bits, ta[k].g_dev, ta[k].packed,
+                                                ta[k].scales, stream, launches);
         if (e != cudaSuccess) return e;
       }
       k_error_stats_tail<FMT, T><<<1, 32, 0, stream>>>(
-          (const T*)ta[k].x, first, count, N, ta[k].g_bits,
+          (const T*)ta[k].x, first, count, N, ta[k].g_bits, ta[k].g_dev,
           MODE == kRecompute ? nullptr : ta[k].packed, ta[k].scales, extra);
       ++*launches;
     }

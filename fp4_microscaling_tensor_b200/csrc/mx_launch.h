@@ -119,6 +119,8 @@ struct TensorArgs {
   void* stats;        // device mx_error_stats_t of the error reduction
   int64_t numel;
   uint16_t g_bits;
+  uint16_t* g_dev;    // when set: g is read from here when the kernel runs (g_bits unused); the
+                      // global-scale group launch writes it
 };
 
 // What the error-reduction pass does with the codes (see mx_error_stats.cu).
@@ -157,8 +159,8 @@ cudaError_t run_quantize_stats(const void* x, bool bf16, int64_t numel, int bloc
 // The `count` elements from `first` on (a multiple of the block size N <= 8, fewer than an item of
 // the calling kernel): quantize + pack them with plain per-element code.
 cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,
-                              uint16_t g_bits, uint8_t* packed, uint8_t* scales,
-                              cudaStream_t stream, int* launches);
+                              uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                              uint8_t* scales, cudaStream_t stream, int* launches);
 // One CTA's partial sums of the error reduction (64 bytes; the workspace holds one per CTA after
 // a header of kMaxGroup 64-byte counters).
 struct StatsPartial {
@@ -186,19 +188,30 @@ cudaError_t launch_counter_reset(unsigned int* counter, cudaStream_t stream, int
 
 // C (m x n, fp32 or bf16) = alpha * dequant(A) dequant(B)^T for A (m x k) and B (n x k) stored
 // with blocks of 16 along k and E4M3 scales; k a positive multiple of 256; scales in the
-// tensor-core order written by run_scales_to_mma.
+// tensor-core order written by run_scales_to_mma.  cta_pairs: 256 x 256 tiles of C computed by
+// CTA pairs (tcgen05 cta_group::2) when m > 128, else 128 x 256 tiles, one per CTA.
 cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
-                             cudaStream_t stream, int* launches);
+                             bool cta_pairs, cudaStream_t stream, int* launches);
 // Bytes of an operand's scales in tensor-core order, and the reordering kernel.
 int64_t mma_scales_bytes(int64_t rows, int64_t k);
 cudaError_t run_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out,
                               cudaStream_t stream, int* launches);
 // Reads and clears the count of matmul CTAs whose bounded waits ran out (synchronizes).
 cudaError_t matmul_gave_up(unsigned int* count);
+// Test hook: marks the most recent matmul launch as abandoned on the current device, as a CTA
+// whose waits ran out does (synchronizes).
+cudaError_t matmul_abandon_last();
 
+// Per-tensor FP16 scale of every tensor of a group: t[k].x -> *t[k].g_dev.
+cudaError_t run_global_scale_group(const TensorArgs* t, int count, bool bf16, int fmt,
+                                   void* workspace, cudaStream_t stream, int* launches);
 cudaError_t run_global_scale(const void* x, bool bf16, int64_t numel, int fmt, uint16_t* out,
                              void* workspace, cudaStream_t stream, int* launches);
+// Zeroes n last-CTA counters 64 bytes apart (counters[16 k], k < n <= 32) once the previous kernel
+// in the stream is done with them (a one-warp kernel launched with programmatic serialization).
+cudaError_t launch_counters_reset(unsigned int* counters, int n, cudaStream_t stream,
+                                  int* launches);
 
 }  // namespace mxk

@@ -9,20 +9,22 @@
 // which is the layout the quantizer writes; C is m x n row-major, float32 or bfloat16.
 //
 // One CTA per 128 x BN tile of C (BN = 256 by default, MMA N = BN), 4 warps:
-//   * warp 0 produces: for each 256-element step of k, one TMA load per operand (128 rows x 128
-//     bytes, 128-byte swizzle) and the 128 x 16 scale bytes of each operand, which the 32 lanes
-//     copy asynchronously (cp.async, 4 bytes each) into the 512-byte scale atoms the scale-copy
-//     instruction expects (row r of a 128-row tile at byte 16 (r % 32) + 4 (r / 32) + j for the
-//     four scales j of one 64-element MMA step);
-//   * warp 1, one thread, issues per step 8 tcgen05.cp (scale atoms -> TMEM) and 4 tcgen05.mma
-//     (128 x BN x 64 each, fp32 accumulator in TMEM), then a tcgen05.commit that frees the stage;
+//   * warp 0, one thread, produces: for each 256-element step of k, one TMA load per operand
+//     (128 or BN rows x 128 bytes, 128-byte swizzle) and one bulk copy per 128-row tile of the
+//     step's scales, which mx_matmul_prepare_scales has already put into tensor-core order (2048
+//     contiguous bytes per 128 rows and step), all completing on the stage's full mbarrier;
+//   * warp 1, one thread, issues per step the tcgen05.cp copies of the scale groups into TMEM
+//     (rotating through MX_MM_SFBUF buffers) and 4 tcgen05.mma (128 x BN x 64 each, fp32
+//     accumulator in TMEM), then a tcgen05.commit that frees the stage;
 //   * all 4 warps then read the accumulator (tcgen05.ld, one row per thread), multiply by gA gB
 //     and store C.
-// Stages are handed over with mbarriers (full: TMA bytes + one arrival per producer lane when its
-// scale copies land; empty: the commit).  Every wait is bounded: a CTA that gives up records it in a device counter, lets its
-// issued copies and MMAs finish (bounded again), frees its TMEM and returns.
+// Every wait is bounded: a CTA that gives up records it in a device counter and marks its launch
+// (a generation number passed per launch) so that the launch's other CTAs stop waiting too; it
+// lets its issued copies and MMAs finish (bounded again), frees its TMEM and returns.  Later
+// launches carry other generation numbers and are not affected.
 #include <cuda.h>
-#include <stdlib.h>
+
+#include <atomic>
 
 #include "mx_device.cuh"
 #include "mx_launch.h"
@@ -75,8 +77,11 @@ struct Tile {
                                      ((uint32_t)(kBM >> 4) << 24);
 };
 
-__device__ unsigned int g_mm_gave_up;     // CTAs that stopped waiting (bounded waits ran out)
-__device__ volatile int g_mm_abandon;     // set by a CTA that gave up: the others stop waiting too
+__device__ unsigned int g_mm_gave_up;  // CTAs that stopped waiting (bounded waits ran out)
+// Generation number of the last launch one of whose CTAs gave up: the launch's other CTAs stop
+// waiting too.  Every launch gets a new number (from 1), so a launch that gave up leaves later
+// launches alone.
+__device__ volatile unsigned int g_mm_abandon_gen;
 
 struct MmArgs {
   const uint8_t* a_scales;
@@ -85,6 +90,7 @@ struct MmArgs {
   int64_t m, n, k;
   float alpha;
   int c_bf16;
+  unsigned int gen;  // this launch's generation number (never 0)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -106,9 +112,9 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 // critical path must not flood the shared-memory pipe that the TMA and the tensor core use.
 // CLUSTER: acquire at cluster scope (the phase was completed by the other CTA of a pair).
 template <int SLEEP_NS = 0, bool CLUSTER = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int gen) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if ((i & 1023u) == 1023u && g_mm_abandon) return false;
+    if ((i & 1023u) == 1023u && g_mm_abandon_gen == gen) return false;
     if (SLEEP_NS > 0 && i > 0) __nanosleep(SLEEP_NS);
     uint32_t ok;
     if constexpr (CLUSTER)
@@ -336,7 +342,8 @@ __global__ void __launch_bounds__(128, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % kStages;
         if (*gave_up ||
-            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
+            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1,
+                                                     args.gen))) {
           *gave_up = 1;
           break;
         }
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(128, 1)
       if (*gave_up) {
         // let the copies already issued land before the CTA can exit (bounded)
         for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt)
-          mbar_wait<100>(smem_u32(full + kt % kStages), (kt / kStages) & 1);
+          mbar_wait<100>(smem_u32(full + kt % kStages), (kt / kStages) & 1, args.gen);
       }
     }
     __syncwarp();
@@ -365,7 +372,7 @@ __global__ void __launch_bounds__(128, 1)
     if (lane == 0) {
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % kStages;
-        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1)) {
+        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1, args.gen)) {
           *gave_up = 1;
           break;
         }
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncwarp();
   bool ok = true;
   if (lane == 0) {
-    ok = mbar_wait<200>(smem_u32(done), 0);  // sleeps through the main loop
+    ok = mbar_wait<200>(smem_u32(done), 0, args.gen);  // sleeps through the main loop
     if (!ok) *gave_up = 1;
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -405,7 +412,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   if (threadIdx.x == 0 && *gave_up) {
     atomicAdd(&g_mm_gave_up, 1u);
-    g_mm_abandon = 1;
+    g_mm_abandon_gen = args.gen;
   }
   if (warp == 0) {
     tc_fence_after();
@@ -546,7 +553,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % kStages;
         if (*gave_up ||
-            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1))) {
+            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1,
+                                                     args.gen))) {
           *gave_up = 1;
           break;
         }
@@ -577,7 +585,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
       const uint32_t empty1 = map_to(smem_u32(empty), 1), done1 = map_to(smem_u32(done), 1);
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % kStages;
-        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1)) {
+        if (!mbar_wait(smem_u32(full + s), (kt / kStages) & 1, args.gen)) {
           *gave_up = 1;
           break;
         }
@@ -609,7 +617,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
   __syncwarp();
   bool ok = true;
   if (lane == 0) {
-    ok = mbar_wait<200>(smem_u32(done), 0);
+    ok = mbar_wait<200>(smem_u32(done), 0, args.gen);
     if (!ok) *gave_up = 1;
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -619,7 +627,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
   __syncthreads();
   if (threadIdx.x == 0 && *gave_up) {
     atomicAdd(&g_mm_gave_up, 1u);
-    g_mm_abandon = 1;
+    g_mm_abandon_gen = args.gen;
   }
   cluster_sync();  // neither CTA releases TMEM or exits while the pair still signals it
   if (warp == 0) {
@@ -680,25 +688,42 @@ bool make_rows_map(CUtensorMap* map, const uint8_t* scales, int64_t rows) {
 
 int64_t mma_scales_bytes(int64_t rows, int64_t k);
 
+// Dynamic shared memory above 48 KiB must be enabled per kernel and per device; the flag of a
+// device is set once the attribute call has succeeded there (a failed call is retried next time).
+constexpr int kMaxDevices = 64;
+static std::atomic<bool> g_smem_one[kMaxDevices], g_smem_pair[kMaxDevices];
+static std::atomic<unsigned int> g_launch_gen{0};
+
+template <typename K>
+static cudaError_t allow_smem(std::atomic<bool>* flags, K* kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && flags[dev].load(std::memory_order_acquire))
+    return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices)
+    flags[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+// A new generation number for a launch (never 0, the flag's initial value).
+static unsigned int next_gen() {
+  unsigned int g = g_launch_gen.fetch_add(1u) + 1u;
+  if (g == 0) g = g_launch_gen.fetch_add(1u) + 1u;
+  return g;
+}
+
 cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
-                             cudaStream_t stream, int* launches) {
-  MmArgs args{a_scales, b_scales, c, m, n, k, alpha, c_bf16 ? 1 : 0};
+                             bool cta_pairs, cudaStream_t stream, int* launches) {
+  MmArgs args{a_scales, b_scales, c, m, n, k, alpha, c_bf16 ? 1 : 0, next_gen()};
   CUtensorMap ma, mb;
-  // The CTA-pair kernel is correct but, with its per-step scale copies, not yet faster than the
-  // one-CTA kernel on B200; MXFP4_MATMUL_PAIRS=1 selects it (for m > 128).
-  const char* env = getenv("MXFP4_MATMUL_PAIRS");
-  const bool pairs_on = env != nullptr && env[0] == '1';
-  if (m > kBM && pairs_on) {
+  if (m > kBM && cta_pairs) {
     // CTA pairs: 256 x 256 tiles of C
-    static bool attr_set = false;
-    if (!attr_set) {
-      const cudaError_t e = cudaFuncSetAttribute(
-          k_matmul_nvfp4_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, Pair::kSmemBytes);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    cudaError_t e = allow_smem(g_smem_pair, k_matmul_nvfp4_pair, Pair::kSmemBytes);
+    if (e != cudaSuccess) return e;
     CUtensorMap msa, msb;
     if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, kBM) ||
         !make_rows_map(&msa, a_scales, mma_scales_bytes(m, k) / 256) ||
@@ -711,13 +736,8 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
     constexpr int BN = MX_MM_BN;
     static_assert(BN == 128 || BN == 256, "tile width");
     using T = Tile<BN>;
-    static bool attr_set = false;
-    if (!attr_set) {
-      const cudaError_t e = cudaFuncSetAttribute(
-          k_matmul_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    cudaError_t e = allow_smem(g_smem_one, k_matmul_nvfp4<BN>, T::kSmemBytes);
+    if (e != cudaSuccess) return e;
     if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, BN))
       return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)((m + kBM - 1) / kBM));
@@ -743,11 +763,14 @@ cudaError_t run_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t k, ui
 
 cudaError_t matmul_gave_up(unsigned int* count) {
   const unsigned int zero = 0;
-  const int izero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(count, g_mm_gave_up, sizeof(unsigned int));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_mm_gave_up, &zero, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_mm_abandon, &izero, sizeof(int));
   return e;
+}
+
+cudaError_t matmul_abandon_last() {
+  const unsigned int gen = g_launch_gen.load();
+  return cudaMemcpyToSymbol(g_mm_abandon_gen, &gen, sizeof(unsigned int));
 }
 
 }  // namespace mxk

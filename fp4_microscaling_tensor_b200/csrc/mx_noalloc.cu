@@ -11,7 +11,9 @@
 // The array lives in every device's copy of this library's module for as long as the process keeps
 // the library loaded.  Host code cannot use the array's name as a device address, so the first call
 // on each device resolves the address with cudaGetSymbolAddress (with that device current) and
-// keeps it; later calls on that device reuse it.
+// keeps it; later calls on that device reuse it.  A lookup that fails is not kept: the call
+// reports MX_ERR_CUDA and the next call tries again.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mx.h"
@@ -26,23 +28,29 @@ constexpr size_t kNoAllocScratchBytes = (size_t)mxk::kMaxReduceCtas * 64;  // 25
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_resolve_mutex[kMaxDevices];
+std::atomic<void*> g_scratch_ptr[kMaxDevices];  // nullptr until resolved on that device
 
-// Device address of the scratch array on the current device, resolved once per device.
+// Device address of the scratch array on the current device.  Only a successful lookup is kept:
+// a failure (for example an error left pending by unrelated earlier work) is returned to this
+// caller, and the next call on the device tries again.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = 0;
   const cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev]() {
-    void* p = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_scratch_ptr[dev] = p;
-  });
-  *out = g_scratch_ptr[dev];
-  return g_scratch_err[dev];
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_resolve_mutex[dev]);
+    p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      const cudaError_t r = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (r != cudaSuccess || p == nullptr) return r != cudaSuccess ? r : cudaErrorUnknown;
+      g_scratch_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -45,6 +45,7 @@ struct QTensor {
   void* y;  // round trip (OUT != kCodes): the dequantized output instead of codes and scales
   int64_t nitems;
   uint32_t g_bits;
+  const uint16_t* g_dev;  // g in device memory (written by the previous kernel) when set
 };
 
 // What a quantize kernel writes: codes and scales, or (the fake-quantize round trip) the
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
   const int64_t nitems = wk.t.nitems;
   __shared__ float s_rcp[256];
   __shared__ float s_D[OUT == kCodes ? 1 : 256];
-  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(wk.t.g_bits, wk.t.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);  // exact (<= 15 significant bits)
     s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;          // zero scale -> every code is +-0
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant
   uint8_t* __restrict__ scales = wk.t.scales;
   const int64_t nitems = wk.t.nitems;
   __shared__ float s_D[256];
-  const float g = fp16_bits_to_float((uint16_t)wk.t.g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(wk.t.g_bits, wk.t.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
   const float g6 = __fmul_rn(6.0f, g);
   __syncthreads();
@@ -293,10 +294,11 @@ __global__ void __launch_bounds__(kThreads) k_quantize_f32(const __grid_constant
 
 template <int FMT, typename T, int OUT = kCodes>
 __global__ void k_quantize_tail(const T* __restrict__ x, int64_t first, int count, int N,
-                                uint16_t g_bits, uint8_t* __restrict__ packed,
-                                uint8_t* __restrict__ scales, void* __restrict__ y = nullptr) {
+                                uint16_t g_bits, const uint16_t* g_dev,
+                                uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                                void* __restrict__ y = nullptr) {
   if (threadIdx.x != 0) return;
-  const float g = fp16_bits_to_float(g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(g_bits, g_dev));
   for (int b0 = 0; b0 < count; b0 += N) {
     const int64_t f = first + b0;
     float v[16], a = 0.0f;  // N <= 16
@@ -341,7 +343,8 @@ static cudaError_t launch_q(const TensorArgs* ta, int count, cudaStream_t stream
   int64_t nitems[kMaxGroup];
   for (int k = 0; k < count; ++k) {
     nitems[k] = ta[k].numel / S::EPT;
-    grp.t[k] = {ta[k].x, ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits};
+    grp.t[k] = {ta[k].x, ta[k].packed, ta[k].scales, ta[k].y, nitems[k], ta[k].g_bits,
+                ta[k].g_dev};
   }
   auto kern = (sizeof(T) == 2) ? (void*)k_quantize_bf16<N, FMT, OUT>
                                : (void*)k_quantize_f32<N, FMT, OUT>;
@@ -357,7 +360,7 @@ static cudaError_t launch_q(const TensorArgs* ta, int count, cudaStream_t stream
     if (ta[k].numel % S::EPT != 0) {  // only N = 4 leaves a remainder (of exactly 4 elements)
       k_quantize_tail<FMT, T, OUT><<<1, 32, 0, stream>>>(
           (const T*)ta[k].x, nitems[k] * S::EPT, (int)(ta[k].numel % S::EPT), N, ta[k].g_bits,
-          ta[k].packed, ta[k].scales, ta[k].y);
+          ta[k].g_dev, ta[k].packed, ta[k].scales, ta[k].y);
       ++*launches;
     }
   }
@@ -379,22 +382,22 @@ static cudaError_t dispatch_block(int block, const TensorArgs* t, int count, cud
 }
 
 cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,
-                              uint16_t g_bits, uint8_t* packed, uint8_t* scales,
-                              cudaStream_t stream, int* launches) {
+                              uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                              uint8_t* scales, cudaStream_t stream, int* launches) {
   if (bf16) {
     if (fmt == kUE5M3)
       k_quantize_tail<kUE5M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, count, N,
-                                                              g_bits, packed, scales);
+                                                              g_bits, g_dev, packed, scales);
     else
       k_quantize_tail<kE4M3, uint16_t><<<1, 32, 0, stream>>>((const uint16_t*)x, first, count, N,
-                                                             g_bits, packed, scales);
+                                                             g_bits, g_dev, packed, scales);
   } else {
     if (fmt == kUE5M3)
       k_quantize_tail<kUE5M3, float><<<1, 32, 0, stream>>>((const float*)x, first, count, N,
-                                                           g_bits, packed, scales);
+                                                           g_bits, g_dev, packed, scales);
     else
       k_quantize_tail<kE4M3, float><<<1, 32, 0, stream>>>((const float*)x, first, count, N,
-                                                          g_bits, packed, scales);
+                                                          g_bits, g_dev, packed, scales);
   }
   ++*launches;
   return cudaGetLastError();

@@ -12,8 +12,6 @@ errors shard by shard with no exchange, except for two per-tensor quantities:
 Each rank runs the library's kernels on its own shard; only these two small collectives cross
 ranks (NCCL over NVLink on GPUs, gloo on the CPU in the tests).
 """
-import struct
-
 import torch
 import torch.distributed as dist
 
@@ -40,16 +38,12 @@ def combine_stats(local, group=None, device=None):
         dist.all_reduce(cnts, op=dist.ReduceOp.SUM, group=group)
     out = dict(zip(_FIELDS[:3], (float(v) for v in sums.tolist())))
     out.update(zip(_FIELDS[3:], (int(v) for v in cnts.tolist())))
-    n = out["numel"] or 1
-    out.update(mse_elem=out["sse_elem"] / n, mse_max=out["sse_max"] / n,
-               mse_zero=out["sse_zero"] / n)
-    out["mse_total"] = out["mse_elem"] + out["mse_max"] + out["mse_zero"]
-    return out
+    return api.record_dict(api.record_bytes(out))
 
 
 def record_from_bytes(raw):
-    """An error record (64 bytes, mx_error_stats_t) as a dict."""
-    return dict(zip(_FIELDS, struct.unpack("<3d5q", bytes(raw))))
+    """An error record (64 bytes, mx_error_stats_t) as a dict (with the means)."""
+    return api.record_dict(raw)
 
 
 def global_scale_sharded(x_local, fmt="e4m3", group=None):

@@ -16,7 +16,12 @@
  *
  * Conventions shared by every entry point:
  *   - All tensors are caller-owned DEVICE memory, contiguous and row-major.  The library never
- *     allocates, never synchronizes and keeps no state between calls.
+ *     allocates and never synchronizes (except the calls documented as synchronizing).  State that
+ *     outlives a call: the diagnostic launch counter (mx_kernel_launches), the scratch array of
+ *     mx_error_stats_noalloc (shared by its calls on a device, see there), the test hook's armed
+ *     failures (mx_test_fail_next_calls), and for mx_matmul a per-device count of thread blocks
+ *     whose bounded waits ran out plus the generation number of the last launch that gave up
+ *     (see mx_matmul_gave_up; later launches are not affected by it).
  *   - Everything is enqueued on `stream` (0 = the legacy default stream); results are valid after
  *     the caller synchronizes that stream.
  *   - Arguments are checked on the host before anything is enqueued; a non-OK status means nothing
@@ -143,6 +148,12 @@ MX_API mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int
                                    uint8_t* packed, uint8_t* scales, mx_error_stats_t* out_dev,
                                    void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* The pages' mean squared errors from a record copied to host memory ([MX] §2.2: each sum over
+ * the tensor's element count, so the three means add up to the total MSE):
+ * mse4[0..3] = sse_elem / numel, sse_max / numel, sse_zero / numel and their sum (all zero for an
+ * empty tensor).  record and mse4 are host memory; NULL gives MX_ERR_INVALID_ARG. */
+MX_API mx_status mx_error_stats_means(const mx_error_stats_t* record, double* mse4);
+
 /* Bytes of device workspace mx_global_scale needs. */
 MX_API size_t mx_global_scale_workspace_size(int64_t rows, int64_t cols);
 
@@ -184,13 +195,19 @@ MX_API mx_status mx_error_stats_noalloc(const void* x, mx_dtype xt, int64_t rows
 
 /* One tensor of a grouped call: rows x cols, row-major, cols % block == 0. */
 typedef struct {
-  const void* x;              /* input of mx_quantize_group / mx_quantize_stats_group */
+  const void* x;              /* input of mx_quantize_group / mx_quantize_stats_group /
+                                 mx_global_scale_group */
   void* y;                    /* output of mx_dequantize_group */
   uint8_t* packed;            /* rows*cols/2 codes: written by quantize, read by dequantize */
   uint8_t* scales;            /* rows*cols/block scale codes, likewise */
   mx_error_stats_t* stats;    /* mx_quantize_stats_group: this tensor's record (device) */
+  uint16_t* global_scale_dev; /* NULL, or the device address (2-byte aligned) of this tensor's g
+                                 as a binary16 bit pattern: written by mx_global_scale_group, read
+                                 by the other grouped calls when their kernels run (so g never
+                                 visits the host; global_scale_fp16 is then ignored) */
   int64_t rows, cols;
-  uint16_t global_scale_fp16; /* per-tensor g, as in mx_quantize */
+  uint16_t global_scale_fp16; /* per-tensor g, as in mx_quantize (used when global_scale_dev is
+                                 NULL) */
   uint16_t reserved[3];       /* must be zero */
 } mx_tensor_t;
 
@@ -207,6 +224,15 @@ MX_API mx_status mx_dequantize_group(const mx_tensor_t* tensors, int count, int 
 MX_API mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtype xt,
                                          int block, mx_scale_fmt fmt, void* workspace,
                                          size_t ws_bytes, cudaStream_t stream);
+
+/* mx_global_scale of every tensor (x -> *global_scale_dev, which must be non-NULL) with one
+ * workspace of mx_global_scale_workspace_size() bytes for the whole group; global_scale_fp16 is
+ * not read.  The same descriptors can then drive mx_quantize_stats_group and mx_dequantize_group
+ * on the same stream: the per-tensor g stays in device memory ([MX] §3.1 item 3, a per-tensor
+ * FP16 factor; how it is chosen is this library's rule, see mx_global_scale). */
+MX_API mx_status mx_global_scale_group(const mx_tensor_t* tensors, int count, mx_dtype xt,
+                                       mx_scale_fmt fmt, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream);
 
 /* ---- Block-scaled matrix product on the tensor cores.
  * C = dequant(A) * dequant(B)^T, the dequantize-then-multiply step of inference in the 4-bit float
@@ -239,17 +265,30 @@ MX_API mx_status mx_matmul_prepare_scales(const uint8_t* scales, int64_t rows, i
  * block != 16 or fmt != MX_SCALE_E4M3 (no native tensor-core form), k == 0 or k % 256 != 0:
  * MX_ERR_UNSUPPORTED; m, n or k negative, or m, n >= 2^31: MX_ERR_INVALID_ARG; m == 0 or n == 0:
  * nothing is enqueued.  Every wait inside the kernel is bounded; a launch whose waits ran out
- * leaves C unspecified and is counted by mx_matmul_gave_up.  Kernel: one CTA per 128 x 256 tile
- * of C; with the environment variable MXFP4_MATMUL_PAIRS=1 (read at each call) and m > 128, CTA
- * pairs (tcgen05 cta_group::2) per 256 x 256 tile instead, with the same results. */
+ * leaves C unspecified and is counted by mx_matmul_gave_up (it does not affect later launches).
+ * Kernel: one CTA per 128 x 256 tile of C. */
 MX_API mx_status mx_matmul(const uint8_t* a_packed, const uint8_t* a_scales_mma, uint16_t a_g,
                            const uint8_t* b_packed, const uint8_t* b_scales_mma, uint16_t b_g,
                            int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt, void* c,
                            mx_dtype ct, cudaStream_t stream);
 
+/* mx_matmul computed by CTA pairs (tcgen05 cta_group::2): a cluster of two CTAs per 256 x 256
+ * tile of C when m > 128 (else the one-CTA kernel).  Same arguments, results and errors as
+ * mx_matmul; an alternative kernel for the same product (slower than mx_matmul on the shapes
+ * measured so far). */
+MX_API mx_status mx_matmul_pair(const uint8_t* a_packed, const uint8_t* a_scales_mma, uint16_t a_g,
+                                const uint8_t* b_packed, const uint8_t* b_scales_mma, uint16_t b_g,
+                                int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt,
+                                void* c, mx_dtype ct, cudaStream_t stream);
+
 /* Number of mx_matmul thread blocks that stopped waiting since the previous call (0 in normal
  * operation), written to *count (host memory); clears the count.  Synchronizes the device. */
 MX_API mx_status mx_matmul_gave_up(unsigned int* count);
+
+/* Test hook (no counterpart in the pages): marks the most recent mx_matmul / mx_matmul_pair launch
+ * on the current device as abandoned, as a thread block whose waits ran out would.  Later
+ * launches must not be affected.  Synchronizes the device. */
+MX_API mx_status mx_test_matmul_abandon_last(void);
 
 /* Test hook for error paths (no counterpart in the pages).  The next `count` calls that pass
  * their argument checks and would enqueue work return MX_ERR_CUDA instead, as a failed launch is
@@ -261,7 +300,7 @@ MX_API int mx_test_fail_next_calls(int count);
 MX_API const char* mx_status_string(mx_status status);
 
 /* Diagnostic: number of kernels this library has enqueued in this process so far (all calls,
- * all threads).  The only state the library keeps; it never affects results. */
+ * all threads).  It never affects results. */
 MX_API long long mx_kernel_launches(void);
 
 #ifdef __cplusplus

@@ -138,11 +138,12 @@ def test_python_binding_marshalling_errors():
     assert mx.g_bits(None) == 0x3C00 and mx.g_bits(1.0) == 0x3C00 and mx.g_bits(0x1234) == 0x1234
 
 
-def group(n, rows=4, cols=64, x=A, y=A, p=A, s=A, st=A, g=0x3C00, reserved=0):
+def group(n, rows=4, cols=64, x=A, y=A, p=A, s=A, st=A, g=0x3C00, reserved=0, gdev=None):
     d = (_lib.Tensor * max(n, 1))()
     for k in range(max(n, 1)):
         d[k].x, d[k].y, d[k].packed, d[k].scales, d[k].stats = x, y, p, s, st
         d[k].rows, d[k].cols, d[k].global_scale_fp16 = rows, cols, g
+        d[k].global_scale_dev = gdev
         d[k].reserved[0] = reserved
     return d
 
@@ -174,6 +175,47 @@ def test_group_calls_reject_bad_arguments():
     d = group(3)
     d[2].cols = 40
     assert L.mx_quantize_group(d, 3, BF16, 32, E4, None) == INV
+
+
+def test_device_global_scales_in_groups():
+    gws = L.mx_global_scale_workspace_size(4, 64)
+    # g read from device memory: the bit-pattern field is then not checked, the address must be
+    # 2-byte aligned
+    L.mx_test_fail_next_calls(1)  # valid arguments on fake pointers: stop before any launch
+    assert L.mx_quantize_group(group(2, g=0, gdev=A + 2), 2, BF16, 32, E4, None) == \
+        _lib.MX_ERR_CUDA
+    assert L.mx_quantize_group(group(2, g=0, gdev=A + 3), 2, BF16, 32, E4, None) == MIS
+    assert L.mx_dequantize_group(group(2, g=0, gdev=A + 1), 2, 32, E4, BF16, None) == MIS
+    assert L.mx_quantize_group(group(2, g=0), 2, BF16, 32, E4, None) == INV  # neither form
+    # the grouped global scale writes g: the address is required, the bit pattern ignored
+    assert L.mx_global_scale_group(group(2, gdev=None), 2, BF16, E4, A, gws, None) == INV
+    assert L.mx_global_scale_group(group(2, gdev=A + 1), 2, BF16, E4, A, gws, None) == MIS
+    assert L.mx_global_scale_group(group(2, gdev=A, x=None), 2, BF16, E4, A, gws, None) == INV
+    assert L.mx_global_scale_group(group(2, gdev=A, x=A + 4), 2, BF16, E4, A, gws, None) == MIS
+    assert L.mx_global_scale_group(group(2, gdev=A), 2, 5, E4, A, gws, None) == INV
+    assert L.mx_global_scale_group(group(2, gdev=A), 2, BF16, 7, A, gws, None) == INV
+    assert L.mx_global_scale_group(group(2, gdev=A), 2, BF16, E4, None, gws, None) == WS
+    assert L.mx_global_scale_group(group(2, gdev=A), 2, BF16, E4, A, gws - 1, None) == WS
+    assert L.mx_global_scale_group(group(0, gdev=A), 0, BF16, E4, A, gws, None) == INV
+    L.mx_test_fail_next_calls(1)  # any cols is fine for the global scale (it has no block)
+    assert L.mx_global_scale_group(group(2, gdev=A, cols=40), 2, BF16, E4, A, gws, None) == \
+        _lib.MX_ERR_CUDA
+    assert L.mx_test_fail_next_calls(0) == 0
+
+
+def test_error_stats_means_on_the_host():
+    import fp4_microscaling_tensor_b200 as mx
+    rec = mx.api.record_bytes(dict(sse_elem=3.0, sse_max=1.5, sse_zero=0.5, numel=8, n_blocks=1,
+                                   n_zero_blocks=0, n_scale_sat=0, n_elem_sat=0))
+    d = mx.api.record_dict(rec)
+    assert (d["mse_elem"], d["mse_max"], d["mse_zero"], d["mse_total"]) == \
+        (3.0 / 8, 1.5 / 8, 0.5 / 8, 5.0 / 8)
+    empty = mx.api.record_dict(mx.api.record_bytes(dict.fromkeys(mx.api.STATS_FIELDS, 0)))
+    assert empty["mse_total"] == 0.0
+    out = (ctypes.c_double * 4)()
+    assert L.mx_error_stats_means(None, out) == INV
+    buf = ctypes.create_string_buffer(rec, 64)
+    assert L.mx_error_stats_means(ctypes.addressof(buf), None) == INV
 
 
 def test_fake_quantize_rejects_bad_arguments():
@@ -214,6 +256,9 @@ def test_matmul_rejects_bad_arguments():
     assert mm(m=0, ap=None, as_=None, c=None) == OK   # empty product: nothing to do
     assert mm(n=0) == OK
     assert L.mx_matmul_gave_up(None) == INV
+    # the CTA-pair entry point checks the same arguments
+    args = (A, A, 0x3C00, A, A, 0x3C00, 128, 64, 256, 32, E4, A, BF16, None)
+    assert L.mx_matmul_pair(*args) == UNS
 
 
 def test_matmul_scale_preparation_arguments():

@@ -1,25 +1,23 @@
-"""Parity at the workload configurations' full sizes, through the launches the benchmark times.
+"""Parity at the workload configurations' full sizes, whole tensors, through the launches the
+benchmark times.
 
 Every tensor is drawn on the GPU with the seeded generators of `inputs.py` and copied to the host
-for the oracle.  A configuration is either compared with the oracle over whole tensors (codes,
-scales and dequantized bits bit-exact, the error record within 1e-5 relative, counts exact) or,
-where a whole-tensor oracle run would take too long, on sampled rows (first, last and seeded
-random rows) plus properties that hold at any size:
-
-* the three error sums add up to sum((x - y)^2) over the tensor, y the exact (fp32) dequantized
-  output (checked in float64 on the device), and the zero-scale sum to sum(x^2) over zero-scale
-  blocks;
-* n_blocks = numel / N and n_zero_blocks = the number of zero scale bytes.
+for the oracle.  Every tensor is compared whole: codes, scales and dequantized bits bit-exact, and
+the error record term by term (sse_elem, sse_max and sse_zero each within 1e-5 relative, the counts
+exactly) against the oracle's record for the same codes.
 
 Configurations (sizes as the workloads state them):
-  2  bf16 4096x4096 x 5 sigma, N in {4..256} x {E4M3, UE5M3}: the 14 points of sigma = 0.02 whole,
-     the other 56 sampled + properties.
-  3  Llama-2-7B-shaped weights (32 layers x 7 tensors, Student-t rows), N = 32, UE5M3 + global
-     scale: layer 0 whole, every layer sampled.
-  4  activations bf16 16384x8192 with outlier channels, N = 16, E4M3: whole.
-  5  Llama-2-70B-shaped layer (2 x 8192^2, 2 x 1024x8192, 3 x 8192x28672), N = 32, UE5M3 + global
-     scale, with the error record: layer 0 whole; layers 1, 13, 27, 40, 53, 66, 79 sampled +
-     properties.
+  2  bf16 4096x4096 x 5 sigma, N in {4..256} x {E4M3, UE5M3}: all 70 points, through the grouped
+     fused pass and grouped dequantize the benchmark's sweep launches (one launch per (N, format)
+     over the five sigma tensors).
+  3  Llama-2-7B-shaped weights (32 layers x 7 tensors, Student-t rows), N = 32, UE5M3 + per-tensor
+     global scale: all 224 tensors, per layer the grouped global scale, fused pass and dequantize
+     with g kept in device memory.
+  4  activations bf16 16384x8192 with outlier channels, N = 16, E4M3: quantize, dequantize and
+     the error record.
+  5  Llama-2-70B-shaped layers (2 x 8192^2, 2 x 1024x8192, 3 x 8192x28672), N = 32, UE5M3 + global
+     scale: the eight layers 0, 1, 13, 27, 40, 53, 66, 79, through the benchmark's three grouped
+     launches per layer (global scale -> fused pass -> dequantize, g in device memory).
 """
 import numpy as np
 import pytest
@@ -34,32 +32,8 @@ from gpu_helpers import assert_same, assert_stats, bits, u8
 pytestmark = pytest.mark.gpu
 
 
-def bench_launches(x, block, fmt, g=0x3C00):
-    """The benchmark's two launches for one tensor: fused pass, then dequantize (bf16 out)."""
-    p, s, st = mx.quantize_with_stats(x, block, fmt, g)
-    y = mx.dequantize(p, s, block, fmt, g)
-    return p, s, st.to_dict(), y
-
-
-def sample_rows(rows, seed, k=6):
-    rng = np.random.default_rng(seed)
-    extra = rng.choice(rows, size=min(k, rows), replace=False).tolist()
-    return sorted(set([0, rows - 1] + extra))
-
-
-def check_rows(x, p, s, y, block, fmt, g, row_ids, what):
-    """Codes, scales and dequantized bits of the chosen rows against the oracle, row by row."""
-    cols = x.shape[1]
-    for r in row_ids:
-        xr = inputs.to_oracle(x[r:r + 1])
-        po, so = oracle.quantize(xr, 1, cols, block, fmt, g)
-        assert_same(u8(s[r]), so, f"{what} scales row {r}")
-        assert_same(u8(p[r]), po, f"{what} packed row {r}")
-        yo = oracle.dequantize(po, so, 1, cols, block, fmt, g, out_bf16=True)
-        assert_same(bits(y[r]), yo, f"{what} dequant row {r}")
-
-
 def check_whole(x, p, s, st, y, block, fmt, g, what):
+    """Codes, scales, dequantized bits and the error record of one tensor against the oracle."""
     rows, cols = x.shape
     xo = inputs.to_oracle(x)
     po, so = oracle.quantize(xo, rows, cols, block, fmt, g)
@@ -71,86 +45,57 @@ def check_whole(x, p, s, st, y, block, fmt, g, what):
     assert_stats(st, ref, f"{what} stats")
 
 
-def check_properties(x, p, s, st, block, fmt, g, what):
-    """Size-independent identities between the error record and the tensors themselves (y is the
-    exact fp32 dequantization of the stored codes)."""
-    y = mx.dequantize(p, s, block, fmt, g, out_dtype=torch.float32)
-    numel = x.numel()
-    assert st["numel"] == numel and st["n_blocks"] == numel // block, what
-    zero = (s == 0)
-    assert st["n_zero_blocks"] == int(zero.sum()), what
-    xd = x.double().reshape(-1, block)
-    d2 = (xd - y.double().reshape(-1, block)).square().sum(dim=1)
-    total = float(d2.sum())
-    got = st["sse_elem"] + st["sse_max"] + st["sse_zero"]
-    assert abs(got - total) <= 1e-5 * total, (what, got, total)
-    zsum = float(xd.square().sum(dim=1)[zero.reshape(-1)].sum())
-    assert abs(st["sse_zero"] - zsum) <= 1e-5 * max(zsum, 1e-300), (what, st["sse_zero"], zsum)
+def layer_launches(xs, block, fmt):
+    """The benchmark's three grouped launches over one layer: global scales into device memory,
+    the fused pass and dequantize reading them there.  Returns (g bits, packed, scales, records,
+    dequantized)."""
+    g = mx.global_scale_group(xs, fmt)
+    p, s, st = mx.quantize_with_stats_group(xs, block, fmt, g=g)
+    y = mx.dequantize_group(p, s, block, fmt, g=g)
+    gh = [int(v) for v in g.cpu().numpy().view(np.uint16)]
+    return gh, p, s, [t.to_dict() for t in st], y
 
 
-def test_config2_sweep(cuda_device):
-    for k in range(len(inputs.SWEEP_SIGMAS)):
-        x = inputs.workload2(k, device=cuda_device)
-        for n in inputs.SWEEP_BLOCKS:
-            for fmt in (mx.E4M3, mx.UE5M3):
-                what = f"config 2 sigma={inputs.SWEEP_SIGMAS[k]} N={n} fmt={fmt}"
-                p, s, st, y = bench_launches(x, n, fmt)
-                if k == 2:
-                    check_whole(x, p, s, st, y, n, fmt, 0x3C00, what)
-                else:
-                    check_rows(x, p, s, y, n, fmt, 0x3C00, sample_rows(x.shape[0], 17 * k + n),
-                               what)
-                    check_properties(x, p, s, st, n, fmt, 0x3C00, what)
+@pytest.mark.parametrize("block", inputs.SWEEP_BLOCKS)
+@pytest.mark.parametrize("fmt", (mx.E4M3, mx.UE5M3))
+def test_config2_sweep_whole(cuda_device, block, fmt):
+    xs = [inputs.workload2(k, device=cuda_device) for k in range(len(inputs.SWEEP_SIGMAS))]
+    p, s, st = mx.quantize_with_stats_group(xs, block, fmt)
+    y = mx.dequantize_group(p, s, block, fmt)
+    for k, x in enumerate(xs):
+        what = f"config 2 sigma={inputs.SWEEP_SIGMAS[k]} N={block} fmt={fmt}"
+        check_whole(x, p[k], s[k], st[k].to_dict(), y[k], block, fmt, 0x3C00, what)
 
 
-def test_config3_llama7b_weights(cuda_device):
-    for layer in range(32):
-        for j in range(len(inputs.LLAMA7B_SHAPES)):
-            x = inputs.workload3_tensor(layer, j, device=cuda_device)
-            what = f"config 3 layer {layer} tensor {j}"
-            g = int(mx.global_scale(x, mx.UE5M3).item()) & 0xFFFF
-            if layer == 0:
-                assert g == oracle.global_scale(inputs.to_oracle(x), mx.UE5M3), what
-            p, s = mx.quantize(x, 32, mx.UE5M3, g)
-            y = mx.dequantize(p, s, 32, mx.UE5M3, g)
-            if layer == 0:
-                xo = inputs.to_oracle(x)
-                rows, cols = x.shape
-                po, so = oracle.quantize(xo, rows, cols, 32, mx.UE5M3, g)
-                assert_same(u8(s), so, what + " scales")
-                assert_same(u8(p), po, what + " packed")
-                yo = oracle.dequantize(po, so, rows, cols, 32, mx.UE5M3, g, out_bf16=True)
-                assert_same(bits(y), yo, what + " dequant")
-            else:
-                check_rows(x, p, s, y, 32, mx.UE5M3, g, sample_rows(x.shape[0], layer, k=2), what)
+@pytest.mark.parametrize("layer", range(32))
+def test_config3_llama7b_weights_whole(cuda_device, layer):
+    xs = [inputs.workload3_tensor(layer, j, device=cuda_device)
+          for j in range(len(inputs.LLAMA7B_SHAPES))]
+    gh, p, s, st, y = layer_launches(xs, 32, mx.UE5M3)
+    for j, x in enumerate(xs):
+        what = f"config 3 layer {layer} tensor {j}"
+        assert gh[j] == oracle.global_scale(inputs.to_oracle(x), oracle.UE5M3), what
+        check_whole(x, p[j], s[j], st[j], y[j], 32, mx.UE5M3, gh[j], what)
 
 
-def test_config4_activations(cuda_device):
+def test_config4_activations_whole(cuda_device):
     x = inputs.workload4(device=cuda_device)
-    rows, cols = x.shape
-    p, s = mx.quantize(x, 16, mx.E4M3)
+    p, s, st = mx.quantize_with_stats(x, 16, mx.E4M3)
     y = mx.dequantize(p, s, 16, mx.E4M3)
-    xo = inputs.to_oracle(x)
-    po, so = oracle.quantize(xo, rows, cols, 16, mx.E4M3)
-    assert_same(u8(s), so, "config 4 scales")
-    assert_same(u8(p), po, "config 4 packed")
-    yo = oracle.dequantize(po, so, rows, cols, 16, mx.E4M3, out_bf16=True)
-    assert_same(bits(y), yo, "config 4 dequant")
+    check_whole(x, p, s, st.to_dict(), y, 16, mx.E4M3, 0x3C00, "config 4")
+    # the plain quantize kernel writes the same codes
+    p2, s2 = mx.quantize(x, 16, mx.E4M3)
+    assert torch.equal(p2, p) and torch.equal(s2, s)
 
 
 @pytest.mark.parametrize("layer", [0, 1, 13, 27, 40, 53, 66, 79])
-def test_config5_llama70b_layer(cuda_device, layer):
-    for j in range(len(inputs.LLAMA70B_SHAPES)):
-        x = inputs.workload5_tensor(layer, j, device=cuda_device)
+def test_config5_llama70b_layer_whole(cuda_device, layer):
+    xs = [inputs.workload5_tensor(layer, j, device=cuda_device)
+          for j in range(len(inputs.LLAMA70B_SHAPES))]
+    gh, p, s, st, y = layer_launches(xs, 32, mx.UE5M3)
+    for j, x in enumerate(xs):
         what = f"config 5 layer {layer} tensor {j}"
-        g = int(mx.global_scale(x, mx.UE5M3).item()) & 0xFFFF
-        p, s, st, y = bench_launches(x, 32, mx.UE5M3, g)
-        if layer == 0:
-            assert g == oracle.global_scale(inputs.to_oracle(x), mx.UE5M3), what
-            check_whole(x, p, s, st, y, 32, mx.UE5M3, g, what)
-        else:
-            check_rows(x, p, s, y, 32, mx.UE5M3, g, sample_rows(x.shape[0], 79 * layer + j, k=2),
-                       what)
-            check_properties(x, p, s, st, 32, mx.UE5M3, g, what)
-        del x, p, s, y
-        torch.cuda.empty_cache()
+        assert gh[j] == oracle.global_scale(inputs.to_oracle(x), oracle.UE5M3), what
+        check_whole(x, p[j], s[j], st[j], y[j], 32, mx.UE5M3, gh[j], what)
+    del xs, p, s, y
+    torch.cuda.empty_cache()

@@ -85,3 +85,73 @@ def test_group_rejects_mixed_dtypes(cuda_device):
         mx.quantize_group([a, b], 32, mx.E4M3)
     with pytest.raises(ValueError):
         mx.quantize_group([a] * (mx.MX_MAX_GROUP + 1), 32, mx.E4M3)
+
+
+@pytest.mark.parametrize("block", [4, 16, 32, 256])
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_device_global_scales_drive_the_group(cuda_device, block, fmt, dtype):
+    """mx_global_scale_group writes every tensor's g to device memory; the other grouped calls
+    read it there (no host round trip).  g equals the oracle's rule per tensor (1.0 for the empty
+    tensor), and codes, scales, dequantized bits and error records equal the oracle's with it."""
+    xs = make_group(block, dtype, cuda_device, seed=block * 11 + fmt + 3)
+    xs[1] = xs[1] * 1e-4  # one tensor whose g sits far below 1
+    g = mx.global_scale_group(xs, fmt)
+    p, s = mx.quantize_group(xs, block, fmt, g=g)
+    y = mx.dequantize_group(p, s, block, fmt, g=g, out_dtype=dtype)
+    p2, s2, st = mx.quantize_with_stats_group(xs, block, fmt, g=g)
+    gh = g.cpu().numpy().view(np.uint16)
+    for k, x in enumerate(xs):
+        gk = oracle.global_scale(inputs.to_oracle(x), fmt)
+        what = f"device g N={block} fmt={fmt} {dtype} tensor {k} {tuple(x.shape)}"
+        assert int(gh[k]) == gk, (what, hex(int(gh[k])), hex(gk))
+        po, so, yo, sto = oracle_tensor(x, block, fmt, gk)
+        assert_same(u8(s[k]), so, what + " scales")
+        assert_same(u8(p[k]), po, what + " packed")
+        assert_same(u8(s2[k]), so, what + " fused scales")
+        assert_same(u8(p2[k]), po, what + " fused packed")
+        ref = yo if dtype == torch.bfloat16 else yo.view(np.uint32)
+        assert_same(bits(y[k]), ref, what + " dequant")
+        assert_stats(st[k].to_dict(), sto, what + " stats")
+
+
+def test_device_global_scales_in_a_graph(cuda_device):
+    """The chain global scale -> fused pass -> dequantize captured in a CUDA graph and replayed on
+    new inputs: the replay reads the g its own first launch wrote."""
+    xs = [inputs.workload5_tensor(0, j, device=cuda_device, shape=(256, 1024)) for j in range(3)]
+    g = torch.empty(3, dtype=torch.int16, device=cuda_device)
+    p = [torch.empty(256, 512, dtype=torch.uint8, device=cuda_device) for _ in xs]
+    s = [torch.empty(256, 32, dtype=torch.uint8, device=cuda_device) for _ in xs]
+    y = [torch.empty(256, 1024, dtype=torch.bfloat16, device=cuda_device) for _ in xs]
+    out = torch.empty(3, 64, dtype=torch.uint8, device=cuda_device)
+    ws = mx.stats_workspace(cuda_device)
+
+    def chain():
+        mx.global_scale_group(xs, "ue5m3", out=g)
+        mx.quantize_with_stats_group(xs, 32, "ue5m3", g=g, packed=p, scales=s, out=out,
+                                     workspace=ws)
+        mx.dequantize_group(p, s, 32, "ue5m3", g=g, out=y)
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        chain()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            chain()
+    stream.synchronize()
+    for scale in (1.0, 37.0):
+        for x in xs:
+            x.mul_(scale)
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        for k, x in enumerate(xs):
+            gk = oracle.global_scale(inputs.to_oracle(x), oracle.UE5M3)
+            po, so, yo, sto = oracle_tensor(x, 32, oracle.UE5M3, gk)
+            assert_same(u8(p[k]), po, f"graph x{scale} tensor {k} packed")
+            assert_same(u8(s[k]), so, f"graph x{scale} tensor {k} scales")
+            assert_same(bits(y[k]), yo, f"graph x{scale} tensor {k} dequant")
+            assert_stats(mx.ErrorStats(out[k]).to_dict(), sto, f"graph x{scale} tensor {k}")
+    del graph

@@ -12,21 +12,25 @@ Gaussian data), built on the host and copied to the device; the oracle multiplie
   bound k * 2^-23 * sum |a b| (twice the round-to-nearest bound, allowing truncating adders), plus
   one rounding of the final scaling by gA gB (2^-24 |c|) and, for bfloat16 output, 2^-8 |c|.
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
 
 import fp4_microscaling_tensor_b200 as mx
 import oracle
-from fp4_microscaling_tensor_b200 import inputs
+from fp4_microscaling_tensor_b200 import _lib, inputs
+from fp4_microscaling_tensor_b200 import api as mx_api
 
 pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(params=["one_cta", "cta_pairs"], autouse=True)
 def kernel(request, monkeypatch):
-    """Every test runs with both kernels (the CTA-pair kernel is used for m > 128)."""
-    monkeypatch.setenv("MXFP4_MATMUL_PAIRS", "1" if request.param == "cta_pairs" else "0")
+    """Every test runs with both kernels: mx_matmul and mx_matmul_pair (CTA pairs for m > 128)."""
+    monkeypatch.setattr(mx, "matmul", functools.partial(mx_api.matmul,
+                                                        cta_pairs=request.param == "cta_pairs"))
     return request.param
 
 ONE = 0x38  # E4M3 code of 1.0
@@ -186,3 +190,21 @@ def test_prepared_scale_layout(rows, k):
                                                  16 * kt + 4 * j: 16 * kt + 4 * j + 4]
     assert got.size == ref.size
     assert np.array_equal(got, ref.reshape(-1))
+
+
+def test_abandoned_launch_leaves_later_launches_alone():
+    """A launch marked as abandoned (as a thread block whose bounded waits ran out marks it) must
+    not make a later launch stop waiting.  One long tile (k = 2^18: each CTA waits for its whole
+    main loop, far beyond the polls after which an abandoned launch's waits give up) is run, its
+    launch marked, then run again: the result is the same bit for bit and nothing gave up."""
+    rng = np.random.default_rng(11)
+    m, n, k = 256, 256, 1 << 18
+    pa, pb = codes(rng, m, k), codes(rng, n, k)
+    sa = np.full((m, k // 16), ONE, np.uint8)
+    sb = np.full((n, k // 16), ONE, np.uint8)
+    first = run(pa, sa, pb, sb, m, n, k)
+    assert mx.matmul_gave_up() == 0
+    assert _lib.lib.mx_test_matmul_abandon_last() == _lib.MX_OK
+    second = run(pa, sa, pb, sb, m, n, k)
+    assert mx.matmul_gave_up() == 0
+    assert np.array_equal(first, second)

@@ -35,7 +35,7 @@ def worker(rank, world, port, out):
         # timings: element-wise max over ranks
         got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5 * rank], "cpu")
         # each rank draws its own tensors: checksums differ across ranks
-        x = inputs.normal((64, 256), inputs.SWEEP_SIGMAS[2], bench.rank_seed(2, rank))
+        x = inputs.workload5_tensor(bench.rank_layer(0, rank), 2, shape=(64, 256))
         chk = torch.tensor([float(x.float().sum())], dtype=torch.float64)
         allc = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(allc, chk)
@@ -68,7 +68,7 @@ def test_two_ranks_gloo():
 
 def test_single_process_identity():
     assert bench.max_over_ranks([3.0, 4.0], "cpu") == [3.0, 4.0]
-    assert bench.rank_seed(0, 0) != bench.rank_seed(0, 1)
+    assert bench.rank_layer(0, 0) != bench.rank_layer(0, 1)
 
 
 def shard_worker(rank, world, port, out):

@@ -1,7 +1,9 @@
 """mx_error_stats_noalloc: the error reduction for callers that cannot allocate a workspace (its
 scratch is a fixed array inside the library).  Called through the C ABI and checked against the
-workspace entry point mx_error_stats on two calls in a row, so the second call runs over the
-scratch contents the first one left behind.  Collected last on purpose (file name)."""
+workspace entry point mx_error_stats and against the oracle on two calls in a row, so the second
+call runs over the scratch contents the first one left behind.  Whole-block tensors and ragged ones
+(cols not a multiple of the block, the row-wise path with its own scratch layout) are both run.
+Collected last on purpose (file name)."""
 import ctypes
 import struct
 
@@ -9,7 +11,8 @@ import numpy as np
 import pytest
 import torch
 
-from fp4_microscaling_tensor_b200 import _lib
+import oracle
+from fp4_microscaling_tensor_b200 import _lib, inputs
 import fp4_microscaling_tensor_b200 as mx
 
 pytestmark = pytest.mark.gpu
@@ -44,22 +47,29 @@ def same(got, ref):
 
 
 def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
-    cases = [  # (rows, cols, block, fmt, dtype, scale): the second case is smaller than the first
+    cases = [  # (rows, cols, block, fmt, dtype, scale): later cases are smaller than the first
         (2048, 4096, 32, mx.E4M3, torch.bfloat16, 0.02),
         (37, 20, 4, mx.UE5M3, torch.bfloat16, 1e-3),
         (256, 256, 32, mx.E4M3, torch.float32, 0.02),
+        (33, 100, 32, mx.UE5M3, torch.bfloat16, 0.02),   # ragged: 100 = 3 * 32 + 4
+        (5, 7, 4, mx.E4M3, torch.float32, 0.5),          # ragged: 7 = 4 + 3
     ]
     gen = torch.Generator(device=cuda_device)
     gen.manual_seed(7)
     for rows, cols, block, fmt, dtype, scale in cases:
         x = (torch.randn(rows, cols, generator=gen, device=cuda_device) * scale).to(dtype)
         packed, scales = mx.quantize(x, block, fmt)
+        xo = inputs.to_oracle(x)
+        po, so = oracle.quantize(xo, rows, cols, block, fmt)
         for given in (False, True):
             p, s = (packed, scales) if given else (None, None)
             ref = mx.error_stats(x, block, fmt, packed=p, scales=s).to_dict()
+            orc = oracle.error_stats(xo, rows, cols, block, fmt,
+                                     packed=po if given else None, scales=so if given else None)
             first = noalloc(x, block, fmt, packed=p, scales=s)
             second = noalloc(x, block, fmt, packed=p, scales=s)
             torch.cuda.synchronize()
-            same(first, ref)
-            same(second, ref)
+            for got in (first, second):
+                same(got, ref)
+                same(got, orc)
             assert first == second
