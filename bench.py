@@ -68,7 +68,7 @@ def parse(argv=None):
     # single-kernel timing / profiling case (not the benchmark line)
     ap.add_argument("--case", choices=["quantize", "dequantize", "stats", "stats-recompute",
                                        "quantize-stats", "global-scale", "fake-quantize",
-                                       "matmul"])
+                                       "matmul", "dequant-matmul"])
     ap.add_argument("--mnk", type=int, nargs=3, default=[8192, 8192, 8192],
                     help="m n k of --case matmul")
     ap.add_argument("--shape", type=int, nargs=2, default=[16384, 8192])
@@ -366,7 +366,7 @@ class Llama70B:
         nt = len(self.shapes)
         self.stats = torch.zeros(layers, nt, 64, dtype=torch.uint8, device=device)
         self.g = torch.zeros(layers, nt, dtype=torch.int16, device=device)
-        self.ws_stats = torch.empty(self.lib.mx_error_stats_workspace_size(0, 0),
+        self.ws_stats = torch.empty(self.lib.mx_error_stats_workspace_size(0, 0, BLOCK),
                                     dtype=torch.uint8, device=device)
         self.ws_g = torch.empty(self.lib.mx_global_scale_workspace_size(0, 0), dtype=torch.uint8,
                                 device=device)
@@ -897,6 +897,53 @@ def run_matmul_case(args):
                       "gave_up": mx.matmul_gave_up(), "reps": args.reps}), flush=True)
 
 
+def run_dequant_matmul_case(args):
+    """Time mx_dequant_matmul (C = A dequant(W)^T: bf16 activations m x k, weights n x k stored
+    with --block / --fmt and a global scale, bf16 out) on a seeded weight tensor quantized by the
+    library, L2 flushed before each launch.  Reports TFLOP/s (2 m n k / time) against the measured
+    bf16 tensor peak and the bytes that must cross HBM (codes + scales + A + C) / time."""
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    from fp4_microscaling_tensor_b200 import inputs
+    m, n, k = args.mnk
+    fmt = mx.fmt_code(args.fmt)
+    dev = torch.device("cuda", 0)
+    w = inputs.normal((n, k), 0.015, 7, device=dev)
+    g = int(mx.global_scale(w, fmt).item()) & 0xFFFF
+    pw, sw = mx.quantize(w, args.block, fmt, g)
+    del w
+    a = inputs.normal((m, k), 1.0, 8, device=dev)
+    c = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    fn = lambda: mx.dequant_matmul(a, pw, sw, args.block, fmt, g, out=c)  # noqa: E731
+    fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_peak, kind = float(json.load(f)["bf16_tflops"]), "measured bf16 burst"
+    except Exception:
+        bf16_peak, kind = 1590.0, "fallback bf16"
+    hbm, hkind = measured_peak()
+    tflops = 2.0 * m * n * k / t / 1e12
+    nbytes = n * k * (0.5 + 1.0 / args.block) + 2.0 * m * k + 2.0 * m * n
+    print(json.dumps({"case": "dequant-matmul", "mnk": [m, n, k], "block": args.block,
+                      "fmt": args.fmt, "median_us": t * 1e6, "tflops": tflops,
+                      "tensor_frac": tflops / bf16_peak, "tensor_peak": bf16_peak,
+                      "tensor_peak_kind": kind, "gbs": nbytes / t / 1e9,
+                      "hbm_frac": nbytes / t / 1e9 / hbm, "hbm_peak_kind": hkind,
+                      "gave_up": mx.matmul_gave_up(), "reps": args.reps}), flush=True)
+
+
 def run_case(args):
     """Time one kernel (or, with --group G, one grouped launch over G tensors) on bf16 tensors
     N(0, 0.02^2): CUDA events around each launch, L2 flushed before each launch by writing a 256 MB
@@ -1001,6 +1048,9 @@ def main():
     args = parse()
     if args.case == "matmul":
         run_matmul_case(args)
+        return
+    if args.case == "dequant-matmul":
+        run_dequant_matmul_case(args)
         return
     if args.case:
         run_case(args)

@@ -11,7 +11,7 @@ Using the API raises ImportError when the library is missing: there is no fallba
 import importlib
 
 _API_NAMES = ("E4M3", "MX_MAX_GROUP", "UE5M3", "ErrorStats", "FakeQuantize", "MXError",
-              "dequantize", "dequantize_group", "error_stats", "fake_quantize", "fmt_code",
+              "dequant_matmul", "dequantize", "dequantize_group", "error_stats", "fake_quantize", "fmt_code",
               "g_bits", "global_scale", "global_scale_group", "kernel_launches", "matmul",
               "matmul_gave_up", "prepare_scales", "quantize", "quantize_group",
               "quantize_with_stats", "quantize_with_stats_group", "stats_workspace")

@@ -28,7 +28,8 @@ EXPORTS = ("mx_quantize", "mx_dequantize", "mx_error_stats_workspace_size", "mx_
            "mx_quantize_group", "mx_dequantize_group", "mx_quantize_stats_group",
            "mx_global_scale_group", "mx_error_stats_means",
            "mx_fake_quantize", "mx_matmul_scales_size", "mx_matmul_prepare_scales",
-           "mx_matmul", "mx_matmul_pair", "mx_matmul_gave_up", "mx_test_matmul_abandon_last",
+           "mx_matmul", "mx_matmul_pair", "mx_dequant_matmul", "mx_matmul_gave_up",
+           "mx_test_matmul_abandon_last",
            "mx_test_fail_next_calls", "mx_status_string", "mx_kernel_launches")
 MX_MAX_GROUP = 16
 
@@ -81,6 +82,8 @@ lib.mx_matmul.restype = _i
 lib.mx_matmul.argtypes = [_vp, _vp, _u16, _vp, _vp, _u16, _i64, _i64, _i64, _i, _i, _vp, _i, _vp]
 lib.mx_matmul_pair.restype = _i
 lib.mx_matmul_pair.argtypes = lib.mx_matmul.argtypes
+lib.mx_dequant_matmul.restype = _i
+lib.mx_dequant_matmul.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _i, _i, _u16, _vp, _vp, _i, _vp]
 lib.mx_test_matmul_abandon_last.restype = _i
 lib.mx_test_matmul_abandon_last.argtypes = []
 lib.mx_matmul_scales_size.restype = _sz

@@ -412,6 +412,39 @@ def matmul(a_packed, a_scales, b_packed, b_scales, a_g=None, b_g=None, out_dtype
     return out
 
 
+def dequant_matmul(a, w_packed, w_scales, block=32, fmt="ue5m3", g=None, out_dtype=torch.bfloat16,
+                   out=None, stream=None):
+    """C = a dequant(W)^T on the tensor cores: a [m, k] bfloat16 activations, W an n x k weight
+    tensor as quantize() stores it (w_packed [n, k/2], w_scales [n, k/block]) with any block size,
+    E4M3 or UE5M3 scales and global scale g (a value, or a CUDA tensor of one 16-bit bit pattern
+    read on the device, e.g. from global_scale).  The weights enter as their bf16 dequantization.
+    Returns C [m, n] of out_dtype."""
+    if out_dtype not in _DT:
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if a.dtype != torch.bfloat16 or a.dim() != 2 or w_packed.dim() != 2:
+        raise ValueError("a must be a 2-D bfloat16 tensor and w_packed 2-D")
+    _shape2d(a, "a")
+    _shape2d(w_packed, "w_packed")
+    _shape2d(w_scales, "w_scales")
+    m, k = a.shape
+    n = w_packed.shape[0]
+    if 2 * w_packed.shape[1] != k:
+        raise ValueError("w_packed must hold n x k codes (k / 2 bytes per row)")
+    g_dev = None
+    if isinstance(g, torch.Tensor):
+        if not g.is_cuda or g.numel() < 1 or g.element_size() != 2:
+            raise ValueError("device global scale: a CUDA tensor of 16-bit values")
+        g_dev, gb = g.data_ptr(), 0
+    else:
+        gb = g_bits(g)
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=a.device)
+    check(lib.mx_dequant_matmul(a.data_ptr(), m, k, w_packed.data_ptr(), w_scales.data_ptr(), n,
+                                int(block), fmt_code(fmt), gb, g_dev, out.data_ptr(),
+                                _DT[out.dtype], _stream(stream, a.device)), "mx_dequant_matmul")
+    return out
+
+
 def matmul_gave_up():
     """Number of matmul thread blocks whose bounded waits ran out since the last call (0 normally);
     synchronizes the device."""

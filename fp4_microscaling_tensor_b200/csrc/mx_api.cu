@@ -286,6 +286,30 @@ mx_status mx_matmul_pair(const uint8_t* a_packed, const uint8_t* a_scales, uint1
                      true, stream);
 }
 
+mx_status mx_dequant_matmul(const void* a, int64_t m, int64_t k, const uint8_t* w_packed,
+                            const uint8_t* w_scales, int64_t n, int block, mx_scale_fmt fmt,
+                            uint16_t w_global_scale_fp16, const uint16_t* w_global_scale_dev,
+                            void* c, mx_dtype ct, cudaStream_t stream) {
+  if (!valid_fmt(fmt) || !valid_dtype(ct)) return MX_ERR_INVALID_ARG;
+  if (!w_global_scale_dev && !valid_g(w_global_scale_fp16)) return MX_ERR_INVALID_ARG;
+  if (m < 0 || n < 0 || k < 0 || m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) ||
+      k >= (int64_t(1) << 31))
+    return MX_ERR_INVALID_ARG;
+  if (!valid_block(block) || k == 0 || k % 64 != 0 || k % block != 0) return MX_ERR_UNSUPPORTED;
+  if (m == 0 || n == 0) return MX_OK;
+  if (!a || !w_packed || !w_scales || !c) return MX_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w_packed) || !aligned16(w_scales) || !aligned16(c) ||
+      (reinterpret_cast<uintptr_t>(w_global_scale_dev) & 1u) != 0)
+    return MX_ERR_MISALIGNED;
+  if (injected_failure()) return MX_ERR_CUDA;
+  int launches = 0;
+  const cudaError_t e = mxk::run_dequant_matmul(a, m, k, w_packed, w_scales, n, block, (int)fmt,
+                                                w_global_scale_fp16, w_global_scale_dev, c,
+                                                ct == MX_BF16, stream, &launches);
+  g_launches += launches;
+  return from_cuda(e);
+}
+
 size_t mx_matmul_scales_size(int64_t rows, int64_t k) {
   if (rows < 0 || rows >= (int64_t(1) << 31) || k <= 0 || k % 256 != 0 || k > (int64_t(1) << 40))
     return 0;

@@ -298,27 +298,47 @@ __device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t 
         "r"(lo), "r"(hi), "r"(w));
 }
 
+// |x| s for the two bf16 halves of aw, s a power of two given as its bf16 bit pattern sc16: two
+// mixed-precision FMAs (bf16 operands, fp32 result) take the halves straight from the word, so the
+// word needs no split into two fp32 values first.  Exact (a power-of-two scaling of a bf16 value).
+__device__ __forceinline__ float2 mag_scaled2(uint32_t aw, uint32_t sc16) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h, s;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.u16.u32 s, %3;\n\t"
+      "fma.rn.f32.bf16 %0, l, s, 0f00000000;\n\t"
+      "fma.rn.f32.bf16 %1, h, s, 0f00000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(aw), "r"(sc16));
+  return make_float2(lo, hi);
+}
+
 // One code word's eight elements (words w[0..3]) with recomputed codes, quantized and reduced in
-// one go.  The quotients are taken of the magnitudes (x r + 48 - 48 rounds |x| r exactly onto the
-// 2^-18 grid, see snap_quotient2; a magnitude needs no sign fix for zero), so the E2M1 conversion
-// gives magnitude codes whose decode is one shift and one mask; x's sign bits are put into the
-// codes afterwards (byte permutes that replicate each half's sign, two masked ORs).  Errors use the
-// magnitudes too: (|x| s - |q| S g s)^2 is the element's scaled square.  Per pair k the block
-// constants are those of block k / PB (PB = pairs per block inside the word: 2 for N = 4, else 4);
-// lt2[k / PB] collects the squares, nsat2 the clipped elements (|x| > RD_bf16(6 S g) = S2).
+// one go.  The scaled magnitudes xs = |x| s (s = 2^k, the slice scaling) come straight from the
+// bf16 words (mag_scaled2).  The quotients are taken of them with the rescaled reciprocal
+// r / s (x r = xs (r / s) exactly: s is a power of two), rounded onto the 2^-18 grid by adding and
+// subtracting 48 (see snap_quotient2; a magnitude needs no sign fix for zero), so the E2M1
+// conversion gives magnitude codes whose decode is one shift and one mask; x's sign bits are put
+// into the codes afterwards (byte permutes that replicate each half's sign, two masked ORs).
+// Errors use the magnitudes too: (xs - |q| S g s)^2 is the element's scaled square.  Per pair k
+// the block constants are those of block k / PB (PB = pairs per block inside the word: 2 for
+// N = 4, else 4); lt2[k / PB] collects the squares, nsat2 the clipped elements
+// (|x| > RD_bf16(6 S g) = S2).
 template <int PB>
 __device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, const float* nDq,
                                               const uint32_t* S2, float sc, float2* lt2,
                                               uint32_t& nsat2) {
   uint32_t aw[4];
-  float2 xa[4];
+  float2 xs[4];
   float q[8];
+  const uint32_t sc16 = __float_as_uint(sc) >> 16;  // a power of two: exact as a bf16
+  const float isc = __frcp_rn(sc);                   // exact (a power of two)
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     aw[k] = w[k] & 0x7FFF7FFFu;
-    xa[k] = make_float2(__uint_as_float(aw[k] << 16), __uint_as_float(aw[k] & 0xFFFF0000u));
-    const float rk = r[k / PB];
-    const float2 y = __ffma2_rn(xa[k], make_float2(rk, rk), make_float2(48.0f, 48.0f));
+    xs[k] = mag_scaled2(aw[k], sc16);
+    const float rk = __fmul_rn(r[k / PB], isc);
+    const float2 y = __ffma2_rn(xs[k], make_float2(rk, rk), make_float2(48.0f, 48.0f));
     const float2 qq = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
     q[2 * k] = qq.x;
     q[2 * k + 1] = qq.y;
@@ -330,9 +350,8 @@ __device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, 
     const uint32_t blo = (k < 3 ? cm << (22 - 8 * k) : cm >> 2) & 0x01C00000u;
     const uint32_t bhi = (k < 3 ? cm << (18 - 8 * k) : cm >> 6) & 0x01C00000u;
     const float nd = nDq[k / PB];
-    const float2 xs = __fmul2_rn(xa[k], make_float2(sc, sc));
     const float2 d = __ffma2_rn(make_float2(__uint_as_float(blo), __uint_as_float(bhi)),
-                                make_float2(nd, nd), xs);
+                                make_float2(nd, nd), xs[k]);
     lt2[k / PB] = __ffma2_rn(d, d, lt2[k / PB]);
     uint32_t m;
     asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(aw[k]), "r"(S2[k / PB]));

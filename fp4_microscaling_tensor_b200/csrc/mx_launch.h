@@ -194,6 +194,13 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
                              const uint8_t* b_packed, const uint8_t* b_scales, int64_t m,
                              int64_t n, int64_t k, float alpha, void* c, bool c_bf16,
                              bool cta_pairs, cudaStream_t stream, int* launches);
+// C (m x n, fp32 or bf16) = A dequant(W)^T for bf16 activations A (m x k) and weights W (n x k)
+// stored by the quantizer with blocks of `block` along k, E4M3 or UE5M3 scales and global scale g
+// (g_bits, or read from g_dev when that is set); k a positive multiple of 64 and of block.
+cudaError_t run_dequant_matmul(const void* a, int64_t m, int64_t k, const uint8_t* w_packed,
+                               const uint8_t* w_scales, int64_t n, int block, int fmt,
+                               uint16_t g_bits, const uint16_t* g_dev, void* c, bool c_bf16,
+                               cudaStream_t stream, int* launches);
 // Bytes of an operand's scales in tensor-core order, and the reordering kernel.
 int64_t mma_scales_bytes(int64_t rows, int64_t k);
 cudaError_t run_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t k, uint8_t* out,

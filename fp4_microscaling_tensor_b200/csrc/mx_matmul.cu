@@ -684,6 +684,320 @@ bool make_rows_map(CUtensorMap* map, const uint8_t* scales, int64_t rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// ------------------------------------------------------------------------------------------------
+// bf16 activations x stored FP4 weights: C = A dequant(W)^T (the inference step of the 4-bit float
+// quantization article, gtnt.cn/news/16247, §3.1: the stored weights are dequantized to the
+// activations' type, then multiplied).  W is n x k as mx_quantize stores it, with any block size
+// N, E4M3 or UE5M3 scales ([MX] §3.1 item 1) and an FP16 global scale; the tensor core has no
+// block-scaled form for UE5M3 or for most of these N, so each CTA dequantizes its tile of W into
+// shared memory itself -- RN_bf16(E2M1 * S * g), the values mx_dequantize writes as bf16 -- and
+// multiplies bf16 x bf16 with tcgen05.mma kind::f16 (fp32 accumulator in TMEM).  Nothing is
+// dequantized to global memory: per element of W the kernel reads 1/2 + 1/N bytes.
+//
+// One CTA per 256 x 256 tile of C (two 128-row accumulators side by side in TMEM, 512 columns),
+// 10 warps:
+//   * warp 0, one thread: per 64-element step of k, TMA loads of the step's two 128 x 64 tiles of
+//     A (128-byte swizzle), completing on the stage's A barrier;
+//   * warps 2..9 (256 threads, one row of the W tile each): load the step's 32 code bytes and
+//     64 / N scale bytes of their row one step ahead, decode the codes (E2M1x2 -> f16x2), multiply
+//     by the block's S g (exact in fp32), round to bf16 and write the 128-byte row into the
+//     stage's W tile in the same 128-byte-swizzled K-major layout the TMA writes for A; then a
+//     proxy fence and one arrival per warp on the stage's W barrier;
+//   * warp 1, one thread: waits for both barriers, issues 4 (or 8) tcgen05.mma of 128 x 256 x 16,
+//     commits to the stage's empty barrier;
+//   * warps 2..9 then read the accumulators back (tcgen05.ld; warp w serves TMEM lanes 32 (w % 4)
+//     of accumulator (w - 2) / 4) and store C.
+// Every wait is bounded, as in the kernels above.
+// ------------------------------------------------------------------------------------------------
+namespace dqmm {
+constexpr int kBN = 256;                      // columns of C per CTA (MMA N)
+constexpr int kBK = 64;                       // k elements per stage
+constexpr int kStages = 3;
+constexpr int kATile = 128 * 128;             // one 128-row half of A: 128 x 64 bf16
+constexpr int kABytes = 2 * kATile;
+constexpr int kBBytes = kBN * 128;            // the W tile: 256 x 64 bf16
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 320;
+constexpr int kDqWarps = 8;
+constexpr int kSmemBytes = kStages * kStageBytes + 256 * 4 + 256 + 1024;
+constexpr uint32_t kTmemCols = 512;
+// Instruction descriptor of kind::f16: fp32 accumulator (bits 4..5 = 1), A and B bf16 (bits 7..9
+// and 10..12 = 1), both K-major, N = 256 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16).
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(128 >> 4) << 24);
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+}  // namespace dqmm
+
+struct DqArgs {
+  const uint8_t* w_packed;
+  const uint8_t* w_scales;
+  const uint16_t* g_dev;  // when set, the global scale is read here (device)
+  void* c;
+  int64_t m, n, k;
+  uint32_t g_bits;
+  int c_bf16;
+  unsigned int gen;
+};
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_shared16(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// The scale bytes of one 64-element step of a row, packed little-endian (64 / N of them for
+// N <= 64, the one covering the step otherwise).
+template <int N>
+struct StepScales {
+  static constexpr int kBytes = N >= 64 ? 1 : 64 / N;
+  uint32_t v[kBytes > 4 ? kBytes / 4 : 1];
+};
+
+template <int N>
+__device__ __forceinline__ void load_step(const uint8_t* wrow, const uint8_t* srow, int kt,
+                                          bool ok, uint4& c0, uint4& c1, StepScales<N>& sc) {
+  c0 = c1 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < (int)(sizeof(sc.v) / 4); ++i) sc.v[i] = 0;
+  if (!ok) return;
+  c0 = ld_stream16(wrow + 32 * (int64_t)kt);
+  c1 = ld_stream16(wrow + 32 * (int64_t)kt + 16);
+  if constexpr (N == 4) {
+    const uint4 t = __ldg(reinterpret_cast<const uint4*>(srow + 16 * (int64_t)kt));
+    sc.v[0] = t.x; sc.v[1] = t.y; sc.v[2] = t.z; sc.v[3] = t.w;
+  } else if constexpr (N == 8) {
+    const uint2 t = __ldg(reinterpret_cast<const uint2*>(srow + 8 * (int64_t)kt));
+    sc.v[0] = t.x; sc.v[1] = t.y;
+  } else if constexpr (N == 16) {
+    sc.v[0] = __ldg(reinterpret_cast<const unsigned int*>(srow + 4 * (int64_t)kt));
+  } else if constexpr (N == 32) {
+    sc.v[0] = __ldg(reinterpret_cast<const unsigned short*>(srow + 2 * (int64_t)kt));
+  } else {
+    sc.v[0] = __ldg(srow + (64 * (int64_t)kt) / N);
+  }
+}
+
+// Scale byte of block b inside the step (b < 64 / N; 0 for N >= 64).
+template <int N>
+__device__ __forceinline__ uint32_t step_scale(const StepScales<N>& sc, int b) {
+  if constexpr (N >= 64) return sc.v[0] & 0xFFu;
+  else return (sc.v[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+}
+
+// One code word (elements 8 w .. 8 w + 7 of the step) -> 8 bf16 = one 16-byte chunk of the row.
+template <int N>
+__device__ __forceinline__ void dq_word(uint32_t cw, int w, const StepScales<N>& sc,
+                                        const float* s_D, uint32_t (&out)[4]) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(cw));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 8 * w + 2 * i;  // element index in the step
+    const float D = s_D[step_scale<N>(sc, N >= 64 ? 0 : e / N)];
+    const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    const float2 y = __fmul2_rn(v, make_float2(D, D));  // exact
+    out[i] = pack_bf16x2(y.x, y.y);                    // round to nearest even
+  }
+}
+
+template <int N, int FMT>
+__global__ void __launch_bounds__(dqmm::kThreads, 1)
+    k_dequant_matmul(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ DqArgs args) {
+  using namespace dqmm;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* s_D = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(s_D + 256);
+  uint64_t* b_full = a_full + kStages;
+  uint64_t* empty = b_full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* gave_up = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.y * 256, n0 = (int64_t)blockIdx.x * kBN;
+  const bool two = m0 + 128 < args.m;  // the second 128-row half has rows
+  const int KT = (int)(args.k / dqmm::kBK);
+  const uint16_t gb = args.g_dev ? __ldg(args.g_dev) : (uint16_t)args.g_bits;
+  const float g = fp16_bits_to_float(gb);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(a_full + s), 1);
+      mbar_init(smem_u32(b_full + s), kDqWarps);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *gave_up = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- A producer (one thread) ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (*gave_up ||
+            (kt >= kStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s),
+                                                           ((kt / kStages) + 1) & 1, args.gen))) {
+          *gave_up = 1;
+          break;
+        }
+        const uint32_t st = smem_u32(smem + s * kStageBytes), bar = smem_u32(a_full + s);
+        mbar_expect_tx(bar, two ? 2 * kATile : kATile);  // OOB rows included
+        tma_load_2d(st, &tma_a, kt * dqmm::kBK, (int)m0, bar);
+        if (two) tma_load_2d(st + kATile, &tma_a, kt * dqmm::kBK, (int)(m0 + 128), bar);
+        issued = kt + 1;
+      }
+      if (*gave_up) {
+        for (int kt = issued - kStages < 0 ? 0 : issued - kStages; kt < issued; ++kt)
+          mbar_wait<100>(smem_u32(a_full + kt % kStages), (kt / kStages) & 1, args.gen);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        if (!mbar_wait(smem_u32(a_full + s), (kt / kStages) & 1, args.gen) ||
+            !mbar_wait(smem_u32(b_full + s), (kt / kStages) & 1, args.gen)) {
+          *gave_up = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes), wt = st + kABytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t bdesc = desc_sw128(wt + 32 * j);
+          tc_mma_f16(tmem, desc_sw128(st + 32 * j), bdesc, kIdesc, (kt | j) != 0);
+          if (two) tc_mma_f16(tmem + 256, desc_sw128(st + kATile + 32 * j), bdesc, kIdesc,
+                              (kt | j) != 0);
+        }
+        tc_commit(smem_u32(empty + s));
+      }
+      tc_commit(smem_u32(done));  // also after giving up: the epilogue waits for issued MMAs
+    }
+    __syncwarp();
+  } else {
+    // ---------------- W dequantization (warps 2..9, one row of the tile per thread) ----------
+    const int d = threadIdx.x - 64;
+    const int64_t row = n0 + d;
+    const bool row_ok = row < args.n;
+    const uint8_t* wrow = args.w_packed + (row_ok ? row : 0) * (args.k / 2);
+    const uint8_t* srow = args.w_scales + (row_ok ? row : 0) * (args.k / N);
+    const uint32_t r8 = (uint32_t)(d & 7);
+    const uint32_t row_off = (uint32_t)(d >> 3) * 1024u + r8 * 128u;
+    uint4 c0, c1;
+    StepScales<N> sc;
+    load_step<N>(wrow, srow, 0, row_ok, c0, c1, sc);
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % kStages;
+      uint4 n0c, n1c;
+      StepScales<N> nsc;
+      load_step<N>(wrow, srow, kt + 1, row_ok && kt + 1 < KT, n0c, n1c, nsc);
+      bool ok = !*gave_up;
+      if (ok && kt >= kStages && lane == 0)
+        ok = mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1, args.gen);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        *gave_up = 1;
+        break;
+      }
+      const uint32_t base = smem_u32(smem + s * kStageBytes + kABytes) + row_off;
+      const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        uint32_t o[4];
+        dq_word<N>(cw[w], w, sc, s_D, o);
+        st_shared16(base + (((uint32_t)w ^ r8) << 4), o[0], o[1], o[2], o[3]);
+      }
+      // the tensor core reads this tile through the async proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(b_full + s));
+      c0 = n0c;
+      c1 = n1c;
+      sc = nsc;
+    }
+  }
+
+  // ---------------- epilogue: warps 2..9 ----------------
+  if (warp >= 2) {
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    bool ok = true;
+    if (lane == 0) {
+      ok = mbar_wait<200>(smem_u32(done), 0, args.gen);
+      if (!ok) *gave_up = 1;
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    tc_fence_after();
+    if (__all_sync(0xffffffffu, ok && !*gave_up) && (h == 0 || two)) {
+      MmArgs ea{nullptr, nullptr, args.c, args.m, args.n, args.k, 1.0f, args.c_bf16, args.gen};
+      store_rows<kBN>(tmem + (uint32_t)(256 * h), q, lane, m0 + 128 * h, n0, ea);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *gave_up) {
+    atomicAdd(&g_mm_gave_up, 1u);
+    g_mm_abandon_gen = args.gen;
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// Map of the bf16 activations: m x k, row pitch 2 k bytes, boxes of 128 rows x 64 elements loaded
+// with the 128-byte swizzle; rows past the end read as zero.
+bool make_bf16_map(CUtensorMap* map, const void* a, int64_t m, int64_t k) {
+  const EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
+  const cuuint64_t strides[1] = {(cuuint64_t)(2 * k)};
+  const cuuint32_t box[2] = {(cuuint32_t)dqmm::kBK, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 }  // namespace
 
 int64_t mma_scales_bytes(int64_t rows, int64_t k);
@@ -745,6 +1059,43 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
   }
   ++*launches;
   return cudaGetLastError();
+}
+
+template <int N, int FMT>
+static cudaError_t launch_dqmm(const CUtensorMap& ma, const DqArgs& args, cudaStream_t stream) {
+  static std::atomic<bool> attr[kMaxDevices];
+  const cudaError_t e = allow_smem(attr, k_dequant_matmul<N, FMT>, dqmm::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((args.n + dqmm::kBN - 1) / dqmm::kBN), (unsigned)((args.m + 255) / 256));
+  k_dequant_matmul<N, FMT><<<grid, dqmm::kThreads, dqmm::kSmemBytes, stream>>>(ma, args);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t dqmm_block(int block, const CUtensorMap& ma, const DqArgs& args,
+                              cudaStream_t st) {
+  switch (block) {
+    case 4: return launch_dqmm<4, FMT>(ma, args, st);
+    case 8: return launch_dqmm<8, FMT>(ma, args, st);
+    case 16: return launch_dqmm<16, FMT>(ma, args, st);
+    case 32: return launch_dqmm<32, FMT>(ma, args, st);
+    case 64: return launch_dqmm<64, FMT>(ma, args, st);
+    case 128: return launch_dqmm<128, FMT>(ma, args, st);
+    default: return launch_dqmm<256, FMT>(ma, args, st);
+  }
+}
+
+cudaError_t run_dequant_matmul(const void* a, int64_t m, int64_t k, const uint8_t* w_packed,
+                               const uint8_t* w_scales, int64_t n, int block, int fmt,
+                               uint16_t g_bits, const uint16_t* g_dev, void* c, bool c_bf16,
+                               cudaStream_t stream, int* launches) {
+  CUtensorMap ma;
+  if (!make_bf16_map(&ma, a, m, k)) return cudaErrorInvalidValue;
+  const DqArgs args{w_packed, w_scales, g_dev, c, m, n, k, g_bits, c_bf16 ? 1 : 0, next_gen()};
+  const cudaError_t e = fmt == kUE5M3 ? dqmm_block<kUE5M3>(block, ma, args, stream)
+                                      : dqmm_block<kE4M3>(block, ma, args, stream);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 int64_t mma_scales_bytes(int64_t rows, int64_t k) {

@@ -281,6 +281,30 @@ MX_API mx_status mx_matmul_pair(const uint8_t* a_packed, const uint8_t* a_scales
                                 int64_t m, int64_t n, int64_t k, int block, mx_scale_fmt fmt,
                                 void* c, mx_dtype ct, cudaStream_t stream);
 
+/* bf16 activations times stored FP4 weights on the tensor cores: the inference step of the 4-bit
+ * float quantization article (gtnt.cn/news/16247, §3.1, dequantize the stored weights, then
+ * multiply), for weights in any of this library's formats ([MX] §3.1 items 1-3: blocks of
+ * 4..256, E4M3 or UE5M3 scales, FP16 global scale):
+ *   C[i][j] = sum_t A[i][t] * Wq[j][t],  Wq = RN_bf16(E2M1 * S * g), the values mx_dequantize
+ *   writes as bf16,
+ * accumulated in float32 by the tensor core (order unspecified; every product is exact).  Each
+ * weight tile is dequantized into shared memory inside the kernel, nothing to global memory.
+ *   a        m x k bf16, row-major (device).
+ *   w_packed, w_scales  n x k weights exactly as mx_quantize stores them with this block / fmt
+ *            (n*k/2 code bytes, n*k/block scale bytes).
+ *   w_global_scale_fp16 / w_global_scale_dev  g as a bit pattern, or (dev non-NULL, 2-byte
+ *            aligned) read from device memory when the kernel runs (e.g. mx_global_scale output).
+ *   c        OUT m x n, row-major, float32 (ct = MX_F32) or bfloat16 rounded to nearest even.
+ * Errors: k not a positive multiple of 64 and of block, or block not one of 4..256:
+ * MX_ERR_UNSUPPORTED; m, n or k negative or >= 2^31, bad fmt / ct / g: MX_ERR_INVALID_ARG;
+ * m == 0 or n == 0: nothing is enqueued.  Kernel: one CTA per 256 x 256 tile of C, tcgen05.mma
+ * kind::f16; its waits are bounded and counted by mx_matmul_gave_up like mx_matmul's. */
+MX_API mx_status mx_dequant_matmul(const void* a, int64_t m, int64_t k, const uint8_t* w_packed,
+                                   const uint8_t* w_scales, int64_t n, int block,
+                                   mx_scale_fmt fmt, uint16_t w_global_scale_fp16,
+                                   const uint16_t* w_global_scale_dev, void* c, mx_dtype ct,
+                                   cudaStream_t stream);
+
 /* Number of mx_matmul thread blocks that stopped waiting since the previous call (0 in normal
  * operation), written to *count (host memory); clears the count.  Synchronizes the device. */
 MX_API mx_status mx_matmul_gave_up(unsigned int* count);

@@ -7,5 +7,5 @@ and readings) and shares nothing with the CUDA library.
 from .oracle import (  # noqa: F401
     F32, BF16, E4M3, UE5M3, Stats, lib, e2m1_value, e4m3_value, ue5m3_value, scale_value,
     fp16_value, round_scale, round_e2m1_mag, scale_max, scale_min, quantize, dequantize,
-    error_stats, global_scale, matmul,
+    error_stats, global_scale, matmul, bf16_values, dequant_matmul,
 )

@@ -144,3 +144,27 @@ def matmul(a_packed, a_scales, a_g_bits, b_packed, b_scales, b_g_bits, m, n, k, 
     B = yb.astype(np.float64).reshape(n, k)
     return A @ B.T
 
+
+
+def bf16_values(bits):
+    """float64 values of bf16 bit patterns: a bf16 value is the float32 whose upper 16 bits are
+    the pattern and whose lower 16 bits are zero."""
+    bits = np.ascontiguousarray(bits, np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def dequant_matmul(a_bits, m, k, w_packed, w_scales, n, block, fmt, w_g_bits=0x3C00):
+    """C = A dequant(W)^T in float64 (m x n): A an m x k bf16 tensor (uint16 bit patterns), W an
+    n x k tensor stored by the quantizer.
+
+    The 4-bit float quantization article (gtnt.cn/news/16247, §3.1) runs inference by dequantizing
+    the stored weights to the activations' type and multiplying.  Here the weights' values are
+    their bf16 dequantization (round to nearest even of E2M1 x S x g, what dequantize() returns
+    with out_bf16=True), the activations their exact bf16 values, and the product is one float64
+    matrix multiply, whose rounding (at most k 2^-53 relative to sum |a w|) is far below any
+    float32 accumulation.
+    """
+    A = bf16_values(a_bits).reshape(m, k)
+    yw = dequantize(w_packed, w_scales, n, k, block, fmt, w_g_bits, out_bf16=True)
+    W = bf16_values(yw).reshape(n, k)
+    return A @ W.T

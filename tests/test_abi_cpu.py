@@ -261,6 +261,37 @@ def test_matmul_rejects_bad_arguments():
     assert L.mx_matmul_pair(*args) == UNS
 
 
+def test_dequant_matmul_rejects_bad_arguments():
+    def dm(a=A, m=128, k=256, pw=A, sw=A, n=64, block=32, fmt=UE, g=0x3C00, gdev=None, c=A,
+           ct=BF16):
+        return L.mx_dequant_matmul(a, m, k, pw, sw, n, block, fmt, g, gdev, c, ct, None)
+    assert dm(k=96) == UNS                       # k not a multiple of 64
+    assert dm(k=128, block=256) == UNS           # k not a multiple of the block
+    assert dm(block=12) == UNS
+    assert dm(k=0) == UNS
+    assert dm(fmt=3) == INV
+    assert dm(ct=9) == INV
+    assert dm(g=0x7C00) == INV                   # g must be finite and positive ...
+    L.mx_test_fail_next_calls(1)
+    assert dm(g=0, gdev=A + 2) == _lib.MX_ERR_CUDA   # ... unless read from device memory
+    assert dm(g=0, gdev=A + 1) == MIS
+    assert dm(m=-1) == INV
+    assert dm(n=1 << 31) == INV
+    assert dm(k=1 << 31) == INV
+    assert dm(a=None) == INV
+    assert dm(sw=None) == INV
+    assert dm(c=None) == INV
+    assert dm(a=A + 8) == MIS
+    assert dm(pw=A + 4) == MIS
+    assert dm(c=A + 2) == MIS
+    assert dm(m=0, a=None, c=None) == OK       # empty product: nothing to do
+    assert dm(n=0) == OK
+    for blk in (4, 8, 16, 32, 64, 128, 256):     # every block size is accepted
+        L.mx_test_fail_next_calls(1)
+        assert dm(k=512, block=blk) == _lib.MX_ERR_CUDA
+    assert L.mx_test_fail_next_calls(0) == 0
+
+
 def test_matmul_scale_preparation_arguments():
     assert L.mx_matmul_scales_size(128, 256) == 256 * 16        # rows padded to 256
     assert L.mx_matmul_scales_size(300, 512) == 512 * 32
