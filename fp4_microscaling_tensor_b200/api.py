@@ -291,10 +291,11 @@ def quantize_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None, s
         rows, cols = _shape2d(x, "x")
         lead = tuple(x.shape[:-1])
         if packed[k] is None:
-            packed[k] = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
-        if scales[k] is None:
-            scales[k] = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+            packed[k] = torch.empty(lead + ((cols + 1) // 2,), dtype=torch.uint8,
                                     device=x.device)
+        if scales[k] is None:
+            scales[k] = torch.empty(lead + (-(-cols // block) if block else 0,),
+                                    dtype=torch.uint8, device=x.device)
         desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
         desc[k].rows, desc[k].cols = rows, cols
@@ -305,8 +306,10 @@ def quantize_group(xs, block=32, fmt="e4m3", g=None, packed=None, scales=None, s
 
 
 def dequantize_group(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=torch.bfloat16,
-                     out=None, stream=None):
-    """dequantize() of every (packed, scales) pair in one launch.  Returns the list of outputs."""
+                     out=None, stream=None, cols=None):
+    """dequantize() of every (packed, scales) pair in one launch.  cols: the row length of each
+    tensor (default 2 * packed.shape[-1]; give it for rows of odd length).  Returns the list of
+    outputs."""
     packed, scales = list(packed), list(scales)
     n = len(packed)
     if len(scales) != n:
@@ -316,15 +319,19 @@ def dequantize_group(packed, scales, block=32, fmt="e4m3", g=None, out_dtype=tor
     desc = _group(n, "dequantize_group")
     gs = _gs(g, n)
     out = list(out) if out is not None else [None] * n
+    cols = list(cols) if cols is not None else [None] * n
     for k in range(n):
         prow, pcols = _shape2d(packed[k], "packed")
         _shape2d(scales[k], "scales")
+        ck = 2 * pcols if cols[k] is None else int(cols[k])
+        if (ck + 1) // 2 != pcols:
+            raise ValueError("cols does not match packed.shape[-1]")
         if out[k] is None:
-            out[k] = torch.empty(tuple(packed[k].shape[:-1]) + (2 * pcols,), dtype=out_dtype,
+            out[k] = torch.empty(tuple(packed[k].shape[:-1]) + (ck,), dtype=out_dtype,
                                  device=packed[k].device)
         desc[k].y, desc[k].packed, desc[k].scales = (out[k].data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
-        desc[k].rows, desc[k].cols = prow, 2 * pcols
+        desc[k].rows, desc[k].cols = prow, ck
         _set_g(desc[k], gs, k)
     check(lib.mx_dequantize_group(desc, n, int(block), fmt_code(fmt), _DT[out_dtype],
                                   _stream(stream, packed[0].device)), "mx_dequantize_group")
@@ -354,10 +361,11 @@ def quantize_with_stats_group(xs, block=32, fmt="e4m3", g=None, packed=None, sca
         rows, cols = _shape2d(x, "x")
         lead = tuple(x.shape[:-1])
         if packed[k] is None:
-            packed[k] = torch.empty(lead + (cols // 2,), dtype=torch.uint8, device=x.device)
-        if scales[k] is None:
-            scales[k] = torch.empty(lead + (cols // block if block else 0,), dtype=torch.uint8,
+            packed[k] = torch.empty(lead + ((cols + 1) // 2,), dtype=torch.uint8,
                                     device=x.device)
+        if scales[k] is None:
+            scales[k] = torch.empty(lead + (-(-cols // block) if block else 0,),
+                                    dtype=torch.uint8, device=x.device)
         desc[k].x, desc[k].packed, desc[k].scales = (x.data_ptr(), packed[k].data_ptr(),
                                                      scales[k].data_ptr())
         desc[k].stats = out[k].data_ptr()

@@ -73,8 +73,8 @@ mx_status mx_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t cols, in
   const cudaError_t e =
       cols % block != 0
           ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
-                            nullptr, nullptr, packed, scales, nullptr, false, nullptr, nullptr,
-                            stream, &n)
+                            nullptr, nullptr, nullptr, packed, scales, nullptr, false, nullptr,
+                            nullptr, stream, &n)
           : mxk::run_quantize(x, xt == MX_BF16, numel, block, (int)fmt, global_scale_fp16, packed,
                               scales, stream, &n);
   g_launches += n;
@@ -96,7 +96,7 @@ mx_status mx_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t ro
   const cudaError_t e =
       cols % block != 0
           ? mxk::run_ragged_dequantize(packed, scales, rows, cols, block, (int)fmt,
-                                       global_scale_fp16, y, yt == MX_BF16, stream, &n)
+                                       global_scale_fp16, nullptr, y, yt == MX_BF16, stream, &n)
           : mxk::run_dequantize(packed, scales, numel, block, (int)fmt, global_scale_fp16, y,
                                 yt == MX_BF16, stream, &n);
   g_launches += n;
@@ -119,8 +119,8 @@ mx_status mx_fake_quantize(const void* x, mx_dtype xt, int64_t rows, int64_t col
   const cudaError_t e =
       cols % block != 0
           ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
-                            nullptr, nullptr, nullptr, nullptr, y, yt == MX_BF16, nullptr,
-                            nullptr, stream, &n)
+                            nullptr, nullptr, nullptr, nullptr, nullptr, y, yt == MX_BF16,
+                            nullptr, nullptr, stream, &n)
           : mxk::run_fake_quantize(x, xt == MX_BF16, numel, block, (int)fmt, global_scale_fp16,
                                    y, yt == MX_BF16, stream, &n);
   g_launches += n;
@@ -154,8 +154,8 @@ mx_status mx_error_stats(const void* x, mx_dtype xt, int64_t rows, int64_t cols,
   const cudaError_t e =
       numel != 0 && cols % block != 0
           ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
-                            packed, scales, nullptr, nullptr, nullptr, false, out_dev, workspace,
-                            stream, &n)
+                            nullptr, packed, scales, nullptr, nullptr, nullptr, false, out_dev,
+                            workspace, stream, &n)
           : mxk::run_error_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
                                  global_scale_fp16, packed, scales, out_dev, workspace, stream,
                                  &n);
@@ -182,8 +182,8 @@ mx_status mx_quantize_stats(const void* x, mx_dtype xt, int64_t rows, int64_t co
   const cudaError_t e =
       numel != 0 && cols % block != 0
           ? mxk::run_ragged(x, xt == MX_BF16, rows, cols, block, (int)fmt, global_scale_fp16,
-                            nullptr, nullptr, packed, scales, nullptr, false, out_dev, workspace,
-                            stream, &n)
+                            nullptr, nullptr, nullptr, packed, scales, nullptr, false, out_dev,
+                            workspace, stream, &n)
           : mxk::run_quantize_stats(numel ? x : nullptr, xt == MX_BF16, numel, block, (int)fmt,
                                     global_scale_fp16, packed, scales, out_dev, workspace, stream,
                                     &n);
@@ -356,7 +356,6 @@ mx_status check_group(const mx_tensor_t* t, int count, int block, unsigned need,
     if (!shape_ok(d.rows, d.cols) || !g_ok || d.reserved[0] || d.reserved[1] || d.reserved[2])
       return MX_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(d.global_scale_dev) & 1u) != 0) return MX_ERR_MISALIGNED;
-    if (d.cols % block != 0) return MX_ERR_INVALID_ARG;
     const int64_t numel = d.rows * d.cols;
     if ((need & kNeedStats) && !d.stats) return MX_ERR_INVALID_ARG;
     if ((need & kNeedStats) && !aligned16(d.stats)) return MX_ERR_MISALIGNED;
@@ -369,9 +368,22 @@ mx_status check_group(const mx_tensor_t* t, int count, int block, unsigned need,
         return MX_ERR_MISALIGNED;
     }
     args[k] = {d.x, d.y, d.packed, d.scales, d.stats, numel, d.global_scale_fp16,
-               d.global_scale_dev};
+               d.global_scale_dev, d.rows, d.cols};
   }
   return MX_OK;
+}
+
+// Splits checked tensors into those of whole blocks (one grouped launch) and ragged ones (cols %
+// block != 0, non-empty: the row-wise kernels, one launch each, after the grouped one).
+int split_ragged(const mxk::TensorArgs* args, int count, int block, mxk::TensorArgs* whole,
+                 mxk::TensorArgs* ragged, int* nragged) {
+  int nw = 0;
+  *nragged = 0;
+  for (int k = 0; k < count; ++k) {
+    if (args[k].numel != 0 && args[k].cols % block != 0) ragged[(*nragged)++] = args[k];
+    else whole[nw++] = args[k];
+  }
+  return nw;
 }
 
 }  // namespace
@@ -380,13 +392,21 @@ mx_status mx_quantize_group(const mx_tensor_t* tensors, int count, mx_dtype xt, 
                             mx_scale_fmt fmt, cudaStream_t stream) {
   if (!valid_dtype(xt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  mxk::TensorArgs args[MX_MAX_GROUP];
+  mxk::TensorArgs args[MX_MAX_GROUP], whole[MX_MAX_GROUP], ragged[MX_MAX_GROUP];
   const mx_status st = check_group(tensors, count, block, kNeedX | kNeedCodes, args);
   if (st != MX_OK) return st;
   if (injected_failure()) return MX_ERR_CUDA;
-  int n = 0;
-  const cudaError_t e =
-      mxk::run_quantize_group(args, count, xt == MX_BF16, block, (int)fmt, stream, &n);
+  int n = 0, nr = 0;
+  const int nw = split_ragged(args, count, block, whole, ragged, &nr);
+  cudaError_t e = nw ? mxk::run_quantize_group(whole, nw, xt == MX_BF16, block, (int)fmt, stream,
+                                               &n)
+                     : cudaSuccess;
+  for (int k = 0; k < nr && e == cudaSuccess; ++k) {
+    const mxk::TensorArgs& t = ragged[k];
+    e = mxk::run_ragged(t.x, xt == MX_BF16, t.rows, t.cols, block, (int)fmt, t.g_bits, t.g_dev,
+                        nullptr, nullptr, t.packed, t.scales, nullptr, false, nullptr, nullptr,
+                        stream, &n);
+  }
   g_launches += n;
   return from_cuda(e);
 }
@@ -395,13 +415,20 @@ mx_status mx_dequantize_group(const mx_tensor_t* tensors, int count, int block, 
                               mx_dtype yt, cudaStream_t stream) {
   if (!valid_dtype(yt) || !valid_fmt(fmt)) return MX_ERR_INVALID_ARG;
   if (!valid_block(block)) return MX_ERR_UNSUPPORTED;
-  mxk::TensorArgs args[MX_MAX_GROUP];
+  mxk::TensorArgs args[MX_MAX_GROUP], whole[MX_MAX_GROUP], ragged[MX_MAX_GROUP];
   const mx_status st = check_group(tensors, count, block, kNeedY | kNeedCodes, args);
   if (st != MX_OK) return st;
   if (injected_failure()) return MX_ERR_CUDA;
-  int n = 0;
-  const cudaError_t e =
-      mxk::run_dequantize_group(args, count, yt == MX_BF16, block, (int)fmt, stream, &n);
+  int n = 0, nr = 0;
+  const int nw = split_ragged(args, count, block, whole, ragged, &nr);
+  cudaError_t e = nw ? mxk::run_dequantize_group(whole, nw, yt == MX_BF16, block, (int)fmt,
+                                                 stream, &n)
+                     : cudaSuccess;
+  for (int k = 0; k < nr && e == cudaSuccess; ++k) {
+    const mxk::TensorArgs& t = ragged[k];
+    e = mxk::run_ragged_dequantize(t.packed, t.scales, t.rows, t.cols, block, (int)fmt, t.g_bits,
+                                   t.g_dev, t.y, yt == MX_BF16, stream, &n);
+  }
   g_launches += n;
   return from_cuda(e);
 }
@@ -417,9 +444,19 @@ mx_status mx_quantize_stats_group(const mx_tensor_t* tensors, int count, mx_dtyp
   if (!workspace || ws_bytes < stats_ws_bytes()) return MX_ERR_WORKSPACE;
   if (!aligned16(workspace)) return MX_ERR_MISALIGNED;
   if (injected_failure()) return MX_ERR_CUDA;
-  int n = 0;
-  const cudaError_t e = mxk::run_stats_group(args, count, xt == MX_BF16, block, (int)fmt,
-                                             mxk::kStore, workspace, stream, &n);
+  mxk::TensorArgs whole[MX_MAX_GROUP], ragged[MX_MAX_GROUP];
+  int n = 0, nr = 0;
+  const int nw = split_ragged(args, count, block, whole, ragged, &nr);
+  // the ragged tensors reuse the workspace after the grouped launch (same stream, in order)
+  cudaError_t e = nw ? mxk::run_stats_group(whole, nw, xt == MX_BF16, block, (int)fmt,
+                                            mxk::kStore, workspace, stream, &n)
+                     : cudaSuccess;
+  for (int k = 0; k < nr && e == cudaSuccess; ++k) {
+    const mxk::TensorArgs& t = ragged[k];
+    e = mxk::run_ragged(t.x, xt == MX_BF16, t.rows, t.cols, block, (int)fmt, t.g_bits, t.g_dev,
+                        nullptr, nullptr, t.packed, t.scales, nullptr, false, t.stats, workspace,
+                        stream, &n);
+  }
   g_launches += n;
   return from_cuda(e);
 }

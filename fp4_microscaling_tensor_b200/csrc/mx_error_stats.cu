@@ -176,8 +176,10 @@ __device__ __forceinline__ double scaled_to_double(float v, int E) {
 
 // Per-block constants of one block slice (see the file comment for the scaling).
 struct SliceSetup {
-  int E;           // biased exponent of the block maximum a (at least 1)
-  float sc;        // 2^(127 - E): a * sc in [1, 2)
+  int E;           // biased exponent of the block maximum a, clamped to [1, 253]
+  float sc;        // 2^(127 - E), a normal number: a * sc in [1, 2) (in [2, 4) for the top
+                   // binade, where the clamp keeps sc normal: the mixed-precision FMAs that
+                   // apply it take it as a bf16 operand, and a subnormal one would be lost)
   float sat6s;     // 6 S g sc, the scaled clip level
   float nDq;       // -S g sc 2^126: one FMA with a code's bits gives -y sc
   float tiny;      // a 2^-30: below it a scaled square could lose digits
@@ -187,8 +189,8 @@ struct SliceSetup {
 
 __device__ __forceinline__ SliceSetup slice_setup(float a, float D) {
   SliceSetup st;
-  st.E = max((int)((__float_as_uint(a) >> 23) & 0xFFu), 1);
-  st.sc = __uint_as_float(st.E <= 253 ? (uint32_t)(254 - st.E) << 23 : 0x00400000u);
+  st.E = min(max((int)((__float_as_uint(a) >> 23) & 0xFFu), 1), 253);
+  st.sc = __uint_as_float((uint32_t)(254 - st.E) << 23);
   const float Ds = __fmul_rn(D, st.sc);
   st.sat6s = __fmul_rn(6.0f, Ds);
   st.nDq = -__fmul_rn(Ds, 0x1p126f);
@@ -313,35 +315,54 @@ __device__ __forceinline__ float2 mag_scaled2(uint32_t aw, uint32_t sc16) {
   return make_float2(lo, hi);
 }
 
-// One code word's eight elements (words w[0..3]) with recomputed codes, quantized and reduced in
-// one go.  The scaled magnitudes xs = |x| s (s = 2^k, the slice scaling) come straight from the
-// bf16 words (mag_scaled2).  The quotients are taken of them with the rescaled reciprocal
-// r / s (x r = xs (r / s) exactly: s is a power of two), rounded onto the 2^-18 grid by adding and
-// subtracting 48 (see snap_quotient2; a magnitude needs no sign fix for zero), so the E2M1
-// conversion gives magnitude codes whose decode is one shift and one mask; x's sign bits are put
-// into the codes afterwards (byte permutes that replicate each half's sign, two masked ORs).
-// Errors use the magnitudes too: (xs - |q| S g s)^2 is the element's scaled square.  Per pair k
-// the block constants are those of block k / PB (PB = pairs per block inside the word: 2 for
-// N = 4, else 4); lt2[k / PB] collects the squares, nsat2 the clipped elements
-// (|x| > RD_bf16(6 S g) = S2).
-template <int PB>
+// One code word's eight elements (words w[0..3], all in one block) with recomputed codes,
+// quantized and reduced in one go.  The scaled magnitudes xs = |x| s (s = 2^k, the slice scaling)
+// come straight from the bf16 words (mag_scaled2).  The quotients are taken of them with the
+// rescaled reciprocal r / s (x r = xs (r / s) exactly: s is a power of two), rounded onto the
+// 2^-18 grid by adding and subtracting 48 (see snap_quotient2; a magnitude needs no sign fix for
+// zero), so the E2M1 conversion gives magnitude codes whose decode is one shift and one mask; x's
+// sign bits are put into the codes afterwards (byte permutes that replicate each half's sign, two
+// masked ORs).  Errors use the magnitudes too: (xs - |q| S g s)^2 is the element's scaled square.
+// A block far beyond its saturation (S g s below 2^-64: possible only with a caller's g far below
+// the tensor's) would overflow r / s; for it the quotients are taken of the unscaled |x| with r,
+// from the fp32 split of the words.  MODE says how that case is found: kFast / kDeep when the
+// caller has decided it for the whole item (deep_item), kCheck per call (where two inlined copies
+// of the item's work would cost registers).  r, nDq, S2: the block's reciprocal, -S g s 2^126 and
+// clip level RD_bf16(6 S g) (twice); lt2 collects the squares, nsat2 the clipped elements.
+enum QsMode { kFast = 0, kDeep = 1, kCheck = 2 };
+template <int PB, int MODE>
 __device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, const float* nDq,
                                               const uint32_t* S2, float sc, float2* lt2,
                                               uint32_t& nsat2) {
+  static_assert(PB == 4, "the code word's four words lie in one block");
   uint32_t aw[4];
   float2 xs[4];
   float q[8];
   const uint32_t sc16 = __float_as_uint(sc) >> 16;  // a power of two: exact as a bf16
-  const float isc = __frcp_rn(sc);                   // exact (a power of two)
+  const float rs = __fmul_rn(r[0], __frcp_rn(sc));  // r / s, exact unless it overflows
+  const bool deep = MODE == kDeep || (MODE == kCheck && !(rs <= 0x1p64f));
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    aw[k] = w[k] & 0x7FFF7FFFu;
-    xs[k] = mag_scaled2(aw[k], sc16);
-    const float rk = __fmul_rn(r[k / PB], isc);
-    const float2 y = __ffma2_rn(xs[k], make_float2(rk, rk), make_float2(48.0f, 48.0f));
-    const float2 qq = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
-    q[2 * k] = qq.x;
-    q[2 * k + 1] = qq.y;
+  for (int k = 0; k < 4; ++k) aw[k] = w[k] & 0x7FFF7FFFu;
+  if (!deep) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      xs[k] = mag_scaled2(aw[k], sc16);
+      const float2 y = __ffma2_rn(xs[k], make_float2(rs, rs), make_float2(48.0f, 48.0f));
+      const float2 qq = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
+      q[2 * k] = qq.x;
+      q[2 * k + 1] = qq.y;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 xa = make_float2(__uint_as_float(aw[k] << 16),
+                                    __uint_as_float(aw[k] & 0xFFFF0000u));
+      xs[k] = __fmul2_rn(xa, make_float2(sc, sc));
+      const float2 y = __ffma2_rn(xa, make_float2(r[0], r[0]), make_float2(48.0f, 48.0f));
+      const float2 qq = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
+      q[2 * k] = qq.x;
+      q[2 * k + 1] = qq.y;
+    }
   }
   const uint32_t cm = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
 #pragma unroll
@@ -366,6 +387,16 @@ __device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, 
   asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(hs) : "r"(x01), "r"(x23));
   asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(ls) : "r"(x01), "r"(x23));
   return (cm | (hs & 0x80808080u)) | (ls & 0x08080808u);
+}
+
+// True when one of the blocks (reciprocals r[0..nb)) is so far beyond its saturation that r / s
+// would overflow (see qs_word8): the item then takes the unscaled quotients.
+template <int NBL>
+__device__ __forceinline__ bool deep_item(const float* r, float sc) {
+  float mr = r[0];
+#pragma unroll
+  for (int b = 1; b < NBL; ++b) mr = fmaxf(mr, r[b]);
+  return __fmul_rn(mr, __frcp_rn(sc)) > 0x1p64f;
 }
 
 // Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
@@ -711,34 +742,33 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       D_b[b] = s_D[s];
       sc_all |= s << (8 * b);
     }
-    // closed form (one block slice per item): codes and squares together, per code word
+    // closed form (one block slice per item): codes and squares together, per code word (also
+    // where a block spans several lanes, N >= 64: measured 0.68 -> 0.74 of the copy peak there
+    // against converting the item's codes first and reducing them afterwards)
     SliceSetup st0;
     float2 lt0 = make_float2(0.0f, 0.0f);
     uint32_t nsat0 = 0u;
-    // (measured: the per-code-word form is faster when a lane holds a whole block, L == 1; with
-    // blocks spread over lanes, converting the item's codes first and then reducing is faster)
-    constexpr bool W8 = CLOSED && L == 1;
+    constexpr bool W8 = CLOSED;
     if constexpr (W8) {
       static_assert(!CLOSED || BPI == 1, "one block slice per item");
       st0 = slice_setup(a_b[0], D_b[0]);
       const uint32_t S2 = (__float_as_uint(__fmul_rn(6.0f, D_b[0])) >> 16) * 0x10001u;
+      // (measured: deciding the saturation case once per item is faster where a lane holds a
+      // whole block; where a block spans lanes the two inlined copies spill, so each code word
+      // checks it itself)
+      if constexpr (L > 1) {
 #pragma unroll
-      for (int j = 0; j < NCW; ++j)
-        it.cw[j] = qs_word8<4>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0, nsat0);
-    } else if constexpr (RECOMPUTE) {
-      // codes: eight quotients per code word, converted right away
+        for (int j = 0; j < NCW; ++j)
+          it.cw[j] = qs_word8<4, kCheck>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0,
+                                         nsat0);
+      } else if (!deep_item<1>(&r_b[0], st0.sc)) {
 #pragma unroll
-      for (int j = 0; j < NCW; ++j) {
-        float q[8];
+        for (int j = 0; j < NCW; ++j)
+          it.cw[j] = qs_word8<4, kFast>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0, nsat0);
+      } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int wi = 4 * j + k;
-          const uint32_t w = it.w[wi];
-          const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
-          q[2 * k] = qq.x;
-          q[2 * k + 1] = qq.y;
-        }
-        it.cw[j] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+        for (int j = 0; j < NCW; ++j)
+          it.cw[j] = qs_word8<4, kDeep>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0, nsat0);
       }
     }
     if constexpr (STORE) {
@@ -767,21 +797,6 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       const uint32_t A2 = m_b[b] * 0x10001u, S2 = sb * 0x10001u;
       float lt = 0.0f, ms = 0.0f, cnt = 0.0f, nsat = 0.0f, dmax = 0.0f;
       const float nD = st.nDq;
-      if constexpr (CLOSED && !W8) {
-        unsigned long long l2 = 0ull;
-#pragma unroll
-        for (int k = 0; k < BW; ++k) {
-          const int wi = b * BW + k;
-          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, cw = it.cw[wi >> 2];
-          switch (wi & 3) {
-            case 0: pair_step_all<0>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
-            case 1: pair_step_all<1>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
-            case 2: pair_step_all<2>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
-            default: pair_step_all<3>(w, lo, hi, cw, st.sc, nD, S2, l2, nsat0); break;
-          }
-        }
-        asm("mov.b64 {%0, %1}, %2;" : "=f"(lt0.x), "=f"(lt0.y) : "l"(l2));
-      }
 #pragma unroll
       for (int k = 0; k < BW && !CLOSED; ++k) {
         const int wi = b * BW + k;
@@ -952,8 +967,9 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     uint32_t mm = M[0];
 #pragma unroll
     for (int j = 1; j < NP; ++j) mm = bf16x2_absmax(mm, M[j]);
-    const int E = max((int)(max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu) >> 7), 1);
-    const float sc = __uint_as_float(E <= 253 ? (uint32_t)(254 - E) << 23 : 0x00400000u);
+    // E clamped to [1, 253]: sc = 2^(127 - E) stays a normal number (see SliceSetup)
+    const int E = min(max((int)(max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu) >> 7), 1), 253);
+    const float sc = __uint_as_float((uint32_t)(254 - E) << 23);
     // scale codes, reciprocals and per-block constants, two blocks at a time
     float r_b[NB], D_b[NB], nDq_b[NB];
     uint32_t S2_b[NB];
@@ -1005,10 +1021,20 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
 #pragma unroll
     for (int b = 0; b < NB; ++b) lt[b] = make_float2(0.0f, 0.0f);
     if constexpr (N >= 8) {
+      if (!deep_item<NB>(r_b, sc)) {
 #pragma unroll
-      for (int c = 0; c < NCW; ++c) {
-        const int b0 = (4 * c) / BW;  // block of the code word's first pair
-        cw[c] = qs_word8<PB>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0], nsat2);
+        for (int c = 0; c < NCW; ++c) {
+          const int b0 = (4 * c) / BW;  // block of the code word's first pair
+          cw[c] = qs_word8<PB, kFast>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                      nsat2);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < NCW; ++c) {
+          const int b0 = (4 * c) / BW;
+          cw[c] = qs_word8<PB, kDeep>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                      nsat2);
+        }
       }
     } else {
 #pragma unroll

@@ -121,6 +121,7 @@ struct TensorArgs {
   uint16_t g_bits;
   uint16_t* g_dev;    // when set: g is read from here when the kernel runs (g_bits unused); the
                       // global-scale group launch writes it
+  int64_t rows, cols; // the shape (used for tensors whose rows the block size does not divide)
 };
 
 // What the error-reduction pass does with the codes (see mx_error_stats.cu).
@@ -174,13 +175,16 @@ cudaError_t launch_stats_final(const StatsPartial* part, int nparts, int64_t num
 // Ragged tensors (cols % block != 0): one thread per block with plain per-element code.  Outputs
 // that are null are not produced: codes + scales (packed / scales), the round trip (y), the error
 // record (out, with workspace; from stored codes when packed_in is given).
+// g_dev: when set, g is read from device memory when the kernel runs (g_bits unused).
 cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int block, int fmt,
-                       uint16_t g_bits, const uint8_t* packed_in, const uint8_t* scales_in,
-                       uint8_t* packed, uint8_t* scales, void* y, bool y_bf16, void* out,
-                       void* workspace, cudaStream_t stream, int* launches);
+                       uint16_t g_bits, const uint16_t* g_dev, const uint8_t* packed_in,
+                       const uint8_t* scales_in, uint8_t* packed, uint8_t* scales, void* y,
+                       bool y_bf16, void* out, void* workspace, cudaStream_t stream,
+                       int* launches);
 cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
-                                  int64_t cols, int block, int fmt, uint16_t g_bits, void* y,
-                                  bool y_bf16, cudaStream_t stream, int* launches);
+                                  int64_t cols, int block, int fmt, uint16_t g_bits,
+                                  const uint16_t* g_dev, void* y, bool y_bf16,
+                                  cudaStream_t stream, int* launches);
 
 // Zeroes one last-CTA counter once the previous kernel in the stream is done with it (a one-thread
 // kernel launched with programmatic serialization).

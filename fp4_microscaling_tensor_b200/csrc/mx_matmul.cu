@@ -696,14 +696,17 @@ bool make_rows_map(CUtensorMap* map, const uint8_t* scales, int64_t rows) {
 // dequantized to global memory: per element of W the kernel reads 1/2 + 1/N bytes.
 //
 // One CTA per 256 x 256 tile of C (two 128-row accumulators side by side in TMEM, 512 columns),
-// 10 warps:
+// 11 warps:
 //   * warp 0, one thread: per 64-element step of k, TMA loads of the step's two 128 x 64 tiles of
 //     A (128-byte swizzle), completing on the stage's A barrier;
-//   * warps 2..9 (256 threads, one row of the W tile each): load the step's 32 code bytes and
-//     64 / N scale bytes of their row one step ahead, decode the codes (E2M1x2 -> f16x2), multiply
-//     by the block's S g (exact in fp32), round to bf16 and write the 128-byte row into the
-//     stage's W tile in the same 128-byte-swizzled K-major layout the TMA writes for A; then a
-//     proxy fence and one arrival per warp on the stage's W barrier;
+//   * warp 10, one thread: TMA loads of the step's code bytes of the W tile (256 rows x 32 bytes)
+//     into a ring of 4 code tiles, up to 4 steps ahead of their use;
+//   * warps 2..9 (256 threads, one row of the W tile each): read the step's 32 code bytes from the
+//     ring (every lane acquires the ring's barrier), take the 64 / N scale bytes loaded two steps
+//     earlier, decode the codes (E2M1x2 -> f16x2), multiply by the block's S g (exact in fp32),
+//     round to bf16 and write the 128-byte row into the stage's W tile in the same 128-byte-swizzled
+//     K-major layout the TMA writes for A; then a proxy fence and one arrival per warp on the
+//     stage's W barrier;
 //   * warp 1, one thread: waits for both barriers, issues 4 (or 8) tcgen05.mma of 128 x 256 x 16,
 //     commits to the stage's empty barrier;
 //   * warps 2..9 then read the accumulators back (tcgen05.ld; warp w serves TMEM lanes 32 (w % 4)
@@ -718,9 +721,12 @@ constexpr int kATile = 128 * 128;             // one 128-row half of A: 128 x 64
 constexpr int kABytes = 2 * kATile;
 constexpr int kBBytes = kBN * 128;            // the W tile: 256 x 64 bf16
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 320;
+constexpr int kCStages = 4;                   // ring of the W tile's code bytes (TMA)
+constexpr int kCBytes = kBN * (kBK / 2);      // 256 rows x 32 bytes
+constexpr int kThreads = 352;  // warp 0: A, warp 1: MMA, warps 2..9: W, warp 10: W codes
 constexpr int kDqWarps = 8;
-constexpr int kSmemBytes = kStages * kStageBytes + 256 * 4 + 256 + 1024;
+constexpr int kSmemBytes = kStages * kStageBytes + kCStages * kCBytes + 256 * 4 + 256 + 1024;
+static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 constexpr uint32_t kTmemCols = 512;
 // Instruction descriptor of kind::f16: fp32 accumulator (bits 4..5 = 1), A and B bf16 (bits 7..9
 // and 10..12 = 1), both K-major, N = 256 (bits 17..22: N / 8), M = 128 (bits 24..28: M / 16).
@@ -766,14 +772,11 @@ struct StepScales {
 };
 
 template <int N>
-__device__ __forceinline__ void load_step(const uint8_t* wrow, const uint8_t* srow, int kt,
-                                          bool ok, uint4& c0, uint4& c1, StepScales<N>& sc) {
-  c0 = c1 = make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void load_scales(const uint8_t* srow, int kt, bool ok,
+                                            StepScales<N>& sc) {
 #pragma unroll
   for (int i = 0; i < (int)(sizeof(sc.v) / 4); ++i) sc.v[i] = 0;
   if (!ok) return;
-  c0 = ld_stream16(wrow + 32 * (int64_t)kt);
-  c1 = ld_stream16(wrow + 32 * (int64_t)kt + 16);
   if constexpr (N == 4) {
     const uint4 t = __ldg(reinterpret_cast<const uint4*>(srow + 16 * (int64_t)kt));
     sc.v[0] = t.x; sc.v[1] = t.y; sc.v[2] = t.z; sc.v[3] = t.w;
@@ -821,21 +824,26 @@ __device__ __forceinline__ void dq_word(uint32_t cw, int w, const StepScales<N>&
 
 template <int N, int FMT>
 __global__ void __launch_bounds__(dqmm::kThreads, 1)
-    k_dequant_matmul(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ DqArgs args) {
+    k_dequant_matmul(const __grid_constant__ CUtensorMap tma_a,
+                     const __grid_constant__ CUtensorMap tma_w, const __grid_constant__ DqArgs args) {
   using namespace dqmm;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* s_D = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  uint8_t* codes = smem + kStages * kStageBytes;  // kCStages code tiles
+  float* s_D = reinterpret_cast<float*>(codes + kCStages * kCBytes);
   uint64_t* a_full = reinterpret_cast<uint64_t*>(s_D + 256);
   uint64_t* b_full = a_full + kStages;
   uint64_t* empty = b_full + kStages;
-  uint64_t* done = empty + kStages;
+  uint64_t* c_full = empty + kStages;
+  uint64_t* c_empty = c_full + kCStages;
+  uint64_t* done = c_empty + kCStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* gave_up = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.y * 256, n0 = (int64_t)blockIdx.x * kBN;
+  const int64_t NT = (args.n + kBN - 1) / kBN;  // tiles of C: n fastest (one 1-D grid)
+  const int64_t m0 = ((int64_t)blockIdx.x / NT) * 256, n0 = ((int64_t)blockIdx.x % NT) * kBN;
   const bool two = m0 + 128 < args.m;  // the second 128-row half has rows
   const int KT = (int)(args.k / dqmm::kBK);
   const uint16_t gb = args.g_dev ? __ldg(args.g_dev) : (uint16_t)args.g_bits;
@@ -847,6 +855,10 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
       mbar_init(smem_u32(a_full + s), 1);
       mbar_init(smem_u32(b_full + s), kDqWarps);
       mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int c = 0; c < kCStages; ++c) {
+      mbar_init(smem_u32(c_full + c), 1);
+      mbar_init(smem_u32(c_empty + c), kDqWarps);
     }
     mbar_init(smem_u32(done), 1);
     *gave_up = 0;
@@ -865,7 +877,32 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 10) {
+    // ---------------- code producer (one thread): the W tile's code bytes, kCStages ahead ----
+    // (a warp of its own: two spinning producers in one warp need not both make progress)
+    if (lane == 0) {
+      int issued = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int c = kt % kCStages;
+        if (*gave_up ||
+            (kt >= kCStages && !mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(c_empty + c),
+                                                            ((kt / kCStages) + 1) & 1, args.gen))) {
+          *gave_up = 1;
+          break;
+        }
+        const uint32_t bar = smem_u32(c_full + c);
+        mbar_expect_tx(bar, kCBytes);  // OOB rows included
+        tma_load_2d(smem_u32(codes + c * kCBytes), &tma_w, kt * (dqmm::kBK / 2), (int)n0, bar);
+        mbar_arrive(bar);
+        issued = kt + 1;
+      }
+      if (*gave_up) {
+        for (int kt = issued - kCStages < 0 ? 0 : issued - kCStages; kt < issued; ++kt)
+          mbar_wait<100>(smem_u32(c_full + kt % kCStages), (kt / kCStages) & 1, args.gen);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ---------------- A producer (one thread) ----------------
     if (lane == 0) {
       int issued = 0;
@@ -881,6 +918,7 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
         mbar_expect_tx(bar, two ? 2 * kATile : kATile);  // OOB rows included
         tma_load_2d(st, &tma_a, kt * dqmm::kBK, (int)m0, bar);
         if (two) tma_load_2d(st + kATile, &tma_a, kt * dqmm::kBK, (int)(m0 + 128), bar);
+        mbar_arrive(bar);  // the barrier's one arrival; the phase completes when the bytes land
         issued = kt + 1;
       }
       if (*gave_up) {
@@ -915,23 +953,35 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
     __syncwarp();
   } else {
     // ---------------- W dequantization (warps 2..9, one row of the tile per thread) ----------
+    // codes from the TMA ring (row d at byte 32 d of a code tile), scales by plain loads two steps
+    // ahead
     const int d = threadIdx.x - 64;
     const int64_t row = n0 + d;
     const bool row_ok = row < args.n;
-    const uint8_t* wrow = args.w_packed + (row_ok ? row : 0) * (args.k / 2);
     const uint8_t* srow = args.w_scales + (row_ok ? row : 0) * (args.k / N);
     const uint32_t r8 = (uint32_t)(d & 7);
     const uint32_t row_off = (uint32_t)(d >> 3) * 1024u + r8 * 128u;
-    uint4 c0, c1;
-    StepScales<N> sc;
-    load_step<N>(wrow, srow, 0, row_ok, c0, c1, sc);
+    StepScales<N> sc0, sc1;
+    load_scales<N>(srow, 0, row_ok && 0 < KT, sc0);
+    load_scales<N>(srow, 1, row_ok && 1 < KT, sc1);
     for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % kStages;
-      uint4 n0c, n1c;
-      StepScales<N> nsc;
-      load_step<N>(wrow, srow, kt + 1, row_ok && kt + 1 < KT, n0c, n1c, nsc);
-      bool ok = !*gave_up;
-      if (ok && kt >= kStages && lane == 0)
+      const int s = kt % kStages, c = kt % kCStages;
+      StepScales<N> sc2;
+      load_scales<N>(srow, kt + 2, row_ok && kt + 2 < KT, sc2);
+      // every lane that reads the tile acquires the barrier the TMA completes
+      bool ok = !*gave_up && mbar_wait(smem_u32(c_full + c), (kt / kCStages) & 1, args.gen);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        *gave_up = 1;
+        break;
+      }
+      uint4 c0, c1;
+      const uint32_t caddr = smem_u32(codes + c * kCBytes) + 32u * (uint32_t)d;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w) : "r"(caddr) : "memory");
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w) : "r"(caddr + 16u) : "memory");
+      if (kt >= kStages && lane == 0)
         ok = mbar_wait<MX_MM_PROD_SLEEP>(smem_u32(empty + s), ((kt / kStages) + 1) & 1, args.gen);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
@@ -943,21 +993,26 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
 #pragma unroll
       for (int w = 0; w < 8; ++w) {
         uint32_t o[4];
-        dq_word<N>(cw[w], w, sc, s_D, o);
+        dq_word<N>(cw[w], w, sc0, s_D, o);
         st_shared16(base + (((uint32_t)w ^ r8) << 4), o[0], o[1], o[2], o[3]);
       }
       // the tensor core reads this tile through the async proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(b_full + s));
-      c0 = n0c;
-      c1 = n1c;
-      sc = nsc;
+      if (lane == 0) {
+        mbar_arrive(smem_u32(b_full + s));
+        // the code tile's slot is released only now that every lane has used the values it read
+        // (released right after the loads were issued, the next TMA into the slot was measured
+        // to overwrite codes some lanes had not read yet)
+        mbar_arrive(smem_u32(c_empty + c));
+      }
+      sc0 = sc1;
+      sc1 = sc2;
     }
   }
 
   // ---------------- epilogue: warps 2..9 ----------------
-  if (warp >= 2) {
+  if (warp >= 2 && warp <= 9) {
     const int q = warp & 3, h = (warp - 2) >> 2;
     bool ok = true;
     if (lane == 0) {
@@ -983,6 +1038,20 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
                  "r"(kTmemCols)
                  : "memory");
   }
+}
+
+// Map of the weights' codes: n rows of k / 2 bytes, boxes of 256 rows x 32 bytes (one 64-element
+// step), no swizzle; rows past the end read as zero.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t n, int64_t k) {
+  const EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n};
+  const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)(dqmm::kBK / 2), (cuuint32_t)dqmm::kBN};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Map of the bf16 activations: m x k, row pitch 2 k bytes, boxes of 128 rows x 64 elements loaded
@@ -1062,26 +1131,29 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
 }
 
 template <int N, int FMT>
-static cudaError_t launch_dqmm(const CUtensorMap& ma, const DqArgs& args, cudaStream_t stream) {
+static cudaError_t launch_dqmm(const CUtensorMap& ma, const CUtensorMap& mw, const DqArgs& args,
+                               cudaStream_t stream) {
   static std::atomic<bool> attr[kMaxDevices];
   const cudaError_t e = allow_smem(attr, k_dequant_matmul<N, FMT>, dqmm::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((args.n + dqmm::kBN - 1) / dqmm::kBN), (unsigned)((args.m + 255) / 256));
-  k_dequant_matmul<N, FMT><<<grid, dqmm::kThreads, dqmm::kSmemBytes, stream>>>(ma, args);
+  const int64_t tiles = ((args.n + dqmm::kBN - 1) / dqmm::kBN) * ((args.m + 255) / 256);
+  if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidConfiguration;
+  k_dequant_matmul<N, FMT><<<(unsigned)tiles, dqmm::kThreads, dqmm::kSmemBytes, stream>>>(ma, mw,
+                                                                                        args);
   return cudaGetLastError();
 }
 
 template <int FMT>
-static cudaError_t dqmm_block(int block, const CUtensorMap& ma, const DqArgs& args,
-                              cudaStream_t st) {
+static cudaError_t dqmm_block(int block, const CUtensorMap& ma, const CUtensorMap& mw,
+                              const DqArgs& args, cudaStream_t st) {
   switch (block) {
-    case 4: return launch_dqmm<4, FMT>(ma, args, st);
-    case 8: return launch_dqmm<8, FMT>(ma, args, st);
-    case 16: return launch_dqmm<16, FMT>(ma, args, st);
-    case 32: return launch_dqmm<32, FMT>(ma, args, st);
-    case 64: return launch_dqmm<64, FMT>(ma, args, st);
-    case 128: return launch_dqmm<128, FMT>(ma, args, st);
-    default: return launch_dqmm<256, FMT>(ma, args, st);
+    case 4: return launch_dqmm<4, FMT>(ma, mw, args, st);
+    case 8: return launch_dqmm<8, FMT>(ma, mw, args, st);
+    case 16: return launch_dqmm<16, FMT>(ma, mw, args, st);
+    case 32: return launch_dqmm<32, FMT>(ma, mw, args, st);
+    case 64: return launch_dqmm<64, FMT>(ma, mw, args, st);
+    case 128: return launch_dqmm<128, FMT>(ma, mw, args, st);
+    default: return launch_dqmm<256, FMT>(ma, mw, args, st);
   }
 }
 
@@ -1089,11 +1161,12 @@ cudaError_t run_dequant_matmul(const void* a, int64_t m, int64_t k, const uint8_
                                const uint8_t* w_scales, int64_t n, int block, int fmt,
                                uint16_t g_bits, const uint16_t* g_dev, void* c, bool c_bf16,
                                cudaStream_t stream, int* launches) {
-  CUtensorMap ma;
-  if (!make_bf16_map(&ma, a, m, k)) return cudaErrorInvalidValue;
+  CUtensorMap ma, mw;
+  if (!make_bf16_map(&ma, a, m, k) || !make_codes_map(&mw, w_packed, n, k))
+    return cudaErrorInvalidValue;
   const DqArgs args{w_packed, w_scales, g_dev, c, m, n, k, g_bits, c_bf16 ? 1 : 0, next_gen()};
-  const cudaError_t e = fmt == kUE5M3 ? dqmm_block<kUE5M3>(block, ma, args, stream)
-                                      : dqmm_block<kE4M3>(block, ma, args, stream);
+  const cudaError_t e = fmt == kUE5M3 ? dqmm_block<kUE5M3>(block, ma, mw, args, stream)
+                                      : dqmm_block<kE4M3>(block, ma, mw, args, stream);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -24,6 +24,7 @@ struct RaggedArgs {
   int64_t rows, cols;
   int N;
   uint32_t g_bits;
+  const uint16_t* g_dev;     // g in device memory when set (g_bits unused)
   const uint8_t* packed_in;  // stored codes (error reduction from codes), or null
   const uint8_t* scales_in;
   uint8_t* packed;           // codes written, or null
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kThreads) k_ragged_rows(const __grid_constant_
   constexpr int BPL = N == 4 ? 2 : 1;          // blocks per lane
   constexpr int G = N <= 8 ? 1 : N / 8;        // lanes per block
   constexpr int EB = N == 4 ? 4 : 8;           // elements of a lane in one block
-  const float g = fp16_bits_to_float((uint16_t)a.g_bits);
+  const float g = fp16_bits_to_float(tensor_g_bits(a.g_bits, a.g_dev));
   const float g6 = __fmul_rn(6.0f, g);                   // exact
   const float r6 = __frcp_rn(g6);
   const float sat_thr = __fmul_rn(g6, scale_max<FMT>());  // exact
@@ -87,25 +88,37 @@ __global__ void __launch_bounds__(kThreads) k_ragged_rows(const __grid_constant_
     const T* xr = static_cast<const T*>(a.x) + r * a.cols;
     const bool x_aligned = ((r * a.cols) & (BF16 ? 7 : 3)) == 0;  // 16-byte row start
     const int64_t prow = r * pb, srow = r * nb;
-    for (int e0 = 0; e0 < cols; e0 += 256) {
-      const int j0 = e0 + 8 * lane;  // this lane's first element
+    // the 8 elements of this lane in the step from e0 (zero past the row end); the next step's
+    // are loaded before the current step's work
+    auto load_step = [&](int e0, float (&v)[8]) {
+      const int j0 = e0 + 8 * lane;
       const int nv = max(0, min(8, cols - j0));
-      float v[8];
       if (nv == 8 && x_aligned) {
         if constexpr (BF16) {
-          const uint4 w = *reinterpret_cast<const uint4*>(xr + j0);
+          const uint4 w = ld_stream16(xr + j0);
           v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
           v[4] = bf16lo(w.z); v[5] = bf16hi(w.z); v[6] = bf16lo(w.w); v[7] = bf16hi(w.w);
         } else {
-          const float4 u0 = *reinterpret_cast<const float4*>(xr + j0);
-          const float4 u1 = *reinterpret_cast<const float4*>(xr + j0 + 4);
-          v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
-          v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+          const uint4 u0 = ld_stream16(xr + j0), u1 = ld_stream16(xr + j0 + 4);
+          v[0] = __uint_as_float(u0.x); v[1] = __uint_as_float(u0.y);
+          v[2] = __uint_as_float(u0.z); v[3] = __uint_as_float(u0.w);
+          v[4] = __uint_as_float(u1.x); v[5] = __uint_as_float(u1.y);
+          v[6] = __uint_as_float(u1.z); v[7] = __uint_as_float(u1.w);
         }
       } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = k < nv ? load_x(xr + j0 + k) : 0.0f;
       }
+    };
+    float vn[8];
+    load_step(0, vn);
+    for (int e0 = 0; e0 < cols; e0 += 256) {
+      const int j0 = e0 + 8 * lane;  // this lane's first element
+      const int nv = max(0, min(8, cols - j0));
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = vn[k];
+      if (e0 + 256 < cols) load_step(e0 + 256, vn);
       uint32_t codes = 0;  // 8 codes, element k in nibble k
 #pragma unroll
       for (int h = 0; h < BPL; ++h) {
@@ -221,26 +234,82 @@ __global__ void __launch_bounds__(kThreads) k_ragged_rows(const __grid_constant_
   }
 }
 
-// One warp per row: lane l takes code bytes l, l + 32, ... of the row; y = E2M1 x S x g (exact),
-// bf16 = its round to nearest even.  Both elements of a byte are in one block (blocks start at
-// even columns).
+// One warp per row, a warp step of 256 elements: lane l takes the 8 consecutive elements
+// 8 l .. 8 l + 7 of the step (4 code bytes: one 4-byte load where the row's code bytes are
+// aligned, else byte loads; one scale byte, two for N = 4), y = E2M1 x S x g (exact; S g from a
+// per-CTA table), bf16 = its round to nearest even, stored as one 16-byte vector (fp32: two)
+// where the row start allows, else element by element.  The next step's loads are issued before
+// the current step's stores.  Elements past the row end are neither read nor written.
 template <int FMT, int LOGN>
 __global__ void __launch_bounds__(kThreads)
     k_ragged_dequantize(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-                        int64_t rows, int64_t cols, uint16_t g_bits, void* y, int y_bf16) {
-  const float g = fp16_bits_to_float(g_bits);
-  const int64_t nb = (cols + (1 << LOGN) - 1) >> LOGN, pb = (cols + 1) / 2;
+                        int64_t rows, int64_t cols, uint16_t g_bits, const uint16_t* g_dev,
+                        void* y, int y_bf16) {
+  constexpr int N = 1 << LOGN;
+  __shared__ float s_D[256];
+  const float g = fp16_bits_to_float(tensor_g_bits(g_bits, g_dev));
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+  __syncthreads();
+  const int64_t nb = (cols + N - 1) >> LOGN, pb = (cols + 1) / 2;
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int icols = (int)cols;
+  struct Step {
+    uint32_t codes, sc;  // 8 codes (element k in nibble k); scale byte(s), N = 4: two
+    int nv;              // elements of this lane in the step (0..8)
+  };
+  auto load = [&](int64_t r, int e0) {
+    Step st{0u, 0u, 0};
+    const int j0 = e0 + 8 * lane;
+    st.nv = max(0, min(8, icols - j0));
+    if (st.nv == 0) return st;
+    const int64_t cb = r * pb + j0 / 2;  // first code byte
+    if (st.nv == 8 && (cb & 3) == 0) {
+      st.codes = __ldg(reinterpret_cast<const unsigned int*>(packed + cb));
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (2 * k < st.nv) st.codes |= (uint32_t)__ldg(packed + cb + k) << (8 * k);
+    }
+    const int64_t sb = r * nb + (j0 >> LOGN);
+    st.sc = __ldg(scales + sb);
+    if (N == 4 && st.nv > 4) st.sc |= (uint32_t)__ldg(scales + sb + 1) << 8;
+    return st;
+  };
   for (int64_t r = warp; r < rows; r += nwarps) {
-    for (int64_t k = lane; k < pb; k += 32) {
-      const int64_t j = 2 * k;
-      const uint32_t c = packed[r * pb + k];
-      const float D = __fmul_rn(scale_value((int)scales[r * nb + (j >> LOGN)], FMT), g);
-      store_y(y, r * cols + j, __fmul_rn(e2m1_to_float(c & 0xF), D), y_bf16);
-      if (j + 1 < cols)
-        store_y(y, r * cols + j + 1, __fmul_rn(e2m1_to_float(c >> 4), D), y_bf16);
+    const int64_t y0 = r * cols;  // first element of the row in y
+    const bool vec = y_bf16 ? (y0 & 7) == 0 : (y0 & 3) == 0;
+    Step cur = load(r, 0);
+    for (int e0 = 0; e0 < icols; e0 += 256) {
+      const Step nxt = e0 + 256 < icols ? load(r, e0 + 256) : Step{0u, 0u, 0};
+      if (cur.nv > 0) {
+        const int j0 = e0 + 8 * lane;
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float D = s_D[N == 4 && k >= 4 ? (cur.sc >> 8) & 0xFF : cur.sc & 0xFF];
+          v[k] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits_at(cur.codes, 4 * k)),
+                                     0x1p126f),
+                           D);  // exact
+        }
+        if (cur.nv == 8 && vec) {
+          if (y_bf16) {
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + y0 + j0) =
+                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(y) + y0 + j0);
+            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < cur.nv) store_y(y, y0 + j0 + k, v[k], y_bf16);
+        }
+      }
+      cur = nxt;
     }
   }
 }
@@ -277,36 +346,44 @@ cudaError_t launch_ragged(const RaggedArgs& args, int64_t nblocks, void* out, cu
 
 template <int FMT, int LOGN>
 cudaError_t launch_dq(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t cols,
-                      uint16_t g_bits, void* y, bool y_bf16, cudaStream_t stream) {
+                      uint16_t g_bits, const uint16_t* g_dev, void* y, bool y_bf16,
+                      cudaStream_t stream) {
   const int grid = persistent_grid((const void*)k_ragged_dequantize<FMT, LOGN>, rows * 32, 1);
   k_ragged_dequantize<FMT, LOGN><<<grid, kThreads, 0, stream>>>(packed, scales, rows, cols,
-                                                                 g_bits, y, y_bf16 ? 1 : 0);
+                                                                 g_bits, g_dev, y, y_bf16 ? 1 : 0);
   return cudaGetLastError();
 }
 
 template <int FMT>
 cudaError_t launch_dq_fmt(const uint8_t* packed, const uint8_t* scales, int64_t rows,
-                          int64_t cols, int block, uint16_t g_bits, void* y, bool y_bf16,
-                          cudaStream_t stream) {
+                          int64_t cols, int block, uint16_t g_bits, const uint16_t* g_dev,
+                          void* y, bool y_bf16, cudaStream_t stream) {
   switch (block) {
-    case 4: return launch_dq<FMT, 2>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    case 8: return launch_dq<FMT, 3>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    case 16: return launch_dq<FMT, 4>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    case 32: return launch_dq<FMT, 5>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    case 64: return launch_dq<FMT, 6>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    case 128: return launch_dq<FMT, 7>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
-    default: return launch_dq<FMT, 8>(packed, scales, rows, cols, g_bits, y, y_bf16, stream);
+    case 4: return launch_dq<FMT, 2>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    case 8: return launch_dq<FMT, 3>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    case 16: return launch_dq<FMT, 4>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    case 32: return launch_dq<FMT, 5>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    case 64: return launch_dq<FMT, 6>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    case 128: return launch_dq<FMT, 7>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16,
+                                             stream);
+    default: return launch_dq<FMT, 8>(packed, scales, rows, cols, g_bits, g_dev, y, y_bf16, stream);
   }
 }
 
 }  // namespace
 
 cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int block, int fmt,
-                       uint16_t g_bits, const uint8_t* packed_in, const uint8_t* scales_in,
+                       uint16_t g_bits, const uint16_t* g_dev, const uint8_t* packed_in,
+                       const uint8_t* scales_in,
                        uint8_t* packed, uint8_t* scales, void* y, bool y_bf16, void* out,
                        void* workspace, cudaStream_t stream, int* launches) {
   if (cols > (int64_t(1) << 30)) return cudaErrorInvalidValue;  // in-row indices are 32-bit
-  RaggedArgs args{x, rows, cols, block, g_bits, packed_in, scales_in, packed, scales, y,
+  RaggedArgs args{x, rows, cols, block, g_bits, g_dev, packed_in, scales_in, packed, scales, y,
                   y_bf16 ? 1 : 0, nullptr};
   if (out)  // partials after the workspace's 64-byte counter headers
     args.part = reinterpret_cast<StatsPartial*>(static_cast<char*>(workspace) + 64 * kMaxGroup);
@@ -319,12 +396,15 @@ cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int
 }
 
 cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
-                                  int64_t cols, int block, int fmt, uint16_t g_bits, void* y,
+                                  int64_t cols, int block, int fmt, uint16_t g_bits,
+                                  const uint16_t* g_dev, void* y,
                                   bool y_bf16, cudaStream_t stream, int* launches) {
   ++*launches;
   return fmt == kUE5M3
-             ? launch_dq_fmt<kUE5M3>(packed, scales, rows, cols, block, g_bits, y, y_bf16, stream)
-             : launch_dq_fmt<kE4M3>(packed, scales, rows, cols, block, g_bits, y, y_bf16, stream);
+             ? launch_dq_fmt<kUE5M3>(packed, scales, rows, cols, block, g_bits, g_dev, y, y_bf16,
+                                     stream)
+             : launch_dq_fmt<kE4M3>(packed, scales, rows, cols, block, g_bits, g_dev, y, y_bf16,
+                                    stream);
 }
 
 }  // namespace mxk

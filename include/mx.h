@@ -32,8 +32,8 @@
  *     the low nibble of byte k, 2k+1 in the high nibble; an odd last element leaves the high
  *     nibble 0) and its scales in ceil(cols/N) bytes.  For cols % N == 0 that is rows*cols/2 and
  *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged") run on a row-wise path (one
- *     warp per row; cols up to 2^30, else MX_ERR_CUDA); the grouped calls accept whole blocks
- *     only (cols % N != 0: MX_ERR_INVALID_ARG).
+ *     warp per row; cols up to 2^30, else MX_ERR_CUDA); in a grouped call they run on that path
+ *     after the group's one launch over its whole-block tensors.
  *   - rows == 0 or cols == 0 is an empty tensor: quantize / dequantize enqueue nothing,
  *     mx_error_stats writes an all-zero result and mx_global_scale writes 1.0.
  *   - x must be finite: NaN or Inf in x gives unspecified codes (no kernel faults or hangs).
@@ -193,7 +193,8 @@ MX_API mx_status mx_error_stats_noalloc(const void* x, mx_dtype xt, int64_t rows
  * MX_ERR_INVALID_ARG. */
 #define MX_MAX_GROUP 16
 
-/* One tensor of a grouped call: rows x cols, row-major, cols % block == 0. */
+/* One tensor of a grouped call: rows x cols, row-major (any cols; the layout of codes and scales
+ * is the one described above). */
 typedef struct {
   const void* x;              /* input of mx_quantize_group / mx_quantize_stats_group /
                                  mx_global_scale_group */

@@ -157,7 +157,9 @@ def test_group_calls_reject_bad_arguments():
     assert L.mx_quantize_group(None, 1, BF16, 32, E4, None) == INV
     assert L.mx_quantize_group(group(2), 2, 9, 32, E4, None) == INV           # dtype
     assert L.mx_quantize_group(group(2), 2, BF16, 12, E4, None) == UNS        # block
-    assert L.mx_quantize_group(group(2, cols=48), 2, BF16, 32, E4, None) == INV
+    L.mx_test_fail_next_calls(1)  # ragged rows (48 % 32 != 0) are accepted: stop before launch
+    assert L.mx_quantize_group(group(2, cols=48), 2, BF16, 32, E4, None) == _lib.MX_ERR_CUDA
+    assert L.mx_test_fail_next_calls(0) == 0
     assert L.mx_quantize_group(group(2, g=0x7C00), 2, BF16, 32, E4, None) == INV
     assert L.mx_quantize_group(group(2, reserved=1), 2, BF16, 32, E4, None) == INV
     assert L.mx_quantize_group(group(2, x=None), 2, BF16, 32, E4, None) == INV
@@ -173,7 +175,7 @@ def test_group_calls_reject_bad_arguments():
     assert L.mx_quantize_stats_group(group(2), 2, BF16, 32, E4, A + 4, ws, None) == MIS
     # one bad tensor among good ones rejects the whole call
     d = group(3)
-    d[2].cols = 40
+    d[2].rows = -1
     assert L.mx_quantize_group(d, 3, BF16, 32, E4, None) == INV
 
 

@@ -101,3 +101,44 @@ def test_ragged_large_sampled_rows():
     po, so = oracle.quantize(xs, len(sel), cols, block, mx.E4M3)
     assert_same(u8(p.view(rows, -1)[torch.from_numpy(sel).cuda()]), po, "sampled packed")
     assert_same(u8(s.view(rows, -1)[torch.from_numpy(sel).cuda()]), so, "sampled scales")
+
+
+@pytest.mark.parametrize("block", [4, 16, 32, 256])
+@pytest.mark.parametrize("fmt", (mx.E4M3, mx.UE5M3))
+def test_grouped_calls_take_ragged_tensors(cuda_device, block, fmt):
+    """A group mixing whole-block tensors and tensors whose rows the block size does not divide
+    (odd row lengths included), with g by value and from device memory: every tensor's codes,
+    scales, dequantized bits and error record equal the oracle's."""
+    rng = np.random.default_rng(block + 5 * fmt)
+    shapes = [(64, 2 * block), (33, 3 * block + 5), (7, block - 1 if block > 4 else 3),
+              (0, block + 1), (129, 8 * block), (5, 2 * block + 1)]
+    xs = []
+    for r, c in shapes:
+        x = rng.standard_normal((r, c)) * np.exp(rng.uniform(-3, 1, (r, 1)))
+        xs.append(torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(cuda_device))
+    for gmode in ("value", "device"):
+        if gmode == "device":
+            g = mx.global_scale_group(xs, fmt)
+            gs = [int(v) for v in g.cpu().numpy().view(np.uint16)]
+        else:
+            gs = [0x3C00, 0x3555, 0x2E66, 0x3C00, 0x4400, 0x0003][:len(xs)]
+            g = gs
+        p, s = mx.quantize_group(xs, block, fmt, g=g)
+        p2, s2, st = mx.quantize_with_stats_group(xs, block, fmt, g=g)
+        y = mx.dequantize_group(p, s, block, fmt, g=g, cols=[c for _, c in shapes])
+        torch.cuda.synchronize()
+        for k, x in enumerate(xs):
+            rows, cols = shapes[k]
+            what = f"ragged group N={block} fmt={fmt} g={gmode} tensor {k} {shapes[k]}"
+            xo = inputs.to_oracle(x)
+            if gmode == "device":
+                assert gs[k] == oracle.global_scale(xo, fmt), what
+            po, so = oracle.quantize(xo, rows, cols, block, fmt, gs[k])
+            assert_same(u8(p[k]), po, what + " packed")
+            assert_same(u8(s[k]), so, what + " scales")
+            assert_same(u8(p2[k]), po, what + " fused packed")
+            assert_same(u8(s2[k]), so, what + " fused scales")
+            yo = oracle.dequantize(po, so, rows, cols, block, fmt, gs[k], out_bf16=True)
+            assert_same(bits(y[k]), yo, what + " dequant")
+            ref = oracle.error_stats(xo, rows, cols, block, fmt, gs[k], packed=po, scales=so)
+            assert_stats(st[k].to_dict(), ref, what + " stats")
