@@ -12,8 +12,11 @@
 // (e2m1_scaled_bits_at), not with a conversion instruction.
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "mx_device.cuh"
 #include "mx_launch.h"
+#include "mx_tma.cuh"
 
 namespace mxk {
 
@@ -219,6 +222,177 @@ static cudaError_t dq_block(int block, const TensorArgs* t, int count, cudaStrea
     case 128: return launch_dq<128, FMT, BF16OUT>(t, count, st, n);
     default: return launch_dq<256, FMT, BF16OUT>(t, count, st, n);
   }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Row tiles written by TMA: bf16 output whose rows start on 16-byte boundaries (cols % 8 == 0),
+// any cols otherwise (mx_tma.cuh)
+// ------------------------------------------------------------------------------------------------
+// Each warp walks tiles of 4 rows x 256 columns of y (a stride of all the grid's warps).  A lane
+// takes one 32-element slice of one row (tma::tile_lane): it loads the slice's 16 code bytes as
+// four 4-byte words (a row's code bytes start on a 4-byte boundary; register word c is word c ^ rot
+// of the slice) and its scale byte(s), the next tile's before the current tile's arithmetic;
+// decodes them (E2M1x2 -> f16x2 conversion, times S g from a per-CTA table: exact; bf16 = its round
+// to nearest even) into the warp's shared-memory copy of the tile (chunk c ^ rot at step c: eight
+// bank groups per row); then lane 0 writes the tile with a 2-D tensor store, which leaves out the
+// part of the box past the tensor's last row or column -- so a ragged last block needs nothing
+// special.  Each warp alternates two tile buffers; a buffer is rewritten only after its previous
+// store has finished reading it.  Warps never wait for one another.
+namespace dqtiles {
+constexpr int kBuffers = 2;
+constexpr int kSmem = 8 * kBuffers * tma::kTileBytes + 128;  // 8 warps' buffers + slack
+}  // namespace dqtiles
+
+struct TileDqArgs {
+  const uint8_t* packed;  // row pitch pb bytes
+  const uint8_t* scales;  // row pitch nb bytes
+  int rows, cols, pb, nb;
+  int ntc, ntr;  // tiles per row of tiles, rows of tiles
+  uint32_t g_bits;
+  const uint16_t* g_dev;
+};
+
+template <int N, int FMT>
+__global__ void __launch_bounds__(kThreads)
+    k_tile_dequantize(const __grid_constant__ CUtensorMap ymap, const __grid_constant__ TileDqArgs a) {
+  static_assert(N >= 16, "blocks of 16 and more");
+  constexpr int BPL = N == 16 ? 2 : 1;  // blocks in a lane's slice
+  extern __shared__ uint8_t tdq_smem_raw[];
+  uint8_t* bufs = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(tdq_smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ float s_D[256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float g = fp16_bits_to_float(tensor_g_bits(a.g_bits, a.g_dev));
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) s_D[c] = __fmul_rn(scale_value(c, FMT), g);
+  __syncthreads();
+  griddep_wait();  // codes and scales may come from the previous kernel in the stream
+  griddep_launch_next();
+
+  const tma::TileLane tl = tma::tile_lane();
+  uint8_t* wbuf = bufs + warp * (dqtiles::kBuffers * tma::kTileBytes);
+  struct Slice {
+    uint32_t cw[4];  // register word c: code word c ^ rot of the slice
+    uint32_t sc;     // scale byte(s): byte b = register block b
+    int nvalid;
+  };
+  auto load = [&](const tma::TileCursor& at) {
+    Slice v{{0u, 0u, 0u, 0u}, 0u, 0};
+    if (at.tr >= a.ntr) return v;
+    const int row = at.tr * tma::kTileRows + tl.row;
+    const int col0 = at.tc * tma::kTileCols + tl.slice * 32;
+    v.nvalid = row < a.rows ? max(0, min(32, a.cols - col0)) : 0;  // a multiple of 8
+    if (v.nvalid == 0) return v;
+    const uint8_t* prow = a.packed + (int64_t)row * a.pb + (col0 >> 1);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int cc = c ^ tl.rot;
+      if (8 * cc < v.nvalid) v.cw[c] = __ldcs(reinterpret_cast<const unsigned int*>(prow + 4 * cc));
+    }
+    const uint8_t* srow = a.scales + (int64_t)row * a.nb;
+    if constexpr (BPL == 2) {
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int bb = b ^ (tl.rot >> 1);  // register block b is block bb of the slice
+        if (16 * bb < v.nvalid) v.sc |= (uint32_t)__ldg(srow + col0 / 16 + bb) << (8 * b);
+      }
+    } else {
+      v.sc = __ldg(srow + col0 / N);
+    }
+    return v;
+  };
+
+  const int64_t gwarp = (int64_t)blockIdx.x * 8 + warp, nwarps = (int64_t)gridDim.x * 8;
+  tma::TileCursor at, ahead;  // the current tile and the next one
+  at.init(gwarp, nwarps, a.ntc);
+  ahead = at;
+  ahead.advance();
+  Slice cur = load(at);
+  for (int k = 0; at.tr < a.ntr; ++k, at = ahead, ahead.advance()) {
+    const Slice nxt = load(ahead);
+    uint4 out[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t hv[4];
+      e2m1x8_to_f16x2(cur.cw[c], hv);
+      const float D = s_D[(cur.sc >> (8 * (BPL == 2 ? c / 2 : 0))) & 0xFF];
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&hv[h]));
+        const float2 y2 = __fmul2_rn(v, make_float2(D, D));  // exact
+        o[h] = pack_bf16x2(y2.x, y2.y);
+      }
+      out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    uint8_t* buf = wbuf + (k % dqtiles::kBuffers) * tma::kTileBytes;
+    if (lane == 0) tma::store_wait_read<dqtiles::kBuffers - 1>();  // the buffer's last store
+    __syncwarp();
+    if (cur.nvalid > 0) {
+      uint8_t* dst = buf + tl.off;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(dst + 16 * (c ^ tl.rot)) = out[c];
+    }
+    tma::fence_smem_to_async();  // the writes come before the store reads them
+    __syncwarp();
+    if (lane == 0) {
+      tma::store_2d(&ymap, at.tc * tma::kTileCols, at.tr * tma::kTileRows, tma::smem_addr(buf));
+      tma::store_commit();
+    }
+    cur = nxt;
+  }
+  if (lane == 0) tma::store_wait_all();
+}
+
+// Row-tile dequantize (k_tile_dequantize) of one tensor with bf16 output, cols % 8 == 0, N >= 16.
+template <int N, int FMT>
+static cudaError_t launch_tile_dq(const uint8_t* packed, const uint8_t* scales, int64_t rows,
+                                  int64_t cols, uint16_t g_bits, const uint16_t* g_dev, void* y,
+                                  cudaStream_t stream, int* launches) {
+  static std::atomic<bool> smem_ok[kMaxDevices];
+  auto kern = k_tile_dequantize<N, FMT>;
+  CUtensorMap map;
+  if (!tma::map_row_tiles(&map, y, rows, cols, 2)) return cudaErrorInvalidValue;
+  cudaError_t e = allow_dynamic_smem(smem_ok, kern, dqtiles::kSmem);
+  if (e != cudaSuccess) return e;
+  const int ntc = (int)((cols + tma::kTileCols - 1) / tma::kTileCols);
+  const int ntr = (int)((rows + tma::kTileRows - 1) / tma::kTileRows);
+  int64_t grid = resident_ctas_smem((const void*)kern, dqtiles::kSmem);
+  const int64_t need = ((int64_t)ntc * ntr + 7) / 8;  // one tile per warp at least
+  if (grid > need) grid = need;
+  const TileDqArgs args{packed, scales, (int)rows, (int)cols, (int)((cols + 1) / 2),
+                        (int)((cols + N - 1) / N), ntc, ntr, g_bits, g_dev};
+  e = launch_pdl_smem(kern, (int)grid, kThreads, dqtiles::kSmem, stream, map, args);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+template <int FMT>
+static cudaError_t tile_dq_block(int block, const uint8_t* packed, const uint8_t* scales,
+                                 int64_t rows, int64_t cols, uint16_t g_bits,
+                                 const uint16_t* g_dev, void* y, cudaStream_t st, int* n) {
+  switch (block) {
+    case 16: return launch_tile_dq<16, FMT>(packed, scales, rows, cols, g_bits, g_dev, y, st, n);
+    case 32: return launch_tile_dq<32, FMT>(packed, scales, rows, cols, g_bits, g_dev, y, st, n);
+    case 64: return launch_tile_dq<64, FMT>(packed, scales, rows, cols, g_bits, g_dev, y, st, n);
+    case 128: return launch_tile_dq<128, FMT>(packed, scales, rows, cols, g_bits, g_dev, y, st, n);
+    default: return launch_tile_dq<256, FMT>(packed, scales, rows, cols, g_bits, g_dev, y, st, n);
+  }
+}
+
+bool tile_dequantize_supported(bool y_bf16, int64_t rows, int64_t cols, int block) {
+  return y_bf16 && block >= 16 && cols % 8 == 0 && rows >= 1 && rows <= 0x7FFFFFFF &&
+         cols <= 0x7FFFFFFF;
+}
+
+cudaError_t run_tile_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
+                                int64_t cols, int block, int fmt, uint16_t g_bits,
+                                const uint16_t* g_dev, void* y, cudaStream_t stream,
+                                int* launches) {
+  return fmt == kUE5M3
+             ? tile_dq_block<kUE5M3>(block, packed, scales, rows, cols, g_bits, g_dev, y, stream,
+                                     launches)
+             : tile_dq_block<kE4M3>(block, packed, scales, rows, cols, g_bits, g_dev, y, stream,
+                                    launches);
 }
 
 cudaError_t run_dequantize_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,

@@ -157,6 +157,29 @@ __device__ __forceinline__ uint16_t tensor_g_bits(uint32_t g_bits, const uint16_
   return __ldcg(g_dev);
 }
 
+// Row and item of a linear item index in a space of rows x ipr items (a row-pitched tensor seen as
+// whole items per row), moved on by a fixed stride without a division per step: the stride is
+// split once into whole rows and an item step.
+struct RowCursor {
+  int64_t row, j;  // current row and item within the row
+  int64_t dr, dj, ipr;
+  __device__ __forceinline__ void init(int64_t i, int64_t stride, int64_t items_per_row) {
+    ipr = items_per_row;
+    row = i / ipr;
+    j = i - row * ipr;
+    dr = stride / ipr;
+    dj = stride - dr * ipr;
+  }
+  __device__ __forceinline__ void advance() {
+    j += dj;
+    row += dr;
+    if (j >= ipr) {
+      j -= ipr;
+      ++row;
+    }
+  }
+};
+
 // Streaming 16-byte load of read-only data (not kept in L1).
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;

@@ -125,6 +125,10 @@ struct STensor {
   int64_t nitems, numel, nblocks;
   uint32_t g_bits;
   const uint16_t* g_dev;   // g in device memory (written by the previous kernel) when set
+  // Row-pitched mode (rows whose length cols the block size does not divide): ipr items per row,
+  // the row's blocks rounded up to whole items (the last ones hold zeros past the row's end); row
+  // pitches of x (cols elements), codes (pb bytes) and scales (nb bytes).
+  int64_t cols, ipr, pb, nb;
 };
 struct SGroup {
   STensor t[kMaxGroup];
@@ -541,13 +545,15 @@ __device__ __forceinline__ void slice_finish_bf16(Acc& acc, int lane, bool ok, f
 // SSE_max and the rest stays in SSE_elem (other max-valued elements included, as they should).
 // The subtraction only loses digits when dmax^2 dominates the slice's sum; a slice whose remainder
 // is below dmax^2 / 8, or whose sum is below 2^-80 (squares below 2^-126 could be lost), is redone
-// exactly in double.  has_max: this lane holds a max-valued element.
+// exactly in double -- unless every element of the slice is zero (lane_zero: zeros of a block's
+// padding past a row's end, or of an all-zero block), whose errors are exactly zero.  has_max:
+// this lane holds a max-valued element.
 template <int NE, int L, typename XF, typename CF>
 __device__ __forceinline__ void slice_finish_closed(Acc& acc, int lane, bool ok, bool has_max,
-                                                    float a, float D, float sat_thr,
-                                                    const SliceSetup& st, float2 lt2,
-                                                    float dmax, uint32_t nsat2, XF xval,
-                                                    CF code) {
+                                                    bool lane_zero, float a, float D,
+                                                    float sat_thr, const SliceSetup& st,
+                                                    float2 lt2, float dmax, uint32_t nsat2,
+                                                    XF xval, CF code) {
   bool is_first_lane = has_max;
   if constexpr (L > 1) {
     const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
@@ -556,7 +562,7 @@ __device__ __forceinline__ void slice_finish_closed(Acc& acc, int lane, bool ok,
   }
   const float lt = __fadd_rn(lt2.x, lt2.y);
   double rest = 0.0, first = 0.0, others = 0.0;
-  bool exact = lt < 0x1p-80f;
+  bool exact = lt < 0x1p-80f && !lane_zero;
   if (!exact) {
     rest = (double)lt * unscale_sq(st.E);
     if (is_first_lane && !st.zero_blk) {
@@ -637,9 +643,17 @@ struct StatsItem {
   uint32_t w[NW];
   uint32_t cw[NCW];
   uint32_t scw;
+  int64_t row, j;  // row-pitched mode: the item's row and its item index in the row
+  int nval;        // row-pitched mode: its elements inside the row (a multiple of 8; <= 0: none)
 };
 
-template <int N, int FMT, int MODE>
+// ROWS: the row-pitched mode (STensor) for rows of cols % 8 == 0 elements that the block size
+// N >= 32 does not divide (recomputed codes): item i of the padded item space is item j of row
+// i / ipr (a RowCursor that follows the loads, no division per item); x at row * cols + 32 j
+// (16-byte aligned), codes at row * pb + 16 j as 4-byte words, scales at row * nb; an item's
+// 8-element chunks past the row's end are neither read (zeros: they change neither the block
+// maximum nor the sums) nor written.
+template <int N, int FMT, int MODE, bool ROWS = false>
 __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MINB)
     k_error_stats_bf16(
     const __grid_constant__ SGroup grp) {
@@ -662,6 +676,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
   constexpr int BE = 2 * BW;    // elements per block inside an item
   using Item = StatsItem<NW, NCW>;
   static_assert(NCW == 1 || NCW == 2 || NCW == 4, "items of 8, 16 or 32 elements");
+  static_assert(!ROWS || (RECOMPUTE && BPI == 1 && NCW == 4), "row-pitched mode: N >= 32");
   __shared__ float s_rcp[256], s_D[256];
   const float g = fp16_bits_to_float(g_bits);
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
@@ -681,13 +696,29 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = tid - lane;
 
+  RowCursor lc;  // ROWS: row and item of the next item loaded (loads go tid, tid + T, ...)
+  if constexpr (ROWS) lc.init(tid, T, wk.t.ipr);
+
   // Loads of one item (zeros past the end).  Issued one item ahead of the arithmetic.
   auto load = [&](Item& it, int64_t i) {
-    const bool ok = i < nitems;
+    bool ok = i < nitems;
+    int64_t off = 0;
+    if constexpr (ROWS) {
+      it.row = lc.row;
+      it.j = lc.j;
+      it.nval = (int)min((int64_t)EPT, wk.t.cols - lc.j * EPT);
+      off = lc.row * wk.t.cols + lc.j * EPT;
+      ok = ok && it.nval > 0;
+      lc.advance();
+    }
 #pragma unroll
     for (int h = 0; h < NW / 4; ++h) {
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (ok) v = ld_stream16(x + i * EPT + h * 8);
+      if constexpr (ROWS) {
+        if (ok && 8 * h < it.nval) v = ld_stream16(x + off + h * 8);
+      } else {
+        if (ok) v = ld_stream16(x + i * EPT + h * 8);
+      }
       it.w[4 * h + 0] = v.x; it.w[4 * h + 1] = v.y; it.w[4 * h + 2] = v.z; it.w[4 * h + 3] = v.w;
     }
     it.scw = 0;
@@ -712,10 +743,12 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
   };
 
   auto process = [&](Item& it, int64_t i) {
-    const bool ok = i < nitems;
+    bool ok = i < nitems;
+    if constexpr (ROWS) ok = ok && it.nval > 0;
     float a_b[BPI], D_b[BPI], r_b[BPI];
     uint32_t m_b[BPI];
     bool own_b[BPI];      // this lane holds a max-valued element of block b
+    bool zero_b[BPI];     // this lane's elements of block b are all zero
     uint32_t sc_all = 0;  // scale codes of the item's blocks, byte b = block b
 #pragma unroll
     for (int b = 0; b < BPI; ++b) {
@@ -739,6 +772,7 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       a_b[b] = a;
       m_b[b] = m;
       own_b[b] = m_lane == m;
+      zero_b[b] = m_lane == 0;
       D_b[b] = s_D[s];
       sc_all |= s << (8 * b);
     }
@@ -771,7 +805,16 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
           it.cw[j] = qs_word8<4, kDeep>(&it.w[4 * j], &r_b[0], &st0.nDq, &S2, st0.sc, &lt0, nsat0);
       }
     }
-    if constexpr (STORE) {
+    if constexpr (STORE && ROWS) {
+      if (ok) {
+        uint8_t* prow = packed_out + it.row * wk.t.pb + it.j * 16;
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          if (8 * h < it.nval) *reinterpret_cast<uint32_t*>(prow + 4 * h) = it.cw[h];
+        if ((lane & (L - 1)) == 0)
+          scales_out[it.row * wk.t.nb + (it.j * EPT) / N] = (uint8_t)sc_all;
+      }
+    } else if constexpr (STORE) {
       if (ok) {
         if constexpr (NCW == 4)
           *reinterpret_cast<uint4*>(packed_out + i * 16) =
@@ -823,7 +866,8 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
       };
       auto code = [&](int k) { return it.cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
       if constexpr (CLOSED)
-        slice_finish_closed<BE, L>(acc, lane, ok, own_b[b], a, D, sat_thr, st, lt0, dmax, nsat0,
+        slice_finish_closed<BE, L>(acc, lane, ok, own_b[b], zero_b[b], a, D, sat_thr, st, lt0,
+                                   dmax, nsat0,
                                    xval, code);
       else
         slice_finish_bf16<BE, L, RECOMPUTE, false>(acc, lane, ok, a, D, sat_thr, st, lt, ms, dmax,
@@ -1500,6 +1544,61 @@ static cudaError_t stats_mode(StatsMode mode, int block, const TensorArgs* t, in
     case kRecompute: return stats_block<FMT, T, kRecompute>(block, t, count, ws, st, n);
     default: return stats_block<FMT, T, kStore>(block, t, count, ws, st, n);
   }
+}
+
+// Row-pitched mode of k_error_stats_bf16 over one bf16 tensor (rows whose length the block size
+// N >= 32 does not divide, cols % 8 == 0), recomputed codes, stored (STORE) or not.
+template <int N, int FMT, bool STORE>
+static cudaError_t launch_stats_rows(const void* x, int64_t rows, int64_t cols, uint16_t g_bits,
+                                     const uint16_t* g_dev, uint8_t* packed, uint8_t* scales,
+                                     void* out, Workspace ws, cudaStream_t stream,
+                                     int* launches) {
+  constexpr int MODE = STORE ? kStore : kRecompute;
+  using S = SShape<N, uint16_t>;
+  static_assert(N >= S::EPT, "whole items per block");
+  const int64_t nb = (cols + N - 1) / N, ipr = nb * (N / S::EPT);
+  const int64_t nitems = rows * ipr;
+  SGroup grp = {};
+  grp.t[0] = {x, nullptr, nullptr, STORE ? packed : nullptr, STORE ? scales : nullptr, ws.part,
+              ws.counter(0), static_cast<StatsOut*>(out), nitems, rows * cols, rows * nb,
+              g_bits, g_dev, cols, ipr, (cols + 1) / 2, nb};
+  const int grid = split_grid((const void*)k_error_stats_bf16<N, FMT, MODE, true>, &nitems, 1,
+                              S::U, kMaxStatsGrid, &grp.split);
+  cudaError_t e = launch_pdl(k_stats_reset, 1, 32, stream, ws.counters, 1);
+  if (e != cudaSuccess) return e;
+  ++*launches;
+  e = launch_pdl(k_error_stats_bf16<N, FMT, MODE, true>, grid, kThreads, stream, grp);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+template <int FMT, bool STORE>
+static cudaError_t stats_rows_block(int block, const void* x, int64_t rows, int64_t cols,
+                                    uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                                    uint8_t* scales, void* out, Workspace ws, cudaStream_t st,
+                                    int* n) {
+  switch (block) {
+    case 32: return launch_stats_rows<32, FMT, STORE>(x, rows, cols, g_bits, g_dev, packed, scales, out, ws, st, n);
+    case 64: return launch_stats_rows<64, FMT, STORE>(x, rows, cols, g_bits, g_dev, packed, scales, out, ws, st, n);
+    case 128: return launch_stats_rows<128, FMT, STORE>(x, rows, cols, g_bits, g_dev, packed, scales, out, ws, st, n);
+    default: return launch_stats_rows<256, FMT, STORE>(x, rows, cols, g_bits, g_dev, packed, scales, out, ws, st, n);
+  }
+}
+
+bool rows_stats_supported(bool bf16, int64_t rows, int64_t cols, int block) {
+  return bf16 && block >= 32 && cols % 8 == 0 && rows >= 1;
+}
+
+cudaError_t run_rows_stats(const void* x, int64_t rows, int64_t cols, int block, int fmt,
+                           uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                           uint8_t* scales, void* out, void* workspace, cudaStream_t stream,
+                           int* launches) {
+  const Workspace ws(workspace);
+  if (packed)
+    return fmt == kUE5M3 ? stats_rows_block<kUE5M3, true>(block, x, rows, cols, g_bits, g_dev, packed, scales, out, ws, stream, launches)
+                         : stats_rows_block<kE4M3, true>(block, x, rows, cols, g_bits, g_dev, packed, scales, out, ws, stream, launches);
+  return fmt == kUE5M3 ? stats_rows_block<kUE5M3, false>(block, x, rows, cols, g_bits, g_dev, nullptr, nullptr, out, ws, stream, launches)
+                       : stats_rows_block<kE4M3, false>(block, x, rows, cols, g_bits, g_dev, nullptr, nullptr, out, ws, stream, launches);
 }
 
 cudaError_t run_stats_group(const TensorArgs* t, int count, bool bf16, int block, int fmt,

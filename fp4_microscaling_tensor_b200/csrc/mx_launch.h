@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace mxk {
 
 // Upper bound on the CTAs of any reduction kernel; sizes the workspaces.
@@ -27,14 +29,33 @@ struct CtaSplit {
 #endif
 };
 
-// Resident CTAs of 256 threads on the whole device for `kern` (SMs x occupancy).
-inline int64_t resident_ctas(const void* kern) {
+// Resident CTAs of 256 threads on the whole device for `kern` (SMs x occupancy), with `smem`
+// bytes of dynamic shared memory per CTA.
+inline int64_t resident_ctas_smem(const void* kern, int smem) {
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
   if (per_sm < 1) per_sm = 1;
   return (int64_t)sms * per_sm;
+}
+inline int64_t resident_ctas(const void* kern) { return resident_ctas_smem(kern, 0); }
+
+// Dynamic shared memory above 48 KiB must be enabled per kernel and per device: flags[dev] (one
+// array per kernel) is set once the attribute call has succeeded on that device; a failed call is
+// retried on the next launch.
+constexpr int kMaxDevices = 64;
+template <typename K>
+inline cudaError_t allow_dynamic_smem(std::atomic<bool>* flags, K* kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && flags[dev].load(std::memory_order_acquire))
+    return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices)
+    flags[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 // Persistent grid for a grid-stride kernel with kThreads threads: enough CTAs to fill every SM
@@ -95,12 +116,12 @@ inline int split_grid(const void* kern, const int64_t* nitems, int count, int it
 // previous grid has completed and its writes are visible; so ordering is as for a plain launch and
 // only the launch latency and the shared-memory setup overlap the previous kernel's tail.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t stream,
-                              Args... args) {
+inline cudaError_t launch_pdl_smem(void (*kern)(KArgs...), int grid, int block, size_t smem,
+                                   cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3((unsigned)block);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -108,6 +129,11 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaS
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t stream,
+                              Args... args) {
+  return launch_pdl_smem(kern, grid, block, 0, stream, args...);
 }
 
 // One tensor of a grouped call (all pointers device memory; numel = rows * cols).
@@ -185,6 +211,29 @@ cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, 
                                   int64_t cols, int block, int fmt, uint16_t g_bits,
                                   const uint16_t* g_dev, void* y, bool y_bf16,
                                   cudaStream_t stream, int* launches);
+
+// Row-pitched modes of the whole-block kernels: bf16 tensors whose rows start on 16-byte
+// boundaries (cols % 8 == 0) and whose length the block size does not divide; one tensor per
+// launch.  Quantize (N >= 16): codes and scales (y null), or the round trip to y (bf16 or fp32;
+// packed / scales unused).
+bool rows_quantize_supported(bool bf16, int64_t rows, int64_t cols, int block);
+cudaError_t run_rows_quantize(const void* x, int64_t rows, int64_t cols, int block, int fmt,
+                              uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                              uint8_t* scales, void* y, bool y_bf16, cudaStream_t stream,
+                              int* launches);
+// The error reduction with recomputed codes (N >= 32), fused with quantize + pack when packed /
+// scales are set; out: device mx_error_stats_t; workspace as for the error reduction.
+bool rows_stats_supported(bool bf16, int64_t rows, int64_t cols, int block);
+cudaError_t run_rows_stats(const void* x, int64_t rows, int64_t cols, int block, int fmt,
+                           uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                           uint8_t* scales, void* out, void* workspace, cudaStream_t stream,
+                           int* launches);
+// Dequantize to bf16 (N >= 16) through row tiles written by TMA (mx_tma.cuh).
+bool tile_dequantize_supported(bool y_bf16, int64_t rows, int64_t cols, int block);
+cudaError_t run_tile_dequantize(const uint8_t* packed, const uint8_t* scales, int64_t rows,
+                                int64_t cols, int block, int fmt, uint16_t g_bits,
+                                const uint16_t* g_dev, void* y, cudaStream_t stream,
+                                int* launches);
 
 // Zeroes one last-CTA counter once the previous kernel in the stream is done with it (a one-thread
 // kernel launched with programmatic serialization).

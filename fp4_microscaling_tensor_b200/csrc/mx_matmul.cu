@@ -1071,24 +1071,10 @@ bool make_bf16_map(CUtensorMap* map, const void* a, int64_t m, int64_t k) {
 
 int64_t mma_scales_bytes(int64_t rows, int64_t k);
 
-// Dynamic shared memory above 48 KiB must be enabled per kernel and per device; the flag of a
-// device is set once the attribute call has succeeded there (a failed call is retried next time).
-constexpr int kMaxDevices = 64;
+// Dynamic shared memory above 48 KiB is enabled per kernel and per device (allow_dynamic_smem).
 static std::atomic<bool> g_smem_one[kMaxDevices], g_smem_pair[kMaxDevices];
 static std::atomic<unsigned int> g_launch_gen{0};
 
-template <typename K>
-static cudaError_t allow_smem(std::atomic<bool>* flags, K* kern, int bytes) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kMaxDevices && flags[dev].load(std::memory_order_acquire))
-    return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices)
-    flags[dev].store(true, std::memory_order_release);
-  return e;
-}
 
 // A new generation number for a launch (never 0, the flag's initial value).
 static unsigned int next_gen() {
@@ -1105,7 +1091,7 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
   CUtensorMap ma, mb;
   if (m > kBM && cta_pairs) {
     // CTA pairs: 256 x 256 tiles of C
-    cudaError_t e = allow_smem(g_smem_pair, k_matmul_nvfp4_pair, Pair::kSmemBytes);
+    cudaError_t e = allow_dynamic_smem(g_smem_pair, k_matmul_nvfp4_pair, Pair::kSmemBytes);
     if (e != cudaSuccess) return e;
     CUtensorMap msa, msb;
     if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, kBM) ||
@@ -1119,7 +1105,7 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
     constexpr int BN = MX_MM_BN;
     static_assert(BN == 128 || BN == 256, "tile width");
     using T = Tile<BN>;
-    cudaError_t e = allow_smem(g_smem_one, k_matmul_nvfp4<BN>, T::kSmemBytes);
+    cudaError_t e = allow_dynamic_smem(g_smem_one, k_matmul_nvfp4<BN>, T::kSmemBytes);
     if (e != cudaSuccess) return e;
     if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, BN))
       return cudaErrorInvalidValue;
@@ -1134,7 +1120,7 @@ template <int N, int FMT>
 static cudaError_t launch_dqmm(const CUtensorMap& ma, const CUtensorMap& mw, const DqArgs& args,
                                cudaStream_t stream) {
   static std::atomic<bool> attr[kMaxDevices];
-  const cudaError_t e = allow_smem(attr, k_dequant_matmul<N, FMT>, dqmm::kSmemBytes);
+  const cudaError_t e = allow_dynamic_smem(attr, k_dequant_matmul<N, FMT>, dqmm::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((args.n + dqmm::kBN - 1) / dqmm::kBN) * ((args.m + 255) / 256);
   if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidConfiguration;

@@ -46,6 +46,10 @@ struct QTensor {
   int64_t nitems;
   uint32_t g_bits;
   const uint16_t* g_dev;  // g in device memory (written by the previous kernel) when set
+  // Row-pitched mode (rows whose length cols the block size does not divide): ipr items per row,
+  // the row's blocks rounded up to whole items (the last ones hold zeros past the row's end);
+  // row pitches of x / y (cols elements), codes (pb bytes) and scales (nb bytes).
+  int64_t cols, ipr, pb, nb;
 };
 
 // What a quantize kernel writes: codes and scales, or (the fake-quantize round trip) the
@@ -115,10 +119,16 @@ __device__ __forceinline__ uint32_t absmax_bits(const uint32_t* w) {
   return max(t & 0xFFFFu, t >> 16);
 }
 
-template <int N, int FMT, int OUT = kCodes>
+// ROWS: the row-pitched mode (QTensor) for rows of cols % 8 == 0 elements that the block size does
+// not divide: item i of the padded item space is item j of row i / ipr (a RowCursor per item in
+// flight, no division per item); x and the round trip at row * cols + j * EPT (16-byte aligned),
+// codes at row * pb + j * EPT / 2 as 4-byte words, scales at row * nb; an item's 8-element chunks
+// past the row's end are neither read (zeros: they do not change the block maximum) nor written.
+template <int N, int FMT, int OUT = kCodes, bool ROWS = false>
 __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constant__ QGroup grp) {
   using S = QShape<N, uint16_t>;
   constexpr int EPT = S::EPT, L = S::L, BPI = S::BPI, U = S::U, NW = EPT / 2;
+  static_assert(!ROWS || (N >= 16 && BPI == 1), "row-pitched mode: blocks of 16 and more");
   const QWork wk = q_work(grp);
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(wk.t.x);
   uint8_t* __restrict__ packed = wk.t.packed;
@@ -141,18 +151,34 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
   const int64_t tid = (int64_t)wk.cta * blockDim.x + threadIdx.x;
   const int64_t warp0 = tid - (threadIdx.x & 31);
   const int lane = threadIdx.x & 31;
+  RowCursor rc[U];  // ROWS: row and item of each item in flight
+  if constexpr (ROWS) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) rc[u].init(tid + (int64_t)u * T, T * U, wk.t.ipr);
+  }
 
   for (int64_t base = 0; warp0 + base < nitems; base += T * U) {
     uint32_t w[U][NW];
     bool ok[U];
+    int nval[U];      // ROWS: elements of the item inside its row (a multiple of 8; <= 0: none)
+    int64_t off[U];   // ROWS: the item's first element in x
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t i = tid + base + (int64_t)u * T;
       ok[u] = i < nitems;
+      if constexpr (ROWS) {
+        nval[u] = (int)min((int64_t)EPT, wk.t.cols - rc[u].j * EPT);
+        off[u] = rc[u].row * wk.t.cols + rc[u].j * EPT;
+        ok[u] = ok[u] && nval[u] > 0;
+      }
 #pragma unroll
       for (int h = 0; h < NW / 4; ++h) {
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (ok[u]) v = ld_stream16(x + i * EPT + h * 8);
+        if constexpr (ROWS) {
+          if (ok[u] && 8 * h < nval[u]) v = ld_stream16(x + off[u] + h * 8);
+        } else {
+          if (ok[u]) v = ld_stream16(x + i * EPT + h * 8);
+        }
         w[u][4 * h + 0] = v.x;
         w[u][4 * h + 1] = v.y;
         w[u][4 * h + 2] = v.z;
@@ -188,6 +214,38 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
         codes[j] = cvt_e2m1x8(qv[8 * j], qv[8 * j + 1], qv[8 * j + 2], qv[8 * j + 3], qv[8 * j + 4],
                               qv[8 * j + 5], qv[8 * j + 6], qv[8 * j + 7]);
       if (!ok[u]) continue;
+      if constexpr (ROWS) {
+        const int64_t row = rc[u].row, j = rc[u].j;
+        if constexpr (OUT != kCodes) {
+          const float D = s_D[sc & 0xFF];
+#pragma unroll
+          for (int h = 0; h < EPT / 8; ++h) {
+            if (8 * h >= nval[u]) continue;
+            float out[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              out[e] = __fmul_rn(__fmul_rn(__uint_as_float(e2m1_scaled_bits_at(codes[h], 4 * e)),
+                                           0x1p126f),
+                                 D);  // exact
+            if constexpr (OUT == kRoundTripBf16) {
+              __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(wk.t.y) + off[u] + 8 * h),
+                     make_uint4(pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
+                                pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7])));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(wk.t.y) + off[u] + 8 * h);
+              __stcs(dst, make_float4(out[0], out[1], out[2], out[3]));
+              __stcs(dst + 1, make_float4(out[4], out[5], out[6], out[7]));
+            }
+          }
+        } else {
+          uint8_t* prow = packed + row * wk.t.pb + j * (EPT / 2);
+#pragma unroll
+          for (int h = 0; h < EPT / 8; ++h)
+            if (8 * h < nval[u]) *reinterpret_cast<uint32_t*>(prow + 4 * h) = codes[h];
+          if ((lane & (L - 1)) == 0) scales[row * wk.t.nb + (j * EPT) / N] = (uint8_t)sc;
+        }
+        continue;
+      }
       if constexpr (OUT != kCodes) {
         store_round_trip<EPT, BPI, OUT>(wk.t.y, i, codes, sc, s_D);
         continue;
@@ -202,6 +260,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize_bf16(const __grid_constan
       } else {
         *reinterpret_cast<uint16_t*>(scales + i * 2) = (uint16_t)sc;
       }
+    }
+    if constexpr (ROWS) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) rc[u].advance();
     }
   }
 }
@@ -379,6 +441,65 @@ static cudaError_t dispatch_block(int block, const TensorArgs* t, int count, cud
     case 128: return launch_q<128, FMT, T, OUT>(t, count, st, n);
     default: return launch_q<256, FMT, T, OUT>(t, count, st, n);
   }
+}
+
+// Row-pitched mode of k_quantize_bf16 (rows whose length the block size N >= 16 does not divide,
+// cols % 8 == 0): one tensor per launch.
+template <int N, int FMT, int OUT>
+static cudaError_t launch_q_rows(const void* x, int64_t rows, int64_t cols, uint16_t g_bits,
+                                 const uint16_t* g_dev, uint8_t* packed, uint8_t* scales, void* y,
+                                 cudaStream_t stream, int* launches) {
+  using S = QShape<N, uint16_t>;
+  static_assert(N >= S::EPT, "whole items per block");
+  const int64_t nb = (cols + N - 1) / N, ipr = nb * (N / S::EPT);
+  const int64_t nitems = rows * ipr;
+  QGroup grp = {};
+  grp.t[0] = {x, packed, scales, y, nitems, g_bits, g_dev, cols, ipr, (cols + 1) / 2, nb};
+  const int grid = split_grid((const void*)k_quantize_bf16<N, FMT, OUT, true>, &nitems, 1, S::U,
+                              1 << 30, &grp.split);
+  if (grid == 0) return cudaSuccess;
+  const cudaError_t e = launch_pdl(k_quantize_bf16<N, FMT, OUT, true>, grid, kThreads, stream, grp);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+template <int FMT, int OUT>
+static cudaError_t q_rows_block(int block, const void* x, int64_t rows, int64_t cols,
+                                uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                                uint8_t* scales, void* y, cudaStream_t st, int* n) {
+  switch (block) {
+    case 16: return launch_q_rows<16, FMT, OUT>(x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+    case 32: return launch_q_rows<32, FMT, OUT>(x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+    case 64: return launch_q_rows<64, FMT, OUT>(x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+    case 128: return launch_q_rows<128, FMT, OUT>(x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+    default: return launch_q_rows<256, FMT, OUT>(x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+  }
+}
+
+template <int OUT>
+static cudaError_t q_rows_fmt(int fmt, int block, const void* x, int64_t rows, int64_t cols,
+                              uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                              uint8_t* scales, void* y, cudaStream_t st, int* n) {
+  return fmt == kUE5M3
+             ? q_rows_block<kUE5M3, OUT>(block, x, rows, cols, g_bits, g_dev, packed, scales, y, st, n)
+             : q_rows_block<kE4M3, OUT>(block, x, rows, cols, g_bits, g_dev, packed, scales, y, st, n);
+}
+
+bool rows_quantize_supported(bool bf16, int64_t rows, int64_t cols, int block) {
+  return bf16 && block >= 16 && cols % 8 == 0 && rows >= 1;
+}
+
+cudaError_t run_rows_quantize(const void* x, int64_t rows, int64_t cols, int block, int fmt,
+                              uint16_t g_bits, const uint16_t* g_dev, uint8_t* packed,
+                              uint8_t* scales, void* y, bool y_bf16, cudaStream_t stream,
+                              int* launches) {
+  if (!y)
+    return q_rows_fmt<kCodes>(fmt, block, x, rows, cols, g_bits, g_dev, packed, scales, nullptr,
+                              stream, launches);
+  return y_bf16 ? q_rows_fmt<kRoundTripBf16>(fmt, block, x, rows, cols, g_bits, g_dev, nullptr,
+                                             nullptr, y, stream, launches)
+                : q_rows_fmt<kRoundTripF32>(fmt, block, x, rows, cols, g_bits, g_dev, nullptr,
+                                            nullptr, y, stream, launches);
 }
 
 cudaError_t run_quantize_tail(const void* x, bool bf16, int64_t first, int count, int N, int fmt,

@@ -8,7 +8,11 @@
 // another.  For cols % N == 0 this is the layout of the whole-block kernels, which handle that
 // case; these kernels cover the rest.
 //
-// One warp per row, lanes over consecutive element pairs (coalesced loads and byte stores), block
+// bf16 tensors whose rows start on 16-byte boundaries (cols % 8 == 0) go to the row-pitched modes
+// of the whole-block kernels (quantize and fake quantize for N >= 16, the error reduction with
+// recomputed codes, fused or not, for N >= 32) and to the row-tile dequantize kernel (bf16 output,
+// N >= 16; tiles written by TMA, mx_tma.cuh).  The rest runs here:
+// one warp per row, lanes over consecutive element pairs (coalesced loads and byte stores), block
 // maxima by segmented warp reductions; scale s = RNE_fmt(a / (6 g)) and quotients x / (S g) by
 // IEEE division (a correctly rounded quotient lands on a rounding midpoint only when the exact
 // quotient does), E2M1 codes by the hardware RNE-saturating conversion.  Errors are formed and
@@ -383,6 +387,13 @@ cudaError_t run_ragged(const void* x, bool bf16, int64_t rows, int64_t cols, int
                        uint8_t* packed, uint8_t* scales, void* y, bool y_bf16, void* out,
                        void* workspace, cudaStream_t stream, int* launches) {
   if (cols > (int64_t(1) << 30)) return cudaErrorInvalidValue;  // in-row indices are 32-bit
+  // bf16 rows on 16-byte boundaries with recomputed codes: the row-pitched whole-block kernels
+  if (!packed_in && out && !y && rows_stats_supported(bf16, rows, cols, block))
+    return run_rows_stats(x, rows, cols, block, fmt, g_bits, g_dev, packed, scales, out, workspace,
+                          stream, launches);
+  if (!packed_in && !out && rows_quantize_supported(bf16, rows, cols, block))
+    return run_rows_quantize(x, rows, cols, block, fmt, g_bits, g_dev, packed, scales, y, y_bf16,
+                             stream, launches);
   RaggedArgs args{x, rows, cols, block, g_bits, g_dev, packed_in, scales_in, packed, scales, y,
                   y_bf16 ? 1 : 0, nullptr};
   if (out)  // partials after the workspace's 64-byte counter headers
@@ -399,6 +410,9 @@ cudaError_t run_ragged_dequantize(const uint8_t* packed, const uint8_t* scales, 
                                   int64_t cols, int block, int fmt, uint16_t g_bits,
                                   const uint16_t* g_dev, void* y,
                                   bool y_bf16, cudaStream_t stream, int* launches) {
+  if (tile_dequantize_supported(y_bf16, rows, cols, block))
+    return run_tile_dequantize(packed, scales, rows, cols, block, fmt, g_bits, g_dev, y, stream,
+                               launches);
   ++*launches;
   return fmt == kUE5M3
              ? launch_dq_fmt<kUE5M3>(packed, scales, rows, cols, block, g_bits, g_dev, y, y_bf16,

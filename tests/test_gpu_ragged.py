@@ -18,7 +18,12 @@ pytestmark = pytest.mark.gpu
 
 GUARD = 64
 SHAPES = [(5, 7, 4), (3, 13, 8), (17, 45, 32), (2, 300, 256), (9, 100, 64), (33, 129, 128),
-          (4, 3, 32), (7, 1, 4), (64, 1000, 16), (300, 33, 32)]
+          (4, 3, 32), (7, 1, 4), (64, 1000, 16), (300, 33, 32),
+          # rows on 16-byte boundaries (cols % 8 == 0), bf16: the row-pitched modes and the
+          # row-tile dequantize -- partial last tiles in both directions, a row shorter than one
+          # block, one-block tensors
+          (40, 8200, 32), (33, 520, 64), (65, 1000, 128), (31, 264, 256), (3, 24, 32),
+          (1, 8, 256), (70, 776, 16), (129, 2056, 32)]
 G_CASES = (0x3C00, 0x2E66)
 
 
@@ -87,6 +92,34 @@ def test_ragged_parity(rows, cols, block, fmt, dtype):
     guard_ok(s2buf, rows * nb, "fused scales")
 
 
+def test_ragged_aligned_rows_full_size():
+    # 8192 x 8200, N = 32, UE5M3 with the tensor's global scale (256 whole blocks and a block of 8
+    # per row; the row-pitched kernels and the row-tile dequantize): the error record of the whole tensor against the oracle,
+    # codes, scales and dequantized bits on 256 seeded rows (the first and last included)
+    rows, cols, block = 8192, 8200, 32
+    x = inputs.normal((rows, cols), 0.015, seed=8200).cuda()
+    xo = inputs.to_oracle(x)
+    g = oracle.global_scale(xo, mx.UE5M3)
+    p, s, st = mx.quantize_with_stats(x, block, "ue5m3", g)
+    y = mx.dequantize(p, s, block, "ue5m3", g, cols=cols)
+    yf = mx.fake_quantize(x, block, "ue5m3", g)
+    rec = mx.error_stats(x, block, "ue5m3", g).to_dict()
+    torch.cuda.synchronize()
+    ref = oracle.error_stats(xo, rows, cols, block, mx.UE5M3, g)
+    assert_stats(st.to_dict(), ref, "row tiles 8192x8200 fused")
+    assert_stats(rec, ref, "row tiles 8192x8200 recomputed")
+    sel = np.unique(np.concatenate([[0, rows - 1],
+                                    np.random.default_rng(8).choice(rows, 254, replace=False)]))
+    xs = xo.reshape(rows, cols)[sel].reshape(-1)
+    po, so = oracle.quantize(xs, len(sel), cols, block, mx.UE5M3, g)
+    idx = torch.from_numpy(sel).cuda()
+    assert_same(u8(p.view(rows, -1)[idx]), po, "row tiles sampled packed")
+    assert_same(u8(s.view(rows, -1)[idx]), so, "row tiles sampled scales")
+    yo = oracle.dequantize(po, so, len(sel), cols, block, mx.UE5M3, g, out_bf16=True)
+    assert_same(bits(y.view(rows, cols)[idx]), yo, "row tiles sampled dequant")
+    assert_same(bits(yf.view(rows, cols)[idx]), yo, "row tiles sampled fake quantize")
+
+
 def test_ragged_large_sampled_rows():
     # 4096 x 4100 (N = 32: 128 whole blocks and a block of 4 per row), N(0, 0.02^2): whole tensor
     # quantized on the GPU, 256 seeded rows compared with the oracle, the error record whole
@@ -111,7 +144,7 @@ def test_grouped_calls_take_ragged_tensors(cuda_device, block, fmt):
     scales, dequantized bits and error record equal the oracle's."""
     rng = np.random.default_rng(block + 5 * fmt)
     shapes = [(64, 2 * block), (33, 3 * block + 5), (7, block - 1 if block > 4 else 3),
-              (0, block + 1), (129, 8 * block), (5, 2 * block + 1)]
+              (0, block + 1), (129, 8 * block), (5, 2 * block + 1), (40, 3 * block + 8)]
     xs = []
     for r, c in shapes:
         x = rng.standard_normal((r, c)) * np.exp(rng.uniform(-3, 1, (r, 1)))
@@ -121,7 +154,7 @@ def test_grouped_calls_take_ragged_tensors(cuda_device, block, fmt):
             g = mx.global_scale_group(xs, fmt)
             gs = [int(v) for v in g.cpu().numpy().view(np.uint16)]
         else:
-            gs = [0x3C00, 0x3555, 0x2E66, 0x3C00, 0x4400, 0x0003][:len(xs)]
+            gs = [0x3C00, 0x3555, 0x2E66, 0x3C00, 0x4400, 0x0003, 0x3C00][:len(xs)]
             g = gs
         p, s = mx.quantize_group(xs, block, fmt, g=g)
         p2, s2, st = mx.quantize_with_stats_group(xs, block, fmt, g=g)
