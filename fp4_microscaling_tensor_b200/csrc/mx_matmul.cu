@@ -8,7 +8,10 @@
 // dequantized to memory.  A is m x k and B is n x k, both row-major with k contiguous ("K-major"),
 // which is the layout the quantizer writes; C is m x n row-major, float32 or bfloat16.
 //
-// One CTA per 128 x BN tile of C (BN = 256 by default, MMA N = BN), 4 warps:
+// One CTA per 128 x BN tile of C (MMA N = BN), 4 warps.  BN = 128 with 3 stages by default: the
+// CTA then needs 108 KiB of shared memory and 256 TMEM columns, so two CTAs share an SM and one
+// CTA's prologue and epilogue overlap the other's main loop (measured 3127 TFLOP/s at 8192^3
+// against 2830 for BN = 256, whose 216 KiB and 512 columns allow one CTA per SM):
 //   * warp 0, one thread, produces: for each 256-element step of k, one TMA load per operand
 //     (128 or BN rows x 128 bytes, 128-byte swizzle) and one bulk copy per 128-row tile of the
 //     step's scales, which mx_matmul_prepare_scales has already put into tensor-core order (2048
@@ -43,7 +46,11 @@ namespace {
 #define MX_MM_SFBUF 2  // for the previous step's MMAs to finish reading the same columns
 #endif
 #ifndef MX_MM_BN  // columns of C per CTA in the one-CTA kernel: 128 or 256 (MMA N)
-#define MX_MM_BN 256
+#define MX_MM_BN 128
+#endif
+#ifndef MX_MM_STAGES128  // pipeline stages of the one-CTA kernel with 128-column tiles: 3 keeps
+#define MX_MM_STAGES128 3  // two CTAs per SM (shared memory and TMEM), so that one CTA's epilogue
+                           // overlaps the other's main loop
 #endif
 
 constexpr int kBM = 128;              // rows of C per CTA (MMA M)
@@ -55,7 +62,7 @@ constexpr uint32_t kWaitLimit = 1u << 20;  // polls of one mbarrier before a CTA
 template <int BN>
 struct Tile {
   static constexpr int kHalves = BN / 128;                     // 128-row scale atoms of B per step
-  static constexpr int kStages = BN == 256 ? 4 : 5;
+  static constexpr int kStages = BN == 256 ? 4 : MX_MM_STAGES128;
   static constexpr int kABytes = kBM * kRowBytes;             // 16 KiB
   static constexpr int kBBytes = BN * kRowBytes;              // 16 or 32 KiB
   static constexpr int kSfaBytes = kBM * (kBK / 16);          // four 512-byte atoms
@@ -434,20 +441,32 @@ __global__ void __launch_bounds__(128, 1)
 // leader's full barrier, which expects the bytes of both; the leader commits its MMAs to its own
 // and to the peer's empty / done barriers with separate single-target commits.
 // ------------------------------------------------------------------------------------------------
-struct Pair {
-  static constexpr int kStages = MX_MM_PAIR_STAGES;
-  static constexpr int kABytes = kBM * kRowBytes;   // this CTA's 128 rows of A
-  static constexpr int kBBytes = kBM * kRowBytes;   // this CTA's 128 of the 256 B rows
-  static constexpr int kSfaBytes = 2048;            // A's scales, this CTA's rows
-  static constexpr int kSfbBytes = 4096;            // B's scales, all 256 rows
+// Geometry of the CTA-pair kernel: 256 x PN tiles of C, each CTA of the pair holding 128 rows of A
+// and PN / 2 rows of B per stage.  PN = 256: 5 stages, 512 TMEM columns, one CTA per SM; PN = 128:
+// 3 stages of 28 KiB and 256 TMEM columns, so two CTAs (of different pairs) share an SM.
+#ifndef MX_MM_PAIR_N
+#define MX_MM_PAIR_N 128
+#endif
+template <int PN>
+struct PairT {
+  static constexpr int kStages = PN == 256 ? MX_MM_PAIR_STAGES : 3;
+  static constexpr int kBRows = PN / 2;              // this CTA's rows of B
+  static constexpr int kGroups = PN / 128;           // 128-row scale groups of B
+  static constexpr int kABytes = kBM * kRowBytes;    // this CTA's 128 rows of A
+  static constexpr int kBBytes = kBRows * kRowBytes;
+  static constexpr int kSfaBytes = 2048;             // A's scales, this CTA's rows
+  static constexpr int kSfbBytes = 2048 * kGroups;   // B's scales, all PN rows
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
-  static constexpr uint32_t kTmemCols = 512, kSfaCol = 256, kSfbCol = 272, kSfCols = 48;
-  static_assert(256 + MX_MM_SFBUF * kSfCols <= kTmemCols, "TMEM columns");
-  // M = 256 (bits 24..28: 16), N = 256 (bits 17..22: 32), otherwise as the one-CTA descriptor
-  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (32u << 17) | (16u << 24);
+  static constexpr uint32_t kTmemCols = PN == 256 ? 512 : 256, kSfaCol = PN, kSfbCol = PN + 16,
+                            kSfCols = 16 + 16 * kGroups;
+  static_assert(PN + MX_MM_SFBUF * kSfCols <= kTmemCols, "TMEM columns");
+  // M = 256 (bits 24..28: 16), N = PN (bits 17..22: PN / 8), otherwise as the one-CTA descriptor
+  static constexpr uint32_t kIdesc =
+      (1u << 7) | (1u << 10) | ((uint32_t)(PN >> 3) << 17) | (16u << 24);
 };
+using Pair = PairT<MX_MM_PAIR_N>;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -516,10 +535,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int64_t pair = blockIdx.x >> 1, NT = (args.n + 255) / 256;
+  constexpr int PN = MX_MM_PAIR_N;
+  const int64_t pair = blockIdx.x >> 1, NT = (args.n + PN - 1) / PN;
   const int64_t mt = pair / NT, nt = pair - mt * NT;
   const int64_t m0 = mt * 256 + 128 * rank;  // this CTA's rows of A and of C
-  const int64_t n0 = nt * 256;               // the pair's columns of C
+  const int64_t n0 = nt * PN;                // the pair's columns of C
   const int KT = (int)(args.k / kBK);
 
   if (threadIdx.x == 0) {
@@ -562,11 +582,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
         if (rank == 0)
           mbar_expect_tx(smem_u32(full + s), 2 * (kABytes + kBBytes + kSfaBytes + kSfbBytes));
         tma2_load_2d(st, &tma_a, kt * kRowBytes, (int)m0, bar);
-        tma2_load_2d(st + kABytes, &tma_b, kt * kRowBytes, (int)(n0 + 128 * rank), bar);
+        tma2_load_2d(st + kABytes, &tma_b, kt * kRowBytes, (int)(n0 + P::kBRows * rank), bar);
         // scale groups: 2048 bytes = 8 rows of 256 in the scale maps
         tma2_load_2d(st + kABytes + kBBytes, &tma_sfa, 0, sfa_row + 8 * kt, bar);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < P::kGroups; ++h)
           tma2_load_2d(st + kABytes + kBBytes + kSfaBytes + 2048 * h, &tma_sfb, 0,
                        sfb_row + 8 * (h * KT + kt), bar);
         if (rank == 0) mbar_arrive(smem_u32(full + s));
@@ -597,13 +617,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
         for (int j = 0; j < 4; ++j) {
           tc2_copy_sf(tsf + P::kSfaCol + 4 * j, desc_sf(sfa + 512 * j));
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tc2_copy_sf(tsf + P::kSfbCol + 4 * (2 * j + h), desc_sf(sfb + 2048 * h + 512 * j));
+          for (int h = 0; h < P::kGroups; ++h)
+            tc2_copy_sf(tsf + P::kSfbCol + 4 * (P::kGroups * j + h),
+                        desc_sf(sfb + 2048 * h + 512 * j));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           tc2_mma(tmem, desc_sw128(st + 32 * j), desc_sw128(st + kABytes + 32 * j), P::kIdesc,
-                  tsf + P::kSfaCol + 4 * j, tsf + P::kSfbCol + 8 * j, (kt | j) != 0);
+                  tsf + P::kSfaCol + 4 * j, tsf + P::kSfbCol + 4 * P::kGroups * j, (kt | j) != 0);
         tc2_commit(smem_u32(empty + s));
         tc2_commit(empty1 + 8 * s);
       }
@@ -622,7 +643,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
   }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   tc_fence_after();
-  if (__all_sync(0xffffffffu, ok && !*gave_up)) store_rows<256>(tmem, warp, lane, m0, n0, args);
+  if (__all_sync(0xffffffffu, ok && !*gave_up)) store_rows<PN>(tmem, warp, lane, m0, n0, args);
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *gave_up) {
@@ -1094,11 +1115,11 @@ cudaError_t run_matmul_nvfp4(const uint8_t* a_packed, const uint8_t* a_scales,
     cudaError_t e = allow_dynamic_smem(g_smem_pair, k_matmul_nvfp4_pair, Pair::kSmemBytes);
     if (e != cudaSuccess) return e;
     CUtensorMap msa, msb;
-    if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, kBM) ||
+    if (!make_map(&ma, a_packed, m, k, kBM) || !make_map(&mb, b_packed, n, k, Pair::kBRows) ||
         !make_rows_map(&msa, a_scales, mma_scales_bytes(m, k) / 256) ||
         !make_rows_map(&msb, b_scales, mma_scales_bytes(n, k) / 256))
       return cudaErrorInvalidValue;
-    const int64_t pairs = ((m + 255) / 256) * ((n + 255) / 256);
+    const int64_t pairs = ((m + 255) / 256) * ((n + MX_MM_PAIR_N - 1) / MX_MM_PAIR_N);
     k_matmul_nvfp4_pair<<<(unsigned)(2 * pairs), 128, Pair::kSmemBytes, stream>>>(ma, mb, msa, msb,
                                                                                  args);
   } else {
