@@ -31,9 +31,12 @@
  *   - Layout of codes and scales: row-major, a row's codes in ceil(cols/2) bytes (element 2k in
  *     the low nibble of byte k, 2k+1 in the high nibble; an odd last element leaves the high
  *     nibble 0) and its scales in ceil(cols/N) bytes.  For cols % N == 0 that is rows*cols/2 and
- *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged") run on a row-wise path (one
- *     warp per row; cols up to 2^30, else MX_ERR_CUDA); in a grouped call they run on that path
- *     after the group's one launch over its whole-block tensors.
+ *     rows*cols/N bytes.  Tensors with cols % N != 0 ("ragged"; cols up to 2^30, else
+ *     MX_ERR_CUDA) run on ragged paths: bf16 rows on 16-byte boundaries (cols % 8 == 0) on the
+ *     whole-block kernels in a row-pitched mode (quantize and fake quantize for N >= 16, the error
+ *     reduction with recomputed codes for N >= 32) or through row tiles written by TMA
+ *     (dequantize to bf16, N >= 16); everything else on a row-wise kernel (one warp per row).  In
+ *     a grouped call they run after the group's one launch over its whole-block tensors.
  *   - rows == 0 or cols == 0 is an empty tensor: quantize / dequantize enqueue nothing,
  *     mx_error_stats writes an all-zero result and mx_global_scale writes 1.0.
  *   - x must be finite: NaN or Inf in x gives unspecified codes (no kernel faults or hangs).
