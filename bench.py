@@ -50,9 +50,9 @@ FMT_UE5M3 = 1
 L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) of one fused-pass launch over one 70B-shaped layer (7 tensors, N = 32,
 # UE5M3, device g), from the ncu capture summarised in
-# profiles/k_error_stats_bf16_fused_llama70b_layer_n32_ue5m3.md (1,711,739,392 read + 401,406,208
+# profiles/k_error_stats_bf16_fused_llama70b_layer_n32_ue5m3.md (1,711,382,272 read + 399,107,328
 # written; the last codes are still in L2 when the launch ends).
-FUSED_TRAFFIC_BYTES = 2113145600
+FUSED_TRAFFIC_BYTES = 2110489600
 
 
 def parse(argv=None):
