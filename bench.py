@@ -21,8 +21,8 @@ Python API from pinned host memory (inputs in, codes + scales + error records ou
 
 Other workloads (N = 1 only, reported under `other_workloads`): the bf16 4096x4096 sigma sweep
 (blocks 4..256 x E4M3/UE5M3), the Llama-2-7B-shaped weight set (32 layers, N = 32, UE5M3 + g), the
-activation tensor 16384x8192 with outlier channels (N = 16, E4M3), the fp32 256x256 tensor
-(latency per call).
+activation tensor 16384x8192 with outlier channels (N = 16, E4M3), a 16384x8200 tensor whose rows
+end in a ragged block (N = 32, UE5M3), the fp32 256x256 tensor (latency per call).
 
 --gpus N > 1 runs under torchrun, one process per GPU: every rank streams its own 80 seeded layers
 (weak scaling; the path has no exchange step), timing is the max over ranks.
@@ -798,6 +798,45 @@ def activation_workload(dev, stream, peak):
                         "flushed before each launch)", **res}
 
 
+def ragged_workload(dev, stream, peak):
+    """bf16 16384 x 8200 N(0, 0.02^2) (rows of 256 whole blocks of 32 and one of 8), UE5M3:
+    quantize + pack, dequantize (bf16), the fused quantize + pack + error reduction; one launch
+    each, L2 flushed before it."""
+    import torch
+    import fp4_microscaling_tensor_b200 as mx
+    from fp4_microscaling_tensor_b200 import inputs
+    rows, cols, n = 16384, 8200, 32
+    x = inputs.normal((rows, cols), 0.02, 8200, device=dev)
+    pb, nb = (cols + 1) // 2, -(-cols // n)
+    p = torch.empty(rows, pb, dtype=torch.uint8, device=dev)
+    s = torch.empty(rows, nb, dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    out = torch.empty(64, dtype=torch.uint8, device=dev)
+    ws = mx.stats_workspace(dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    nbytes = rows * cols * 2.0 + rows * (pb + nb)
+    res = {}
+    for name, fn in (
+            ("quantize_pack", lambda: mx.quantize(x, n, "ue5m3", packed=p, scales=s)),
+            ("dequantize", lambda: mx.dequantize(p, s, n, "ue5m3", out=y, cols=cols)),
+            ("quantize_pack_stats", lambda: mx.quantize_with_stats(
+                x, n, "ue5m3", packed=p, scales=s, out=out, workspace=ws))):
+        times = []
+        for _ in range(10):
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+            stream.synchronize()
+            times.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(times)
+        res[name] = {"gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak, "us": t * 1e6}
+    return {"workload": "bf16 16384x8200 N(0,0.02^2), N=32 (a ragged block of 8 per row), UE5M3 "
+                        "(L2 flushed before each launch)", **res}
+
+
 def small_tensor_latency(dev, stream, calls=1000):
     """Microseconds per call for the fp32 256 x 256 tensor (N = 32, E4M3): quantize, dequantize
     (fp32 out), error reduction from the stored codes, each replayed as one graph of `calls`."""
@@ -826,7 +865,8 @@ def other_workloads(dev, stream, peak):
     out = {}
     for name, fn in (("sweep_bf16_4096x4096", sweep_workload),
                      ("llama2_7b_weights", llama7b_workload),
-                     ("activations_16384x8192", activation_workload)):
+                     ("activations_16384x8192", activation_workload),
+                     ("ragged_16384x8200", ragged_workload)):
         try:
             out[name] = fn(dev, stream, peak)
         except Exception as e:  # reported, never fatal for the line

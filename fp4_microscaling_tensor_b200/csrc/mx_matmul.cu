@@ -31,6 +31,7 @@
 
 #include "mx_device.cuh"
 #include "mx_launch.h"
+#include "mx_tma.cuh"
 
 namespace mxk {
 namespace {
@@ -659,29 +660,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
   }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeTiled>(nullptr);
-    return reinterpret_cast<EncodeTiled>(p);
-  }();
-  return fn;
-}
 
 // Map of one operand's codes: rows x (k / 2) bytes, row pitch k / 2, boxes of box_rows x 128
 // bytes loaded with the 128-byte swizzle; rows past the end read as zero.
 bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k, int box_rows) {
-  const EncodeTiled enc = encode_fn();
+  const tma::EncodeTiledFn enc = tma::encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
@@ -694,7 +677,7 @@ bool make_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k, i
 
 // Map of a prepared scale array seen as rows of 256 bytes, boxes of 8 rows (one 2048-byte group).
 bool make_rows_map(CUtensorMap* map, const uint8_t* scales, int64_t rows) {
-  const EncodeTiled enc = encode_fn();
+  const tma::EncodeTiledFn enc = tma::encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[2] = {256, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {256};
@@ -1064,7 +1047,7 @@ __global__ void __launch_bounds__(dqmm::kThreads, 1)
 // Map of the weights' codes: n rows of k / 2 bytes, boxes of 256 rows x 32 bytes (one 64-element
 // step), no swizzle; rows past the end read as zero.
 bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t n, int64_t k) {
-  const EncodeTiled enc = encode_fn();
+  const tma::EncodeTiledFn enc = tma::encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)n};
   const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
@@ -1078,7 +1061,7 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t n, int64_t k
 // Map of the bf16 activations: m x k, row pitch 2 k bytes, boxes of 128 rows x 64 elements loaded
 // with the 128-byte swizzle; rows past the end read as zero.
 bool make_bf16_map(CUtensorMap* map, const void* a, int64_t m, int64_t k) {
-  const EncodeTiled enc = encode_fn();
+  const tma::EncodeTiledFn enc = tma::encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
   const cuuint64_t strides[1] = {(cuuint64_t)(2 * k)};
