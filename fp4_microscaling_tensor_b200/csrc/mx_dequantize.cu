@@ -5,11 +5,13 @@
 // scale (<= 4) and the FP16 g (<= 11) has at most 17 significant bits and stays inside the fp32
 // normal range, so y = e2m1 * (S g) is exact in fp32; bf16 output is its round-to-nearest-even.
 //
-// Layout mirrors the quantize kernel: a thread owns EPT consecutive codes (16 for bf16 output with
-// N >= 16, else 8), reads EPT/2 packed bytes and the scale byte(s) of its block(s), decodes the
-// codes, multiplies by the per-code constant S g from a
-// shared-memory table and writes 16-byte vectors.  Codes are decoded with exact bit arithmetic
-// (e2m1_scaled_bits_at), not with a conversion instruction.
+// Layout mirrors the quantize kernel: a thread owns EPT = 8 consecutive codes (MX_DQ_EPT_BF16 = 16
+// for bf16 output with N >= 16 was measured slower: 0.64 against 0.85 of the copy peak), two items
+// in flight, reads EPT/2 packed bytes and the scale byte(s) of its block(s), decodes the codes with
+// the E2M1x2 -> f16x2 conversion on the loaded word (exact: E2M1 values are f16 values; bit
+// arithmetic with MX_DQ_HWDEC = 0), multiplies by the per-code constant S g from a shared-memory
+// table and writes 16-byte vectors.  Ragged rows with bf16 output go through k_tile_dequantize
+// below: row tiles assembled in shared memory and written by TMA.
 #include <cuda_fp16.h>
 
 #include <atomic>

@@ -14,6 +14,11 @@
 // is: absmax, one multiply + snap + FP8 encode, one shared-memory lookup.  The grid is persistent
 // (a multiple of the SM count) and walks the items with a grid stride, two items per thread in
 // flight.  No kernel here waits on another CTA.
+//
+// Rows whose length the block size does not divide (cols % N != 0, bf16, cols % 8 == 0) use the
+// same kernel in its row-pitched mode (ROWS): each row's blocks rounded up to whole items, a
+// RowCursor turning the item index into (row, item), the chunks past a row's end neither read nor
+// written.
 #include "mx_device.cuh"
 #include "mx_launch.h"
 
