@@ -269,41 +269,6 @@ __device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, 
 #undef MX_PAIR_TAIL
 }
 
-// Error step of one word (two elements) whose codes were computed beforehand (the signed form of
-// qs_word8's error part, used where the codes of a whole item are converted first): every
-// element's scaled error d goes into the f32x2 sum of squares lt2 -- the max-valued ones included,
-// the first of them is taken out per block, see slice_finish_closed -- and the clipped elements
-// (|x| above S2 = RD_bf16(6 S g)) are counted per half in nsat2 as bf16x2 integers.
-template <int J>
-__device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
-                                              float sc, float nDq, uint32_t S2,
-                                              unsigned long long& lt2, uint32_t& nsat2) {
-  static_assert(J >= 0 && J < 4, "byte index");
-  asm("{\n\t"
-      ".reg .b32 blo, bhi, aw, t, m;\n\t"
-      ".reg .b64 x2, s2, b2, q2, d2;\n\t"
-      "mov.b64 x2, {%8, %9};\n\t"
-      "mov.b64 s2, {%3, %3};\n\t"
-      "mul.rn.f32x2 x2, x2, s2;\n\t"
-      "mul.lo.u32 t, %2, %6;\n\t"
-      "shr.s32 t, t, 6;\n\t"
-      "and.b32 blo, t, 0x81c00000;\n\t"
-      "mul.lo.u32 t, %2, %7;\n\t"
-      "shr.s32 t, t, 6;\n\t"
-      "and.b32 bhi, t, 0x81c00000;\n\t"
-      "mov.b64 b2, {blo, bhi};\n\t"
-      "mov.b64 q2, {%4, %4};\n\t"
-      "fma.rn.f32x2 d2, b2, q2, x2;\n\t"
-      "fma.rn.f32x2 %0, d2, d2, %0;\n\t"
-      "and.b32 aw, %10, 0x7fff7fff;\n\t"
-      "set.gt.bf16x2.bf16x2 m, aw, %5;\n\t"
-      "add.rn.bf16x2 %1, %1, m;\n\t"
-      "}"
-      : "+l"(lt2), "+r"(nsat2)
-      : "r"(cw), "f"(sc), "f"(nDq), "r"(S2), "n"(1u << (28 - 8 * J)), "n"(1u << (24 - 8 * J)),
-        "r"(lo), "r"(hi), "r"(w));
-}
-
 // |x| s for the two bf16 halves of aw, s a power of two given as its bf16 bit pattern sc16: two
 // mixed-precision FMAs (bf16 operands, fp32 result) take the halves straight from the word, so the
 // word needs no split into two fp32 values first.  Exact (a power-of-two scaling of a bf16 value).
@@ -317,6 +282,20 @@ __device__ __forceinline__ float2 mag_scaled2(uint32_t aw, uint32_t sc16) {
       : "=f"(lo), "=f"(hi)
       : "r"(aw), "r"(sc16));
   return make_float2(lo, hi);
+}
+
+// Code word of four bf16 words w0..w3 from their magnitude codes cm (byte k: word k's two codes,
+// sign bits clear): each code takes its element's sign bit.  Per word, bytes 1 and 3 (the halves'
+// high bytes) with their sign bit replicated over the byte (prmt selector nibbles with the top bit
+// set), then regrouped so that byte k of hs / ls holds the sign of word k's high / low half.
+__device__ __forceinline__ uint32_t put_signs(uint32_t cm, uint32_t w0, uint32_t w1, uint32_t w2,
+                                              uint32_t w3) {
+  uint32_t x01, x23, hs, ls;
+  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x01) : "r"(w0), "r"(w1));
+  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x23) : "r"(w2), "r"(w3));
+  asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(hs) : "r"(x01), "r"(x23));
+  asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(ls) : "r"(x01), "r"(x23));
+  return (cm | (hs & 0x80808080u)) | (ls & 0x08080808u);
 }
 
 // One code word's eight elements (words w[0..3], all in one block) with recomputed codes,
@@ -382,15 +361,7 @@ __device__ __forceinline__ uint32_t qs_word8(const uint32_t* w, const float* r, 
     asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(aw[k]), "r"(S2[k / PB]));
     asm("add.rn.bf16x2 %0, %0, %1;" : "+r"(nsat2) : "r"(m));
   }
-  // sign bits: per word, bytes 1 and 3 (the halves' high bytes) with their sign bit replicated
-  // over the byte (prmt selector nibbles with the top bit set), then regrouped so that byte k of
-  // hs / ls holds the sign of word k's high / low half
-  uint32_t x01, x23, hs, ls;
-  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x01) : "r"(w[0]), "r"(w[1]));
-  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(x23) : "r"(w[2]), "r"(w[3]));
-  asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(hs) : "r"(x01), "r"(x23));
-  asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(ls) : "r"(x01), "r"(x23));
-  return (cm | (hs & 0x80808080u)) | (ls & 0x08080808u);
+  return put_signs(cm, w[0], w[1], w[2], w[3]);
 }
 
 // True when one of the blocks (reciprocals r[0..nb)) is so far beyond its saturation that r / s
@@ -401,6 +372,17 @@ __device__ __forceinline__ bool deep_item(const float* r, float sc) {
 #pragma unroll
   for (int b = 1; b < NBL; ++b) mr = fmaxf(mr, r[b]);
   return __fmul_rn(mr, __frcp_rn(sc)) > 0x1p64f;
+}
+
+// One E2M1 conversion of two values: the code of lo in bits 0..3, of hi in bits 4..7.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.u32.u8 %0, b;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Tail of a block slice: lt / ms are the scaled squares of the other / the max-valued elements,
@@ -907,6 +889,11 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
 // item is redone exactly in double when squares could have been lost to fp32 underflow: a non-zero
 // block maximum with a sum below 2^-80, or (in a block summed apart) a non-zero scaled error below
 // 2^-63.
+// N = 4 goes further: each block pair's two blocks sit side by side in f32x2 form through the
+// whole item (qs4_pair), a block's reciprocal, scale value and clip level come from one 16-byte
+// shared-memory entry, and the split of the sums is made for both blocks of a pair with one test
+// (the per-block handling above runs only where a pair has a zero block, a dominating max element
+// or a possibly underflowed sum).  N = 8 and 16 reduce one code word at a time (qs_word8).
 
 // Quotients of two elements with their own reciprocals (see snap_quotient2).
 __device__ __forceinline__ float2 snap_quotient2v(float2 x, float2 r) {
@@ -940,6 +927,57 @@ __device__ __forceinline__ float bf16x2_hsum(uint32_t v) {
   return __fadd_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
+// Blocks of 4: one block pair (words w[0], w[1]: block 2j; w[2], w[3]: block 2j + 1) quantized and
+// reduced with the two blocks side by side in f32x2 form -- .x an element of block 2j, .y the
+// element at the same place in block 2j + 1 -- so that each pair operand (the reciprocals rq, the
+// code scalings nDq = -S g s 2^126, the sums lt) is the two blocks' own values and needs no copy.
+// As in qs_word8 the quotients are taken of magnitudes, xs = |x| s from the mixed-precision FMAs
+// with rq = r / s (DEEP: of the unscaled |x| with rq = r, for an item with a block so far beyond
+// its saturation that r / s would overflow), the magnitude codes decode with one shift and one
+// mask, and x's signs are put into the code word at the end.  S2a / S2b: the two blocks' clip
+// levels RD_bf16(6 S g), twice; clipped elements are counted in nsat2 (bf16x2 integers).
+template <bool DEEP>
+__device__ __forceinline__ uint32_t qs4_pair(const uint32_t* w, float2 rq, float2 nDq,
+                                             uint32_t S2a, uint32_t S2b, float sc, uint32_t sc16,
+                                             float2& lt, uint32_t& nsat2) {
+  uint32_t aw[4];
+  float2 xs[4], xq[4];  // per word: (low half, high half) scaled, and the quotients' operands
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    aw[k] = w[k] & 0x7FFF7FFFu;
+    if constexpr (!DEEP) {
+      xs[k] = mag_scaled2(aw[k], sc16);
+      xq[k] = xs[k];
+    } else {
+      xq[k] = make_float2(__uint_as_float(aw[k] << 16), __uint_as_float(aw[k] & 0xFFFF0000u));
+      xs[k] = __fmul2_rn(xq[k], make_float2(sc, sc));
+    }
+  }
+  // element pair p: half p & 1 of word p >> 1 in each block
+  float2 X[4], Q[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int m = p >> 1;
+    X[p] = (p & 1) ? make_float2(xs[m].y, xs[m + 2].y) : make_float2(xs[m].x, xs[m + 2].x);
+    const float2 o = (p & 1) ? make_float2(xq[m].y, xq[m + 2].y) : make_float2(xq[m].x, xq[m + 2].x);
+    const float2 y = __ffma2_rn(o, rq, make_float2(48.0f, 48.0f));
+    Q[p] = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
+  }
+  // byte k of cm: word k's two magnitude codes (words 0, 1 from the .x lanes, 2, 3 from the .y)
+  const uint32_t cm = cvt_e2m1x8(Q[0].x, Q[1].x, Q[2].x, Q[3].x, Q[0].y, Q[1].y, Q[2].y, Q[3].y);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    // nibble 4p holds pair p's .x code, nibble 16 + 4p its .y code: magnitude bits to 22..24
+    const uint32_t bx = (cm << (22 - 4 * p)) & 0x01C00000u;
+    const uint32_t by = (p < 2 ? cm << (6 - 4 * p) : cm >> (4 * p - 6)) & 0x01C00000u;
+    const float2 d = __ffma2_rn(make_float2(__uint_as_float(bx), __uint_as_float(by)), nDq, X[p]);
+    lt = __ffma2_rn(d, d, lt);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) nsat2 = bf16x2_add(nsat2, bf16x2_set_gt(aw[k], k < 2 ? S2a : S2b));
+  return put_signs(cm, w[0], w[1], w[2], w[3]);
+}
+
 // Item shape of the small-block kernel: 16 elements for N = 4 (four blocks), 32 for N = 8 and 16
 // (four or two blocks), so that blocks always come in pairs.
 #ifndef MX_QS_EPT8  // elements per item of the small-block kernel for N = 8 (16 or 32)
@@ -965,11 +1003,21 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
   constexpr int NP = NB / 2;
   static_assert(NB % 2 == 0 && NB <= 4 && (NCW == 2 || NCW == 4), "2 or 4 blocks per item");
   __shared__ float s_rcp[256], s_D[256];
+  // N = 4: per scale code {1 / (S g) (0 for S = 0), S g, the clip level RD_bf16(6 S g) twice as
+  // bf16x2 bits (the largest finite bf16 for S = 0, which no finite |x| exceeds), unused}
+  __shared__ float4 s_tab[N == 4 ? 256 : 1];
   const float g = fp16_bits_to_float(tensor_g_bits(wk.t.g_bits, wk.t.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);
-    s_D[c] = D;
-    s_rcp[c] = D > 0.0f ? __frcp_rn(D) : 0.0f;
+    const float rcp = D > 0.0f ? __frcp_rn(D) : 0.0f;
+    if constexpr (N == 4) {
+      uint32_t thr = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // exact product, truncated
+      if (thr == 0u) thr = 0x7F7Fu;
+      s_tab[c] = make_float4(rcp, D, __uint_as_float(thr * 0x10001u), 0.0f);
+    } else {
+      s_D[c] = D;
+      s_rcp[c] = rcp;
+    }
   }
   const float r6 = __frcp_rn(__fmul_rn(6.0f, g));
   const float sat_thr = __fmul_rn(__fmul_rn(6.0f, g), scale_max<FMT>());  // exact
@@ -1014,7 +1062,162 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     // E clamped to [1, 253]: sc = 2^(127 - E) stays a normal number (see SliceSetup)
     const int E = min(max((int)(max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu) >> 7), 1), 253);
     const float sc = __uint_as_float((uint32_t)(254 - E) << 23);
-    // scale codes, reciprocals and per-block constants, two blocks at a time
+    if constexpr (N == 4) {
+      // Blocks of 4: the item's two block pairs, each with its blocks side by side in f32x2 form
+      // (qs4_pair); the per-block split of the sums is made for both blocks of a pair at once
+      // where neither needs the special handling below (a zero block, a block whose max element
+      // dominates its sum, or a sum that could have lost squares to underflow).
+      const float rcs = __uint_as_float((uint32_t)E << 23);  // 1 / sc, exact
+      const uint32_t sc16 = __float_as_uint(sc) >> 16;       // sc as a bf16 (a power of two)
+      float2 af[2], r2[2], D2[2], nDq2[2], rs2[2];
+      uint32_t S2[4];
+      uint32_t sc_all = 0, ss2 = 0;  // scale bytes; saturated-scale count
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        af[j] = make_float2(__uint_as_float(M[j] << 16), __uint_as_float(M[j] & 0xFFFF0000u));
+        const float2 u = __fmul2_rn(af[j], make_float2(r6, r6));
+        uint32_t s0, s1;
+        if constexpr (FMT == kE4M3) {
+          unsigned short h;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+              : "=h"(h) : "f"(snap21(u.y)), "f"(snap21(u.x)));
+          s0 = h & 0xFFu;
+          s1 = (uint32_t)h >> 8;
+        } else {
+          s0 = encode_scale<FMT>(snap21(u.x));
+          s1 = encode_scale<FMT>(snap21(u.y));
+        }
+        sc_all |= (s0 | (s1 << 8)) << (16 * j);
+        const float4 t0 = s_tab[s0], t1 = s_tab[s1];
+        r2[j] = make_float2(t0.x, t1.x);
+        D2[j] = make_float2(t0.y, t1.y);
+        S2[2 * j] = __float_as_uint(t0.z);
+        S2[2 * j + 1] = __float_as_uint(t1.z);
+        nDq2[j] = __fmul2_rn(__fmul2_rn(D2[j], make_float2(sc, sc)),
+                             make_float2(-0x1p126f, -0x1p126f));
+        rs2[j] = __fmul2_rn(r2[j], make_float2(rcs, rcs));  // r / s (see qs_word8)
+        ss2 = bf16x2_add(ss2, bf16x2_set_gt(M[j], SAT2));
+      }
+      const bool deep = fmaxf(fmaxf(rs2[0].x, rs2[0].y), fmaxf(rs2[1].x, rs2[1].y)) > 0x1p64f;
+      uint32_t cw[2];
+      float2 lt[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      uint32_t nsat2 = 0u;
+      if (!deep) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          cw[j] = qs4_pair<false>(&it.w[4 * j], rs2[j], nDq2[j], S2[2 * j], S2[2 * j + 1], sc,
+                                  sc16, lt[j], nsat2);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          cw[j] = qs4_pair<true>(&it.w[4 * j], r2[j], nDq2[j], S2[2 * j], S2[2 * j + 1], sc,
+                                 sc16, lt[j], nsat2);
+      }
+      if constexpr (STORE) {
+        if (ok) {
+          *reinterpret_cast<uint2*>(packed_out + i * 8) = make_uint2(cw[0], cw[1]);
+          *reinterpret_cast<uint32_t*>(scales_out + i * 4) = sc_all;
+        }
+      }
+      float2 ae2 = make_float2(0.0f, 0.0f), am2 = make_float2(0.0f, 0.0f);
+      float az = 0.0f, nz = 0.0f;  // zero blocks' sums and their count
+      bool exact = false;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        // the two blocks' max elements: code of a / (S g) (unscaled quotients, which never
+        // overflow), scaled error, square
+        const float2 y = __ffma2_rn(af[j], r2[j], make_float2(48.0f, 48.0f));
+        const float2 qa = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
+        const uint32_t ca = cvt_e2m1x2(qa.y, qa.x);
+        const float2 dec = make_float2(__uint_as_float((ca << 22) & 0x01C00000u),
+                                       __uint_as_float((ca << 18) & 0x01C00000u));
+        const float2 dm = __ffma2_rn(dec, nDq2[j], __fmul2_rn(af[j], make_float2(sc, sc)));
+        const float2 f2 = __fmul2_rn(dm, dm);
+        const float2 rest = __ffma2_rn(f2, make_float2(-1.0f, -1.0f), lt[j]);
+        const float2 lim = __fmul2_rn(f2, make_float2(0x1p-6f, 0x1p-6f));
+        const bool plain = D2[j].x > 0.0f && D2[j].y > 0.0f && !(rest.x < lim.x) &&
+                           !(rest.y < lim.y) && !(lt[j].x < 0x1p-80f) && !(lt[j].y < 0x1p-80f);
+        if (plain) {
+          ae2 = __fadd2_rn(ae2, rest);
+          am2 = __fadd2_rn(am2, f2);
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int b = 2 * j + h;
+            const float tb = h ? lt[j].y : lt[j].x;
+            const float first = h ? f2.y : f2.x;
+            const float ab = h ? af[j].y : af[j].x;
+            const float Db = h ? D2[j].y : D2[j].x;
+            const float nDqb = h ? nDq2[j].y : nDq2[j].x;
+            exact |= ab > 0.0f && tb < 0x1p-80f;
+            if (Db > 0.0f) {
+              float rb = __fsub_rn(tb, first);
+              if (rb < __fmul_rn(first, 0x1p-6f)) {
+                // dmax^2 dominates the block: sum the elements below the maximum apart (no
+                // cancellation) and add the other max-valued elements' copies of dmax^2
+                float rs = 0.0f, nt = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int e = b * 4 + k;
+                  const uint32_t wd = it.w[e >> 1];
+                  const float xv = (e & 1) ? bf16hi(wd) : bf16lo(wd);
+                  const float dq = __uint_as_float(e2m1_scaled_bits_at(cw[e >> 3], 4 * (e & 7)));
+                  const float d = __fmaf_rn(dq, nDqb, __fmul_rn(xv, sc));
+                  if (fabsf(xv) != ab) rs = __fmaf_rn(d, d, rs);
+                  else nt += 1.0f;
+                  exact |= d != 0.0f && fabsf(d) < 0x1p-63f;  // its square would be lost
+                }
+                rb = __fmaf_rn(nt - 1.0f, first, rs);
+              }
+              if (h) {
+                ae2.y = __fadd_rn(ae2.y, rb);
+                am2.y = __fadd_rn(am2.y, first);
+              } else {
+                ae2.x = __fadd_rn(ae2.x, rb);
+                am2.x = __fadd_rn(am2.x, first);
+              }
+            } else {
+              az = __fadd_rn(az, tb);
+              nz += 1.0f;
+            }
+          }
+        }
+      }
+      if (!exact) {
+        const double us = unscale_sq(E);
+        acc.elem += (double)__fadd_rn(ae2.x, ae2.y) * us;
+        acc.mx += (double)__fadd_rn(am2.x, am2.y) * us;
+        acc.zero += (double)az * us;
+      } else {
+        // exact in double, block by block (first max element by index)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int e0 = b * 4;
+          auto xval = [&](int k) {
+            const uint32_t wd = it.w[(e0 + k) >> 1];
+            return ((e0 + k) & 1) ? bf16hi(wd) : bf16lo(wd);
+          };
+          auto code = [&](int k) { return cw[(e0 + k) >> 3] >> (4 * ((e0 + k) & 7)); };
+          const float ab = (b & 1) ? af[b >> 1].y : af[b >> 1].x;
+          const float Db = (b & 1) ? D2[b >> 1].y : D2[b >> 1].x;
+          double rest = 0.0, first = 0.0, others = 0.0;
+          exact_slice<4, false>(ab, Db, xval, code, rest, first, others);
+          if (Db > 0.0f) {
+            acc.elem += rest + others;
+            acc.mx += first;
+          } else {
+            acc.zero += rest + first + others;
+          }
+        }
+      }
+      if (ok) {
+        acc.n_esat += bf16x2_hsum(nsat2);
+        acc.n_zero_f += nz;
+        acc.n_ssat_f += bf16x2_hsum(ss2);
+      }
+      return;
+    }
+    // N = 8, 16: scale codes, reciprocals and per-block constants, two blocks at a time
     float r_b[NB], D_b[NB], nDq_b[NB];
     uint32_t S2_b[NB];
     uint32_t sc_all = 0, zc2 = 0, ss2 = 0;  // scale bytes; zero-block and saturated-scale counts
@@ -1057,58 +1260,25 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     }
     // codes and every element's scaled square (into its block's sum), one code word at a time;
     // clipped elements counted
-    // (measured: for N = 4, converting the item's codes first and then reducing is faster)
-    constexpr int PB = BW < 4 ? BW : 4;  // pairs per block inside a code word
+    constexpr int PB = 4;  // a code word's four words lie in one block (N >= 8)
     uint32_t cw[NCW];
     float2 lt[NB];
     uint32_t nsat2 = 0u;
 #pragma unroll
     for (int b = 0; b < NB; ++b) lt[b] = make_float2(0.0f, 0.0f);
-    if constexpr (N >= 8) {
-      if (!deep_item<NB>(r_b, sc)) {
+    if (!deep_item<NB>(r_b, sc)) {
 #pragma unroll
-        for (int c = 0; c < NCW; ++c) {
-          const int b0 = (4 * c) / BW;  // block of the code word's first pair
-          cw[c] = qs_word8<PB, kFast>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
-                                      nsat2);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < NCW; ++c) {
-          const int b0 = (4 * c) / BW;
-          cw[c] = qs_word8<PB, kDeep>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
-                                      nsat2);
-        }
+      for (int c = 0; c < NCW; ++c) {
+        const int b0 = (4 * c) / BW;  // block of the code word's first pair
+        cw[c] = qs_word8<PB, kFast>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                    nsat2);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < NCW; ++c) {
-        float q[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int wi = 4 * c + k;
-          const uint32_t w = it.w[wi];
-          const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
-          q[2 * k] = qq.x;
-          q[2 * k + 1] = qq.y;
-        }
-        cw[c] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-      }
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        unsigned long long l2 = 0ull;
-#pragma unroll
-        for (int k = 0; k < BW; ++k) {
-          const int wi = b * BW + k;
-          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, c = cw[wi >> 2];
-          switch (wi & 3) {
-            case 0: pair_step_all<0>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
-            case 1: pair_step_all<1>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
-            case 2: pair_step_all<2>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
-            default: pair_step_all<3>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
-          }
-        }
-        asm("mov.b64 {%0, %1}, %2;" : "=f"(lt[b].x), "=f"(lt[b].y) : "l"(l2));
+        const int b0 = (4 * c) / BW;
+        cw[c] = qs_word8<PB, kDeep>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                    nsat2);
       }
     }
     if constexpr (STORE) {
