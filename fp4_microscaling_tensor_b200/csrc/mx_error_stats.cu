@@ -269,6 +269,41 @@ __device__ __forceinline__ void pair_step(uint32_t w, uint32_t lo, uint32_t hi, 
 #undef MX_PAIR_TAIL
 }
 
+// Error step of one word (two elements) whose codes were computed beforehand (the signed form of
+// qs_word8's error part, used where the codes of a whole item are converted first): every
+// element's scaled error d goes into the f32x2 sum of squares lt2 -- the max-valued ones included,
+// the first of them is taken out per block, see slice_finish_closed -- and the clipped elements
+// (|x| above S2 = RD_bf16(6 S g)) are counted per half in nsat2 as bf16x2 integers.
+template <int J>
+__device__ __forceinline__ void pair_step_all(uint32_t w, uint32_t lo, uint32_t hi, uint32_t cw,
+                                              float sc, float nDq, uint32_t S2,
+                                              unsigned long long& lt2, uint32_t& nsat2) {
+  static_assert(J >= 0 && J < 4, "byte index");
+  asm("{\n\t"
+      ".reg .b32 blo, bhi, aw, t, m;\n\t"
+      ".reg .b64 x2, s2, b2, q2, d2;\n\t"
+      "mov.b64 x2, {%8, %9};\n\t"
+      "mov.b64 s2, {%3, %3};\n\t"
+      "mul.rn.f32x2 x2, x2, s2;\n\t"
+      "mul.lo.u32 t, %2, %6;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 blo, t, 0x81c00000;\n\t"
+      "mul.lo.u32 t, %2, %7;\n\t"
+      "shr.s32 t, t, 6;\n\t"
+      "and.b32 bhi, t, 0x81c00000;\n\t"
+      "mov.b64 b2, {blo, bhi};\n\t"
+      "mov.b64 q2, {%4, %4};\n\t"
+      "fma.rn.f32x2 d2, b2, q2, x2;\n\t"
+      "fma.rn.f32x2 %0, d2, d2, %0;\n\t"
+      "and.b32 aw, %10, 0x7fff7fff;\n\t"
+      "set.gt.bf16x2.bf16x2 m, aw, %5;\n\t"
+      "add.rn.bf16x2 %1, %1, m;\n\t"
+      "}"
+      : "+l"(lt2), "+r"(nsat2)
+      : "r"(cw), "f"(sc), "f"(nDq), "r"(S2), "n"(1u << (28 - 8 * J)), "n"(1u << (24 - 8 * J)),
+        "r"(lo), "r"(hi), "r"(w));
+}
+
 // |x| s for the two bf16 halves of aw, s a power of two given as its bf16 bit pattern sc16: two
 // mixed-precision FMAs (bf16 operands, fp32 result) take the halves straight from the word, so the
 // word needs no split into two fp32 values first.  Exact (a power-of-two scaling of a bf16 value).
@@ -889,11 +924,16 @@ __global__ void __launch_bounds__(kThreads, N <= 8 ? MX_ST_MINB_SMALL : MX_ST_MI
 // item is redone exactly in double when squares could have been lost to fp32 underflow: a non-zero
 // block maximum with a sum below 2^-80, or (in a block summed apart) a non-zero scaled error below
 // 2^-63.
-// N = 4 goes further: each block pair's two blocks sit side by side in f32x2 form through the
-// whole item (qs4_pair), a block's reciprocal, scale value and clip level come from one 16-byte
-// shared-memory entry, and the split of the sums is made for both blocks of a pair with one test
-// (the per-block handling above runs only where a pair has a zero block, a dominating max element
-// or a possibly underflowed sum).  N = 8 and 16 reduce one code word at a time (qs_word8).
+// N = 4 with UE5M3 scales goes further: each block pair's two blocks sit side by side in f32x2
+// form through the whole item (qs4_pair), a block's reciprocal, scale value and clip level come
+// from one 16-byte shared-memory entry, and the split of the sums is made for both blocks of a
+// pair with one test (the per-block handling above runs only where a pair has a zero block, a
+// dominating max element or a possibly underflowed sum).  N = 4 with E4M3 scales keeps the
+// per-block form: without a global scale, data of small magnitude puts E4M3 scales in its coarse
+// subnormal range, where a block's max element often dominates its sum; some lane of nearly every
+// warp then needs the per-block handling, and the pair test only adds to it (measured: 0.41 of the
+// copy peak per-block against 0.37 paired on a 70B-shaped layer, while UE5M3 goes from 0.44 to
+// 0.52).  N = 8 and 16 reduce one code word at a time (qs_word8).
 
 // Quotients of two elements with their own reciprocals (see snap_quotient2).
 __device__ __forceinline__ float2 snap_quotient2v(float2 x, float2 r) {
@@ -927,10 +967,11 @@ __device__ __forceinline__ float bf16x2_hsum(uint32_t v) {
   return __fadd_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
-// Blocks of 4: one block pair (words w[0], w[1]: block 2j; w[2], w[3]: block 2j + 1) quantized and
-// reduced with the two blocks side by side in f32x2 form -- .x an element of block 2j, .y the
-// element at the same place in block 2j + 1 -- so that each pair operand (the reciprocals rq, the
-// code scalings nDq = -S g s 2^126, the sums lt) is the two blocks' own values and needs no copy.
+// Blocks of 4 (UE5M3): one block pair (words w[0], w[1]: block 2j; w[2], w[3]: block 2j + 1)
+// quantized and reduced with the two blocks side by side in f32x2 form -- .x an element of block
+// 2j, .y the element at the same place in block 2j + 1 -- so that each pair operand (the
+// reciprocals rq, the code scalings nDq = -S g s 2^126, the sums lt) is the two blocks' own values
+// and needs no copy.
 // As in qs_word8 the quotients are taken of magnitudes, xs = |x| s from the mixed-precision FMAs
 // with rq = r / s (DEEP: of the unscaled |x| with rq = r, for an item with a block so far beyond
 // its saturation that r / s would overflow), the magnitude codes decode with one shift and one
@@ -959,7 +1000,8 @@ __device__ __forceinline__ uint32_t qs4_pair(const uint32_t* w, float2 rq, float
   for (int p = 0; p < 4; ++p) {
     const int m = p >> 1;
     X[p] = (p & 1) ? make_float2(xs[m].y, xs[m + 2].y) : make_float2(xs[m].x, xs[m + 2].x);
-    const float2 o = (p & 1) ? make_float2(xq[m].y, xq[m + 2].y) : make_float2(xq[m].x, xq[m + 2].x);
+    const float2 o =
+        (p & 1) ? make_float2(xq[m].y, xq[m + 2].y) : make_float2(xq[m].x, xq[m + 2].x);
     const float2 y = __ffma2_rn(o, rq, make_float2(48.0f, 48.0f));
     Q[p] = __fadd2_rn(y, make_float2(-48.0f, -48.0f));
   }
@@ -1002,15 +1044,18 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
   constexpr int EPT = QSShape<N>::EPT, NW = EPT / 2, NCW = EPT / 8, NB = EPT / N, BW = N / 2;
   constexpr int NP = NB / 2;
   static_assert(NB % 2 == 0 && NB <= 4 && (NCW == 2 || NCW == 4), "2 or 4 blocks per item");
+  // Blocks of 4 with UE5M3 scales take the block-pair form (qs4_pair); E4M3 keeps the per-block
+  // form, which measured faster there (see the note above qs4_pair)
+  constexpr bool PAIRS4 = N == 4 && FMT == kUE5M3;
   __shared__ float s_rcp[256], s_D[256];
-  // N = 4: per scale code {1 / (S g) (0 for S = 0), S g, the clip level RD_bf16(6 S g) twice as
+  // PAIRS4: per scale code {1 / (S g) (0 for S = 0), S g, the clip level RD_bf16(6 S g) twice as
   // bf16x2 bits (the largest finite bf16 for S = 0, which no finite |x| exceeds), unused}
-  __shared__ float4 s_tab[N == 4 ? 256 : 1];
+  __shared__ float4 s_tab[PAIRS4 ? 256 : 1];
   const float g = fp16_bits_to_float(tensor_g_bits(wk.t.g_bits, wk.t.g_dev));
   for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     const float D = __fmul_rn(scale_value(c, FMT), g);
     const float rcp = D > 0.0f ? __frcp_rn(D) : 0.0f;
-    if constexpr (N == 4) {
+    if constexpr (PAIRS4) {
       uint32_t thr = __float_as_uint(__fmul_rn(6.0f, D)) >> 16;  // exact product, truncated
       if (thr == 0u) thr = 0x7F7Fu;
       s_tab[c] = make_float4(rcp, D, __uint_as_float(thr * 0x10001u), 0.0f);
@@ -1062,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     // E clamped to [1, 253]: sc = 2^(127 - E) stays a normal number (see SliceSetup)
     const int E = min(max((int)(max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu) >> 7), 1), 253);
     const float sc = __uint_as_float((uint32_t)(254 - E) << 23);
-    if constexpr (N == 4) {
+    if constexpr (PAIRS4) {
       // Blocks of 4: the item's two block pairs, each with its blocks side by side in f32x2 form
       // (qs4_pair); the per-block split of the sums is made for both blocks of a pair at once
       // where neither needs the special handling below (a zero block, a block whose max element
@@ -1217,7 +1262,7 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
       }
       return;
     }
-    // N = 8, 16: scale codes, reciprocals and per-block constants, two blocks at a time
+    // scale codes, reciprocals and per-block constants, two blocks at a time
     float r_b[NB], D_b[NB], nDq_b[NB];
     uint32_t S2_b[NB];
     uint32_t sc_all = 0, zc2 = 0, ss2 = 0;  // scale bytes; zero-block and saturated-scale counts
@@ -1260,25 +1305,58 @@ __global__ void __launch_bounds__(kThreads, MX_QS_MINB)
     }
     // codes and every element's scaled square (into its block's sum), one code word at a time;
     // clipped elements counted
-    constexpr int PB = 4;  // a code word's four words lie in one block (N >= 8)
+    // (measured: for N = 4, converting the item's codes first and then reducing is faster)
+    constexpr int PB = BW < 4 ? BW : 4;  // pairs per block inside a code word
     uint32_t cw[NCW];
     float2 lt[NB];
     uint32_t nsat2 = 0u;
 #pragma unroll
     for (int b = 0; b < NB; ++b) lt[b] = make_float2(0.0f, 0.0f);
-    if (!deep_item<NB>(r_b, sc)) {
+    if constexpr (N >= 8) {
+      if (!deep_item<NB>(r_b, sc)) {
 #pragma unroll
-      for (int c = 0; c < NCW; ++c) {
-        const int b0 = (4 * c) / BW;  // block of the code word's first pair
-        cw[c] = qs_word8<PB, kFast>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
-                                    nsat2);
+        for (int c = 0; c < NCW; ++c) {
+          const int b0 = (4 * c) / BW;  // block of the code word's first pair
+          cw[c] = qs_word8<PB, kFast>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                      nsat2);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < NCW; ++c) {
+          const int b0 = (4 * c) / BW;
+          cw[c] = qs_word8<PB, kDeep>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
+                                      nsat2);
+        }
       }
     } else {
 #pragma unroll
       for (int c = 0; c < NCW; ++c) {
-        const int b0 = (4 * c) / BW;
-        cw[c] = qs_word8<PB, kDeep>(&it.w[4 * c], &r_b[b0], &nDq_b[b0], &S2_b[b0], sc, &lt[b0],
-                                    nsat2);
+        float q[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int wi = 4 * c + k;
+          const uint32_t w = it.w[wi];
+          const float2 qq = snap_quotient2(w << 16, w & 0xFFFF0000u, r_b[wi / BW]);
+          q[2 * k] = qq.x;
+          q[2 * k + 1] = qq.y;
+        }
+        cw[c] = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        unsigned long long l2 = 0ull;
+#pragma unroll
+        for (int k = 0; k < BW; ++k) {
+          const int wi = b * BW + k;
+          const uint32_t w = it.w[wi], lo = w << 16, hi = w & 0xFFFF0000u, c = cw[wi >> 2];
+          switch (wi & 3) {
+            case 0: pair_step_all<0>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            case 1: pair_step_all<1>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            case 2: pair_step_all<2>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+            default: pair_step_all<3>(w, lo, hi, c, sc, nDq_b[b], S2_b[b], l2, nsat2); break;
+          }
+        }
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lt[b].x), "=f"(lt[b].y) : "l"(l2));
       }
     }
     if constexpr (STORE) {
