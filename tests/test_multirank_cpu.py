@@ -55,7 +55,7 @@ def worker(rank, world, port, out):
 def test_two_ranks_gloo():
     world = 2
     port = free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this (threaded) process
         out = m.dict()
         mp.spawn(worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
@@ -96,7 +96,7 @@ def test_row_sharded_tensor_combines_to_whole():
     from fp4_microscaling_tensor_b200 import inputs
     world = 2
     port = free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of this (threaded) process
         out = m.dict()
         mp.spawn(shard_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
